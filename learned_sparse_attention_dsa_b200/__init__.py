@@ -1,0 +1,23 @@
+"""DeepSeek Sparse Attention (DSA) forward path for NVIDIA B200 (sm_100a).
+
+Three stages, each a hand-written CUDA kernel behind a C ABI (``libdsa.so``,
+declared in ``include/dsa.h``):
+
+  indexer_scores   I[t,s] = sum_j w[t,j] * ReLU(q^I[t,j] . k^I[s]), s <= t
+  topk             S_t = the k largest I[t,s], ties to the lower s
+  sparse_attn      softmax attention of every query head over S_t
+  forward          the three back to back on one stream
+
+The Python functions are argument marshalling only; every step runs in the
+CUDA library, which is loaded on first use and raises if it is missing.
+"""
+from .inputs import WORKLOADS, Workload, make_inputs, to_device  # noqa: F401
+
+
+def __getattr__(name):
+    # The binding loads libdsa.so; import it lazily so that CPU-only users of
+    # the input generator do not need the CUDA library.
+    from . import binding
+    if hasattr(binding, name):
+        return getattr(binding, name)
+    raise AttributeError(name)
