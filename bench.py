@@ -1,0 +1,475 @@
+"""Benchmark of the DSA forward path (indexer -> top-k -> sparse attention).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step is one dsa_forward call over one batch of synthetic input: the
+lightning-indexer scores, the top-k selection and the attention over the
+selected rows. The default workload is the decode step of 32 sequences at
+context 32,768 with k = 2048 (16 query heads sharing one 128-wide KV head);
+its unit is decode steps per second. Prefill workloads report tokens per
+second. Rank 0 prints one JSON line.
+
+Timing: W untimed warm-up steps, then exactly K steps between two CUDA events
+on the launching stream, bracketed by a barrier and a device synchronize,
+max over ranks. Every step streams the 268 MB indexer-key cache (larger than
+the 126 MB L2), so L2 is not flushed between steps. Per-stage times (for the
+roofline) are taken the same way in separate loops after the main region.
+--impl reference times the CPU oracle on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from learned_sparse_attention_dsa_b200.inputs import WORKLOADS, make_inputs, to_device  # noqa: E402
+
+METRIC = "prefill tokens/s and decode steps/s at k=2048; % HBM/tensor roofline per stage"
+
+
+# ------------------------------------------------------------------ helpers
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+def stage_work(wl):
+    """Algorithmic bytes and flops per forward pass, per stage.
+
+    indexer: reads K^I once, q^I and w once, writes one fp32 score per causal
+             pair; flops = 2 * H_I * d_I per causal pair (the contraction).
+    top-k:   reads one fp32 score per causal pair, writes k int32 per row.
+    attn:    reads each selected KV row once per KV head (K and V; a V that is
+             a view of the K row adds nothing), Q once, writes the output;
+             flops = 2 * Hq * (Dqk + Dv) per selected row.
+    """
+    eb = 4 if wl.dtype == "f32" else 2
+    rows = wl.B * wl.Tq
+    pairs = wl.causal_pairs()
+    sel = wl.selected_rows()
+    idx_bytes = (wl.B * wl.L * wl.d_I * eb + rows * wl.H_I * wl.d_I * eb + rows * wl.H_I * 4
+                 + pairs * 4)
+    idx_flops = 2.0 * wl.H_I * wl.d_I * pairs
+    topk_bytes = pairs * 4 + rows * wl.k * 4
+    kv_row = wl.Hkv * (wl.Dqk if wl.kv_alias else wl.Dqk + wl.Dv) * eb
+    attn_bytes = sel * kv_row + rows * wl.Hq * (wl.Dqk + wl.Dv) * eb + rows * wl.k * 4
+    attn_flops = 2.0 * wl.Hq * (wl.Dqk + wl.Dv) * sel
+    return {"indexer": (idx_bytes, idx_flops), "topk": (topk_bytes, 0.0), "attn": (attn_bytes, attn_flops)}
+
+
+class ClockSampler:
+    """Polls NVML for SM clock and throttle reasons on a background thread."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown", 0x1: "gpu_idle",
+               0x2: "applications_clocks_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.002):
+        self.samples = []
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thread = None
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # NVML missing: no clock record
+            self._nvml = None
+
+    def _run(self):
+        nv = self._nvml
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                self.samples.append((time.perf_counter(), mhz, reasons))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self._nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
+
+    def summary(self, t0: float, t1: float):
+        if self._nvml is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "NVML unavailable"}
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        note = "sampled during the timed region"
+        if not inside:  # region shorter than the polling period: nearest samples
+            inside = sorted(self.samples, key=lambda s: min(abs(s[0] - t0), abs(s[0] - t1)))[:3]
+            note = "timed region shorter than the polling period; nearest samples"
+        mhz = [s[1] for s in inside]
+        mask = 0
+        for s in inside:
+            mask |= int(s[2])
+        reasons = [name for bit, name in self.REASONS.items() if mask & bit and name != "gpu_idle"]
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(inside), "note": note}
+
+
+def _dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def _max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def _units(wl, steps: int) -> tuple[float, str]:
+    if wl.is_decode:
+        return float(steps), "decode steps/s"
+    return float(steps * wl.B * wl.Tq), "prefill tokens/s"
+
+
+# ------------------------------------------------------------------ oracle timing
+
+def time_oracle(wl, cpu, n_rows: int, nthreads: int = 0):
+    """Run the CPU oracle on the first n_rows query rows (flat order, evenly
+    spread over the batch) and return (seconds, rows)."""
+    import oracle
+
+    def bits(t):
+        t = t.contiguous()
+        return t.view(torch.int16).numpy().view(np.uint16) if t.dtype == torch.bfloat16 else t.numpy()
+
+    total = wl.B * wl.Tq
+    flat = np.linspace(0, total - 1, num=min(n_rows, total)).round().astype(np.int64)
+    row_b = (flat // wl.Tq).astype(np.int32)
+    row_i = (flat % wl.Tq).astype(np.int32)
+    row_t = row_i + wl.q_pos0
+    q_idx = bits(cpu["q_idx"][row_b, row_i])
+    w = cpu["w"][row_b, row_i].numpy()
+    q = bits(cpu["q"][row_b, row_i])
+    kc = cpu["k_cache"]
+    kbuf = bits(kc)
+    ks = (kc.shape[1] * kc.shape[2] * kc.shape[3], kc.shape[2] * kc.shape[3], kc.shape[3])
+    if wl.kv_alias:
+        vbuf, vs = kbuf, ks
+    else:
+        vc = cpu["v_cache"]
+        vbuf = bits(vc)
+        vs = (vc.shape[1] * vc.shape[2] * vc.shape[3], vc.shape[2] * vc.shape[3], vc.shape[3])
+    k_idx = bits(cpu["k_idx"])
+    t0 = time.perf_counter()
+    scores = oracle.indexer_rows(q_idx, w, k_idx, row_b, row_t, nthreads)
+    idx = oracle.topk_rows(scores, row_t, wl.k, nthreads)
+    oracle.attn_rows(q, kbuf, vbuf, idx, row_b, wl.scale, k_strides=ks, v_strides=vs, Hkv=wl.Hkv,
+                     Dv=wl.Dv, nthreads=nthreads)
+    return time.perf_counter() - t0, len(flat)
+
+
+def _oracle_rate(wl, seconds: float, rows: int) -> float:
+    """Metric value of the oracle: decode steps/s or prefill tokens/s."""
+    total = wl.B * wl.Tq
+    step_seconds = seconds * total / rows
+    if wl.is_decode:
+        return 1.0 / step_seconds
+    return wl.B * wl.Tq / step_seconds
+
+
+def _sample_rows_for(wl, budget_s: float, nthreads: int, cpu) -> int:
+    """Rows of the oracle that fit a wall-clock budget (probe with a few rows)."""
+    probe = max(1, min(wl.B * wl.Tq, max(1, nthreads)))
+    sec, rows = time_oracle(wl, cpu, probe, nthreads)
+    per_row = sec / rows
+    return int(max(1, min(wl.B * wl.Tq, budget_s / per_row)))
+
+
+# ------------------------------------------------------------------ reference arm
+
+def run_reference(args, wl):
+    world, rank, _ = _dist()
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    cpu = make_inputs(wl)
+    nthreads = oracle.max_threads()
+    # Size each step so that the whole run ends within a few minutes.
+    budget = max(0.5, 150.0 / max(1, args.steps + args.warmup))
+    rows = _sample_rows_for(wl, budget, nthreads, cpu)
+    for _ in range(args.warmup):
+        time_oracle(wl, cpu, rows, nthreads)
+    secs = []
+    for _ in range(args.steps):
+        s, r = time_oracle(wl, cpu, rows, nthreads)
+        secs.append(s)
+    mean_s = sum(secs) / len(secs)
+    value = _oracle_rate(wl, mean_s, rows)
+    _, unit = _units(wl, 1)
+    sample = f"{rows} of {wl.B * wl.Tq} query rows per step (all three stages), scaled to a full step"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": 0,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * mean_s * (wl.B * wl.Tq) / rows,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": _config(wl, world),
+        "cpu_baseline": {"value": value, "unit": unit, "cores": nthreads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def _config(wl, world):
+    return {"workload": wl.name, "global_batch": wl.B * world, "seq_len": wl.L, "query_rows": wl.Tq,
+            "k": wl.k, "indexer_heads": wl.H_I, "indexer_dim": wl.d_I, "q_heads": wl.Hq,
+            "kv_heads": wl.Hkv, "d_qk": wl.Dqk, "d_v": wl.Dv, "kv_alias": wl.kv_alias,
+            "parallelism": f"replicas{world}",
+            "l2": "no flush: every step streams the indexer-key cache "
+                  f"({wl.B * wl.L * wl.d_I * (4 if wl.dtype == 'f32' else 2) / 1e6:.0f} MB), "
+                  "larger than the 126 MB L2"}
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args, wl):
+    from learned_sparse_attention_dsa_b200 import binding
+
+    world, rank, local = _dist()
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    binding.load_library()
+
+    cpu = make_inputs(wl, seed=wl.seed + rank)
+    dev = to_device(cpu, device)
+    out = torch.empty((wl.B, wl.Tq, wl.Hq, wl.Dv), dtype=dev["q"].dtype, device=device)
+    fargs = binding.forward_args(dev["q_idx"], dev["k_idx"], dev["w"], dev["q"], dev["k_cache"],
+                                 dev["v_cache"], wl.k, wl.q_pos0, wl.scale, out=out)
+    ws_bytes = binding.forward_workspace_bytes(fargs)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        binding.forward(dev["q_idx"], dev["k_idx"], dev["w"], dev["q"], dev["k_cache"], dev["v_cache"],
+                        wl.k, wl.q_pos0, wl.scale, out=out, ws=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    _barrier(world)
+    torch.cuda.synchronize(device)
+    launches0 = binding.kernel_launch_count()
+    h0 = time.perf_counter()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize(device)
+    h1 = time.perf_counter()
+    launches = binding.kernel_launch_count() - launches0
+    _barrier(world)
+    sampler.stop()
+    sec = ev0.elapsed_time(ev1) / 1000.0
+    sec_max = _max_over_ranks(sec, world, device)
+    units, unit = _units(wl, args.steps)
+    value = units * world / sec_max
+    clocks = sampler.summary(h0, h1)
+
+    # ---- per-stage timing (same stream, separate loops) for the roofline
+    stages = stage_timings(wl, dev, binding, stream, max(3, min(args.steps, 50)))
+    peaks = _peaks()
+    work = stage_work(wl)
+    stage_report = {}
+    for name, ms in stages.items():
+        nbytes, flops = work[name]
+        sec_s = ms / 1000.0
+        gbs = nbytes / sec_s / 1e9
+        tfs = flops / sec_s / 1e12 if flops else 0.0
+        entry = {"ms": ms, "GB/s": gbs, "hbm_frac": gbs / peaks["hbm_gbs"],
+                 "algorithmic_bytes": nbytes, "algorithmic_flops": flops}
+        if flops:
+            entry["TFLOP/s"] = tfs
+            entry["tensor_frac"] = tfs / peaks["bf16_tflops"]
+        stage_report[name] = entry
+    dominant = max(stages, key=lambda n: stages[n])
+    d = stage_report[dominant]
+    bound = "hbm"
+    if dominant == "indexer" and not wl.is_decode:
+        bound = "tensor"
+    if bound == "tensor":
+        roofline = {"bound": "tensor", "kernel": dominant, "achieved": d["TFLOP/s"],
+                    "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                    "frac": d["TFLOP/s"] / peaks["bf16_tflops"], "traffic": None,
+                    "peak_source": peaks["source"]}
+    else:
+        roofline = {"bound": "hbm", "kernel": dominant, "achieved": d["GB/s"], "peak": peaks["hbm_gbs"],
+                    "unit": "GB/s", "frac": d["GB/s"] / peaks["hbm_gbs"], "traffic": None,
+                    "peak_source": peaks["source"]}
+
+    # ---- end to end through the public API with host buffers
+    e2e = run_e2e(wl, cpu, binding, device, stream, max(1, min(args.steps, args.e2e_steps)), world)
+
+    # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
+    cpu_baseline = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        nthreads = oracle.max_threads()
+        rows = _sample_rows_for(wl, args.cpu_budget, nthreads, cpu)
+        secs, rows = time_oracle(wl, cpu, rows, nthreads)
+        cpu_baseline = {"value": _oracle_rate(wl, secs, rows), "unit": unit, "cores": nthreads,
+                        "kind": "oracle",
+                        "sample": f"{rows} of {wl.B * wl.Tq} query rows (all three stages) in "
+                                  f"{secs:.1f} s, scaled to a full step"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1000.0 * sec_max / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16"
+            if wl.dtype == "bf16" else "f32", "data": "synthetic", "config": _config(wl, world),
+            "roofline": roofline, "stages": stage_report, "cpu_baseline": cpu_baseline, "e2e": e2e,
+            "gpu_launches": int(launches), "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def stage_timings(wl, dev, binding, stream, iters):
+    """Average device time (ms) per launch of each stage, CUDA events on the
+    launching stream."""
+    scores = torch.empty((wl.B, wl.Tq, wl.L), dtype=torch.float32, device=dev["q"].device)
+    idx = torch.empty((wl.B, wl.Tq, wl.k), dtype=torch.int32, device=dev["q"].device)
+    out = torch.empty((wl.B, wl.Tq, wl.Hq, wl.Dv), dtype=dev["q"].dtype, device=dev["q"].device)
+
+    def t_of(fn):
+        for _ in range(3):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(iters):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / iters
+
+    res = {}
+    res["indexer"] = t_of(lambda: binding.indexer_scores(dev["q_idx"], dev["k_idx"], dev["w"], wl.q_pos0,
+                                                         scores=scores, stream=stream))
+    res["topk"] = t_of(lambda: binding.topk(scores, wl.k, wl.q_pos0, idx=idx, stream=stream))
+    res["attn"] = t_of(lambda: binding.sparse_attn(dev["q"], dev["k_cache"], dev["v_cache"], idx, wl.scale,
+                                                   out=out, stream=stream))
+    return res
+
+
+def run_e2e(wl, cpu, binding, device, stream, steps, world):
+    """Same metric through dsa_forward with inputs in pinned host memory:
+    every step copies all of its inputs host->device and reads the output
+    back device->host inside the timed region."""
+    host = {k: v.contiguous().pin_memory() for k, v in cpu.items() if k != "v_cache"}
+    if not wl.kv_alias:
+        host["v_cache"] = cpu["v_cache"].contiguous().pin_memory()
+    dev = {k: torch.empty_like(v, device=device) for k, v in host.items()}
+    v_dev = dev["k_cache"][..., : wl.Dv] if wl.kv_alias else dev["v_cache"]
+    out = torch.empty((wl.B, wl.Tq, wl.Hq, wl.Dv), dtype=dev["q"].dtype, device=device)
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    fargs = binding.forward_args(dev["q_idx"], dev["k_idx"], dev["w"], dev["q"], dev["k_cache"], v_dev,
+                                 wl.k, wl.q_pos0, wl.scale, out=out)
+    ws = torch.empty(max(binding.forward_workspace_bytes(fargs), 1), dtype=torch.uint8, device=device)
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = out.numel() * out.element_size()
+
+    def step():
+        for k2, v in host.items():
+            dev[k2].copy_(v, non_blocking=True)
+        binding.forward(dev["q_idx"], dev["k_idx"], dev["w"], dev["q"], dev["k_cache"], v_dev, wl.k,
+                        wl.q_pos0, wl.scale, out=out, ws=ws, stream=stream)
+        out_host.copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        step()
+    _barrier(world)
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    sec = _max_over_ranks(e0.elapsed_time(e1) / 1000.0, world, device)
+    units, unit = _units(wl, steps)
+    return {"value": units * world / sec, "unit": unit, "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "steps": steps,
+            "note": "all step inputs copied from pinned host memory, output read back, every step"}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="decode32k", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle wall time")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)  # at least three untimed warm-up steps
+    wl = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, wl)
+    else:
+        run_ours(args, wl)
+
+
+if __name__ == "__main__":
+    main()

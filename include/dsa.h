@@ -1,0 +1,197 @@
+/*
+ * dsa.h -- C ABI of the DeepSeek Sparse Attention (DSA) forward path on
+ * NVIDIA B200 (sm_100a). Library: libdsa.so.
+ *
+ * The path, as defined on "DeepSeek Sparse Attention: Learned Token Selection
+ * from Scratch" (first page) and "DeepSeek NSA and DSA" §3.2:
+ *
+ *   1. lightning-indexer scores   I[t,s] = sum_j w[t,j] * ReLU(q^I[t,j] . k^I[s])
+ *      (first page §2.1, boxed equation), for candidates s <= t;
+ *   2. top-k selection            S_t = positions of the k largest I[t,s]
+ *      (first page §3.1, boxed equation);
+ *   3. attention over S_t         u[t,h] = sum_{s in S_t} softmax_s(q[t,h].k[s]*scale) v[s]
+ *      (first page §3.3 and §10.1), one S_t shared by every query head
+ *      (first page §4.1-4.2: the MQA mode of MLA).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Query row i of batch entry b sits at absolute position t = q_pos0 + i.
+ *   Prefill: Tq = L, q_pos0 = 0. Decode: Tq = 1, q_pos0 = L - 1 (the cache of
+ *   L entries includes the new token).
+ * - Candidates of row t are positions 0..t (the page's running example says
+ *   "preceding tokens ... (plus itself)").
+ * - Equal scores are ordered by position, lower position first. When t+1 <= k,
+ *   every candidate is selected (first page §7.6 note: DSA collapses to full
+ *   attention when the context is shorter than the budget).
+ * - Selected positions are written in ascending order, followed by -1 padding
+ *   up to k entries.
+ * - All pointers are DEVICE pointers owned by the caller. The library never
+ *   allocates or frees device memory; scratch space is passed in as a
+ *   workspace. Every call is asynchronous on the given stream: it validates its
+ *   arguments on the host, enqueues kernels and returns.
+ * - Tensors are dense and row-major unless a stride says otherwise. Strides
+ *   are in elements. Every base pointer must be 16-byte aligned and every
+ *   stride must be a multiple of 16 bytes (the kernels move 16-byte vectors).
+ * - Errors: arguments are checked before any launch; a failed check returns a
+ *   status other than DSA_OK and enqueues nothing. A failed launch returns
+ *   DSA_ERR_CUDA. Kernels never trap or assert. No exception crosses the ABI.
+ * - Thread safety: calls on different streams may run concurrently. The only
+ *   global state is a per-device cache of device attributes.
+ */
+#ifndef DSA_H_
+#define DSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* An opaque CUDA stream (cudaStream_t / CUstream). NULL is the legacy default
+ * stream. */
+typedef void *dsa_stream_t;
+
+typedef enum {
+    DSA_OK = 0,
+    DSA_ERR_INVALID_ARG = 1,  /* null pointer, bad size, bad alignment or stride */
+    DSA_ERR_UNSUPPORTED = 2,  /* valid but not implemented (dtype, head width) */
+    DSA_ERR_WORKSPACE = 3,    /* workspace pointer null or ws_bytes too small */
+    DSA_ERR_CUDA = 4,         /* a CUDA runtime call or a kernel launch failed */
+    DSA_ERR_TIMEOUT = 5       /* reserved: a bounded device-side wait gave up */
+} dsa_status;
+
+typedef enum {
+    DSA_F32 = 0,   /* IEEE fp32 */
+    DSA_BF16 = 1   /* bfloat16 */
+} dsa_dtype;
+
+/* Library version, e.g. 100 for 0.1.0. */
+int dsa_version(void);
+
+/* Number of kernels this library has enqueued in this process, over all
+ * devices and streams (a diagnostic counter; it never resets). */
+uint64_t dsa_kernel_launch_count(void);
+
+/* Static text for a status code (never NULL). */
+const char *dsa_status_string(dsa_status status);
+
+/*
+ * dsa_indexer_scores -- stage 1, lightning-indexer scores (first page §2.1).
+ *
+ *   scores[b,i,s] = sum_{j<H_I} w[b,i,j] * max(0, sum_{e<d_I} q_idx[b,i,j,e] * k_idx[b,s,e])
+ *                   for s <= q_pos0 + i,   and -inf for s > q_pos0 + i.
+ *
+ * q_idx  [B, Tq, H_I, d_I]  dtype dt (indexer queries)
+ * k_idx  [B, L, d_I]        dtype dt (indexer key cache, one key per position,
+ *                           shared by all indexer heads)
+ * w      [B, Tq, H_I]       fp32 per-head weights
+ * scores [B, Tq, L]         fp32 output; every element is written
+ *
+ * Products are accumulated in fp32 (tensor cores for bf16 with d_I % 64 == 0;
+ * CUDA cores otherwise). With integer-valued inputs and power-of-two weights
+ * every partial sum is an exact fp32 value, so the result does not depend on
+ * the summation order.
+ * Requires B, Tq, L, H_I, d_I >= 1, 0 <= q_pos0, q_pos0 + Tq <= L.
+ */
+dsa_status dsa_indexer_scores(const void *q_idx, const void *k_idx, const float *w,
+                              int B, int Tq, int L, int q_pos0, int H_I, int d_I,
+                              dsa_dtype dt, float *scores, dsa_stream_t stream);
+
+/*
+ * dsa_topk -- stage 2, per-row top-k selection (first page §3.1).
+ *
+ * For each row (b, i), t = q_pos0 + i, reads scores[b,i,0..t] and writes the
+ * positions of the k largest values to idx[b,i,:] in ascending order, then -1
+ * up to k entries. Ties go to the lower position; -0.0 equals +0.0; -inf is
+ * an ordinary (lowest) value. NaN scores are not supported.
+ * Entries scores[b,i,s] with s > t are never read.
+ *
+ * scores [B, Tq, L] fp32;  idx [B, Tq, k] int32 output.
+ * ws / ws_bytes: workspace of at least dsa_topk_workspace_bytes(...) bytes
+ * (may be NULL when that is 0).
+ * Requires k >= 1, 0 <= q_pos0, q_pos0 + Tq <= L.
+ */
+dsa_status dsa_topk(const float *scores, int B, int Tq, int L, int q_pos0, int k,
+                    int32_t *idx, void *ws, size_t ws_bytes, dsa_stream_t stream);
+
+size_t dsa_topk_workspace_bytes(int B, int Tq, int L, int q_pos0, int k);
+
+/* Shape of the attention stage. */
+typedef struct dsa_attn_shape {
+    int B, Tq, L, k;          /* batch, query rows, cache length, idx entries per row */
+    int Hq, Hkv;              /* query heads, KV heads (Hq % Hkv == 0) */
+    int Dqk, Dv;              /* query/key width, value width */
+    float scale;              /* logit scale, usually 1/sqrt(Dqk) */
+    /* element strides of the caches: element (b, s, g, e) of K is at
+     * k_cache[b*k_stride_b + s*k_stride_s + g*k_stride_h + e]; same for V.
+     * V may alias K (a latent row whose first Dv columns are the value). */
+    int64_t k_stride_b, k_stride_s, k_stride_h;
+    int64_t v_stride_b, v_stride_s, v_stride_h;
+} dsa_attn_shape;
+
+/*
+ * dsa_sparse_attn -- stage 3, attention over the selected rows (first page
+ * §3.3, §10.1; one selection shared by all heads, §4.1-4.2).
+ *
+ *   out[b,i,h,:] = sum_{s in S} softmax_s(scale * q[b,i,h,:] . K[b,s,g,:]) * V[b,s,g,:]
+ *   with g = h / (Hq / Hkv) and S = { idx[b,i,j] : idx[b,i,j] >= 0 }.
+ *
+ * q   [B, Tq, Hq, Dqk] dtype dt;  out [B, Tq, Hq, Dv] dtype dt
+ * idx [B, Tq, k] int32: positions in [0, L) or -1 (skipped); order is free;
+ *     a position must not appear twice in one row.
+ * lse [B, Tq, Hq] fp32 or NULL: log sum_{s in S} exp(scale * q.k_s).
+ * A row whose idx holds only -1 gets out = 0 and lse = -inf.
+ * Logits, softmax and the weighted sum are accumulated in fp32.
+ * ws: at least dsa_sparse_attn_workspace_bytes(sh) bytes.
+ */
+dsa_status dsa_sparse_attn(const void *q, const void *k_cache, const void *v_cache,
+                           const int32_t *idx, const dsa_attn_shape *sh, dsa_dtype dt,
+                           void *out, float *lse, void *ws, size_t ws_bytes,
+                           dsa_stream_t stream);
+
+size_t dsa_sparse_attn_workspace_bytes(const dsa_attn_shape *sh, dsa_dtype dt);
+
+/* Arguments of the fused forward pass. */
+typedef struct dsa_forward_args {
+    int B, Tq, L, q_pos0, k;
+    /* indexer (stage 1) */
+    const void *q_idx;        /* [B, Tq, H_I, d_I] */
+    const void *k_idx;        /* [B, L, d_I] */
+    const float *w;           /* [B, Tq, H_I] */
+    int H_I, d_I;
+    dsa_dtype idx_dtype;
+    /* attention (stage 3) */
+    const void *q;            /* [B, Tq, Hq, Dqk] */
+    const void *k_cache;      /* strided as in dsa_attn_shape */
+    const void *v_cache;
+    int Hq, Hkv, Dqk, Dv;
+    float scale;
+    int64_t k_stride_b, k_stride_s, k_stride_h;
+    int64_t v_stride_b, v_stride_s, v_stride_h;
+    dsa_dtype attn_dtype;
+    /* outputs */
+    void *out;                /* [B, Tq, Hq, Dv] attn_dtype */
+    float *lse;               /* [B, Tq, Hq] or NULL */
+    int32_t *idx_out;         /* [B, Tq, k] or NULL: the selected positions */
+    float *scores_out;        /* [B, Tq, L] or NULL: the indexer scores (then
+                                 filled with -inf above the diagonal) */
+} dsa_forward_args;
+
+/*
+ * dsa_forward -- stages 1-3 back to back on one stream.
+ * Scores and indices go to caller memory when scores_out / idx_out are set,
+ * otherwise to the workspace. Results equal those of the three stage calls.
+ * ws: at least dsa_forward_workspace_bytes(a) bytes.
+ */
+dsa_status dsa_forward(const dsa_forward_args *a, void *ws, size_t ws_bytes,
+                       dsa_stream_t stream);
+
+/* Workspace needed by dsa_forward; 0 when the arguments are invalid. */
+size_t dsa_forward_workspace_bytes(const dsa_forward_args *a);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H_ */

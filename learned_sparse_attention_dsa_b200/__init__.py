@@ -14,10 +14,14 @@ CUDA library, which is loaded on first use and raises if it is missing.
 from .inputs import WORKLOADS, Workload, make_inputs, to_device  # noqa: F401
 
 
+_BINDING_NAMES = ("indexer_scores", "topk", "sparse_attn", "forward", "forward_args",
+                  "forward_workspace_bytes", "attn_shape", "load_library", "DSAError")
+
+
 def __getattr__(name):
-    # The binding loads libdsa.so; import it lazily so that CPU-only users of
-    # the input generator do not need the CUDA library.
-    from . import binding
-    if hasattr(binding, name):
-        return getattr(binding, name)
+    # The binding loads libdsa.so on first call; it is imported lazily so that
+    # CPU-only users of the input generator do not need the CUDA library.
+    if name in _BINDING_NAMES:
+        import importlib
+        return getattr(importlib.import_module(".binding", __name__), name)
     raise AttributeError(name)

@@ -1,0 +1,232 @@
+"""ctypes binding of libdsa.so: argument marshalling only.
+
+Each function takes CUDA tensors, reads their shapes, strides and data
+pointers, and calls the C entry point of the same name on the current torch
+stream. No arithmetic of the method happens here. The library is loaded on
+first use; a missing library raises immediately (there is no CPU fallback).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libdsa.so")
+
+DSA_F32 = 0
+DSA_BF16 = 1
+
+STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED",
+                3: "DSA_ERR_WORKSPACE", 4: "DSA_ERR_CUDA", 5: "DSA_ERR_TIMEOUT"}
+
+# Symbols declared in include/dsa.h.
+EXPORTED = ("dsa_version", "dsa_kernel_launch_count", "dsa_status_string", "dsa_indexer_scores", "dsa_topk",
+            "dsa_topk_workspace_bytes", "dsa_sparse_attn", "dsa_sparse_attn_workspace_bytes",
+            "dsa_forward", "dsa_forward_workspace_bytes")
+
+
+class DSAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)}")
+
+
+class AttnShape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("Tq", ctypes.c_int), ("L", ctypes.c_int), ("k", ctypes.c_int),
+                ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int), ("Dqk", ctypes.c_int), ("Dv", ctypes.c_int),
+                ("scale", ctypes.c_float),
+                ("k_stride_b", ctypes.c_int64), ("k_stride_s", ctypes.c_int64), ("k_stride_h", ctypes.c_int64),
+                ("v_stride_b", ctypes.c_int64), ("v_stride_s", ctypes.c_int64), ("v_stride_h", ctypes.c_int64)]
+
+
+class ForwardArgs(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("Tq", ctypes.c_int), ("L", ctypes.c_int), ("q_pos0", ctypes.c_int),
+                ("k", ctypes.c_int),
+                ("q_idx", ctypes.c_void_p), ("k_idx", ctypes.c_void_p), ("w", ctypes.c_void_p),
+                ("H_I", ctypes.c_int), ("d_I", ctypes.c_int), ("idx_dtype", ctypes.c_int),
+                ("q", ctypes.c_void_p), ("k_cache", ctypes.c_void_p), ("v_cache", ctypes.c_void_p),
+                ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int), ("Dqk", ctypes.c_int), ("Dv", ctypes.c_int),
+                ("scale", ctypes.c_float),
+                ("k_stride_b", ctypes.c_int64), ("k_stride_s", ctypes.c_int64), ("k_stride_h", ctypes.c_int64),
+                ("v_stride_b", ctypes.c_int64), ("v_stride_s", ctypes.c_int64), ("v_stride_h", ctypes.c_int64),
+                ("attn_dtype", ctypes.c_int),
+                ("out", ctypes.c_void_p), ("lse", ctypes.c_void_p), ("idx_out", ctypes.c_void_p),
+                ("scores_out", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libdsa.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"libdsa.so not found at {path}; build it with "
+                          "`python -m learned_sparse_attention_dsa_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, ci, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    lib.dsa_version.argtypes, lib.dsa_version.restype = [], ci
+    lib.dsa_kernel_launch_count.argtypes, lib.dsa_kernel_launch_count.restype = [], ctypes.c_uint64
+    lib.dsa_status_string.argtypes, lib.dsa_status_string.restype = [ci], ctypes.c_char_p
+    lib.dsa_indexer_scores.argtypes = [vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, vp, vp]
+    lib.dsa_indexer_scores.restype = ci
+    lib.dsa_topk.argtypes = [vp, ci, ci, ci, ci, ci, vp, vp, sz, vp]
+    lib.dsa_topk.restype = ci
+    lib.dsa_topk_workspace_bytes.argtypes = [ci, ci, ci, ci, ci]
+    lib.dsa_topk_workspace_bytes.restype = sz
+    lib.dsa_sparse_attn.argtypes = [vp, vp, vp, vp, ctypes.POINTER(AttnShape), ci, vp, vp, vp, sz, vp]
+    lib.dsa_sparse_attn.restype = ci
+    lib.dsa_sparse_attn_workspace_bytes.argtypes = [ctypes.POINTER(AttnShape), ci]
+    lib.dsa_sparse_attn_workspace_bytes.restype = sz
+    lib.dsa_forward.argtypes = [ctypes.POINTER(ForwardArgs), vp, sz, vp]
+    lib.dsa_forward.restype = ci
+    lib.dsa_forward_workspace_bytes.argtypes = [ctypes.POINTER(ForwardArgs)]
+    lib.dsa_forward_workspace_bytes.restype = sz
+    _lib = lib
+    return lib
+
+
+def kernel_launch_count() -> int:
+    """Kernels libdsa has enqueued in this process so far."""
+    return int(load_library().dsa_kernel_launch_count())
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise DSAError(status, what)
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return DSA_F32
+    if t.dtype == torch.bfloat16:
+        return DSA_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("all tensors must live on a CUDA device")
+
+
+def _cache_strides(t: torch.Tensor):
+    if t.dim() != 4 or t.stride(3) != 1:
+        raise ValueError("caches are [B, L, H_kv, D] with unit innermost stride")
+    return t.stride(0), t.stride(1), t.stride(2)
+
+
+def _workspace(nbytes: int, device, ws):
+    if nbytes == 0:
+        return None
+    if ws is not None:
+        if ws.numel() * ws.element_size() < nbytes:
+            raise ValueError(f"workspace too small: need {nbytes} bytes")
+        return ws
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def indexer_scores(q_idx, k_idx, w, q_pos0: int = 0, scores=None, stream=None):
+    """dsa_indexer_scores: fp32 [B, Tq, L] scores, -inf above the diagonal."""
+    lib = load_library()
+    _need_cuda(q_idx, k_idx, w, scores)
+    B, Tq, H, d = q_idx.shape
+    L = k_idx.shape[1]
+    if scores is None:
+        scores = torch.empty((B, Tq, L), dtype=torch.float32, device=q_idx.device)
+    st = lib.dsa_indexer_scores(_p(q_idx), _p(k_idx), _p(w), B, Tq, L, q_pos0, H, d, _dt(q_idx),
+                                _p(scores), _stream(stream))
+    _check(st, "dsa_indexer_scores")
+    return scores
+
+
+def topk(scores, k: int, q_pos0: int = 0, idx=None, ws=None, stream=None):
+    """dsa_topk: int32 [B, Tq, k], ascending positions then -1."""
+    lib = load_library()
+    _need_cuda(scores, idx)
+    B, Tq, L = scores.shape
+    if idx is None:
+        idx = torch.empty((B, Tq, k), dtype=torch.int32, device=scores.device)
+    nbytes = lib.dsa_topk_workspace_bytes(B, Tq, L, q_pos0, k)
+    ws = _workspace(nbytes, scores.device, ws)
+    st = lib.dsa_topk(_p(scores), B, Tq, L, q_pos0, k, _p(idx), _p(ws), nbytes, _stream(stream))
+    _check(st, "dsa_topk")
+    return idx
+
+
+def attn_shape(q, k_cache, v_cache, k: int, scale=None) -> AttnShape:
+    B, Tq, Hq, Dqk = q.shape
+    ksb, kss, ksh = _cache_strides(k_cache)
+    vsb, vss, vsh = _cache_strides(v_cache)
+    return AttnShape(B, Tq, k_cache.shape[1], k, Hq, k_cache.shape[2], Dqk, v_cache.shape[3],
+                     float(scale if scale is not None else Dqk ** -0.5),
+                     ksb, kss, ksh, vsb, vss, vsh)
+
+
+def sparse_attn(q, k_cache, v_cache, idx, scale=None, out=None, lse=None, want_lse=False, ws=None,
+                stream=None):
+    """dsa_sparse_attn: [B, Tq, Hq, Dv] in q's dtype (and fp32 lse if asked)."""
+    lib = load_library()
+    _need_cuda(q, k_cache, v_cache, idx, out, lse)
+    sh = attn_shape(q, k_cache, v_cache, idx.shape[-1], scale)
+    if out is None:
+        out = torch.empty((sh.B, sh.Tq, sh.Hq, sh.Dv), dtype=q.dtype, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((sh.B, sh.Tq, sh.Hq), dtype=torch.float32, device=q.device)
+    nbytes = lib.dsa_sparse_attn_workspace_bytes(ctypes.byref(sh), _dt(q))
+    ws = _workspace(nbytes, q.device, ws)
+    st = lib.dsa_sparse_attn(_p(q), _p(k_cache), _p(v_cache), _p(idx), ctypes.byref(sh), _dt(q), _p(out),
+                             _p(lse), _p(ws), nbytes, _stream(stream))
+    _check(st, "dsa_sparse_attn")
+    return (out, lse) if (want_lse or lse is not None) else out
+
+
+def forward_args(q_idx, k_idx, w, q, k_cache, v_cache, k: int, q_pos0: int = 0, scale=None,
+                 out=None, lse=None, idx_out=None, scores_out=None) -> ForwardArgs:
+    B, Tq, H, d = q_idx.shape
+    sh = attn_shape(q, k_cache, v_cache, k, scale)
+    return ForwardArgs(B, Tq, k_idx.shape[1], q_pos0, k,
+                       q_idx.data_ptr(), k_idx.data_ptr(), w.data_ptr(), H, d, _dt(q_idx),
+                       q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                       sh.Hq, sh.Hkv, sh.Dqk, sh.Dv, sh.scale,
+                       sh.k_stride_b, sh.k_stride_s, sh.k_stride_h,
+                       sh.v_stride_b, sh.v_stride_s, sh.v_stride_h, _dt(q),
+                       out.data_ptr() if out is not None else None,
+                       lse.data_ptr() if lse is not None else None,
+                       idx_out.data_ptr() if idx_out is not None else None,
+                       scores_out.data_ptr() if scores_out is not None else None)
+
+
+def forward_workspace_bytes(args: ForwardArgs) -> int:
+    return int(load_library().dsa_forward_workspace_bytes(ctypes.byref(args)))
+
+
+def forward(q_idx, k_idx, w, q, k_cache, v_cache, k: int, q_pos0: int = 0, scale=None,
+            out=None, lse=None, idx_out=None, scores_out=None, ws=None, stream=None):
+    """dsa_forward: all three stages; returns out (and fills lse/idx_out/scores_out if given)."""
+    lib = load_library()
+    _need_cuda(q_idx, k_idx, w, q, k_cache, v_cache, out, lse, idx_out, scores_out)
+    if out is None:
+        out = torch.empty((q.shape[0], q.shape[1], q.shape[2], v_cache.shape[3]), dtype=q.dtype,
+                          device=q.device)
+    args = forward_args(q_idx, k_idx, w, q, k_cache, v_cache, k, q_pos0, scale, out, lse, idx_out,
+                        scores_out)
+    nbytes = lib.dsa_forward_workspace_bytes(ctypes.byref(args))
+    ws = _workspace(nbytes, q.device, ws)
+    st = lib.dsa_forward(ctypes.byref(args), _p(ws), nbytes, _stream(stream))
+    _check(st, "dsa_forward")
+    return out

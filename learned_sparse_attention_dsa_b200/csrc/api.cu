@@ -1,0 +1,286 @@
+// C ABI of the DSA forward path: argument checks, workspace layout, dispatch.
+//
+// Every entry point validates on the host before enqueuing anything; a failed
+// check returns a status and leaves the stream untouched.
+#include <math.h>
+#include <atomic>
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace dsa {
+
+size_t indexer_cuda_core_smem_bytes(int H, int d);
+size_t attn_cuda_core_smem_bytes(int Dqk, int k);
+
+namespace {
+constexpr int kMaxDevices = 64;
+DeviceInfo g_info[kMaxDevices];
+std::mutex g_info_mutex;
+std::atomic<uint64_t> g_launches{0};
+}  // namespace
+
+void count_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+cudaError_t device_info(DeviceInfo *out) {
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_info_mutex);
+    if (g_info[dev].device != dev) {
+        DeviceInfo d;
+        d.device = dev;
+        if ((err = cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+            return err;
+        if ((err = cudaDeviceGetAttribute(&d.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) !=
+            cudaSuccess)
+            return err;
+        if ((err = cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess)
+            return err;
+        if ((err = cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess)
+            return err;
+        g_info[dev] = d;
+    }
+    *out = g_info[dev];
+    return cudaSuccess;
+}
+
+}  // namespace dsa
+
+using namespace dsa;
+
+namespace {
+
+constexpr size_t kWsAlign = 256;
+
+bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+size_t dtype_bytes(dsa_dtype dt) { return dt == DSA_F32 ? 4 : 2; }
+bool valid_dtype(dsa_dtype dt) { return dt == DSA_F32 || dt == DSA_BF16; }
+
+dsa_status from_cuda(cudaError_t err) { return err == cudaSuccess ? DSA_OK : DSA_ERR_CUDA; }
+
+// Host-side shared-memory limit of the current device (0 when unknown).
+int smem_limit() {
+    DeviceInfo info;
+    return device_info(&info) == cudaSuccess ? info.max_smem_optin : 0;
+}
+
+dsa_status check_rows(int B, int Tq, int L, int q_pos0) {
+    if (B < 1 || Tq < 1 || L < 1 || q_pos0 < 0) return DSA_ERR_INVALID_ARG;
+    if ((int64_t)q_pos0 + Tq > L) return DSA_ERR_INVALID_ARG;
+    return DSA_OK;
+}
+
+dsa_status check_indexer(const void *q_idx, const void *k_idx, const float *w, int B, int Tq, int L,
+                         int q_pos0, int H_I, int d_I, dsa_dtype dt, const float *scores) {
+    if (!q_idx || !k_idx || !w || !scores) return DSA_ERR_INVALID_ARG;
+    dsa_status st = check_rows(B, Tq, L, q_pos0);
+    if (st != DSA_OK) return st;
+    if (H_I < 1 || d_I < 1) return DSA_ERR_INVALID_ARG;
+    if (!valid_dtype(dt)) return DSA_ERR_UNSUPPORTED;
+    const size_t eb = dtype_bytes(dt);
+    if (!aligned(q_idx, eb) || !aligned(k_idx, eb) || !aligned(w, 4) || !aligned(scores, 4))
+        return DSA_ERR_INVALID_ARG;
+    return DSA_OK;
+}
+
+dsa_status check_indexer_fits(int H_I, int d_I) {
+    // The CUDA-core kernel is the fallback for every shape: its staging must fit.
+    const int lim = smem_limit();
+    if (lim == 0) return DSA_ERR_CUDA;
+    if (indexer_cuda_core_smem_bytes(H_I, d_I) > (size_t)lim) return DSA_ERR_UNSUPPORTED;
+    return DSA_OK;
+}
+
+dsa_status check_topk(const float *scores, int B, int Tq, int L, int q_pos0, int k, const int32_t *idx) {
+    if (!scores || !idx) return DSA_ERR_INVALID_ARG;
+    dsa_status st = check_rows(B, Tq, L, q_pos0);
+    if (st != DSA_OK) return st;
+    if (k < 1) return DSA_ERR_INVALID_ARG;
+    if (!aligned(scores, 4) || !aligned(idx, 4)) return DSA_ERR_INVALID_ARG;
+    return DSA_OK;
+}
+
+dsa_status check_attn(const void *q, const void *k_cache, const void *v_cache, const int32_t *idx,
+                      const dsa_attn_shape *sh, dsa_dtype dt, const void *out, const float *lse) {
+    if (!sh || !q || !k_cache || !v_cache || !idx || !out) return DSA_ERR_INVALID_ARG;
+    if (sh->B < 1 || sh->Tq < 1 || sh->L < 1 || sh->k < 1) return DSA_ERR_INVALID_ARG;
+    if (sh->Hq < 1 || sh->Hkv < 1 || sh->Hq % sh->Hkv != 0) return DSA_ERR_INVALID_ARG;
+    if (sh->Dqk < 1 || sh->Dv < 1) return DSA_ERR_INVALID_ARG;
+    if (!(sh->scale == sh->scale) || isinf(sh->scale)) return DSA_ERR_INVALID_ARG;
+    if (sh->k_stride_s < 1 || sh->v_stride_s < 1 || sh->k_stride_b < 0 || sh->v_stride_b < 0 ||
+        sh->k_stride_h < 0 || sh->v_stride_h < 0)
+        return DSA_ERR_INVALID_ARG;
+    if (!valid_dtype(dt)) return DSA_ERR_UNSUPPORTED;
+    const size_t eb = dtype_bytes(dt);
+    if (!aligned(q, eb) || !aligned(k_cache, eb) || !aligned(v_cache, eb) || !aligned(out, eb) ||
+        !aligned(idx, 4) || (lse && !aligned(lse, 4)))
+        return DSA_ERR_INVALID_ARG;
+    if (sh->Dv > 512) return DSA_ERR_UNSUPPORTED;
+    const int lim = smem_limit();
+    if (lim == 0) return DSA_ERR_CUDA;
+    if (attn_cuda_core_smem_bytes(sh->Dqk, sh->k) > (size_t)lim) return DSA_ERR_UNSUPPORTED;
+    return DSA_OK;
+}
+
+AttnProblem make_attn_problem(const void *q, const void *k_cache, const void *v_cache, const int32_t *idx,
+                              const dsa_attn_shape *sh, dsa_dtype dt, void *out, float *lse, void *ws,
+                              size_t ws_bytes) {
+    AttnProblem p;
+    p.q = q; p.k_cache = k_cache; p.v_cache = v_cache; p.idx = idx;
+    p.B = sh->B; p.Tq = sh->Tq; p.L = sh->L; p.k = sh->k;
+    p.Hq = sh->Hq; p.Hkv = sh->Hkv; p.Dqk = sh->Dqk; p.Dv = sh->Dv; p.scale = sh->scale;
+    p.k_sb = sh->k_stride_b; p.k_ss = sh->k_stride_s; p.k_sh = sh->k_stride_h;
+    p.v_sb = sh->v_stride_b; p.v_ss = sh->v_stride_s; p.v_sh = sh->v_stride_h;
+    p.dt = dt; p.out = out; p.lse = lse; p.ws = ws; p.ws_bytes = ws_bytes;
+    return p;
+}
+
+dsa_attn_shape forward_attn_shape(const dsa_forward_args *a) {
+    dsa_attn_shape sh;
+    sh.B = a->B; sh.Tq = a->Tq; sh.L = a->L; sh.k = a->k;
+    sh.Hq = a->Hq; sh.Hkv = a->Hkv; sh.Dqk = a->Dqk; sh.Dv = a->Dv; sh.scale = a->scale;
+    sh.k_stride_b = a->k_stride_b; sh.k_stride_s = a->k_stride_s; sh.k_stride_h = a->k_stride_h;
+    sh.v_stride_b = a->v_stride_b; sh.v_stride_s = a->v_stride_s; sh.v_stride_h = a->v_stride_h;
+    return sh;
+}
+
+struct ForwardLayout {
+    size_t scores = 0, idx = 0, topk = 0, attn = 0, total = 0;
+    size_t topk_bytes = 0, attn_bytes = 0;
+};
+
+ForwardLayout forward_layout(const dsa_forward_args *a) {
+    ForwardLayout lay;
+    size_t off = 0;
+    if (!a->scores_out) {
+        lay.scores = off;
+        off += align_up(sizeof(float) * (size_t)a->B * a->Tq * a->L, kWsAlign);
+    }
+    if (!a->idx_out) {
+        lay.idx = off;
+        off += align_up(sizeof(int32_t) * (size_t)a->B * a->Tq * a->k, kWsAlign);
+    }
+    lay.topk = off;
+    lay.topk_bytes = topk_workspace_bytes(a->B, a->Tq, a->L, a->q_pos0, a->k);
+    off += align_up(lay.topk_bytes, kWsAlign);
+    lay.attn = off;
+    dsa_attn_shape sh = forward_attn_shape(a);
+    AttnProblem p = make_attn_problem(a->q, a->k_cache, a->v_cache, nullptr, &sh, a->attn_dtype, a->out,
+                                      a->lse, nullptr, 0);
+    lay.attn_bytes = attn_workspace_bytes(p);
+    off += align_up(lay.attn_bytes, kWsAlign);
+    lay.total = off;
+    return lay;
+}
+
+dsa_status check_forward(const dsa_forward_args *a) {
+    if (!a) return DSA_ERR_INVALID_ARG;
+    dsa_status st = check_indexer(a->q_idx, a->k_idx, a->w, a->B, a->Tq, a->L, a->q_pos0, a->H_I, a->d_I,
+                                  a->idx_dtype, a->scores_out ? a->scores_out : a->w);
+    if (st != DSA_OK) return st;
+    if (a->k < 1) return DSA_ERR_INVALID_ARG;
+    if (a->idx_out && !aligned(a->idx_out, 4)) return DSA_ERR_INVALID_ARG;
+    dsa_attn_shape sh = forward_attn_shape(a);
+    // idx is produced internally: pass a non-null placeholder to the check
+    st = check_attn(a->q, a->k_cache, a->v_cache, reinterpret_cast<const int32_t *>(a->w), &sh,
+                    a->attn_dtype, a->out, a->lse);
+    if (st != DSA_OK) return st;
+    return check_indexer_fits(a->H_I, a->d_I);
+}
+
+}  // namespace
+
+extern "C" {
+
+int dsa_version(void) { return 100; }
+
+uint64_t dsa_kernel_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char *dsa_status_string(dsa_status status) {
+    switch (status) {
+        case DSA_OK: return "DSA_OK";
+        case DSA_ERR_INVALID_ARG: return "DSA_ERR_INVALID_ARG: invalid argument";
+        case DSA_ERR_UNSUPPORTED: return "DSA_ERR_UNSUPPORTED: unsupported shape or dtype";
+        case DSA_ERR_WORKSPACE: return "DSA_ERR_WORKSPACE: workspace missing or too small";
+        case DSA_ERR_CUDA: return "DSA_ERR_CUDA: CUDA runtime or launch failure";
+        case DSA_ERR_TIMEOUT: return "DSA_ERR_TIMEOUT: bounded device wait expired";
+    }
+    return "unknown dsa_status";
+}
+
+dsa_status dsa_indexer_scores(const void *q_idx, const void *k_idx, const float *w, int B, int Tq, int L,
+                              int q_pos0, int H_I, int d_I, dsa_dtype dt, float *scores,
+                              dsa_stream_t stream) {
+    dsa_status st = check_indexer(q_idx, k_idx, w, B, Tq, L, q_pos0, H_I, d_I, dt, scores);
+    if (st != DSA_OK) return st;
+    if ((st = check_indexer_fits(H_I, d_I)) != DSA_OK) return st;
+    IndexerProblem p{q_idx, k_idx, w, B, Tq, L, q_pos0, H_I, d_I, dt, scores, true};
+    return from_cuda(launch_indexer(p, static_cast<cudaStream_t>(stream)));
+}
+
+size_t dsa_topk_workspace_bytes(int B, int Tq, int L, int q_pos0, int k) {
+    if (check_rows(B, Tq, L, q_pos0) != DSA_OK || k < 1) return 0;
+    return topk_workspace_bytes(B, Tq, L, q_pos0, k);
+}
+
+dsa_status dsa_topk(const float *scores, int B, int Tq, int L, int q_pos0, int k, int32_t *idx, void *ws,
+                    size_t ws_bytes, dsa_stream_t stream) {
+    dsa_status st = check_topk(scores, B, Tq, L, q_pos0, k, idx);
+    if (st != DSA_OK) return st;
+    const size_t need = topk_workspace_bytes(B, Tq, L, q_pos0, k);
+    if (need > 0 && (!ws || ws_bytes < need || !aligned(ws, 16))) return DSA_ERR_WORKSPACE;
+    TopkProblem p{scores, B, Tq, L, q_pos0, k, idx, ws, ws_bytes};
+    return from_cuda(launch_topk(p, static_cast<cudaStream_t>(stream)));
+}
+
+size_t dsa_sparse_attn_workspace_bytes(const dsa_attn_shape *sh, dsa_dtype dt) {
+    if (!sh) return 0;
+    AttnProblem p = make_attn_problem(nullptr, nullptr, nullptr, nullptr, sh, dt, nullptr, nullptr, nullptr, 0);
+    return attn_workspace_bytes(p);
+}
+
+dsa_status dsa_sparse_attn(const void *q, const void *k_cache, const void *v_cache, const int32_t *idx,
+                           const dsa_attn_shape *sh, dsa_dtype dt, void *out, float *lse, void *ws,
+                           size_t ws_bytes, dsa_stream_t stream) {
+    dsa_status st = check_attn(q, k_cache, v_cache, idx, sh, dt, out, lse);
+    if (st != DSA_OK) return st;
+    AttnProblem p = make_attn_problem(q, k_cache, v_cache, idx, sh, dt, out, lse, ws, ws_bytes);
+    const size_t need = attn_workspace_bytes(p);
+    if (need > 0 && (!ws || ws_bytes < need || !aligned(ws, 16))) return DSA_ERR_WORKSPACE;
+    return from_cuda(launch_attn(p, static_cast<cudaStream_t>(stream)));
+}
+
+size_t dsa_forward_workspace_bytes(const dsa_forward_args *a) {
+    if (check_forward(a) != DSA_OK) return 0;
+    return forward_layout(a).total;
+}
+
+dsa_status dsa_forward(const dsa_forward_args *a, void *ws, size_t ws_bytes, dsa_stream_t stream) {
+    dsa_status st = check_forward(a);
+    if (st != DSA_OK) return st;
+    const ForwardLayout lay = forward_layout(a);
+    if (lay.total > 0 && (!ws || ws_bytes < lay.total || !aligned(ws, kWsAlign))) return DSA_ERR_WORKSPACE;
+    char *base = static_cast<char *>(ws);
+    float *scores = a->scores_out ? a->scores_out : reinterpret_cast<float *>(base + lay.scores);
+    int32_t *idx = a->idx_out ? a->idx_out : reinterpret_cast<int32_t *>(base + lay.idx);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    IndexerProblem ip{a->q_idx, a->k_idx, a->w, a->B, a->Tq, a->L, a->q_pos0, a->H_I, a->d_I,
+                      a->idx_dtype, scores, a->scores_out != nullptr};
+    cudaError_t err = launch_indexer(ip, s);
+    if (err != cudaSuccess) return DSA_ERR_CUDA;
+
+    TopkProblem tp{scores, a->B, a->Tq, a->L, a->q_pos0, a->k, idx,
+                   lay.topk_bytes ? base + lay.topk : nullptr, lay.topk_bytes};
+    if ((err = launch_topk(tp, s)) != cudaSuccess) return DSA_ERR_CUDA;
+
+    dsa_attn_shape sh = forward_attn_shape(a);
+    AttnProblem ap = make_attn_problem(a->q, a->k_cache, a->v_cache, idx, &sh, a->attn_dtype, a->out, a->lse,
+                                       lay.attn_bytes ? base + lay.attn : nullptr, lay.attn_bytes);
+    return from_cuda(launch_attn(ap, s));
+}
+
+}  // extern "C"

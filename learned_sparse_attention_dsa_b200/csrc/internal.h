@@ -1,0 +1,65 @@
+// Host-side launch interface between the C ABI (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "dsa.h"
+
+namespace dsa {
+
+// Cached per-device attributes.
+struct DeviceInfo {
+    int device = -1;
+    int sm_count = 0;
+    int max_smem_optin = 0;
+    int cc_major = 0, cc_minor = 0;
+};
+cudaError_t device_info(DeviceInfo *out);
+
+// Process-wide count of kernels this library has enqueued (diagnostics).
+void count_launch(int n = 1);
+
+// ----------------------------------------------------------------- indexer
+struct IndexerProblem {
+    const void *q_idx;   // [B, Tq, H, d]
+    const void *k_idx;   // [B, L, d]
+    const float *w;      // [B, Tq, H]
+    int B, Tq, L, q_pos0, H, d;
+    dsa_dtype dt;
+    float *scores;       // [B, Tq, L]
+    bool fill_masked;    // write -inf at s > t (else those entries are untouched)
+};
+cudaError_t launch_indexer(const IndexerProblem &p, cudaStream_t stream);
+
+// ----------------------------------------------------------------- top-k
+struct TopkProblem {
+    const float *scores;  // [B, Tq, L]
+    int B, Tq, L, q_pos0, k;
+    int32_t *idx;         // [B, Tq, k]
+    void *ws;
+    size_t ws_bytes;
+};
+size_t topk_workspace_bytes(int B, int Tq, int L, int q_pos0, int k);
+cudaError_t launch_topk(const TopkProblem &p, cudaStream_t stream);
+
+// ----------------------------------------------------------------- attention
+struct AttnProblem {
+    const void *q;        // [B, Tq, Hq, Dqk]
+    const void *k_cache;
+    const void *v_cache;
+    const int32_t *idx;   // [B, Tq, k]
+    int B, Tq, L, k, Hq, Hkv, Dqk, Dv;
+    float scale;
+    int64_t k_sb, k_ss, k_sh, v_sb, v_ss, v_sh;
+    dsa_dtype dt;
+    void *out;            // [B, Tq, Hq, Dv]
+    float *lse;           // [B, Tq, Hq] or null
+    void *ws;
+    size_t ws_bytes;
+};
+size_t attn_workspace_bytes(const AttnProblem &p);
+cudaError_t launch_attn(const AttnProblem &p, cudaStream_t stream);
+
+}  // namespace dsa

@@ -1,0 +1,85 @@
+"""Host-side checks of the C ABI: the library loads, exports every entry point
+that include/dsa.h declares, and rejects bad arguments before touching a GPU.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"\b(dsa_[a-z0-9_]+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_header_declares_the_entry_points():
+    names = _declared_functions()
+    for n in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_attn", "dsa_forward"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(dsa_lib):
+    from learned_sparse_attention_dsa_b200 import binding
+    for name in _declared_functions():
+        assert hasattr(dsa_lib, name), name
+    assert set(binding.EXPORTED) <= set(_declared_functions())
+
+
+def test_version_and_status_strings(dsa_lib):
+    assert dsa_lib.dsa_version() >= 100
+    for code in range(6):
+        assert dsa_lib.dsa_status_string(code)
+    assert b"unknown" in dsa_lib.dsa_status_string(99)
+
+
+def test_null_pointers_rejected_before_any_launch(dsa_lib):
+    assert dsa_lib.dsa_indexer_scores(None, None, None, 1, 1, 1, 0, 1, 1, 1, None, None) == 1
+    assert dsa_lib.dsa_topk(None, 1, 1, 1, 0, 1, None, None, 0, None) == 1
+    assert dsa_lib.dsa_sparse_attn(None, None, None, None, None, 1, None, None, None, 0, None) == 1
+    assert dsa_lib.dsa_forward(None, None, 0, None) == 1
+    assert dsa_lib.dsa_forward_workspace_bytes(None) == 0
+
+
+def test_bad_sizes_rejected(dsa_lib):
+    fake = ctypes.c_void_p(0x1000)  # never dereferenced: the checks fail first
+    # q_pos0 + Tq > L
+    assert dsa_lib.dsa_topk(fake, 1, 4, 3, 0, 2, fake, None, 0, None) == 1
+    # k < 1
+    assert dsa_lib.dsa_topk(fake, 1, 1, 3, 0, 0, fake, None, 0, None) == 1
+    # negative q_pos0
+    assert dsa_lib.dsa_indexer_scores(fake, fake, fake, 1, 1, 4, -1, 2, 2, 0, fake, None) == 1
+    # unsupported dtype
+    assert dsa_lib.dsa_indexer_scores(fake, fake, fake, 1, 1, 4, 0, 2, 2, 7, fake, None) == 2
+    # misaligned bf16 pointer
+    odd = ctypes.c_void_p(0x1001)
+    assert dsa_lib.dsa_indexer_scores(odd, fake, fake, 1, 1, 4, 0, 2, 2, 1, fake, None) == 1
+
+
+def test_attention_shape_checks(dsa_lib):
+    from learned_sparse_attention_dsa_b200.binding import AttnShape
+    fake = ctypes.c_void_p(0x1000)
+    sh = AttnShape(1, 1, 8, 4, 6, 4, 64, 64, 0.125, 512, 64, 64, 512, 64, 64)  # Hq % Hkv != 0
+    assert dsa_lib.dsa_sparse_attn(fake, fake, fake, fake, ctypes.byref(sh), 1, fake, None, None, 0, None) == 1
+    sh = AttnShape(1, 1, 8, 4, 8, 4, 64, 64, float("nan"), 512, 64, 64, 512, 64, 64)
+    assert dsa_lib.dsa_sparse_attn(fake, fake, fake, fake, ctypes.byref(sh), 1, fake, None, None, 0, None) == 1
+    sh = AttnShape(1, 1, 8, 4, 8, 4, 64, 64, 0.1, 512, 0, 64, 512, 64, 64)  # zero row stride
+    assert dsa_lib.dsa_sparse_attn(fake, fake, fake, fake, ctypes.byref(sh), 1, fake, None, None, 0, None) == 1
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    from learned_sparse_attention_dsa_b200 import binding
+    saved = binding._lib
+    binding._lib = None
+    try:
+        with pytest.raises(ImportError):
+            binding.load_library(str(tmp_path / "missing.so"))
+    finally:
+        binding._lib = saved

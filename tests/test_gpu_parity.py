@@ -1,0 +1,193 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Index sets and (for integer-valued indexer inputs) scores must match bit for
+bit; attention outputs must be within max-abs 2e-2 and norm-wise relative
+1e-2 of the fp64 oracle.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from learned_sparse_attention_dsa_b200 import binding
+from learned_sparse_attention_dsa_b200.inputs import (WORKLOADS, Workload, make_inputs,
+                                                      random_score_rows, to_device)
+from parity_helpers import assert_attn_close, bits, oracle_forward, rows_of
+
+pytestmark = pytest.mark.gpu
+
+MEDIUM = {
+    "prefill_mqa_700": Workload("prefill_mqa_700", B=2, Tq=700, L=700, q_pos0=0, H_I=64, d_I=128,
+                                k=96, Hq=16, Hkv=1, Dqk=192, Dv=128, seed=11),
+    "prefill_perhead_520": Workload("prefill_perhead_520", B=1, Tq=520, L=520, q_pos0=0, H_I=64,
+                                    d_I=128, k=64, Hq=8, Hkv=8, Dqk=64, Dv=64, seed=12),
+    "chunked_prefill": Workload("chunked_prefill", B=1, Tq=200, L=900, q_pos0=700, H_I=64, d_I=128,
+                                k=128, Hq=16, Hkv=1, Dqk=128, Dv=128, seed=13),
+    "decode_5000": Workload("decode_5000", B=3, Tq=1, L=5000, q_pos0=4999, H_I=64, d_I=128,
+                            k=2048, Hq=16, Hkv=1, Dqk=128, Dv=128, seed=14),
+    "decode_latent_3000": Workload("decode_latent_3000", B=2, Tq=1, L=3000, q_pos0=2999, H_I=64,
+                                   d_I=128, k=256, Hq=128, Hkv=1, Dqk=576, Dv=512, kv_alias=True,
+                                   seed=15),
+    "short_context": Workload("short_context", B=2, Tq=40, L=40, q_pos0=0, H_I=64, d_I=128, k=64,
+                              Hq=8, Hkv=8, Dqk=64, Dv=64, seed=16),
+    "odd_heads": Workload("odd_heads", B=1, Tq=300, L=300, q_pos0=0, H_I=32, d_I=64, k=50, Hq=4,
+                          Hkv=2, Dqk=64, Dv=32, seed=17),
+    "tiny_f32": Workload("tiny_f32", B=2, Tq=45, L=45, q_pos0=0, H_I=3, d_I=5, k=7, Hq=6, Hkv=3,
+                         Dqk=20, Dv=12, dtype="f32", idx_range=4, seed=18),
+    "single_position": Workload("single_position", B=2, Tq=1, L=1, q_pos0=0, H_I=64, d_I=128, k=1,
+                                Hq=16, Hkv=1, Dqk=128, Dv=128, seed=19),
+}
+
+FULL_ROWS = {
+    "toy16": None,  # every row
+    "decode32k": [0, 13, 31],
+    "prefill8k": [0, 1, 2046, 2047, 2048, 5000, 8191],
+    "prefill32k": [0, 2047, 2048, 20000, 32767],
+    "decode128k": [0, 5],
+}
+
+_cache = {}
+
+
+def _inputs(wl):
+    if wl.name not in _cache:
+        _cache.clear()
+        cpu = make_inputs(wl)
+        _cache[wl.name] = (cpu, to_device(cpu, "cuda"))
+    return _cache[wl.name]
+
+
+def _gpu_forward(wl, dev):
+    out = torch.empty((wl.B, wl.Tq, wl.Hq, wl.Dv), dtype=dev["q"].dtype, device="cuda")
+    idx = torch.empty((wl.B, wl.Tq, wl.k), dtype=torch.int32, device="cuda")
+    scores = torch.empty((wl.B, wl.Tq, wl.L), dtype=torch.float32, device="cuda")
+    binding.forward(dev["q_idx"], dev["k_idx"], dev["w"], dev["q"], dev["k_cache"], dev["v_cache"],
+                    wl.k, wl.q_pos0, wl.scale, out=out, idx_out=idx, scores_out=scores)
+    torch.cuda.synchronize()
+    return scores, idx, out
+
+
+def _check_forward(wl, flat_rows):
+    cpu, dev = _inputs(wl)
+    scores, idx, out = _gpu_forward(wl, dev)
+    if flat_rows is None:
+        flat_rows = list(range(wl.B * wl.Tq))
+    o_scores, o_idx, o_out = oracle_forward(wl, cpu, flat_rows)
+    row_b, row_i, _ = rows_of(wl, flat_rows)
+    rb = torch.from_numpy(row_b.astype(np.int64))
+    ri = torch.from_numpy(row_i.astype(np.int64))
+    g_scores = scores.cpu()[rb, ri].numpy()
+    g_idx = idx.cpu()[rb, ri].numpy()
+    g_out = out.float().cpu()[rb, ri].numpy()
+    # integer-valued indexer inputs with power-of-two weights: exact scores
+    assert np.array_equal(g_scores, o_scores), f"{wl.name}: scores differ"
+    assert np.array_equal(g_idx, o_idx), f"{wl.name}: selected positions differ"
+    assert_attn_close(g_out, o_out, wl.name)
+
+
+@pytest.mark.parametrize("name", sorted(MEDIUM))
+def test_forward_medium(cuda, name):
+    _check_forward(MEDIUM[name], None)
+
+
+@pytest.mark.parametrize("name", list(FULL_ROWS))
+def test_forward_full_size_sampled_rows(cuda, name):
+    _check_forward(WORKLOADS[name], FULL_ROWS[name])
+
+
+def test_hand_trace_on_gpu(cuda):
+    """The t=10 example: 10 keys at positions 0..9, H=2, d=2, k=3 -> S = {3, 8, 9}."""
+    q = torch.tensor([[[[1.0, 2.0], [2.0, -1.0]]]], device="cuda")              # [1,1,2,2]
+    k = torch.tensor([[[1, 0], [0, 1], [-1, 1], [2, 1], [0, -1], [1, 1], [-1, 0], [1, -1],
+                       [0, 2], [2, 0]]], dtype=torch.float32, device="cuda")     # [1,10,2]
+    w = torch.tensor([[[0.5, 0.3]]], device="cuda")
+    scores = binding.indexer_scores(q, k, w, q_pos0=9)
+    expect = [1.1, 1.0, 0.5, 2.9, 0.3, 1.8, 0.0, 0.9, 2.0, 2.2]
+    assert np.allclose(scores.cpu().numpy()[0, 0], expect, rtol=0, atol=1e-6)
+    idx = binding.topk(scores, 3, q_pos0=9)
+    assert idx.cpu().tolist() == [[[3, 8, 9]]]
+
+
+@pytest.mark.parametrize("name", ["prefill_mqa_700", "chunked_prefill", "decode_5000", "odd_heads",
+                                  "tiny_f32"])
+def test_indexer_stage_all_rows(cuda, name):
+    wl = MEDIUM[name]
+    cpu, dev = _inputs(wl)
+    scores = binding.indexer_scores(dev["q_idx"], dev["k_idx"], dev["w"], wl.q_pos0).cpu().numpy()
+    flat = np.arange(wl.B * wl.Tq)
+    row_b, row_i, row_t = rows_of(wl, flat)
+    ref = oracle.indexer_rows(bits(cpu["q_idx"][row_b, row_i]), cpu["w"][row_b, row_i].numpy(),
+                              bits(cpu["k_idx"]), row_b, row_t)
+    assert np.array_equal(scores.reshape(-1, wl.L), ref)
+
+
+@pytest.mark.parametrize("kind", ["int", "equal", "normal", "neg", "mixed"])
+@pytest.mark.parametrize("L,Tq,q_pos0,k", [(37, 37, 0, 5), (5000, 3, 4997, 2048), (3000, 2, 2998, 1),
+                                           (70000, 2, 69998, 2048), (140000, 1, 139999, 2048),
+                                           (2100, 2100, 0, 2048)])
+def test_topk_stage(cuda, kind, L, Tq, q_pos0, k):
+    gen = torch.Generator().manual_seed(L + Tq + k)
+    scores = random_score_rows(gen, Tq, L, kind)[None]            # [1, Tq, L]
+    got = binding.topk(scores.cuda(), k, q_pos0=q_pos0).cpu().numpy()[0]
+    row_t = q_pos0 + np.arange(Tq)
+    ref = oracle.topk_rows(scores[0].numpy(), row_t, k)
+    assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("name", ["prefill_mqa_700", "decode_latent_3000", "prefill_perhead_520",
+                                  "tiny_f32"])
+def test_sparse_attn_stage_shuffled_and_padded(cuda, name):
+    """Attention on its own, with the oracle's index sets shuffled and padded."""
+    wl = MEDIUM[name]
+    cpu, dev = _inputs(wl)
+    flat = np.arange(wl.B * wl.Tq)
+    _, o_idx, _ = oracle_forward(wl, cpu, flat)
+    rng = np.random.default_rng(0)
+    idx = o_idx.copy()
+    for r in range(idx.shape[0]):
+        rng.shuffle(idx[r])
+    _, _, ref = oracle_forward(wl, cpu, flat, idx_override=idx)
+    idx_t = torch.from_numpy(idx).reshape(wl.B, wl.Tq, wl.k).cuda()
+    out, lse = binding.sparse_attn(dev["q"], dev["k_cache"], dev["v_cache"], idx_t, wl.scale,
+                                   want_lse=True)
+    assert_attn_close(out.float().cpu().numpy().reshape(-1, wl.Hq, wl.Dv), ref, name)
+    assert torch.isfinite(lse).all()
+
+
+def test_sparse_attn_all_padding_row(cuda):
+    wl = MEDIUM["odd_heads"]
+    _, dev = _inputs(wl)
+    idx = torch.full((wl.B, wl.Tq, 4), -1, dtype=torch.int32, device="cuda")
+    idx[:, 1:, 0] = 0
+    out, lse = binding.sparse_attn(dev["q"], dev["k_cache"], dev["v_cache"], idx, wl.scale,
+                                   want_lse=True)
+    assert torch.count_nonzero(out[:, 0]) == 0
+    assert torch.isneginf(lse[:, 0]).all()
+    # |S| = 1: the output is the value row itself (rounded to bf16)
+    v0 = dev["v_cache"][:, 0]                                                   # [B, Hkv, Dv]
+    g = torch.arange(wl.Hq, device="cuda") // (wl.Hq // wl.Hkv)
+    assert torch.equal(out[:, 1], v0[:, g])
+
+
+def test_forward_equals_stage_calls(cuda):
+    wl = MEDIUM["prefill_mqa_700"]
+    _, dev = _inputs(wl)
+    scores_f, idx_f, out_f = _gpu_forward(wl, dev)
+    scores = binding.indexer_scores(dev["q_idx"], dev["k_idx"], dev["w"], wl.q_pos0)
+    idx = binding.topk(scores, wl.k, wl.q_pos0)
+    out = binding.sparse_attn(dev["q"], dev["k_cache"], dev["v_cache"], idx, wl.scale)
+    assert torch.equal(scores, scores_f)
+    assert torch.equal(idx, idx_f)
+    assert torch.equal(out, out_f)
+
+
+def test_invalid_arguments_enqueue_nothing(cuda):
+    wl = MEDIUM["odd_heads"]
+    _, dev = _inputs(wl)
+    with pytest.raises(binding.DSAError):
+        binding.indexer_scores(dev["q_idx"], dev["k_idx"], dev["w"], q_pos0=wl.L)   # q_pos0+Tq > L
+    with pytest.raises(binding.DSAError):
+        binding.topk(torch.zeros((1, 2, 8), device="cuda"), 0)
+    torch.cuda.synchronize()
