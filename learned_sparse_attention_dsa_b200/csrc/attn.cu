@@ -175,6 +175,8 @@ cudaError_t launch_attn(const AttnProblem &p, cudaStream_t stream) {
     return launch_attn_cuda_core(p, stream);
 }
 
-size_t attn_workspace_bytes(const AttnProblem &) { return 0; }
+size_t attn_tc_workspace_bytes(const AttnProblem &p);
+
+size_t attn_workspace_bytes(const AttnProblem &p) { return attn_tc_workspace_bytes(p); }
 
 }  // namespace dsa

@@ -1,9 +1,481 @@
-// Tensor-core sparse-attention kernels: not yet enabled.
+// Sparse attention on tensor cores for groups of 16 query heads that share
+// one KV head (the MQA mode of MLA: "DeepSeek Sparse Attention: Learned
+// Token Selection from Scratch" §4.1-4.2; "Sparse Attention LLM Design ...",
+// "Implemented on MLA's MQA mode").
+//
+//   u[t,h] = sum_{s in S_t} softmax_s(scale * q[t,h] . k[s]) v[s]   (§3.3, §10.1)
+//
+// One CTA owns (query row, group of 16 heads, split of the selected list).
+// The selected positions are compacted in shared memory (padding dropped),
+// then gathered 64 at a time -- K and V rows -- with 16-byte cp.async into a
+// multi-stage ring (16-byte chunks XOR-swizzled by row so that ldmatrix reads
+// are conflict-free). Each of the four warps takes 16 of the 64 rows:
+// S = Q K^T with mma.sync m16n8k16 (bf16 in, fp32 accumulate; Q stays in
+// registers), an online softmax in fp32 (exp2 with the log2(e) prescale, as in
+// FlashAttention), and O += P V with P re-packed from the S accumulators as
+// the A operand. The four warps' (max, sum, O) are merged at the end; with a
+// split selected list the CTA writes fp32 partials and a combine kernel
+// merges the splits. Every selected row is loaded once for all 16 heads.
+#include <math.h>
+
+#include "common.cuh"
 #include "internal.h"
 
 namespace dsa {
-cudaError_t launch_attn_tc(const AttnProblem &, cudaStream_t, bool *taken) {
-    *taken = false;
-    return cudaSuccess;
+
+cudaError_t launch_attn_cuda_core(const AttnProblem &p, cudaStream_t stream);
+
+namespace {
+
+constexpr int kRowsPerTile = 64;
+constexpr int kWarps = 4;
+constexpr int kThreads = kWarps * 32;
+constexpr int kHeads = 16;
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int DQK, int DV>
+struct Cfg {
+    static constexpr int kKChunks = DQK / 8;  // 16-byte chunks per K row
+    static constexpr int kVChunks = DV / 8;
+    static constexpr int kKBytes = kRowsPerTile * DQK * 2;
+    static constexpr int kVBytes = kRowsPerTile * DV * 2;
+    static constexpr int kStageBytes = kKBytes + kVBytes;
+    static constexpr int kStages = (DQK + DV) > 256 ? 2 : 3;
+    static constexpr int kMaxSel = 2048;  // selected entries one CTA handles
+    static constexpr int kMergeBytes = kWarps * kHeads * (DV + 2) * 4;
+    static constexpr int kPipeBytes = kStages * kStageBytes;
+    static constexpr size_t kSmem =
+        (size_t)(kPipeBytes > kMergeBytes ? kPipeBytes : kMergeBytes) + kMaxSel * 4 + 64;
+};
+
+struct Args {
+    const __nv_bfloat16 *q, *k_cache, *v_cache;
+    const int32_t *idx;
+    int Tq, L, k, Hq, Hkv, splits, per_split;
+    float scale_log2;
+    int64_t k_sb, k_ss, k_sh, v_sb, v_ss, v_sh;
+    __nv_bfloat16 *out;
+    float *lse;
+    float *part_o;   // [rows, Hq, splits, DV] when splits > 1
+    float *part_ml;  // [rows, Hq, splits, 2]
+};
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid) {
+    const int n = valid ? 16 : 0;  // 0 source bytes: the 16 bytes are zero-filled
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n) : "memory");
 }
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+__device__ __forceinline__ void mma_bf16(float *c, const uint32_t *a, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+template <int DQK, int DV>
+__global__ void __launch_bounds__(kThreads)
+attn_mma_kernel(const Args a) {
+    using C = Cfg<DQK, DV>;
+    extern __shared__ __align__(128) uint8_t smem[];
+    int32_t *sel = reinterpret_cast<int32_t *>(smem + (C::kPipeBytes > C::kMergeBytes ? C::kPipeBytes
+                                                                                        : C::kMergeBytes));
+    __shared__ int s_count;
+
+    const int row = blockIdx.x;                 // flat query row b*Tq + i
+    const int hgroup = blockIdx.y;              // 16-head group
+    const int split = blockIdx.z;
+    const int b = row / a.Tq;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int h0 = hgroup * kHeads;
+    const int g = h0 / (a.Hq / a.Hkv);
+
+    // ---- compact this split's valid selected positions (order kept)
+    const int j0 = split * a.per_split;
+    const int j1 = min(a.k, j0 + a.per_split);
+    if (threadIdx.x == 0) s_count = 0;
+    __syncthreads();
+    {
+        __shared__ int warp_base[kWarps];
+        int base = 0;
+        for (int c0 = j0; c0 < j1; c0 += kThreads) {
+            const int j = c0 + threadIdx.x;
+            int s = j < j1 ? a.idx[(size_t)row * a.k + j] : -1;
+            const bool valid = s >= 0 && s < a.L;
+            const unsigned m = __ballot_sync(0xffffffffu, valid);
+            if (lane == 0) warp_base[warp] = __popc(m);
+            __syncthreads();
+            int off = base;
+            for (int w = 0; w < warp; ++w) off += warp_base[w];
+            if (valid) sel[off + __popc(m & ((1u << lane) - 1u))] = s;
+            int tot = 0;
+            for (int w = 0; w < kWarps; ++w) tot += warp_base[w];
+            base += tot;
+            __syncthreads();
+        }
+        if (threadIdx.x == 0) s_count = base;
+    }
+    __syncthreads();
+    const int n_sel = s_count;
+    const int n_tiles = (n_sel + kRowsPerTile - 1) / kRowsPerTile;
+
+    const __nv_bfloat16 *kbase = a.k_cache + b * a.k_sb + g * a.k_sh;
+    const __nv_bfloat16 *vbase = a.v_cache + b * a.v_sb + g * a.v_sh;
+    const uint32_t smem_base = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+
+    auto issue_tile = [&](int tile, int stage) {
+        const uint32_t kdst = smem_base + stage * C::kStageBytes;
+        const uint32_t vdst = kdst + C::kKBytes;
+        constexpr int kChunks = kRowsPerTile * (C::kKChunks + C::kVChunks);
+        for (int c = threadIdx.x; c < kChunks; c += kThreads) {
+            const int r = c / (C::kKChunks + C::kVChunks);
+            const int ch = c - r * (C::kKChunks + C::kVChunks);
+            const int jj = tile * kRowsPerTile + r;
+            const bool valid = jj < n_sel;
+            const int s = valid ? sel[jj] : 0;
+            if (ch < C::kKChunks) {
+                const uint32_t dst = kdst + r * (DQK * 2) + ((ch ^ (r & 7)) << 4);
+                cp_async16(dst, kbase + (int64_t)s * a.k_ss + ch * 8, valid);
+            } else {
+                const int cv = ch - C::kKChunks;
+                const uint32_t dst = vdst + r * (DV * 2) + ((cv ^ (r & 7)) << 4);
+                cp_async16(dst, vbase + (int64_t)s * a.v_ss + cv * 8, valid);
+            }
+        }
+    };
+
+    // ---- Q fragments (A operand, 16 heads x DQK) straight from global memory
+    uint32_t qf[DQK / 16][4];
+    {
+        const int hr = lane >> 2, kc = (lane & 3) * 2;
+        const __nv_bfloat16 *q0 = a.q + ((size_t)row * a.Hq + h0 + hr) * DQK;
+        const __nv_bfloat16 *q8 = q0 + 8 * DQK;
+#pragma unroll
+        for (int kk = 0; kk < DQK / 16; ++kk) {
+            qf[kk][0] = *reinterpret_cast<const uint32_t *>(q0 + kk * 16 + kc);
+            qf[kk][1] = *reinterpret_cast<const uint32_t *>(q8 + kk * 16 + kc);
+            qf[kk][2] = *reinterpret_cast<const uint32_t *>(q0 + kk * 16 + 8 + kc);
+            qf[kk][3] = *reinterpret_cast<const uint32_t *>(q8 + kk * 16 + 8 + kc);
+        }
+    }
+
+    float o[DV / 8][4];
+#pragma unroll
+    for (int n = 0; n < DV / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.0f;
+    float m_r[2] = {-INFINITY, -INFINITY};  // running max of heads lane/4 and lane/4+8 (log2 units)
+    float l_r[2] = {0.0f, 0.0f};            // this thread's partial running sums
+
+    // ---- pipeline prologue
+#pragma unroll
+    for (int st = 0; st < C::kStages - 1; ++st) {
+        if (st < n_tiles) issue_tile(st, st);
+        cp_async_commit();
+    }
+
+    for (int tile = 0; tile < n_tiles; ++tile) {
+        const int stage = tile % C::kStages;
+        {
+            const int next = tile + C::kStages - 1;
+            if (next < n_tiles) issue_tile(next, next % C::kStages);
+            cp_async_commit();
+        }
+        cp_async_wait<C::kStages - 1>();
+        __syncthreads();
+
+        const uint32_t kt = smem_base + stage * C::kStageBytes;
+        const uint32_t vt = kt + C::kKBytes;
+
+        // S = Q K^T for this warp's 16 rows (two n-tiles of 8 rows)
+        float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        {
+            const int r = warp * 16 + (lane & 7) + ((lane >> 4) << 3);
+            const uint32_t rbase = kt + r * (DQK * 2);
+            const int rx = r & 7;
+#pragma unroll
+            for (int kk = 0; kk < DQK / 16; ++kk) {
+                const int ch = 2 * kk + ((lane >> 3) & 1);
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4(rbase + ((ch ^ rx) << 4), b0, b1, b2, b3);
+                mma_bf16(s[0], qf[kk], b0, b1);
+                mma_bf16(s[1], qf[kk], b2, b3);
+            }
+        }
+        // mask rows beyond the selected count, scale into log2 units
+        const int valid_rows = n_sel - tile * kRowsPerTile;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int rr = warp * 16 + nt * 8 + (lane & 3) * 2 + (e & 1);
+                s[nt][e] = rr < valid_rows ? s[nt][e] * a.scale_log2 : -INFINITY;
+            }
+        }
+        // online softmax update for heads lane/4 (e = 0,1) and lane/4+8 (e = 2,3)
+        float p[2][4];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            float mx = fmaxf(fmaxf(s[0][2 * hh], s[0][2 * hh + 1]), fmaxf(s[1][2 * hh], s[1][2 * hh + 1]));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+            const float m_new = fmaxf(m_r[hh], mx);
+            const float corr = m_new == -INFINITY ? 1.0f : exp2f(m_r[hh] - m_new);
+            float sum = 0.0f;
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const float v = s[nt][2 * hh + e];
+                    const float pv = v == -INFINITY ? 0.0f : exp2f(v - m_new);
+                    p[nt][2 * hh + e] = pv;
+                    sum += pv;
+                }
+            }
+            l_r[hh] = l_r[hh] * corr + sum;
+            m_r[hh] = m_new;
+#pragma unroll
+            for (int n = 0; n < DV / 8; ++n) {
+                o[n][2 * hh] *= corr;
+                o[n][2 * hh + 1] *= corr;
+            }
+        }
+        // O += P V: P (16 heads x 16 rows) as the A operand
+        uint32_t pa[4];
+        pa[0] = pack_bf16(p[0][0], p[0][1]);
+        pa[1] = pack_bf16(p[0][2], p[0][3]);
+        pa[2] = pack_bf16(p[1][0], p[1][1]);
+        pa[3] = pack_bf16(p[1][2], p[1][3]);
+        {
+            const int r = warp * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
+            const uint32_t rbase = vt + r * (DV * 2);
+            const int rx = r & 7;
+#pragma unroll
+            for (int nn = 0; nn < DV / 16; ++nn) {
+                const int ch = 2 * nn + (lane >> 4);
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4_t(rbase + ((ch ^ rx) << 4), b0, b1, b2, b3);
+                mma_bf16(o[2 * nn], pa, b0, b1);
+                mma_bf16(o[2 * nn + 1], pa, b2, b3);
+            }
+        }
+        __syncthreads();  // this stage may be refilled next iteration
+    }
+    cp_async_wait<0>();
+    __syncthreads();
+
+    // ---- merge the four warps: full row sums, then (m, l, O) across warps
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+        l_r[hh] += __shfl_xor_sync(0xffffffffu, l_r[hh], 1);
+        l_r[hh] += __shfl_xor_sync(0xffffffffu, l_r[hh], 2);
+    }
+    float *mrg_o = reinterpret_cast<float *>(smem);                    // [warp][16][DV]
+    float *mrg_ml = mrg_o + kWarps * kHeads * DV;                      // [warp][16][2]
+    {
+        const int hr = lane >> 2, cc = (lane & 3) * 2;
+#pragma unroll
+        for (int n = 0; n < DV / 8; ++n) {
+            float *d0 = mrg_o + ((warp * kHeads + hr) * DV) + n * 8 + cc;
+            float *d8 = mrg_o + ((warp * kHeads + hr + 8) * DV) + n * 8 + cc;
+            d0[0] = o[n][0];
+            d0[1] = o[n][1];
+            d8[0] = o[n][2];
+            d8[1] = o[n][3];
+        }
+        if ((lane & 3) == 0) {
+            mrg_ml[(warp * kHeads + hr) * 2 + 0] = m_r[0];
+            mrg_ml[(warp * kHeads + hr) * 2 + 1] = l_r[0];
+            mrg_ml[(warp * kHeads + hr + 8) * 2 + 0] = m_r[1];
+            mrg_ml[(warp * kHeads + hr + 8) * 2 + 1] = l_r[1];
+        }
+    }
+    __syncthreads();
+    // thread t handles head t / 8 and columns (t % 8) + 8 * c
+    const int hh = threadIdx.x >> 3;
+    const int c0 = threadIdx.x & 7;
+    float mw[kWarps], m_all = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+        mw[w] = mrg_ml[(w * kHeads + hh) * 2];
+        m_all = fmaxf(m_all, mw[w]);
+    }
+    float fw[kWarps], l_all = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+        fw[w] = m_all == -INFINITY ? 0.0f : exp2f(mw[w] - m_all);
+        l_all += fw[w] * mrg_ml[(w * kHeads + hh) * 2 + 1];
+    }
+    const int h = h0 + hh;
+    if (a.splits == 1) {
+        const float inv = l_all > 0.0f ? 1.0f / l_all : 0.0f;
+        __nv_bfloat16 *dst = a.out + ((size_t)row * a.Hq + h) * DV;
+        for (int c = c0; c < DV; c += 8) {
+            float acc = 0.0f;
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) acc += fw[w] * mrg_o[(w * kHeads + hh) * DV + c];
+            dst[c] = __float2bfloat16_rn(acc * inv);
+        }
+        if (a.lse != nullptr && c0 == 0)
+            a.lse[(size_t)row * a.Hq + h] = l_all > 0.0f ? (m_all + log2f(l_all)) / kLog2e : -INFINITY;
+    } else {
+        const size_t pidx = ((size_t)row * a.Hq + h) * a.splits + split;
+        float *dst = a.part_o + pidx * DV;
+        for (int c = c0; c < DV; c += 8) {
+            float acc = 0.0f;
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) acc += fw[w] * mrg_o[(w * kHeads + hh) * DV + c];
+            dst[c] = acc;
+        }
+        if (c0 == 0) {
+            a.part_ml[pidx * 2 + 0] = m_all;
+            a.part_ml[pidx * 2 + 1] = l_all;
+        }
+    }
+}
+
+// Merge the split partials of one (row, head): one warp, lanes over columns.
+__global__ void attn_combine_kernel(const float *__restrict__ part_o, const float *__restrict__ part_ml,
+                                    int n_pairs, int splits, int DV, __nv_bfloat16 *__restrict__ out,
+                                    float *__restrict__ lse) {
+    const int pair = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (pair >= n_pairs) return;
+    const float *ml = part_ml + (size_t)pair * splits * 2;
+    float m_all = -INFINITY;
+    for (int sp = 0; sp < splits; ++sp) m_all = fmaxf(m_all, ml[2 * sp]);
+    float l_all = 0.0f;
+    for (int sp = 0; sp < splits; ++sp)
+        l_all += m_all == -INFINITY ? 0.0f : exp2f(ml[2 * sp] - m_all) * ml[2 * sp + 1];
+    const float inv = l_all > 0.0f ? 1.0f / l_all : 0.0f;
+    const float *po = part_o + (size_t)pair * splits * DV;
+    for (int c = lane; c < DV; c += 32) {
+        float acc = 0.0f;
+        for (int sp = 0; sp < splits; ++sp) {
+            const float f = m_all == -INFINITY ? 0.0f : exp2f(ml[2 * sp] - m_all);
+            acc += f * po[(size_t)sp * DV + c];
+        }
+        out[(size_t)pair * DV + c] = __float2bfloat16_rn(acc * inv);
+    }
+    if (lse != nullptr && lane == 0)
+        lse[pair] = l_all > 0.0f ? (m_all + log2f(l_all)) / kLog2e : -INFINITY;
+}
+
+// Splits of the selected list: enough CTAs to cover the GPU about twice, and
+// at most kMaxSel entries per split.
+int choose_splits(const AttnProblem &p, int sm_count) {
+    const long long ctas = (long long)p.B * p.Tq * (p.Hq / kHeads);
+    const int max_tiles = (p.k + kRowsPerTile - 1) / kRowsPerTile;
+    int splits = 1;
+    if (ctas < 2LL * sm_count) splits = (int)((2LL * sm_count + ctas - 1) / ctas);
+    const int min_splits = (max_tiles * kRowsPerTile + 2047) / 2048;
+    if (splits < min_splits) splits = min_splits;
+    if (splits > max_tiles) splits = max_tiles;
+    const int tiles_per = (max_tiles + splits - 1) / splits;  // equal whole tiles per split
+    return (max_tiles + tiles_per - 1) / tiles_per;
+}
+
+bool shape_supported(const AttnProblem &p, int *dqk_dv) {
+    if (p.dt != DSA_BF16) return false;
+    if ((p.Hq / p.Hkv) % kHeads != 0) return false;
+    const int cfgs[][2] = {{64, 64}, {128, 128}, {192, 128}};
+    int which = -1;
+    for (int i = 0; i < 3; ++i)
+        if (p.Dqk == cfgs[i][0] && p.Dv == cfgs[i][1]) which = i;
+    if (which < 0) return false;
+    // 16-byte aligned rows for cp.async and 4-byte aligned Q for fragment loads
+    if (((uintptr_t)p.k_cache | (uintptr_t)p.v_cache) % 16 != 0 || (uintptr_t)p.q % 4 != 0) return false;
+    if (p.k_ss % 8 || p.k_sb % 8 || p.k_sh % 8 || p.v_ss % 8 || p.v_sb % 8 || p.v_sh % 8) return false;
+    *dqk_dv = which;
+    return true;
+}
+
+template <int DQK, int DV>
+cudaError_t launch_mma(const AttnProblem &p, const DeviceInfo &info, cudaStream_t stream) {
+    using C = Cfg<DQK, DV>;
+    const int splits = choose_splits(p, info.sm_count);
+    const int max_tiles = (p.k + kRowsPerTile - 1) / kRowsPerTile;
+    const int per_split = ((max_tiles + splits - 1) / splits) * kRowsPerTile;
+    if (per_split > C::kMaxSel) return cudaErrorInvalidValue;
+    Args a;
+    a.q = static_cast<const __nv_bfloat16 *>(p.q);
+    a.k_cache = static_cast<const __nv_bfloat16 *>(p.k_cache);
+    a.v_cache = static_cast<const __nv_bfloat16 *>(p.v_cache);
+    a.idx = p.idx;
+    a.Tq = p.Tq; a.L = p.L; a.k = p.k; a.Hq = p.Hq; a.Hkv = p.Hkv;
+    a.splits = splits; a.per_split = per_split;
+    a.scale_log2 = p.scale * kLog2e;
+    a.k_sb = p.k_sb; a.k_ss = p.k_ss; a.k_sh = p.k_sh;
+    a.v_sb = p.v_sb; a.v_ss = p.v_ss; a.v_sh = p.v_sh;
+    a.out = static_cast<__nv_bfloat16 *>(p.out);
+    a.lse = p.lse;
+    const int rows = p.B * p.Tq;
+    const size_t n_pairs = (size_t)rows * p.Hq;
+    a.part_o = nullptr;
+    a.part_ml = nullptr;
+    if (splits > 1) {
+        a.part_o = static_cast<float *>(p.ws);
+        a.part_ml = a.part_o + n_pairs * splits * DV;
+    }
+    auto kern = attn_mma_kernel<DQK, DV>;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
+    if (err != cudaSuccess) return err;
+    dim3 grid(rows, p.Hq / kHeads, splits);
+    kern<<<grid, kThreads, C::kSmem, stream>>>(a);
+    count_launch();
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    if (splits > 1) {
+        const int warps_per_block = 8;
+        attn_combine_kernel<<<(int)((n_pairs + warps_per_block - 1) / warps_per_block), warps_per_block * 32, 0,
+                              stream>>>(a.part_o, a.part_ml, (int)n_pairs, splits, DV, a.out, a.lse);
+        count_launch();
+        err = cudaGetLastError();
+    }
+    return err;
+}
+
+}  // namespace
+
+size_t attn_tc_workspace_bytes(const AttnProblem &p) {
+    int which;
+    if (!shape_supported(p, &which)) return 0;
+    DeviceInfo info;
+    if (device_info(&info) != cudaSuccess) return 0;
+    const int splits = choose_splits(p, info.sm_count);
+    if (splits <= 1) return 0;
+    const size_t n_pairs = (size_t)p.B * p.Tq * p.Hq;
+    return n_pairs * splits * ((size_t)p.Dv + 2) * sizeof(float);
+}
+
+cudaError_t launch_attn_tc(const AttnProblem &p, cudaStream_t stream, bool *taken) {
+    *taken = false;
+    int which;
+    if (!shape_supported(p, &which)) return cudaSuccess;
+    DeviceInfo info;
+    cudaError_t err = device_info(&info);
+    if (err != cudaSuccess) return err;
+    if (attn_tc_workspace_bytes(p) > p.ws_bytes) return cudaSuccess;
+    *taken = true;
+    switch (which) {
+        case 0: return launch_mma<64, 64>(p, info, stream);
+        case 1: return launch_mma<128, 128>(p, info, stream);
+        default: return launch_mma<192, 128>(p, info, stream);
+    }
+}
+
 }  // namespace dsa

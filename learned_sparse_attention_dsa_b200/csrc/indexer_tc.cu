@@ -1,9 +1,391 @@
-// Tensor-core (tcgen05) lightning-indexer kernel: not yet enabled.
+// Lightning-indexer scores on the 5th-generation tensor cores (tcgen05).
+//
+//   I[t,s] = sum_j w[t,j] * ReLU(q[t,j] . k[s]),  s <= t
+// ("DeepSeek Sparse Attention: Learned Token Selection from Scratch" §2.1;
+// "DeepSeek NSA and DSA" §3.2 for H=64 heads of width 128).
+//
+// The contraction over d is a GEMM with the KEYS on M and (query, head) pairs
+// on N:  X[s, (i,j)] = sum_e K[s,e] * Q[(i,j),e].  One CTA tile is 128 keys by
+// N_TILE = QPT * H columns (QPT queries of one batch entry), K = d. Putting
+// keys on M gives every epilogue thread one key (one TMEM lane) and all heads
+// of a query in its own registers, so the ReLU, the weights and the head sum
+// need no cross-thread reduction, and the per-head scores never leave the SM.
+//
+// Warp roles (192 threads, one CTA per SM, persistent over work units):
+//   warp 0      TMA producer: Q tile of the unit once, then key tiles through
+//               a K_STAGES-deep ring (128-byte swizzle, K-major).
+//   warp 1      allocates TMEM; one thread issues tcgen05.mma (bf16 in, fp32
+//               accumulate) into one of two TMEM accumulators.
+//   warps 2-5   epilogue: tcgen05.ld of the accumulator, ReLU, weight, head
+//               sum, one fp32 score per (query, key), causal mask.
+// The two accumulators let the epilogue of tile n overlap the MMAs of tile
+// n+1. A work unit is (batch entry, query group, chunk of at most C key
+// tiles); units are spread over the CTAs round-robin. Causal: a query group
+// only visits key tiles up to its last query position.
+//
+// Exactness: integer-valued bf16 inputs give integer dot products far below
+// 2^24, and power-of-two weights keep every partial sum exact in fp32, so the
+// scores equal the exact result regardless of accumulation order.
+#include <math.h>
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
 #include "internal.h"
+#include "sm100.cuh"
 
 namespace dsa {
-cudaError_t launch_indexer_tc(const IndexerProblem &, cudaStream_t, bool *taken) {
-    *taken = false;
-    return cudaSuccess;
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kBlockM = 128;       // keys per tile (TMEM lanes)
+constexpr int kThreads = 192;      // 6 warps
+constexpr uint32_t kSmemBudget = 224 * 1024;
+
+__device__ unsigned int g_indexer_error = 0;  // 1 = a bounded wait gave up
+
+struct Params {
+    const float *w;
+    float *scores;
+    int B, Tq, L, q_pos0, H, QPT, ngroups, G, C, units;
+    int fill;
+};
+
+struct Unit {
+    int b, i0, qcount, kt0, kt1;
+};
+
+// Work unit u -> (batch entry, query group, key-tile chunk). Chunk-major
+// order; a unit whose chunk lies beyond the group's causal extent is empty.
+__device__ __forceinline__ bool decode_unit(int u, const Params &p, Unit &un) {
+    const int c_idx = u / p.G;
+    const int g = u - c_idx * p.G;
+    const int b = g / p.ngroups;
+    const int qg = g - b * p.ngroups;
+    const int i0 = qg * p.QPT;
+    const int qcount = min(p.QPT, p.Tq - i0);
+    const int t_max = p.q_pos0 + i0 + qcount - 1;
+    const int nkt = t_max / kBlockM + 1;
+    const int kt0 = c_idx * p.C;
+    if (kt0 >= nkt) return false;
+    un.b = b;
+    un.i0 = i0;
+    un.qcount = qcount;
+    un.kt0 = kt0;
+    un.kt1 = min(kt0 + p.C, nkt);
+    return true;
 }
+
+template <int D, int N_TILE>
+struct Cfg {
+    static constexpr int kHalves = D / 64;                          // 64-element (128-byte) K slices
+    static constexpr uint32_t kQHalf = N_TILE * 128;
+    static constexpr uint32_t kQBytes = kQHalf * kHalves;
+    static constexpr uint32_t kKHalf = kBlockM * 128;
+    static constexpr uint32_t kKBytes = kKHalf * kHalves;
+    static constexpr int kQBufs = 2;
+    static constexpr int kStagesRaw = (int)((kSmemBudget - kQBufs * kQBytes) / kKBytes);
+    static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
+    static constexpr uint32_t kTmemCols = 2 * N_TILE;
+    static constexpr int kBars = 2 * kStages + 2 * kQBufs + 4;
+    static constexpr size_t kSmem = 1024 + (size_t)kQBufs * kQBytes + (size_t)kStages * kKBytes + kBars * 8 + 16;
+    static_assert(kStages >= 2, "shared memory too small for the pipeline");
+    static_assert(kTmemCols == 128 || kTmemCols == 256 || kTmemCols == 512, "TMEM columns");
+};
+
+template <int D, int N_TILE>
+__global__ void __launch_bounds__(kThreads, 1)
+indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const Params p) {
+    using C = Cfg<D, N_TILE>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *q_sm = smem;
+    uint8_t *k_sm = q_sm + C::kQBufs * C::kQBytes;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(k_sm + C::kStages * C::kKBytes);
+    uint64_t *k_full = bars;
+    uint64_t *k_empty = k_full + C::kStages;
+    uint64_t *q_full = k_empty + C::kStages;
+    uint64_t *q_empty = q_full + C::kQBufs;
+    uint64_t *acc_full = q_empty + C::kQBufs;
+    uint64_t *acc_empty = acc_full + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(&k_full[s], 1);
+            mbar_init(&k_empty[s], 1);
+        }
+        for (int s = 0; s < C::kQBufs; ++s) {
+            mbar_init(&q_full[s], 1);
+            mbar_init(&q_empty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&acc_full[s], 1);
+            mbar_init(&acc_empty[s], 128);
+        }
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    bool ok = true;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------------ TMA producer
+            prefetch_tensor_map(&tm_q);
+            prefetch_tensor_map(&tm_k);
+            int ks = 0, qb = 0;
+            uint32_t kph = 0, qph = 0;
+            for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
+                Unit un;
+                if (!decode_unit(u, p, un)) continue;
+                if (!mbar_wait(&q_empty[qb], qph ^ 1u)) { ok = false; break; }
+                mbar_arrive_expect_tx(&q_full[qb], C::kQBytes);
+                const int qrow = (un.b * p.Tq + un.i0) * p.H;
+#pragma unroll
+                for (int h = 0; h < C::kHalves; ++h)
+                    tma_load_2d(q_sm + qb * C::kQBytes + h * C::kQHalf, &tm_q, &q_full[qb], h * 64, qrow);
+                if (++qb == C::kQBufs) { qb = 0; qph ^= 1u; }
+                for (int kt = un.kt0; kt < un.kt1; ++kt) {
+                    if (!mbar_wait(&k_empty[ks], kph ^ 1u)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&k_full[ks], C::kKBytes);
+                    const int krow = un.b * p.L + kt * kBlockM;
+#pragma unroll
+                    for (int h = 0; h < C::kHalves; ++h)
+                        tma_load_2d(k_sm + ks * C::kKBytes + h * C::kKHalf, &tm_k, &k_full[ks], h * 64, krow);
+                    if (++ks == C::kStages) { ks = 0; kph ^= 1u; }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ------------------------------------------------ MMA issuer
+            int ks = 0, qb = 0, ab = 0;
+            uint32_t kph = 0, qph = 0, aph = 0;
+            for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
+                Unit un;
+                if (!decode_unit(u, p, un)) continue;
+                if (!mbar_wait(&q_full[qb], qph)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t idesc = idesc_bf16_f32(kBlockM, un.qcount * p.H);
+                const uint32_t q_base = smem_addr(q_sm + qb * C::kQBytes);
+                for (int kt = un.kt0; kt < un.kt1; ++kt) {
+                    if (!mbar_wait(&k_full[ks], kph)) { ok = false; break; }
+                    if (!mbar_wait(&acc_empty[ab], aph ^ 1u)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t k_base = smem_addr(k_sm + ks * C::kKBytes);
+                    const uint32_t d_tmem = tmem_base + (uint32_t)(ab * N_TILE);
+#pragma unroll
+                    for (int h = 0; h < C::kHalves; ++h) {
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) {  // 4 x K=16 per 128-byte swizzle row
+                            const uint64_t a = smem_desc_k_sw128(k_base + h * C::kKHalf + kk * 32);
+                            const uint64_t b = smem_desc_k_sw128(q_base + h * C::kQHalf + kk * 32);
+                            mma_f16_ss(d_tmem, a, b, idesc, (h | kk) != 0);
+                        }
+                    }
+                    mma_commit(&k_empty[ks]);   // key stage free once these MMAs finish
+                    mma_commit(&acc_full[ab]);  // accumulator ready for the epilogue
+                    if (++ks == C::kStages) { ks = 0; kph ^= 1u; }
+                    if (++ab == 2) { ab = 0; aph ^= 1u; }
+                }
+                if (!ok) break;
+                mma_commit(&q_empty[qb]);
+                if (++qb == C::kQBufs) { qb = 0; qph ^= 1u; }
+            }
+        }
+    } else {
+        // ---------------------------------------------------- epilogue
+        const int quarter = warp & 3;                 // TMEM lanes this warp may read
+        const int key_in_tile = quarter * 32 + lane;  // TMEM lane = key
+        const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+        int ab = 0;
+        uint32_t aph = 0;
+        for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
+            Unit un;
+            if (!decode_unit(u, p, un)) continue;
+            const size_t row0 = (size_t)un.b * p.Tq + un.i0;
+            const float4 *w4 = reinterpret_cast<const float4 *>(p.w + row0 * p.H);
+            for (int kt = un.kt0; kt < un.kt1; ++kt) {
+                if (!mbar_wait(&acc_full[ab], aph)) { ok = false; break; }
+                tc_fence_after();
+                const int s = kt * kBlockM + key_in_tile;
+                const uint32_t tbase = tmem_base + lane_addr + (uint32_t)(ab * N_TILE);
+                for (int q = 0; q < un.qcount; ++q) {
+                    float acc = 0.0f;
+                    for (int c = 0; c < p.H; c += 32) {
+                        uint32_t x[32];
+                        tmem_ld_32x32b_x32(tbase + (uint32_t)(q * p.H + c), x);
+                        tmem_ld_wait();
+                        const float4 *wq = w4 + (q * p.H + c) / 4;
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const float4 wv = __ldg(wq + j);
+                            acc = fmaf(wv.x, fmaxf(__uint_as_float(x[4 * j + 0]), 0.0f), acc);
+                            acc = fmaf(wv.y, fmaxf(__uint_as_float(x[4 * j + 1]), 0.0f), acc);
+                            acc = fmaf(wv.z, fmaxf(__uint_as_float(x[4 * j + 2]), 0.0f), acc);
+                            acc = fmaf(wv.w, fmaxf(__uint_as_float(x[4 * j + 3]), 0.0f), acc);
+                        }
+                    }
+                    const int t = p.q_pos0 + un.i0 + q;
+                    if (s < p.L) {
+                        float *dst = p.scores + (row0 + q) * (size_t)p.L + s;
+                        if (s <= t) {
+                            *dst = acc;
+                        } else if (p.fill) {
+                            *dst = -INFINITY;
+                        }
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(&acc_empty[ab]);
+                if (++ab == 2) { ab = 0; aph ^= 1u; }
+            }
+        }
+    }
+
+    if (!ok) atomicOr(&g_indexer_error, 1u);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::kTmemCols);
+    }
+}
+
+// -inf for the keys of row t beyond the key tiles the GEMM visits.
+__global__ void fill_beyond_tiles_kernel(float *__restrict__ scores, int Tq, int L, int q_pos0) {
+    const int row = blockIdx.x;
+    const int t = q_pos0 + row % Tq;
+    const int start = (t / kBlockM + 1) * kBlockM;
+    float *out = scores + (size_t)row * L;
+    for (int s = start + threadIdx.x; s < L; s += blockDim.x) out[s] = -INFINITY;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (fn == nullptr) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult qres;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qres) == cudaSuccess &&
+            qres == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// Row-major bf16 matrix [rows, cols] read as boxes of box_rows x 64 columns
+// with the 128-byte swizzle.
+bool make_map_bf16(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    auto encode = get_encode_fn();
+    if (!encode) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 2};
+    const cuuint32_t box[2] = {64, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int D, int N_TILE>
+cudaError_t launch_tc(const IndexerProblem &pr, const DeviceInfo &info, cudaStream_t stream) {
+    using C = Cfg<D, N_TILE>;
+    if ((size_t)info.max_smem_optin < C::kSmem) return cudaErrorInvalidValue;
+    CUtensorMap tm_q, tm_k;
+    if (!make_map_bf16(&tm_q, pr.q_idx, (uint64_t)pr.B * pr.Tq * pr.H, (uint64_t)D, N_TILE) ||
+        !make_map_bf16(&tm_k, pr.k_idx, (uint64_t)pr.B * pr.L, (uint64_t)D, kBlockM))
+        return cudaErrorInvalidValue;
+
+    Params p;
+    p.w = pr.w;
+    p.scores = pr.scores;
+    p.B = pr.B; p.Tq = pr.Tq; p.L = pr.L; p.q_pos0 = pr.q_pos0; p.H = pr.H;
+    p.QPT = N_TILE / pr.H;
+    p.ngroups = ceil_div(pr.Tq, p.QPT);
+    p.G = pr.B * p.ngroups;
+    p.fill = pr.fill_masked ? 1 : 0;
+    // total key tiles over all groups, to size the chunks
+    long long tiles = 0;
+    int nkt_max = 0;
+    for (int g = 0; g < p.ngroups; ++g) {
+        const int qcount = pr.Tq - g * p.QPT < p.QPT ? pr.Tq - g * p.QPT : p.QPT;
+        const int nkt = (pr.q_pos0 + g * p.QPT + qcount - 1) / kBlockM + 1;
+        tiles += nkt;
+        nkt_max = nkt > nkt_max ? nkt : nkt_max;
+    }
+    tiles *= pr.B;
+    long long chunk = (tiles + (long long)info.sm_count * 32 - 1) / ((long long)info.sm_count * 32);
+    p.C = (int)(chunk < 1 ? 1 : (chunk > 64 ? 64 : chunk));
+    const long long units = (long long)ceil_div(nkt_max, p.C) * p.G;
+    if (units > 0x7fffffffLL) return cudaErrorInvalidValue;
+    p.units = (int)units;
+
+    auto kern = indexer_tc_kernel<D, N_TILE>;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
+    if (err != cudaSuccess) return err;
+    const int grid = p.units < info.sm_count ? p.units : info.sm_count;
+    kern<<<grid, kThreads, C::kSmem, stream>>>(tm_q, tm_k, p);
+    count_launch();
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    if (pr.fill_masked) {
+        fill_beyond_tiles_kernel<<<pr.B * pr.Tq, 256, 0, stream>>>(pr.scores, pr.Tq, pr.L, pr.q_pos0);
+        count_launch();
+        err = cudaGetLastError();
+    }
+    return err;
+}
+
+}  // namespace
+
+unsigned int indexer_take_device_error() {
+    unsigned int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_indexer_error, sizeof(v)) != cudaSuccess) return 0;
+    cudaMemcpyToSymbol(g_indexer_error, &zero, sizeof(zero));
+    return v;
+}
+
+cudaError_t launch_indexer_tc(const IndexerProblem &p, cudaStream_t stream, bool *taken) {
+    *taken = false;
+    if (p.dt != DSA_BF16) return cudaSuccess;
+    if (!(p.d == 64 || p.d == 128)) return cudaSuccess;
+    if (!(p.H == 32 || p.H == 64 || p.H == 128)) return cudaSuccess;
+    if (((uintptr_t)p.q_idx | (uintptr_t)p.k_idx | (uintptr_t)p.w) % 16 != 0) return cudaSuccess;
+    DeviceInfo info;
+    cudaError_t err = device_info(&info);
+    if (err != cudaSuccess) return err;
+    if (info.cc_major != 10) return cudaSuccess;
+    // queries per tile: as many as fit 256 columns, but no more than the rows
+    int qpt = 256 / p.H;
+    if (p.Tq < qpt) qpt = p.Tq;
+    int n = qpt * p.H;
+    const int n_tile = n <= 64 ? 64 : (n <= 128 ? 128 : 256);
+    // a TMA box may not be taller than the tensor it reads
+    if ((long long)p.B * p.Tq * p.H < n_tile || (long long)p.B * p.L < kBlockM) return cudaSuccess;
+    *taken = true;
+    if (p.d == 128) {
+        if (n_tile == 64) return launch_tc<128, 64>(p, info, stream);
+        if (n_tile == 128) return launch_tc<128, 128>(p, info, stream);
+        return launch_tc<128, 256>(p, info, stream);
+    }
+    if (n_tile == 64) return launch_tc<64, 64>(p, info, stream);
+    if (n_tile == 128) return launch_tc<64, 128>(p, info, stream);
+    return launch_tc<64, 256>(p, info, stream);
+}
+
 }  // namespace dsa

@@ -1,0 +1,87 @@
+"""Host-side logic of the benchmark: algorithmic work per stage, the
+closed-form counts it relies on, and the max-over-ranks timing reduction on
+two gloo ranks."""
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+from learned_sparse_attention_dsa_b200.inputs import WORKLOADS
+
+
+def test_selected_rows_closed_form():
+    """sum_t min(t+1, k) = k(k+1)/2 + (n-k)k ("DeepSeek Sparse Attention ..." §7.2)."""
+    for name, expect in (("prefill8k", 14_681_088), ("prefill32k", 65_012_736)):
+        wl = WORKLOADS[name]
+        n, k = wl.L, wl.k
+        assert wl.selected_rows() == k * (k + 1) // 2 + (n - k) * k == expect
+    wl = WORKLOADS["toy16"]
+    assert wl.selected_rows() == 45  # §7.3
+    assert WORKLOADS["decode32k"].selected_rows() == 32 * 2048
+
+
+def test_causal_pairs():
+    wl = WORKLOADS["prefill32k"]
+    assert wl.causal_pairs() == 32768 * 32769 // 2
+    wl = WORKLOADS["decode128k"]
+    assert wl.causal_pairs() == 8 * 131072
+
+
+def test_stage_work_figures():
+    w = bench.stage_work(WORKLOADS["decode32k"])
+    idx_bytes, idx_flops = w["indexer"]
+    # K^I cache 32 x 32768 x 128 bf16 = 268 MB dominates
+    assert abs(idx_bytes - 268.4e6) / 268.4e6 < 0.03
+    assert abs(idx_flops - 17.18e9) / 17.18e9 < 0.01
+    attn_bytes, attn_flops = w["attn"]
+    assert abs(attn_bytes - 33.5e6) / 33.5e6 < 0.05
+    p4 = bench.stage_work(WORKLOADS["prefill32k"])
+    assert abs(p4["indexer"][1] - 8.80e12) / 8.80e12 < 0.01
+    assert abs(p4["topk"][0] - 2.15e9) / 2.15e9 < 0.15
+    p3 = bench.stage_work(WORKLOADS["prefill8k"])
+    assert abs(p3["indexer"][1] - 5.50e11) / 5.50e11 < 0.01
+    d5 = bench.stage_work(WORKLOADS["decode128k"])
+    # latent rows: V is a view of the 576-wide K row and adds no bytes
+    assert abs(d5["attn"][0] - (8 * 2048 * 1152 + 8 * 128 * (576 + 512) * 2 + 8 * 2048 * 4)) < 1
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        got = bench._max_over_ranks(1.5 + rank, world, torch.device("cpu"))
+        bench._barrier(world)
+        q.put((rank, got))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    res = dict(q.get(timeout=5) for _ in range(2))
+    assert res == {0: 2.5, 1: 2.5}
+
+
+def test_units_and_metric():
+    units, unit = bench._units(WORKLOADS["decode32k"], 10)
+    assert (units, unit) == (10.0, "decode steps/s")
+    units, unit = bench._units(WORKLOADS["prefill8k"], 2)
+    assert (units, unit) == (2 * 8192.0, "prefill tokens/s")
