@@ -349,28 +349,47 @@ attn_mma_kernel(const Args a) {
     }
 }
 
-// Merge the split partials of one (row, head): one warp, lanes over columns.
+// Merge the split partials of one (row, head): one warp; lane j holds the
+// (max, sum) of split j, then every lane owns four output columns and reads
+// all splits' partials for them with independent 16-byte loads.
+template <int DV>
 __global__ void attn_combine_kernel(const float *__restrict__ part_o, const float *__restrict__ part_ml,
-                                    int n_pairs, int splits, int DV, __nv_bfloat16 *__restrict__ out,
+                                    int n_pairs, int splits, __nv_bfloat16 *__restrict__ out,
                                     float *__restrict__ lse) {
     const int pair = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (pair >= n_pairs) return;
     const float *ml = part_ml + (size_t)pair * splits * 2;
-    float m_all = -INFINITY;
-    for (int sp = 0; sp < splits; ++sp) m_all = fmaxf(m_all, ml[2 * sp]);
-    float l_all = 0.0f;
-    for (int sp = 0; sp < splits; ++sp)
-        l_all += m_all == -INFINITY ? 0.0f : exp2f(ml[2 * sp] - m_all) * ml[2 * sp + 1];
+    const float m_s = lane < splits ? ml[2 * lane] : -INFINITY;
+    const float l_s = lane < splits ? ml[2 * lane + 1] : 0.0f;
+    const float m_all = warp_max(m_s);
+    const float f_s = (m_all == -INFINITY || lane >= splits) ? 0.0f : exp2f(m_s - m_all);
+    const float l_all = warp_sum(f_s * l_s);
     const float inv = l_all > 0.0f ? 1.0f / l_all : 0.0f;
-    const float *po = part_o + (size_t)pair * splits * DV;
-    for (int c = lane; c < DV; c += 32) {
-        float acc = 0.0f;
+    const float4 *po = reinterpret_cast<const float4 *>(part_o + (size_t)pair * splits * DV);
+    constexpr int kCols4 = DV / 4;
+    for (int cb = 0; cb < kCols4; cb += 32) {  // uniform trip count: the shuffles see all lanes
+        const int c4 = cb + lane;
+        const bool active = c4 < kCols4;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
         for (int sp = 0; sp < splits; ++sp) {
-            const float f = m_all == -INFINITY ? 0.0f : exp2f(ml[2 * sp] - m_all);
-            acc += f * po[(size_t)sp * DV + c];
+            const float f = __shfl_sync(0xffffffffu, f_s, sp);
+            if (active) {
+                const float4 v = __ldg(po + (size_t)sp * kCols4 + c4);
+                acc.x = fmaf(f, v.x, acc.x);
+                acc.y = fmaf(f, v.y, acc.y);
+                acc.z = fmaf(f, v.z, acc.z);
+                acc.w = fmaf(f, v.w, acc.w);
+            }
         }
-        out[(size_t)pair * DV + c] = __float2bfloat16_rn(acc * inv);
+        if (!active) continue;
+        __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+        __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+        uint2 packed;
+        packed.x = *reinterpret_cast<uint32_t *>(&lo);
+        packed.y = *reinterpret_cast<uint32_t *>(&hi);
+        *reinterpret_cast<uint2 *>(out + (size_t)pair * DV + 4 * c4) = packed;
     }
     if (lse != nullptr && lane == 0)
         lse[pair] = l_all > 0.0f ? (m_all + log2f(l_all)) / kLog2e : -INFINITY;
@@ -386,6 +405,7 @@ int choose_splits(const AttnProblem &p, int sm_count) {
     const int min_splits = (max_tiles * kRowsPerTile + 2047) / 2048;
     if (splits < min_splits) splits = min_splits;
     if (splits > max_tiles) splits = max_tiles;
+    if (splits > 32) splits = 32;  // the combine kernel keeps one split per lane
     const int tiles_per = (max_tiles + splits - 1) / splits;  // equal whole tiles per split
     return (max_tiles + tiles_per - 1) / tiles_per;
 }
@@ -399,7 +419,9 @@ bool shape_supported(const AttnProblem &p, int *dqk_dv) {
         if (p.Dqk == cfgs[i][0] && p.Dv == cfgs[i][1]) which = i;
     if (which < 0) return false;
     // 16-byte aligned rows for cp.async and 4-byte aligned Q for fragment loads
-    if (((uintptr_t)p.k_cache | (uintptr_t)p.v_cache) % 16 != 0 || (uintptr_t)p.q % 4 != 0) return false;
+    if (((uintptr_t)p.k_cache | (uintptr_t)p.v_cache | (uintptr_t)p.out) % 16 != 0 || (uintptr_t)p.q % 4 != 0)
+        return false;
+    if (p.k > 32 * 2048) return false;  // at most 32 splits of 2048 entries
     if (p.k_ss % 8 || p.k_sb % 8 || p.k_sh % 8 || p.v_ss % 8 || p.v_sb % 8 || p.v_sh % 8) return false;
     *dqk_dv = which;
     return true;
@@ -441,8 +463,8 @@ cudaError_t launch_mma(const AttnProblem &p, const DeviceInfo &info, cudaStream_
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     if (splits > 1) {
         const int warps_per_block = 8;
-        attn_combine_kernel<<<(int)((n_pairs + warps_per_block - 1) / warps_per_block), warps_per_block * 32, 0,
-                              stream>>>(a.part_o, a.part_ml, (int)n_pairs, splits, DV, a.out, a.lse);
+        attn_combine_kernel<DV><<<(int)((n_pairs + warps_per_block - 1) / warps_per_block), warps_per_block * 32, 0,
+                                  stream>>>(a.part_o, a.part_ml, (int)n_pairs, splits, a.out, a.lse);
         count_launch();
         err = cudaGetLastError();
     }
