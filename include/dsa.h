@@ -152,6 +152,36 @@ dsa_status dsa_sparse_attn(const void *q, const void *k_cache, const void *v_cac
 
 size_t dsa_sparse_attn_workspace_bytes(const dsa_attn_shape *sh, dsa_dtype dt);
 
+/*
+ * dsa_sparse_attn_noalloc -- dsa_sparse_attn for callers that cannot pass a
+ * workspace. (The pages have no counterpart: this is a library convenience.)
+ *
+ * Some callers cannot allocate device memory when they call the library: an
+ * engine plugin that is handed a stream but no allocator, or a serving loop
+ * that must never call cudaMalloc because it can synchronise the device. This
+ * entry point takes the same arguments as dsa_sparse_attn minus the
+ * workspace, and keeps the split-k partial results in a fixed array inside
+ * the library (dsa_sparse_attn_noalloc_max_scratch_bytes() bytes, 4 MiB, held
+ * by every GPU that loads libdsa.so until the process exits). It calls no
+ * allocator.
+ *
+ * - Returns DSA_ERR_WORKSPACE without launching anything when the problem
+ *   needs more scratch than that (dsa_sparse_attn_workspace_bytes(sh, dt) >
+ *   the maximum); use dsa_sparse_attn with a workspace then.
+ * - The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress, that device current) and caches it: make that first
+ *   call before any stream capture.
+ * - All calls on a device share the array. Calls whose kernels may overlap on
+ *   the GPU (unordered streams) race on it and produce wrong results.
+ * - Results are those of dsa_sparse_attn for the same arguments.
+ */
+dsa_status dsa_sparse_attn_noalloc(const void *q, const void *k_cache, const void *v_cache,
+                                   const int32_t *idx, const dsa_attn_shape *sh, dsa_dtype dt,
+                                   void *out, float *lse, dsa_stream_t stream);
+
+/* Size of the built-in scratch array used by dsa_sparse_attn_noalloc. */
+size_t dsa_sparse_attn_noalloc_max_scratch_bytes(void);
+
 /* Arguments of the fused forward pass. */
 typedef struct dsa_forward_args {
     int B, Tq, L, q_pos0, k;
