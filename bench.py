@@ -516,8 +516,42 @@ def run_e2e(wl, cpu, binding, device, stream, steps, world):
             "note": "all step inputs copied from pinned host memory, output read back, every step"}
 
 
+def run_stage(args, wl):
+    """Eager launches of one stage only (for profiler captures): W warm-up
+    calls then K timed calls; prints the average device time per call."""
+    from learned_sparse_attention_dsa_b200 import binding
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    dev = to_device(make_inputs(wl), device)
+    scores = torch.empty((wl.B, wl.Tq, wl.L), dtype=torch.float32, device=device)
+    idx = torch.empty((wl.B, wl.Tq, wl.k), dtype=torch.int32, device=device)
+    out = torch.empty((wl.B, wl.Tq, wl.Hq, wl.Dv), dtype=dev["q"].dtype, device=device)
+    binding.indexer_scores(dev["q_idx"], dev["k_idx"], dev["w"], wl.q_pos0, scores=scores)
+    binding.topk(scores, wl.k, wl.q_pos0, idx=idx)
+    calls = {
+        "indexer": lambda: binding.indexer_scores(dev["q_idx"], dev["k_idx"], dev["w"], wl.q_pos0,
+                                                  scores=scores),
+        "topk": lambda: binding.topk(scores, wl.k, wl.q_pos0, idx=idx),
+        "attn": lambda: binding.sparse_attn(dev["q"], dev["k_cache"], dev["v_cache"], idx, wl.scale, out=out),
+    }
+    fn = calls[args.stage]
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    print(json.dumps({"stage": args.stage, "workload": wl.name, "calls": args.steps,
+                      "ms_per_call": e0.elapsed_time(e1) / args.steps}))
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--stage", choices=["indexer", "topk", "attn"], default=None,
+                    help="launch only this stage (profiler captures); prints its time")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
@@ -529,7 +563,9 @@ def main():
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)  # at least three untimed warm-up steps
     wl = WORKLOADS[args.workload]
-    if args.impl == "reference":
+    if args.stage is not None:
+        run_stage(args, wl)
+    elif args.impl == "reference":
         run_reference(args, wl)
     else:
         run_ours(args, wl)

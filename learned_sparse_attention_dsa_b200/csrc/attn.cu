@@ -168,9 +168,13 @@ cudaError_t launch_attn_cuda_core(const AttnProblem &p, cudaStream_t stream) {
                : launch_cuda_core<__nv_bfloat16, false>(p, stream);
 }
 
+cudaError_t launch_attn_perhead(const AttnProblem &p, cudaStream_t stream, bool *taken);
+
 cudaError_t launch_attn(const AttnProblem &p, cudaStream_t stream) {
     bool taken = false;
     cudaError_t err = launch_attn_tc(p, stream, &taken);
+    if (taken || err != cudaSuccess) return err;
+    err = launch_attn_perhead(p, stream, &taken);
     if (taken || err != cudaSuccess) return err;
     return launch_attn_cuda_core(p, stream);
 }

@@ -18,8 +18,12 @@
 // merges the splits. Every selected row is loaded once for all 16 heads.
 #include <math.h>
 
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 #include "internal.h"
+
+namespace cg = cooperative_groups;
 
 namespace dsa {
 
@@ -42,7 +46,8 @@ struct Cfg {
     static constexpr int kStageBytes = kKBytes + kVBytes;
     static constexpr int kStages = (DQK + DV) > 256 ? 2 : 3;
     static constexpr int kMaxSel = 2048;  // selected entries one CTA handles
-    static constexpr int kMergeBytes = kWarps * kHeads * (DV + 2) * 4;
+    // four warps' (O, m, l), then the CTA's merged (O, m, l) for the cluster merge
+    static constexpr int kMergeBytes = (kWarps + 1) * kHeads * (DV + 2) * 4;
     static constexpr int kPipeBytes = kStages * kStageBytes;
     static constexpr size_t kSmem =
         (size_t)(kPipeBytes > kMergeBytes ? kPipeBytes : kMergeBytes) + kMaxSel * 4 + 64;
@@ -58,7 +63,12 @@ struct Args {
     float *lse;
     float *part_o;   // [rows, Hq, splits, DV] when splits > 1
     float *part_ml;  // [rows, Hq, splits, 2]
+    int cluster_merge;  // splits merged inside their cluster (no workspace)
 };
+
+// Up to eight splits (a portable cluster) merge through distributed shared
+// memory; more splits go through the workspace and the combine kernel.
+inline bool uses_cluster_merge(int splits) { return splits > 1 && splits <= 8; }
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid) {
     const int n = valid ? 16 : 0;  // 0 source bytes: the 16 bytes are zero-filled
@@ -333,6 +343,50 @@ attn_mma_kernel(const Args a) {
         }
         if (a.lse != nullptr && c0 == 0)
             a.lse[(size_t)row * a.Hq + h] = l_all > 0.0f ? (m_all + log2f(l_all)) / kLog2e : -INFINITY;
+    } else if (a.cluster_merge) {
+        // the splits of this (row, head group) form one cluster: publish this
+        // CTA's (max, sum, O) in shared memory, then every CTA merges a slice
+        // of the 16 x DV outputs from all of them through distributed shared
+        // memory
+        float *cta_o = mrg_ml + kWarps * kHeads * 2;  // [16][DV]
+        float *cta_ml = cta_o + kHeads * DV;          // [16][2]
+        for (int c = c0; c < DV; c += 8) {
+            float acc = 0.0f;
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) acc += fw[w] * mrg_o[(w * kHeads + hh) * DV + c];
+            cta_o[hh * DV + c] = acc;
+        }
+        if (c0 == 0) {
+            cta_ml[hh * 2 + 0] = m_all;
+            cta_ml[hh * 2 + 1] = l_all;
+        }
+        cg::cluster_group cluster = cg::this_cluster();
+        cluster.sync();
+        const int P = a.splits;
+        const int per = (kHeads * DV + P - 1) / P;
+        const int e0 = split * per, e1 = min(kHeads * DV, e0 + per);
+        for (int e = e0 + threadIdx.x; e < e1; e += kThreads) {
+            const int he = e / DV, ce = e - he * DV;
+            float ms[8], m_x = -INFINITY;
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                ms[r] = r < P ? cluster.map_shared_rank(cta_ml, r)[he * 2] : -INFINITY;
+                m_x = fmaxf(m_x, ms[r]);
+            }
+            float acc = 0.0f, l_x = 0.0f;
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                if (r < P) {
+                    const float f = m_x == -INFINITY ? 0.0f : exp2f(ms[r] - m_x);
+                    l_x += f * cluster.map_shared_rank(cta_ml, r)[he * 2 + 1];
+                    acc += f * cluster.map_shared_rank(cta_o, r)[he * DV + ce];
+                }
+            }
+            a.out[((size_t)row * a.Hq + h0 + he) * DV + ce] = __float2bfloat16_rn(l_x > 0.0f ? acc / l_x : 0.0f);
+            if (a.lse != nullptr && ce == 0)
+                a.lse[(size_t)row * a.Hq + h0 + he] = l_x > 0.0f ? (m_x + log2f(l_x)) / kLog2e : -INFINITY;
+        }
+        cluster.sync();  // no CTA leaves while another may still read its shared memory
     } else {
         const size_t pidx = ((size_t)row * a.Hq + h) * a.splits + split;
         float *dst = a.part_o + pidx * DV;
@@ -450,7 +504,8 @@ cudaError_t launch_mma(const AttnProblem &p, const DeviceInfo &info, cudaStream_
     const size_t n_pairs = (size_t)rows * p.Hq;
     a.part_o = nullptr;
     a.part_ml = nullptr;
-    if (splits > 1) {
+    a.cluster_merge = uses_cluster_merge(splits) ? 1 : 0;
+    if (splits > 1 && !a.cluster_merge) {
         a.part_o = static_cast<float *>(p.ws);
         a.part_ml = a.part_o + n_pairs * splits * DV;
     }
@@ -458,6 +513,23 @@ cudaError_t launch_mma(const AttnProblem &p, const DeviceInfo &info, cudaStream_
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
     if (err != cudaSuccess) return err;
     dim3 grid(rows, p.Hq / kHeads, splits);
+    if (a.cluster_merge) {  // the splits of one (row, head group) form a cluster
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = grid;
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = C::kSmem;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 1;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = splits;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        err = cudaLaunchKernelEx(&cfg, kern, a);
+        count_launch();
+        return err;
+    }
     kern<<<grid, kThreads, C::kSmem, stream>>>(a);
     count_launch();
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
@@ -473,24 +545,48 @@ cudaError_t launch_mma(const AttnProblem &p, const DeviceInfo &info, cudaStream_
 
 }  // namespace
 
+bool attn_mla_supported(const AttnProblem &p);
+size_t attn_mla_workspace_bytes(const AttnProblem &p, int sm_count);
+cudaError_t launch_attn_mla(const AttnProblem &p, const DeviceInfo &info, cudaStream_t stream);
+
+cudaError_t launch_attn_combine(const float *part_o, const float *part_ml, int n_pairs, int splits, int DV,
+                                __nv_bfloat16 *out, float *lse, cudaStream_t stream) {
+    const int warps_per_block = 8;
+    const int blocks = (n_pairs + warps_per_block - 1) / warps_per_block;
+    switch (DV) {
+        case 64: attn_combine_kernel<64><<<blocks, warps_per_block * 32, 0, stream>>>(part_o, part_ml, n_pairs, splits, out, lse); break;
+        case 128: attn_combine_kernel<128><<<blocks, warps_per_block * 32, 0, stream>>>(part_o, part_ml, n_pairs, splits, out, lse); break;
+        case 512: attn_combine_kernel<512><<<blocks, warps_per_block * 32, 0, stream>>>(part_o, part_ml, n_pairs, splits, out, lse); break;
+        default: return cudaErrorInvalidValue;
+    }
+    count_launch();
+    return cudaGetLastError();
+}
+
 size_t attn_tc_workspace_bytes(const AttnProblem &p) {
-    int which;
-    if (!shape_supported(p, &which)) return 0;
     DeviceInfo info;
     if (device_info(&info) != cudaSuccess) return 0;
+    if (attn_mla_supported(p)) return attn_mla_workspace_bytes(p, info.sm_count);
+    int which;
+    if (!shape_supported(p, &which)) return 0;
     const int splits = choose_splits(p, info.sm_count);
-    if (splits <= 1) return 0;
+    if (splits <= 1 || uses_cluster_merge(splits)) return 0;
     const size_t n_pairs = (size_t)p.B * p.Tq * p.Hq;
     return n_pairs * splits * ((size_t)p.Dv + 2) * sizeof(float);
 }
 
 cudaError_t launch_attn_tc(const AttnProblem &p, cudaStream_t stream, bool *taken) {
     *taken = false;
-    int which;
-    if (!shape_supported(p, &which)) return cudaSuccess;
     DeviceInfo info;
     cudaError_t err = device_info(&info);
     if (err != cudaSuccess) return err;
+    if (attn_mla_supported(p)) {
+        if (attn_tc_workspace_bytes(p) > p.ws_bytes) return cudaSuccess;
+        *taken = true;
+        return launch_attn_mla(p, info, stream);
+    }
+    int which;
+    if (!shape_supported(p, &which)) return cudaSuccess;
     if (attn_tc_workspace_bytes(p) > p.ws_bytes) return cudaSuccess;
     *taken = true;
     switch (which) {
