@@ -37,6 +37,13 @@ from learned_sparse_attention_dsa_b200.inputs import WORKLOADS, make_inputs, to_
 
 METRIC = "prefill tokens/s and decode steps/s at k=2048; % HBM/tensor roofline per stage"
 
+# dram__bytes_read.sum + dram__bytes_write.sum per launch of a stage's kernel,
+# from one ncu capture of the current kernel (profiles/ holds each capture's
+# summary and command). An entry is removed when its kernel changes.
+DRAM_TRAFFIC_PER_LAUNCH = {
+    ("decode32k", "indexer"): 275.6e6,    # profiles/indexer_tc_decode32k.md
+}
+
 
 # ------------------------------------------------------------------ helpers
 
@@ -365,14 +372,15 @@ def run_ours(args, wl):
     bound = "hbm"
     if dominant == "indexer" and not wl.is_decode:
         bound = "tensor"
+    traffic = DRAM_TRAFFIC_PER_LAUNCH.get((wl.name, dominant))
     if bound == "tensor":
         roofline = {"bound": "tensor", "kernel": dominant, "achieved": d["TFLOP/s"],
                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                    "frac": d["TFLOP/s"] / peaks["bf16_tflops"], "traffic": None,
+                    "frac": d["TFLOP/s"] / peaks["bf16_tflops"], "traffic": traffic,
                     "peak_source": peaks["source"]}
     else:
         roofline = {"bound": "hbm", "kernel": dominant, "achieved": d["GB/s"], "peak": peaks["hbm_gbs"],
-                    "unit": "GB/s", "frac": d["GB/s"] / peaks["hbm_gbs"], "traffic": None,
+                    "unit": "GB/s", "frac": d["GB/s"] / peaks["hbm_gbs"], "traffic": traffic,
                     "peak_source": peaks["source"]}
 
     # ---- end to end through the public API with host buffers

@@ -47,7 +47,8 @@ struct Cfg {
     static constexpr int kStages = (DQK + DV) > 256 ? 2 : 3;
     static constexpr int kMaxSel = 2048;  // selected entries one CTA handles
     // four warps' (O, m, l), then the CTA's merged (O, m, l) for the cluster merge
-    static constexpr int kMergeBytes = (kWarps + 1) * kHeads * (DV + 2) * 4;
+    // (plus one merge weight per split and head)
+    static constexpr int kMergeBytes = (kWarps + 1) * kHeads * (DV + 2) * 4 + 8 * kHeads * 4;
     static constexpr int kPipeBytes = kStages * kStageBytes;
     static constexpr size_t kSmem =
         (size_t)(kPipeBytes > kMergeBytes ? kPipeBytes : kMergeBytes) + kMaxSel * 4 + 64;
@@ -117,6 +118,21 @@ attn_mma_kernel(const Args a) {
     const int h0 = hgroup * kHeads;
     const int g = h0 / (a.Hq / a.Hkv);
 
+    // ---- Q fragments (A operand, 16 heads x DQK) straight from global memory
+    uint32_t qf[DQK / 16][4];
+    {
+        const int hr = lane >> 2, kc = (lane & 3) * 2;
+        const __nv_bfloat16 *q0 = a.q + ((size_t)row * a.Hq + h0 + hr) * DQK;
+        const __nv_bfloat16 *q8 = q0 + 8 * DQK;
+#pragma unroll
+        for (int kk = 0; kk < DQK / 16; ++kk) {
+            qf[kk][0] = *reinterpret_cast<const uint32_t *>(q0 + kk * 16 + kc);
+            qf[kk][1] = *reinterpret_cast<const uint32_t *>(q8 + kk * 16 + kc);
+            qf[kk][2] = *reinterpret_cast<const uint32_t *>(q0 + kk * 16 + 8 + kc);
+            qf[kk][3] = *reinterpret_cast<const uint32_t *>(q8 + kk * 16 + 8 + kc);
+        }
+    }
+
     // ---- compact this split's valid selected positions (order kept)
     const int j0 = split * a.per_split;
     const int j1 = min(a.k, j0 + a.per_split);
@@ -124,10 +140,19 @@ attn_mma_kernel(const Args a) {
     __syncthreads();
     {
         __shared__ int warp_base[kWarps];
+        // all of this split's entries are loaded up front: one memory latency
+        constexpr int kIters = C::kMaxSel / kThreads;
+        int sv[kIters];
+#pragma unroll
+        for (int it = 0; it < kIters; ++it) {
+            const int j = j0 + it * kThreads + threadIdx.x;
+            sv[it] = j < j1 ? __ldg(a.idx + (size_t)row * a.k + j) : -1;
+        }
         int base = 0;
-        for (int c0 = j0; c0 < j1; c0 += kThreads) {
-            const int j = c0 + threadIdx.x;
-            int s = j < j1 ? a.idx[(size_t)row * a.k + j] : -1;
+#pragma unroll
+        for (int it = 0; it < kIters; ++it) {
+            if (j0 + it * kThreads >= j1) break;  // uniform
+            const int s = sv[it];
             const bool valid = s >= 0 && s < a.L;
             const unsigned m = __ballot_sync(0xffffffffu, valid);
             if (lane == 0) warp_base[warp] = __popc(m);
@@ -170,21 +195,6 @@ attn_mma_kernel(const Args a) {
             }
         }
     };
-
-    // ---- Q fragments (A operand, 16 heads x DQK) straight from global memory
-    uint32_t qf[DQK / 16][4];
-    {
-        const int hr = lane >> 2, kc = (lane & 3) * 2;
-        const __nv_bfloat16 *q0 = a.q + ((size_t)row * a.Hq + h0 + hr) * DQK;
-        const __nv_bfloat16 *q8 = q0 + 8 * DQK;
-#pragma unroll
-        for (int kk = 0; kk < DQK / 16; ++kk) {
-            qf[kk][0] = *reinterpret_cast<const uint32_t *>(q0 + kk * 16 + kc);
-            qf[kk][1] = *reinterpret_cast<const uint32_t *>(q8 + kk * 16 + kc);
-            qf[kk][2] = *reinterpret_cast<const uint32_t *>(q0 + kk * 16 + 8 + kc);
-            qf[kk][3] = *reinterpret_cast<const uint32_t *>(q8 + kk * 16 + 8 + kc);
-        }
-    }
 
     float o[DV / 8][4];
 #pragma unroll
@@ -363,28 +373,60 @@ attn_mma_kernel(const Args a) {
         cg::cluster_group cluster = cg::this_cluster();
         cluster.sync();
         const int P = a.splits;
-        const int per = (kHeads * DV + P - 1) / P;
-        const int e0 = split * per, e1 = min(kHeads * DV, e0 + per);
-        for (int e = e0 + threadIdx.x; e < e1; e += kThreads) {
-            const int he = e / DV, ce = e - he * DV;
-            float ms[8], m_x = -INFINITY;
+        // (max, sum) of every split for the 16 heads: read once, then one
+        // weight per (split, head) with the 1/sum folded in
+        float *wts = cta_ml + kHeads * 2;  // [8][16]
+        if (threadIdx.x < kHeads) {
+            const int he = threadIdx.x;
+            float ms[8], ls[8], m_x = -INFINITY;
 #pragma unroll
             for (int r = 0; r < 8; ++r) {
-                ms[r] = r < P ? cluster.map_shared_rank(cta_ml, r)[he * 2] : -INFINITY;
+                ms[r] = -INFINITY;
+                ls[r] = 0.0f;
+                if (r < P) {
+                    const float2 v = *reinterpret_cast<const float2 *>(cluster.map_shared_rank(cta_ml, r) + he * 2);
+                    ms[r] = v.x;
+                    ls[r] = v.y;
+                }
                 m_x = fmaxf(m_x, ms[r]);
             }
-            float acc = 0.0f, l_x = 0.0f;
+            float l_x = 0.0f;
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                ms[r] = (r < P && m_x != -INFINITY) ? exp2f(ms[r] - m_x) : 0.0f;
+                l_x += ms[r] * ls[r];
+            }
+            const float inv = l_x > 0.0f ? 1.0f / l_x : 0.0f;
+#pragma unroll
+            for (int r = 0; r < 8; ++r) wts[r * kHeads + he] = ms[r] * inv;
+            if (a.lse != nullptr && split == 0)
+                a.lse[(size_t)row * a.Hq + h0 + he] = l_x > 0.0f ? (m_x + log2f(l_x)) / kLog2e : -INFINITY;
+        }
+        __syncthreads();
+        // this CTA writes a 1/P slice of the 16 x DV outputs, four columns per step
+        constexpr int kQuads = kHeads * DV / 4;
+        const int per = (kQuads + P - 1) / P;
+        const int e0 = split * per, e1 = min(kQuads, e0 + per);
+        for (int e = e0 + threadIdx.x; e < e1; e += kThreads) {
+            const int he = (4 * e) / DV, ce = 4 * e - he * DV;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
             for (int r = 0; r < 8; ++r) {
                 if (r < P) {
-                    const float f = m_x == -INFINITY ? 0.0f : exp2f(ms[r] - m_x);
-                    l_x += f * cluster.map_shared_rank(cta_ml, r)[he * 2 + 1];
-                    acc += f * cluster.map_shared_rank(cta_o, r)[he * DV + ce];
+                    const float f = wts[r * kHeads + he];
+                    const float4 v = *reinterpret_cast<const float4 *>(cluster.map_shared_rank(cta_o, r) + he * DV + ce);
+                    acc.x = fmaf(f, v.x, acc.x);
+                    acc.y = fmaf(f, v.y, acc.y);
+                    acc.z = fmaf(f, v.z, acc.z);
+                    acc.w = fmaf(f, v.w, acc.w);
                 }
             }
-            a.out[((size_t)row * a.Hq + h0 + he) * DV + ce] = __float2bfloat16_rn(l_x > 0.0f ? acc / l_x : 0.0f);
-            if (a.lse != nullptr && ce == 0)
-                a.lse[(size_t)row * a.Hq + h0 + he] = l_x > 0.0f ? (m_x + log2f(l_x)) / kLog2e : -INFINITY;
+            __nv_bfloat162 lo2 = __floats2bfloat162_rn(acc.x, acc.y);
+            __nv_bfloat162 hi2 = __floats2bfloat162_rn(acc.z, acc.w);
+            uint2 packed;
+            packed.x = *reinterpret_cast<uint32_t *>(&lo2);
+            packed.y = *reinterpret_cast<uint32_t *>(&hi2);
+            *reinterpret_cast<uint2 *>(a.out + ((size_t)row * a.Hq + h0 + he) * DV + ce) = packed;
         }
         cluster.sync();  // no CTA leaves while another may still read its shared memory
     } else {

@@ -11,13 +11,15 @@
 // of a query in its own registers, so the ReLU, the weights and the head sum
 // need no cross-thread reduction, and the per-head scores never leave the SM.
 //
-// Warp roles (192 threads, one CTA per SM, persistent over work units):
+// Warp roles (320 threads, one CTA per SM, persistent over work units):
 //   warp 0      TMA producer: Q tile of the unit once, then key tiles through
 //               a K_STAGES-deep ring (128-byte swizzle, K-major).
 //   warp 1      allocates TMEM; one thread issues tcgen05.mma (bf16 in, fp32
 //               accumulate) into one of two TMEM accumulators.
-//   warps 2-5   epilogue: tcgen05.ld of the accumulator, ReLU, weight, head
-//               sum, one fp32 score per (query, key), causal mask.
+//   warps 2-9   epilogue, two warps per TMEM lane quarter (each takes every
+//               other query of the tile): tcgen05.ld of the accumulator, ReLU,
+//               weight and head sum with packed fp32x2 FMAs, one fp32 score
+//               per (query, key), causal mask.
 // The two accumulators let the epilogue of tile n overlap the MMAs of tile
 // n+1. A work unit is (batch entry, query group, chunk of at most C key
 // tiles); units are spread over the CTAs round-robin. Causal: a query group
@@ -42,7 +44,18 @@ namespace {
 using namespace sm100;
 
 constexpr int kBlockM = 128;       // keys per tile (TMEM lanes)
-constexpr int kThreads = 192;      // 6 warps
+constexpr int kEpilogueThreads = 256;            // 8 warps: two per TMEM lane quarter
+constexpr int kThreads = 64 + kEpilogueThreads;  // + the TMA and MMA warps
+
+// acc(lo, hi) += (a_lo * b_lo, a_hi * b_hi), two independent IEEE fp32 FMAs
+__device__ __forceinline__ void fma2(uint64_t &acc, float a_lo, float a_hi, float b_lo, float b_hi) {
+    uint64_t a, b;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(a_lo), "f"(a_hi));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(b) : "f"(b_lo), "f"(b_hi));
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(a), "l"(b));
+}
+__device__ __forceinline__ float lo_f32(uint64_t v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float hi_f32(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
 constexpr uint32_t kSmemBudget = 224 * 1024;
 
 __device__ unsigned int g_indexer_error = 0;  // 1 = a bounded wait gave up
@@ -128,7 +141,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&acc_full[s], 1);
-            mbar_init(&acc_empty[s], 128);
+            mbar_init(&acc_empty[s], kEpilogueThreads);
         }
         fence_barrier_init();
     }
@@ -210,6 +223,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     } else {
         // ---------------------------------------------------- epilogue
         const int quarter = warp & 3;                 // TMEM lanes this warp may read
+        const int q_first = (warp - 2) >> 2;          // 0 or 1: this warp takes queries q_first, q_first+2, ...
         const int key_in_tile = quarter * 32 + lane;  // TMEM lane = key
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
         int ab = 0;
@@ -224,8 +238,9 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 tc_fence_after();
                 const int s = kt * kBlockM + key_in_tile;
                 const uint32_t tbase = tmem_base + lane_addr + (uint32_t)(ab * N_TILE);
-                for (int q = 0; q < un.qcount; ++q) {
-                    float acc = 0.0f;
+                for (int q = q_first; q < un.qcount; q += 2) {
+                    // four independent packed (f32x2) partial sums
+                    uint64_t part[4] = {0ull, 0ull, 0ull, 0ull};
                     for (int c = 0; c < p.H; c += 32) {
                         uint32_t x[32];
                         tmem_ld_32x32b_x32(tbase + (uint32_t)(q * p.H + c), x);
@@ -234,12 +249,16 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 #pragma unroll
                         for (int j = 0; j < 8; ++j) {
                             const float4 wv = __ldg(wq + j);
-                            acc = fmaf(wv.x, fmaxf(__uint_as_float(x[4 * j + 0]), 0.0f), acc);
-                            acc = fmaf(wv.y, fmaxf(__uint_as_float(x[4 * j + 1]), 0.0f), acc);
-                            acc = fmaf(wv.z, fmaxf(__uint_as_float(x[4 * j + 2]), 0.0f), acc);
-                            acc = fmaf(wv.w, fmaxf(__uint_as_float(x[4 * j + 3]), 0.0f), acc);
+                            const float r0 = fmaxf(__uint_as_float(x[4 * j + 0]), 0.0f);
+                            const float r1 = fmaxf(__uint_as_float(x[4 * j + 1]), 0.0f);
+                            const float r2 = fmaxf(__uint_as_float(x[4 * j + 2]), 0.0f);
+                            const float r3 = fmaxf(__uint_as_float(x[4 * j + 3]), 0.0f);
+                            fma2(part[(2 * j) & 3], wv.x, wv.y, r0, r1);
+                            fma2(part[(2 * j + 1) & 3], wv.z, wv.w, r2, r3);
                         }
                     }
+                    const float acc = (lo_f32(part[0]) + hi_f32(part[0]) + (lo_f32(part[1]) + hi_f32(part[1]))) +
+                                      (lo_f32(part[2]) + hi_f32(part[2]) + (lo_f32(part[3]) + hi_f32(part[3])));
                     const int t = p.q_pos0 + un.i0 + q;
                     if (s < p.L) {
                         float *dst = p.scores + (row0 + q) * (size_t)p.L + s;
@@ -330,7 +349,11 @@ cudaError_t launch_tc(const IndexerProblem &pr, const DeviceInfo &info, cudaStre
         nkt_max = nkt > nkt_max ? nkt : nkt_max;
     }
     tiles *= pr.B;
-    long long chunk = (tiles + (long long)info.sm_count * 32 - 1) / ((long long)info.sm_count * 32);
+    // About 32 units per CTA when the query tile is small (decode: cheap
+    // reloads, fine balance), about 8 when it is 64 KB (prefill: each unit
+    // reloads its query tile).
+    const long long units_per_cta = pr.Tq == 1 ? 32 : 8;
+    long long chunk = (tiles + (long long)info.sm_count * units_per_cta - 1) / ((long long)info.sm_count * units_per_cta);
     p.C = (int)(chunk < 1 ? 1 : (chunk > 64 ? 64 : chunk));
     const long long units = (long long)ceil_div(nkt_max, p.C) * p.G;
     if (units > 0x7fffffffLL) return cudaErrorInvalidValue;

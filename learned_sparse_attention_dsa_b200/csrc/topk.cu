@@ -13,12 +13,13 @@
 // A row is handled by a cluster of P CTAs (P = 1..16; P > 1 when there are
 // fewer rows than SMs, as in decode), each owning a contiguous slice. Digit
 // histograms are summed across the cluster through distributed shared memory
-// so every CTA derives the same threshold. The row is streamed from global
-// memory (L2 after the first read) rather than cached, so several CTAs fit on
-// an SM. After the first pass the keys of the threshold bucket -- usually a
-// few percent of the row -- are compacted into shared memory with their
-// positions, and the later passes and the per-warp counts run on that list
-// only (rows with more candidates than the list holds are re-streamed).
+// so every CTA derives the same threshold. A slice of at most 512 * KPT keys
+// is held in registers (KPT keys per thread); longer slices are streamed from
+// global memory (L2 after the first read), so several CTAs fit on an SM.
+// After the first pass the keys of the threshold bucket -- usually a few
+// percent of the row -- are compacted into shared memory with their
+// positions; the later passes and the per-warp counts run on that list only
+// (slices with more candidates than the list holds are swept again).
 // Output: each warp owns a contiguous segment of its CTA's slice; with the
 // number of keys > T and = T before the segment (from the list, the warps
 // before it and the CTAs before it) every kept position's output slot is
@@ -54,61 +55,103 @@ __device__ __forceinline__ unsigned lanemask_lt() {
     return m;
 }
 
-// Exclusive block scan (kThreads threads); scratch holds kWarps + 1 ints.
-__device__ __forceinline__ int block_exclusive_scan(int v, int *scratch) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int incl = warp_inclusive_scan(v);
-    if (lane == 31) scratch[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-        const int wv = lane < kWarps ? scratch[lane] : 0;
-        const int wincl = warp_inclusive_scan(wv);
-        if (lane < kWarps) scratch[lane] = wincl - wv;
-    }
-    __syncthreads();
-    const int r = scratch[warp] + incl - v;
-    __syncthreads();
-    return r;
+__device__ __forceinline__ void cluster_arrive() {
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// Sum the cluster's NBINS-bin histograms and find the digit whose bucket
-// holds the remaining-th largest key; all P loads of a bin group are issued
-// together. Writes *s_digit and *s_above (keys in higher buckets).
+struct FindScratch {
+    int local[kThreads];     // bucket total per thread (descending digit order)
+    int red[kBins];          // this CTA's segment of the cluster-summed histogram
+    int seg_total;           // sum of that segment
+};
+
+// Cluster-wide digit search by reduce-scatter: CTA `part` sums bins
+// [part*seg, (part+1)*seg) over all P histograms (seg = NBINS / P) into its
+// own shared memory; after a cluster barrier every CTA reads the P segment
+// totals, picks the segment holding the remaining-th largest key (highest
+// bins first) and reads only that segment from its owner. Each CTA moves
+// NBINS + P + seg values over distributed shared memory per pass instead of
+// P * NBINS. Ends with s_digit / s_above set.
 template <int NBINS>
-__device__ __forceinline__ void find_digit(const cg::cluster_group &cluster, int *hist, int P, int remaining,
-                                           int *scratch, int *s_digit, int *s_above) {
-    constexpr int PER = NBINS / kThreads;  // 4 or 2 consecutive bins per thread
-    const int first = NBINS - PER * (threadIdx.x + 1);  // thread 0 owns the highest bins
-    int c[PER];
+__device__ __forceinline__ void find_digit_rs(const cg::cluster_group &cluster, int *hist, int P, int part,
+                                              int remaining, FindScratch &fs, int *s_digit, int *s_above,
+                                              int *s_seg) {
+    const int seg = NBINS / P;  // >= 64, a multiple of 4
+    const int lo = part * seg;
+    // 1. reduce this CTA's segment over the cluster (int4 columns x ranks)
+    for (int c = threadIdx.x; c < seg / 4; c += kThreads) {
+        int4 acc = make_int4(0, 0, 0, 0);
 #pragma unroll
-    for (int j = 0; j < PER; ++j) c[j] = 0;
-#pragma unroll
-    for (int r = 0; r < kMaxCluster; ++r) {
-        if (r < P) {
-            const int *h = cluster.map_shared_rank(hist, r) + first;
-            if constexpr (PER == 4) {
-                const int4 v = *reinterpret_cast<const int4 *>(h);
-                c[0] += v.x; c[1] += v.y; c[2] += v.z; c[3] += v.w;
-            } else {
-                const int2 v = *reinterpret_cast<const int2 *>(h);
-                c[0] += v.x; c[1] += v.y;
+        for (int r = 0; r < kMaxCluster; ++r) {
+            if (r < P) {
+                const int4 v = *reinterpret_cast<const int4 *>(cluster.map_shared_rank(hist, r) + lo + 4 * c);
+                acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
             }
         }
+        *reinterpret_cast<int4 *>(fs.red + lo + 4 * c) = acc;
     }
+    __syncthreads();
+    if (threadIdx.x < kWarp) {
+        int s = 0;
+        for (int b = lo + threadIdx.x; b < lo + seg; b += kWarp) s += fs.red[b];
+        s = warp_sum_int(s);
+        if (threadIdx.x == 0) fs.seg_total = s;
+    }
+    cluster.sync();
+    // 2. which segment (highest bins first), then which bin inside it
+    if (threadIdx.x < kWarp) {
+        const int lane = threadIdx.x;
+        const int sg = P - 1 - lane;  // lane 0 looks at the highest segment
+        const int tot = lane < P ? *cluster.map_shared_rank(&fs.seg_total, sg) : 0;
+        const int incl = warp_inclusive_scan(tot);
+        const int excl = incl - tot;
+        if (lane < P && excl < remaining && incl >= remaining) {
+            *s_seg = sg;
+            *s_above = excl;
+        }
+    }
+    __syncthreads();
+    const int sg = *s_seg;
+    const int base_above = *s_above;
+    const int *red_owner = cluster.map_shared_rank(fs.red, sg) + sg * seg;
+    // every thread takes (seg / kThreads, at least 1) consecutive bins from the top of the segment
+    const int per = seg >= kThreads ? seg / kThreads : 1;
     int local = 0;
+    if (threadIdx.x * per < seg) {
+        for (int j = 0; j < per; ++j) {
+            local += red_owner[seg - 1 - (threadIdx.x * per + j)];  // descending bins
+        }
+    }
+    fs.local[threadIdx.x] = local;
+    __syncthreads();
+    if (threadIdx.x < kWarp) {
+        const int lane = threadIdx.x;
+        constexpr int kPerLane = kThreads / kWarp;
+        int sum = 0;
 #pragma unroll
-    for (int j = 0; j < PER; ++j) local += c[j];
-    const int excl = block_exclusive_scan(local, scratch);
-    if (excl < remaining && excl + local >= remaining) {
-        int run = excl;
-#pragma unroll
-        for (int j = PER - 1; j >= 0; --j) {  // descending digit order
-            if (run + c[j] >= remaining) {
-                *s_digit = first + j;
-                *s_above = run;
-                break;
+        for (int i = 0; i < kPerLane; ++i) sum += fs.local[lane * kPerLane + i];
+        const int incl = warp_inclusive_scan(sum);
+        int run = base_above + incl - sum;
+        if (run < remaining && base_above + incl >= remaining) {
+            for (int i = 0; i < kPerLane; ++i) {
+                const int t = lane * kPerLane + i;
+                if (run + fs.local[t] >= remaining) {
+                    for (int j = 0; j < per; ++j) {
+                        const int cj = red_owner[seg - 1 - (t * per + j)];
+                        if (run + cj >= remaining) {
+                            *s_digit = sg * seg + seg - 1 - (t * per + j);
+                            *s_above = run;
+                            break;
+                        }
+                        run += cj;
+                    }
+                    break;
+                }
+                run += fs.local[t];
             }
-            run += c[j];
         }
     }
     __syncthreads();
@@ -120,35 +163,51 @@ struct Slice {
     int w_lo, w_hi;    // this warp's segment [w_lo, w_hi) of the slice
 };
 
-// Apply fn(pos, key, valid) to the warp's segment, 32 consecutive positions
-// per step, four steps' loads in flight.
-template <typename F>
-__device__ __forceinline__ void sweep(const Slice &sl, F fn) {
+template <int KPT>
+struct RegKeys {
+    uint32_t k[KPT > 0 ? KPT : 1];
+};
+
+// Apply fn(pos, key, valid) to the warp's segment in position order: 32
+// consecutive positions per step. KPT > 0: the keys are the registers loaded
+// by load_keys; KPT == 0: streamed from global memory, four steps' loads in
+// flight.
+template <int KPT, typename F>
+__device__ __forceinline__ void sweep(const Slice &sl, const RegKeys<KPT> &rk, F fn) {
     const int lane = threadIdx.x & 31;
-    for (int base = sl.w_lo; base < sl.w_hi; base += 4 * kWarp) {
-        float v[4];
+    if constexpr (KPT > 0) {
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int s = base + u * kWarp + lane;
-            v[u] = s < sl.w_hi ? __ldg(sl.src + s) : 0.0f;
+        for (int i = 0; i < KPT; ++i) {
+            const int s = sl.w_lo + i * kWarp + lane;
+            fn(s, rk.k[i], s < sl.w_hi);
         }
+    } else {
+        for (int base = sl.w_lo; base < sl.w_hi; base += 4 * kWarp) {
+            float v[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int s = base + u * kWarp + lane;
-            fn(s, order_key(v[u]), s < sl.w_hi);
+            for (int u = 0; u < 4; ++u) {
+                const int s = base + u * kWarp + lane;
+                v[u] = s < sl.w_hi ? __ldg(sl.src + s) : 0.0f;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int s = base + u * kWarp + lane;
+                fn(s, order_key(v[u]), s < sl.w_hi);
+            }
         }
     }
 }
 
+template <int KPT>
 __global__ void __launch_bounds__(kThreads)
 topk_kernel(const float *__restrict__ scores, int Tq, int L, int q_pos0, int k, int32_t *__restrict__ idx) {
-    __shared__ __align__(16) int hist[2][kBins];
+    __shared__ __align__(16) int hist[3][kBins];
     extern __shared__ __align__(16) uint8_t dyn_smem[];
     uint32_t *list_key = reinterpret_cast<uint32_t *>(dyn_smem);                // [kListCap]
     int32_t *list_pos = reinterpret_cast<int32_t *>(dyn_smem + 4 * kListCap);   // [kListCap]
-    __shared__ int scratch[kWarps + 1];
+    FindScratch &fs = *reinterpret_cast<FindScratch *>(dyn_smem + 8 * kListCap);
     __shared__ int w_gt[kWarps], w_eq[kWarps];
-    __shared__ int s_digit, s_above, s_nlist;
+    __shared__ int s_digit, s_above, s_nlist, s_seg;
     __shared__ int s_counts[2];
 
     cg::cluster_group cluster = cg::this_cluster();
@@ -170,27 +229,46 @@ topk_kernel(const float *__restrict__ scores, int Tq, int L, int q_pos0, int k, 
     Slice sl;
     sl.src = scores + (size_t)row * L + lo;
     sl.cnt = max(0, min(n, lo + per) - lo);
-    const int seg = ((sl.cnt + kWarps - 1) / kWarps + 31) & ~31;
+    const int seg = KPT > 0 ? KPT * kWarp : ((sl.cnt + kWarps - 1) / kWarps + 31) & ~31;
     sl.w_lo = min(sl.cnt, warp * seg);
     sl.w_hi = min(sl.cnt, sl.w_lo + seg);
 
-    // ---- pass 1: bits 31..21 of every key
-    for (int b = threadIdx.x; b < kBins; b += kThreads) hist[0][b] = 0;
-    if (threadIdx.x == 0) s_nlist = 0;
+    for (int b = threadIdx.x; b < kBins; b += kThreads) {
+        hist[0][b] = 0;
+        hist[1][b] = 0;
+        hist[2][b] = 0;
+    }
+    if (threadIdx.x == 0) {
+        s_nlist = 0;
+        s_seg = 0;  // always a valid cluster rank, even if a search found nothing
+        s_digit = 0;
+        s_above = 0;
+    }
     __syncthreads();
-    sweep(sl, [&](int, uint32_t key, bool ok) {
+
+    // ---- pass 1: bits 31..21 of every key (the keys land in registers)
+    RegKeys<KPT> rk;
+    if constexpr (KPT > 0) {
+#pragma unroll
+        for (int i = 0; i < KPT; ++i) {
+            const int s = sl.w_lo + i * kWarp + lane;
+            const float v = s < sl.w_hi ? __ldg(sl.src + s) : 0.0f;
+            rk.k[i] = order_key(v);
+        }
+    }
+    sweep<KPT>(sl, rk, [&](int, uint32_t key, bool ok) {
         if (ok) atomicAdd(&hist[0][key >> 21], 1);
     });
     __syncthreads();
     cluster.sync();
     int remaining = k;
-    find_digit<kBins>(cluster, hist[0], P, remaining, scratch, &s_digit, &s_above);
+    find_digit_rs<kBins>(cluster, hist[0], P, part, remaining, fs, &s_digit, &s_above, &s_seg);
     const uint32_t d1 = (uint32_t)s_digit;
     remaining -= s_above;
 
     // ---- compact the threshold bucket; count keys in higher buckets per warp
     int gt1 = 0;
-    sweep(sl, [&](int s, uint32_t key, bool ok) {
+    sweep<KPT>(sl, rk, [&](int s, uint32_t key, bool ok) {
         const bool cand = ok && (key >> 21) == d1;
         gt1 += ok && (key >> 21) > d1;
         const unsigned m = __ballot_sync(0xffffffffu, cand);
@@ -210,7 +288,6 @@ topk_kernel(const float *__restrict__ scores, int Tq, int L, int q_pos0, int k, 
         w_gt[warp] = gt1;
         w_eq[warp] = 0;
     }
-    for (int b = threadIdx.x; b < kBins; b += kThreads) hist[1][b] = 0;
     __syncthreads();
     const int n_list = s_nlist;
     const bool use_list = n_list <= kListCap;
@@ -220,32 +297,30 @@ topk_kernel(const float *__restrict__ scores, int Tq, int L, int q_pos0, int k, 
         for (int j = threadIdx.x; j < n_list; j += kThreads)
             atomicAdd(&hist[1][(list_key[j] >> 10) & 2047u], 1);
     } else {
-        sweep(sl, [&](int, uint32_t key, bool ok) {
+        sweep<KPT>(sl, rk, [&](int, uint32_t key, bool ok) {
             if (ok && (key >> 21) == d1) atomicAdd(&hist[1][(key >> 10) & 2047u], 1);
         });
     }
     __syncthreads();
-    cluster.sync();  // also: every CTA is done reading the pass-1 histograms
-    find_digit<kBins>(cluster, hist[1], P, remaining, scratch, &s_digit, &s_above);
+    cluster.sync();
+    find_digit_rs<kBins>(cluster, hist[1], P, part, remaining, fs, &s_digit, &s_above, &s_seg);
     const uint32_t p2 = (d1 << 11) | (uint32_t)s_digit;
     remaining -= s_above;
 
     // ---- pass 3: bits 9..0 of the keys whose top 22 bits are p2
-    for (int b = threadIdx.x; b < 1024; b += kThreads) hist[0][b] = 0;
-    __syncthreads();
     if (use_list) {
         for (int j = threadIdx.x; j < n_list; j += kThreads) {
             const uint32_t key = list_key[j];
-            if ((key >> 10) == p2) atomicAdd(&hist[0][key & 1023u], 1);
+            if ((key >> 10) == p2) atomicAdd(&hist[2][key & 1023u], 1);
         }
     } else {
-        sweep(sl, [&](int, uint32_t key, bool ok) {
-            if (ok && (key >> 10) == p2) atomicAdd(&hist[0][key & 1023u], 1);
+        sweep<KPT>(sl, rk, [&](int, uint32_t key, bool ok) {
+            if (ok && (key >> 10) == p2) atomicAdd(&hist[2][key & 1023u], 1);
         });
     }
     __syncthreads();
     cluster.sync();
-    find_digit<1024>(cluster, hist[0], P, remaining, scratch, &s_digit, &s_above);
+    find_digit_rs<1024>(cluster, hist[2], P, part, remaining, fs, &s_digit, &s_above, &s_seg);
     const uint32_t T = (p2 << 10) | (uint32_t)s_digit;
     remaining -= s_above;
     const int r = remaining;  // keys equal to T that still fit, lowest positions first
@@ -260,7 +335,7 @@ topk_kernel(const float *__restrict__ scores, int Tq, int L, int q_pos0, int k, 
         }
     } else {
         int gt = 0, eq = 0;
-        sweep(sl, [&](int, uint32_t key, bool ok) {
+        sweep<KPT>(sl, rk, [&](int, uint32_t key, bool ok) {
             gt += ok && key > T;
             eq += ok && key == T;
         });
@@ -292,13 +367,13 @@ topk_kernel(const float *__restrict__ scores, int Tq, int L, int q_pos0, int k, 
         gt_b += rc[0];
         eq_b += rc[1];
     }
-    cluster.sync();  // no CTA leaves while another may still read its shared memory
+    cluster_arrive();  // done with the other CTAs' shared memory
 
     // ---- write the kept positions of this warp's segment in order
     gt_b += w_gt[warp];
     eq_b += w_eq[warp];
     const unsigned lt = lanemask_lt();
-    sweep(sl, [&](int s, uint32_t key, bool ok) {
+    sweep<KPT>(sl, rk, [&](int s, uint32_t key, bool ok) {
         const bool gt = ok && key > T;
         const bool eq = ok && key == T;
         const unsigned gm = __ballot_sync(0xffffffffu, gt);
@@ -311,7 +386,10 @@ topk_kernel(const float *__restrict__ scores, int Tq, int L, int q_pos0, int k, 
         gt_b += __popc(gm);
         eq_b += __popc(em);
     });
+    cluster_wait();  // no CTA leaves while another may still read its shared memory
 }
+
+constexpr size_t kDynSmem = 8 * (size_t)kListCap + sizeof(FindScratch);
 
 }  // namespace
 
@@ -324,12 +402,13 @@ static int cluster_parts(int rows, int sm_count) {
     return P;
 }
 
+template <int KPT>
 static cudaError_t launch_parts(const TopkProblem &p, int P, cudaStream_t stream) {
-    constexpr size_t kDynSmem = 8 * (size_t)kListCap;
-    cudaError_t err = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDynSmem);
+    auto kern = topk_kernel<KPT>;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDynSmem);
     if (err != cudaSuccess) return err;
     if (P > 8) {
-        err = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        err = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         if (err != cudaSuccess) return err;
     }
     cudaLaunchConfig_t cfg = {};
@@ -346,15 +425,24 @@ static cudaError_t launch_parts(const TopkProblem &p, int P, cudaStream_t stream
     cfg.numAttrs = 1;
     if (P > 8) {  // a non-portable cluster size: make sure one can be scheduled
         int clusters = 0;
-        err = cudaOccupancyMaxActiveClusters(&clusters, topk_kernel, &cfg);
+        err = cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg);
         if (err != cudaSuccess || clusters == 0) {
             (void)cudaGetLastError();
             return cudaErrorNotSupported;
         }
     }
-    err = cudaLaunchKernelEx(&cfg, topk_kernel, p.scores, p.Tq, p.L, p.q_pos0, p.k, p.idx);
+    err = cudaLaunchKernelEx(&cfg, kern, p.scores, p.Tq, p.L, p.q_pos0, p.k, p.idx);
     count_launch();
     return err;
+}
+
+// Keys per thread held in registers for a slice of `per` scores (0: stream).
+static cudaError_t launch_with(const TopkProblem &p, int P, cudaStream_t stream) {
+    const int n_max = p.q_pos0 + p.Tq;
+    const int per = (n_max + P - 1) / P;
+    if (per <= kThreads * 8) return launch_parts<8>(p, P, stream);
+    if (per <= kThreads * 16) return launch_parts<16>(p, P, stream);
+    return launch_parts<0>(p, P, stream);
 }
 
 cudaError_t launch_topk(const TopkProblem &p, cudaStream_t stream) {
@@ -365,8 +453,8 @@ cudaError_t launch_topk(const TopkProblem &p, cudaStream_t stream) {
     if (rows == 0) return cudaSuccess;
     int P = cluster_parts((int)(rows < 0x7fffffffLL ? rows : 0x7fffffffLL), info.sm_count);
     if (rows * P >= 0x7fffffffLL) return cudaErrorInvalidValue;
-    err = launch_parts(p, P, stream);
-    if (err == cudaErrorNotSupported && P > 8) err = launch_parts(p, 8, stream);
+    err = launch_with(p, P, stream);
+    if (err == cudaErrorNotSupported && P > 8) err = launch_with(p, 8, stream);
     return err;
 }
 
