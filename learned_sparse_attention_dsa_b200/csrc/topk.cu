@@ -40,7 +40,10 @@ namespace {
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / kWarp;
 constexpr int kBins = 2048;
-constexpr int kListCap = 6144;  // candidate keys + positions kept in shared memory
+constexpr int kListCap = 4096;    // candidate keys + positions of this CTA, in shared memory
+constexpr int kGatherCap = 4096;  // candidate keys of the whole row gathered by every CTA
+// (list + gather buffer + scratch + histograms stay under half the shared
+// memory of an SM, so two 512-thread CTAs fit)
 constexpr int kMaxCluster = 16;
 
 __device__ __forceinline__ uint32_t order_key(float f) {
@@ -67,6 +70,9 @@ struct FindScratch {
     int red[kBins];          // this CTA's segment of the cluster-summed histogram
     int seg_total;           // sum of that segment
 };
+
+__device__ __forceinline__ void pick_in_segment(const int *seg_bins, int seg, int first_digit, int base_above,
+                                                int remaining, FindScratch &fs, int *s_digit, int *s_above);
 
 // Cluster-wide digit search by reduce-scatter: CTA `part` sums bins
 // [part*seg, (part+1)*seg) over all P histograms (seg = NBINS / P) into its
@@ -116,14 +122,21 @@ __device__ __forceinline__ void find_digit_rs(const cg::cluster_group &cluster, 
     __syncthreads();
     const int sg = *s_seg;
     const int base_above = *s_above;
-    const int *red_owner = cluster.map_shared_rank(fs.red, sg) + sg * seg;
-    // every thread takes (seg / kThreads, at least 1) consecutive bins from the top of the segment
+    pick_in_segment(cluster.map_shared_rank(fs.red, sg) + sg * seg, seg, sg * seg, base_above, remaining, fs,
+                    s_digit, s_above);
+}
+
+// Bins seg_bins[0..seg) hold the counts of digits first_digit .. first_digit +
+// seg - 1; base_above keys lie in higher digits. Find the digit whose bucket
+// holds the remaining-th largest key: each thread sums (seg / kThreads, at
+// least one) consecutive bins from the top, warp 0 scans the totals. Sets
+// s_digit / s_above. Two block barriers.
+__device__ __forceinline__ void pick_in_segment(const int *seg_bins, int seg, int first_digit, int base_above,
+                                                int remaining, FindScratch &fs, int *s_digit, int *s_above) {
     const int per = seg >= kThreads ? seg / kThreads : 1;
     int local = 0;
     if (threadIdx.x * per < seg) {
-        for (int j = 0; j < per; ++j) {
-            local += red_owner[seg - 1 - (threadIdx.x * per + j)];  // descending bins
-        }
+        for (int j = 0; j < per; ++j) local += seg_bins[seg - 1 - (threadIdx.x * per + j)];  // descending
     }
     fs.local[threadIdx.x] = local;
     __syncthreads();
@@ -140,9 +153,9 @@ __device__ __forceinline__ void find_digit_rs(const cg::cluster_group &cluster, 
                 const int t = lane * kPerLane + i;
                 if (run + fs.local[t] >= remaining) {
                     for (int j = 0; j < per; ++j) {
-                        const int cj = red_owner[seg - 1 - (t * per + j)];
+                        const int cj = seg_bins[seg - 1 - (t * per + j)];
                         if (run + cj >= remaining) {
-                            *s_digit = sg * seg + seg - 1 - (t * per + j);
+                            *s_digit = first_digit + seg - 1 - (t * per + j);
                             *s_above = run;
                             break;
                         }
@@ -199,16 +212,18 @@ __device__ __forceinline__ void sweep(const Slice &sl, const RegKeys<KPT> &rk, F
 }
 
 template <int KPT>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 2)  // two CTAs per SM: at most 64 registers
 topk_kernel(const float *__restrict__ scores, int Tq, int L, int q_pos0, int k, int32_t *__restrict__ idx) {
     __shared__ __align__(16) int hist[3][kBins];
     extern __shared__ __align__(16) uint8_t dyn_smem[];
     uint32_t *list_key = reinterpret_cast<uint32_t *>(dyn_smem);                // [kListCap]
     int32_t *list_pos = reinterpret_cast<int32_t *>(dyn_smem + 4 * kListCap);   // [kListCap]
     FindScratch &fs = *reinterpret_cast<FindScratch *>(dyn_smem + 8 * kListCap);
+    uint32_t *gkey = reinterpret_cast<uint32_t *>(dyn_smem + 8 * kListCap + sizeof(FindScratch));  // [kGatherCap]
     __shared__ int w_gt[kWarps], w_eq[kWarps];
-    __shared__ int s_digit, s_above, s_nlist, s_seg;
-    __shared__ int s_counts[2];
+    __shared__ int s_digit, s_above, s_nlist, s_seg, s_gather;
+    __shared__ int s_counts[2], s_pub[2], s_before[2];
+    __shared__ int g_n[kMaxCluster], g_gt1[kMaxCluster], g_off[kMaxCluster + 1];
 
     cg::cluster_group cluster = cg::this_cluster();
     const int P = (int)cluster.num_blocks();
@@ -243,6 +258,8 @@ topk_kernel(const float *__restrict__ scores, int Tq, int L, int q_pos0, int k, 
         s_seg = 0;  // always a valid cluster rank, even if a search found nothing
         s_digit = 0;
         s_above = 0;
+        s_before[0] = 0;
+        s_before[1] = 0;
     }
     __syncthreads();
 
@@ -292,6 +309,96 @@ topk_kernel(const float *__restrict__ scores, int Tq, int L, int q_pos0, int k, 
     const int n_list = s_nlist;
     const bool use_list = n_list <= kListCap;
 
+    // ---- publish (candidates, keys above the bucket) and read everyone's
+    if (threadIdx.x == 0) {
+        int g = 0;
+        for (int w = 0; w < kWarps; ++w) g += w_gt[w];
+        s_pub[0] = n_list;
+        s_pub[1] = g;
+    }
+    __syncthreads();
+    cluster.sync();
+    if (threadIdx.x < P) {
+        const int *rc = cluster.map_shared_rank(s_pub, threadIdx.x);
+        g_n[threadIdx.x] = rc[0];
+        g_gt1[threadIdx.x] = rc[1];
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int off = 0, ok = 1;
+        for (int c = 0; c < P; ++c) {
+            g_off[c] = off;
+            off += g_n[c];
+            ok &= g_n[c] <= kListCap;
+        }
+        g_off[P] = off;
+        s_gather = ok && off <= kGatherCap;
+    }
+    __syncthreads();
+
+    uint32_t T;
+    int r, gt_b = 0, eq_b = 0;
+    if (s_gather) {
+        // ---- every CTA gathers all candidate keys of the row and finishes
+        // the selection alone: no more cluster-wide rounds
+        const int total = g_off[P];
+        for (int c = 0; c < P; ++c) {
+            const uint32_t *src = cluster.map_shared_rank(list_key, c);
+            for (int j = threadIdx.x; j < g_n[c]; j += kThreads) gkey[g_off[c] + j] = src[j];
+        }
+        cluster_arrive();  // done with the other CTAs' shared memory
+        __syncthreads();
+        for (int j = threadIdx.x; j < total; j += kThreads) atomicAdd(&hist[1][(gkey[j] >> 10) & 2047u], 1);
+        __syncthreads();
+        pick_in_segment(hist[1], kBins, 0, 0, remaining, fs, &s_digit, &s_above);
+        const uint32_t p2 = (d1 << 11) | (uint32_t)s_digit;
+        remaining -= s_above;
+        for (int j = threadIdx.x; j < total; j += kThreads) {
+            const uint32_t key = gkey[j];
+            if ((key >> 10) == p2) atomicAdd(&hist[2][key & 1023u], 1);
+        }
+        __syncthreads();
+        pick_in_segment(hist[2], 1024, 0, 0, remaining, fs, &s_digit, &s_above);
+        T = (p2 << 10) | (uint32_t)s_digit;
+        remaining -= s_above;
+        r = remaining;
+        // keys > T and = T before this CTA (gathered), and per warp of this CTA (own list)
+        int gb = 0, eb = 0;
+        for (int j = threadIdx.x; j < g_off[part]; j += kThreads) {
+            gb += gkey[j] > T;
+            eb += gkey[j] == T;
+        }
+        for (int j = threadIdx.x; j < n_list; j += kThreads) {
+            const uint32_t key = list_key[j];
+            const int w = list_pos[j] / seg;
+            if (key > T) atomicAdd(&w_gt[w], 1);
+            else if (key == T) atomicAdd(&w_eq[w], 1);
+        }
+        gb = warp_sum_int(gb);
+        eb = warp_sum_int(eb);
+        if (lane == 0) {
+            atomicAdd(&s_before[0], gb);
+            atomicAdd(&s_before[1], eb);
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            int g = 0, e = 0;
+            for (int w = 0; w < kWarps; ++w) {
+                const int gw = w_gt[w], ew = w_eq[w];
+                w_gt[w] = g;
+                w_eq[w] = e;
+                g += gw;
+                e += ew;
+            }
+        }
+        __syncthreads();
+        gt_b = s_before[0];
+        eq_b = s_before[1];
+        for (int c = 0; c < part; ++c) gt_b += g_gt1[c];
+    } else {
+        // ---- too many candidates (heavy ties): cluster-wide passes 2 and 3
+        uint32_t p2;
+        {
     // ---- pass 2: bits 20..10 of the keys in bucket d1
     if (use_list) {
         for (int j = threadIdx.x; j < n_list; j += kThreads)
@@ -304,7 +411,7 @@ topk_kernel(const float *__restrict__ scores, int Tq, int L, int q_pos0, int k, 
     __syncthreads();
     cluster.sync();
     find_digit_rs<kBins>(cluster, hist[1], P, part, remaining, fs, &s_digit, &s_above, &s_seg);
-    const uint32_t p2 = (d1 << 11) | (uint32_t)s_digit;
+    p2 = (d1 << 11) | (uint32_t)s_digit;
     remaining -= s_above;
 
     // ---- pass 3: bits 9..0 of the keys whose top 22 bits are p2
@@ -321,9 +428,9 @@ topk_kernel(const float *__restrict__ scores, int Tq, int L, int q_pos0, int k, 
     __syncthreads();
     cluster.sync();
     find_digit_rs<1024>(cluster, hist[2], P, part, remaining, fs, &s_digit, &s_above, &s_seg);
-    const uint32_t T = (p2 << 10) | (uint32_t)s_digit;
+    T = (p2 << 10) | (uint32_t)s_digit;
     remaining -= s_above;
-    const int r = remaining;  // keys equal to T that still fit, lowest positions first
+    r = remaining;  // keys equal to T that still fit, lowest positions first
 
     // ---- keys > T and = T per warp segment
     if (use_list) {
@@ -361,13 +468,14 @@ topk_kernel(const float *__restrict__ scores, int Tq, int L, int q_pos0, int k, 
     }
     __syncthreads();
     cluster.sync();
-    int gt_b = 0, eq_b = 0;
     for (int c = 0; c < part; ++c) {
         const int *rc = cluster.map_shared_rank(s_counts, c);
         gt_b += rc[0];
         eq_b += rc[1];
     }
     cluster_arrive();  // done with the other CTAs' shared memory
+        }
+    }
 
     // ---- write the kept positions of this warp's segment in order
     gt_b += w_gt[warp];
@@ -389,7 +497,7 @@ topk_kernel(const float *__restrict__ scores, int Tq, int L, int q_pos0, int k, 
     cluster_wait();  // no CTA leaves while another may still read its shared memory
 }
 
-constexpr size_t kDynSmem = 8 * (size_t)kListCap + sizeof(FindScratch);
+constexpr size_t kDynSmem = 8 * (size_t)kListCap + sizeof(FindScratch) + 4 * (size_t)kGatherCap;
 
 }  // namespace
 
