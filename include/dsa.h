@@ -58,7 +58,7 @@ typedef enum {
     DSA_ERR_UNSUPPORTED = 2,  /* valid but not implemented (dtype, head width) */
     DSA_ERR_WORKSPACE = 3,    /* workspace pointer null or ws_bytes too small */
     DSA_ERR_CUDA = 4,         /* a CUDA runtime call or a kernel launch failed */
-    DSA_ERR_TIMEOUT = 5       /* reserved: a bounded device-side wait gave up */
+    DSA_ERR_TIMEOUT = 5       /* a bounded device-side wait gave up (dsa_device_error) */
 } dsa_status;
 
 typedef enum {
@@ -75,6 +75,21 @@ uint64_t dsa_kernel_launch_count(void);
 
 /* Static text for a status code (never NULL). */
 const char *dsa_status_string(dsa_status status);
+
+/*
+ * dsa_device_error -- report and clear the device-side error words of the
+ * current device. The library has no counterpart on the pages: its
+ * tensor-core kernels bound every wait on an mbarrier (2 s); a wait that
+ * gives up makes the kernel set an error word, release its resources and
+ * return without finishing its outputs, instead of hanging the GPU.
+ *   stream  cudaStream_t (as void*) that ran the calls to check; it is
+ *           synchronised first.
+ * Returns DSA_OK if no kernel recorded an error since the last call,
+ * DSA_ERR_TIMEOUT if one did (the outputs of that call are invalid), and
+ * DSA_ERR_CUDA if synchronising or reading the words failed. Blocking; not
+ * for use inside stream capture.
+ */
+dsa_status dsa_device_error(dsa_stream_t stream);
 
 /*
  * dsa_indexer_scores -- stage 1, lightning-indexer scores (first page §2.1).

@@ -15,7 +15,8 @@ from .inputs import WORKLOADS, Workload, make_inputs, to_device  # noqa: F401
 
 
 _BINDING_NAMES = ("indexer_scores", "topk", "sparse_attn", "forward", "forward_args",
-                  "forward_workspace_bytes", "attn_shape", "load_library", "DSAError")
+                  "forward_workspace_bytes", "attn_shape", "load_library", "DSAError", "device_error",
+                  "kernel_launch_count")
 
 
 def __getattr__(name):

@@ -24,7 +24,7 @@ STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED",
 # Symbols declared in include/dsa.h.
 EXPORTED = ("dsa_version", "dsa_kernel_launch_count", "dsa_status_string", "dsa_indexer_scores", "dsa_topk",
             "dsa_topk_workspace_bytes", "dsa_sparse_attn", "dsa_sparse_attn_workspace_bytes",
-            "dsa_forward", "dsa_forward_workspace_bytes")
+            "dsa_forward", "dsa_forward_workspace_bytes", "dsa_device_error")
 
 
 class DSAError(RuntimeError):
@@ -86,6 +86,7 @@ def load_library(path: str = LIB_PATH):
     lib.dsa_forward.restype = ci
     lib.dsa_forward_workspace_bytes.argtypes = [ctypes.POINTER(ForwardArgs)]
     lib.dsa_forward_workspace_bytes.restype = sz
+    lib.dsa_device_error.argtypes, lib.dsa_device_error.restype = [vp], ci
     _lib = lib
     return lib
 
@@ -93,6 +94,11 @@ def load_library(path: str = LIB_PATH):
 def kernel_launch_count() -> int:
     """Kernels libdsa has enqueued in this process so far."""
     return int(load_library().dsa_kernel_launch_count())
+
+
+def device_error(stream=None) -> None:
+    """Synchronise `stream` and raise DSAError if a kernel gave up on a bounded wait."""
+    _check(load_library().dsa_device_error(_stream(stream)), "dsa_device_error")
 
 
 def _check(status: int, what: str):

@@ -199,6 +199,13 @@ int dsa_version(void) { return 100; }
 
 uint64_t dsa_kernel_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
+dsa_status dsa_device_error(dsa_stream_t stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return DSA_ERR_CUDA;
+    unsigned int words = dsa::indexer_take_device_error() | dsa::attn_mla_tc_take_device_error();
+    if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+    return words ? DSA_ERR_TIMEOUT : DSA_OK;
+}
+
 const char *dsa_status_string(dsa_status status) {
     switch (status) {
         case DSA_OK: return "DSA_OK";

@@ -590,6 +590,9 @@ cudaError_t launch_mma(const AttnProblem &p, const DeviceInfo &info, cudaStream_
 bool attn_mla_supported(const AttnProblem &p);
 size_t attn_mla_workspace_bytes(const AttnProblem &p, int sm_count);
 cudaError_t launch_attn_mla(const AttnProblem &p, const DeviceInfo &info, cudaStream_t stream);
+bool attn_mla_tc_supported(const AttnProblem &p);
+size_t attn_mla_tc_workspace_bytes(const AttnProblem &p, int sm_count);
+cudaError_t launch_attn_mla_tc(const AttnProblem &p, const DeviceInfo &info, cudaStream_t stream);
 
 cudaError_t launch_attn_combine(const float *part_o, const float *part_ml, int n_pairs, int splits, int DV,
                                 __nv_bfloat16 *out, float *lse, cudaStream_t stream) {
@@ -608,6 +611,7 @@ cudaError_t launch_attn_combine(const float *part_o, const float *part_ml, int n
 size_t attn_tc_workspace_bytes(const AttnProblem &p) {
     DeviceInfo info;
     if (device_info(&info) != cudaSuccess) return 0;
+    if (attn_mla_tc_supported(p)) return attn_mla_tc_workspace_bytes(p, info.sm_count);
     if (attn_mla_supported(p)) return attn_mla_workspace_bytes(p, info.sm_count);
     int which;
     if (!shape_supported(p, &which)) return 0;
@@ -622,6 +626,11 @@ cudaError_t launch_attn_tc(const AttnProblem &p, cudaStream_t stream, bool *take
     DeviceInfo info;
     cudaError_t err = device_info(&info);
     if (err != cudaSuccess) return err;
+    if (attn_mla_tc_supported(p)) {
+        if (attn_tc_workspace_bytes(p) > p.ws_bytes) return cudaSuccess;
+        *taken = true;
+        return launch_attn_mla_tc(p, info, stream);
+    }
     if (attn_mla_supported(p)) {
         if (attn_tc_workspace_bytes(p) > p.ws_bytes) return cudaSuccess;
         *taken = true;

@@ -31,7 +31,6 @@
 #include <math.h>
 
 #include <cuda.h>
-#include <cudaTypedefs.h>
 
 #include "common.cuh"
 #include "internal.h"
@@ -295,40 +294,13 @@ __global__ void fill_beyond_tiles_kernel(float *__restrict__ scores, int Tq, int
     for (int s = start + threadIdx.x; s < L; s += blockDim.x) out[s] = -INFINITY;
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (fn == nullptr) {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult qres;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qres) == cudaSuccess &&
-            qres == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    }
-    return fn;
-}
-
-// Row-major bf16 matrix [rows, cols] read as boxes of box_rows x 64 columns
-// with the 128-byte swizzle.
-bool make_map_bf16(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
-    auto encode = get_encode_fn();
-    if (!encode) return false;
-    const cuuint64_t dims[2] = {cols, rows};
-    const cuuint64_t strides[1] = {cols * 2};
-    const cuuint32_t box[2] = {64, box_rows};
-    const cuuint32_t estr[2] = {1, 1};
-    CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
-                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
 template <int D, int N_TILE>
 cudaError_t launch_tc(const IndexerProblem &pr, const DeviceInfo &info, cudaStream_t stream) {
     using C = Cfg<D, N_TILE>;
     if ((size_t)info.max_smem_optin < C::kSmem) return cudaErrorInvalidValue;
     CUtensorMap tm_q, tm_k;
-    if (!make_map_bf16(&tm_q, pr.q_idx, (uint64_t)pr.B * pr.Tq * pr.H, (uint64_t)D, N_TILE) ||
-        !make_map_bf16(&tm_k, pr.k_idx, (uint64_t)pr.B * pr.L, (uint64_t)D, kBlockM))
+    if (!make_map_bf16_sw128(&tm_q, pr.q_idx, (uint64_t)pr.B * pr.Tq * pr.H, (uint64_t)D, (uint64_t)D * 2, N_TILE) ||
+        !make_map_bf16_sw128(&tm_k, pr.k_idx, (uint64_t)pr.B * pr.L, (uint64_t)D, (uint64_t)D * 2, kBlockM))
         return cudaErrorInvalidValue;
 
     Params p;

@@ -1,6 +1,7 @@
 // Host-side launch interface between the C ABI (api.cu) and the kernels.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -20,6 +21,12 @@ cudaError_t device_info(DeviceInfo *out);
 
 // Process-wide count of kernels this library has enqueued (diagnostics).
 void count_launch(int n = 1);
+
+// TMA tensor map over a row-major bf16 matrix [rows, cols] whose rows are
+// pitch_bytes apart (a multiple of 16), read as boxes of box_rows x 64
+// columns (128 bytes) with the 128-byte swizzle. False if the driver rejects it.
+bool make_map_bf16_sw128(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint64_t pitch_bytes,
+                         uint32_t box_rows);
 
 // ----------------------------------------------------------------- indexer
 struct IndexerProblem {
@@ -61,5 +68,10 @@ struct AttnProblem {
 };
 size_t attn_workspace_bytes(const AttnProblem &p);
 cudaError_t launch_attn(const AttnProblem &p, cudaStream_t stream);
+
+// Read and clear the error word of a kernel family with bounded waits
+// (non-zero: some launch gave up on a wait).
+unsigned int indexer_take_device_error();
+unsigned int attn_mla_tc_take_device_error();
 
 }  // namespace dsa

@@ -15,6 +15,8 @@ import oracle
 # bf16/fp32 outputs against the fp64 oracle.
 ATOL = 2e-2
 RTOL = 1e-2
+# log-sum-exp: fp32 logits of bf16 inputs against fp64
+LSE_ATOL = 2e-3
 
 
 def bits(t: torch.Tensor) -> np.ndarray:
@@ -39,8 +41,11 @@ def cache_strides(t: torch.Tensor):
     return t.stride(0), t.stride(1), t.stride(2)
 
 
-def oracle_forward(wl, inp, flat_rows, nthreads=0, idx_override=None):
-    """Run the oracle on the given rows of a make_inputs() dict (CPU tensors)."""
+def oracle_forward(wl, inp, flat_rows, nthreads=0, idx_override=None, want_lse=False):
+    """Run the oracle on the given rows of a make_inputs() dict (CPU tensors).
+
+    Returns (scores, idx, out), plus the log-sum-exp per (row, head) when
+    want_lse is set."""
     row_b, row_i, row_t = rows_of(wl, flat_rows)
     q_idx = inp["q_idx"][row_b, row_i]
     w = inp["w"][row_b, row_i]
@@ -61,9 +66,11 @@ def oracle_forward(wl, inp, flat_rows, nthreads=0, idx_override=None):
         vs = ks
     else:
         vs = (vc.shape[1] * vc.shape[2] * vc.shape[3], vc.shape[2] * vc.shape[3], vc.shape[3])
-    out = oracle.attn_rows(bits(q), kbuf, vbuf, idx, row_b, wl.scale, k_strides=ks, v_strides=vs,
-                           Hkv=wl.Hkv, Dv=wl.Dv, nthreads=nthreads)
-    return scores, idx, out
+    res = oracle.attn_rows(bits(q), kbuf, vbuf, idx, row_b, wl.scale, k_strides=ks, v_strides=vs,
+                           Hkv=wl.Hkv, Dv=wl.Dv, nthreads=nthreads, want_lse=want_lse)
+    if want_lse:
+        return (scores, idx) + tuple(res)
+    return scores, idx, res
 
 
 def assert_attn_close(got: np.ndarray, ref: np.ndarray, what: str = ""):

@@ -14,7 +14,7 @@ import oracle
 from learned_sparse_attention_dsa_b200 import binding
 from learned_sparse_attention_dsa_b200.inputs import (WORKLOADS, Workload, make_inputs,
                                                       random_score_rows, to_device)
-from parity_helpers import assert_attn_close, bits, oracle_forward, rows_of
+from parity_helpers import LSE_ATOL, assert_attn_close, bits, oracle_forward, rows_of
 
 pytestmark = pytest.mark.gpu
 
@@ -30,6 +30,16 @@ MEDIUM = {
     "decode_latent_3000": Workload("decode_latent_3000", B=2, Tq=1, L=3000, q_pos0=2999, H_I=64,
                                    d_I=128, k=256, Hq=128, Hkv=1, Dqk=576, Dv=512, kv_alias=True,
                                    seed=15),
+    # latent rows with t+1 < k: -1 padding, partly and fully masked tiles
+    "latent_short": Workload("latent_short", B=2, Tq=1, L=150, q_pos0=149, H_I=64, d_I=128, k=256,
+                             Hq=128, Hkv=1, Dqk=576, Dv=512, kv_alias=True, seed=20),
+    # latent rows, many query rows (no split of S_t), k not a multiple of the tile
+    "latent_chunk": Workload("latent_chunk", B=1, Tq=80, L=400, q_pos0=320, H_I=64, d_I=128, k=100,
+                             Hq=128, Hkv=1, Dqk=576, Dv=512, kv_alias=True, seed=21),
+    # one latent row decoding over 2048 selected positions: 32 splits merged by
+    # the split-k combine kernel
+    "latent_single": Workload("latent_single", B=1, Tq=1, L=3000, q_pos0=2999, H_I=64, d_I=128, k=2048,
+                              Hq=128, Hkv=1, Dqk=576, Dv=512, kv_alias=True, seed=22),
     "short_context": Workload("short_context", B=2, Tq=40, L=40, q_pos0=0, H_I=64, d_I=128, k=64,
                               Hq=8, Hkv=8, Dqk=64, Dv=64, seed=16),
     "odd_heads": Workload("odd_heads", B=1, Tq=300, L=300, q_pos0=0, H_I=32, d_I=64, k=50, Hq=4,
@@ -65,7 +75,7 @@ def _gpu_forward(wl, dev):
     scores = torch.empty((wl.B, wl.Tq, wl.L), dtype=torch.float32, device="cuda")
     binding.forward(dev["q_idx"], dev["k_idx"], dev["w"], dev["q"], dev["k_cache"], dev["v_cache"],
                     wl.k, wl.q_pos0, wl.scale, out=out, idx_out=idx, scores_out=scores)
-    torch.cuda.synchronize()
+    binding.device_error()  # synchronises; raises if a kernel gave up on a bounded wait
     return scores, idx, out
 
 
@@ -136,8 +146,8 @@ def test_topk_stage(cuda, kind, L, Tq, q_pos0, k):
     assert np.array_equal(got, ref)
 
 
-@pytest.mark.parametrize("name", ["prefill_mqa_700", "decode_latent_3000", "prefill_perhead_520",
-                                  "tiny_f32"])
+@pytest.mark.parametrize("name", ["prefill_mqa_700", "decode_latent_3000", "latent_chunk",
+                                  "latent_single", "prefill_perhead_520", "tiny_f32"])
 def test_sparse_attn_stage_shuffled_and_padded(cuda, name):
     """Attention on its own, with the oracle's index sets shuffled and padded."""
     wl = MEDIUM[name]
@@ -148,12 +158,15 @@ def test_sparse_attn_stage_shuffled_and_padded(cuda, name):
     idx = o_idx.copy()
     for r in range(idx.shape[0]):
         rng.shuffle(idx[r])
-    _, _, ref = oracle_forward(wl, cpu, flat, idx_override=idx)
+    _, _, ref, ref_lse = oracle_forward(wl, cpu, flat, idx_override=idx, want_lse=True)
     idx_t = torch.from_numpy(idx).reshape(wl.B, wl.Tq, wl.k).cuda()
     out, lse = binding.sparse_attn(dev["q"], dev["k_cache"], dev["v_cache"], idx_t, wl.scale,
                                    want_lse=True)
+    binding.device_error()
     assert_attn_close(out.float().cpu().numpy().reshape(-1, wl.Hq, wl.Dv), ref, name)
-    assert torch.isfinite(lse).all()
+    got_lse = lse.cpu().numpy().reshape(-1, wl.Hq).astype(np.float64)
+    assert np.all(np.isfinite(got_lse))
+    assert np.max(np.abs(got_lse - ref_lse)) <= LSE_ATOL, f"{name}: lse differs"
 
 
 def test_sparse_attn_all_padding_row(cuda):

@@ -71,16 +71,16 @@ def test_noalloc_matches_workspace_entry_point_twice(cuda, dsa_lib):
 
 def test_noalloc_rejects_problems_beyond_its_scratch(cuda, dsa_lib):
     _declare(dsa_lib)
-    # 8 sequences x 128 heads over a 576-wide latent row, the selection split
-    # four ways: 8*128*4*(512+2)*4 bytes of partials > 4 MiB
-    B, L, k, Hq = 8, 2048, 2048, 128
-    q = torch.zeros((B, 1, Hq, 576), dtype=torch.bfloat16, device="cuda")
-    kc = torch.zeros((B, L, 1, 576), dtype=torch.bfloat16, device="cuda")
-    vc = kc[..., :512]
+    # 16 sequences x 16 heads selecting 65,536 positions: the selection is
+    # split 32 ways, 16*16*32*(128+2)*4 bytes of partials > 4 MiB
+    B, L, k, Hq, D = 16, 65536, 65536, 16, 128
+    q = torch.zeros((B, 1, Hq, D), dtype=torch.bfloat16, device="cuda")
+    kc = torch.zeros((B, L, 1, D), dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros((B, L, 1, D), dtype=torch.bfloat16, device="cuda")
     idx = torch.zeros((B, 1, k), dtype=torch.int32, device="cuda")
-    out = torch.empty((B, 1, Hq, 512), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty((B, 1, Hq, D), dtype=torch.bfloat16, device="cuda")
     lse = torch.empty((B, 1, Hq), dtype=torch.float32, device="cuda")
-    sh = binding.attn_shape(q, kc, vc, k, 576 ** -0.5)
+    sh = binding.attn_shape(q, kc, vc, k, D ** -0.5)
     need = dsa_lib.dsa_sparse_attn_workspace_bytes(ctypes.byref(sh), binding._dt(q))
     assert need > dsa_lib.dsa_sparse_attn_noalloc_max_scratch_bytes()
     assert _noalloc(dsa_lib, q, kc, vc, idx, sh, out, lse) == DSA_ERR_WORKSPACE
