@@ -3,15 +3,16 @@
  * NVIDIA B200 (sm_100a). Library: libdsa.so.
  *
  * The path, as defined on "DeepSeek Sparse Attention: Learned Token Selection
- * from Scratch" (first page) and "DeepSeek NSA and DSA" §3.2:
+ * from Scratch" (cited below as "Learned Token Selection") and "DeepSeek NSA
+ * and DSA" §3.2:
  *
  *   1. lightning-indexer scores   I[t,s] = sum_j w[t,j] * ReLU(q^I[t,j] . k^I[s])
- *      (first page §2.1, boxed equation), for candidates s <= t;
+ *      ("Learned Token Selection" §2.1, boxed equation), for candidates s <= t;
  *   2. top-k selection            S_t = positions of the k largest I[t,s]
- *      (first page §3.1, boxed equation);
+ *      ("Learned Token Selection" §3.1, boxed equation);
  *   3. attention over S_t         u[t,h] = sum_{s in S_t} softmax_s(q[t,h].k[s]*scale) v[s]
- *      (first page §3.3 and §10.1), one S_t shared by every query head
- *      (first page §4.1-4.2: the MQA mode of MLA).
+ *      ("Learned Token Selection" §3.3 and §10.1), one S_t shared by every query head
+ *      ("Learned Token Selection" §4.1-4.2: the MQA mode of MLA).
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -21,7 +22,7 @@
  * - Candidates of row t are positions 0..t (the page's running example says
  *   "preceding tokens ... (plus itself)").
  * - Equal scores are ordered by position, lower position first. When t+1 <= k,
- *   every candidate is selected (first page §7.6 note: DSA collapses to full
+ *   every candidate is selected ("Learned Token Selection" §7.6 note: DSA collapses to full
  *   attention when the context is shorter than the budget).
  * - Selected positions are written in ascending order, followed by -1 padding
  *   up to k entries.
@@ -92,7 +93,7 @@ const char *dsa_status_string(dsa_status status);
 dsa_status dsa_device_error(dsa_stream_t stream);
 
 /*
- * dsa_indexer_scores -- stage 1, lightning-indexer scores (first page §2.1).
+ * dsa_indexer_scores -- stage 1, lightning-indexer scores ("Learned Token Selection" §2.1).
  *
  *   scores[b,i,s] = sum_{j<H_I} w[b,i,j] * max(0, sum_{e<d_I} q_idx[b,i,j,e] * k_idx[b,s,e])
  *                   for s <= q_pos0 + i,   and -inf for s > q_pos0 + i.
@@ -114,7 +115,7 @@ dsa_status dsa_indexer_scores(const void *q_idx, const void *k_idx, const float 
                               dsa_dtype dt, float *scores, dsa_stream_t stream);
 
 /*
- * dsa_topk -- stage 2, per-row top-k selection (first page §3.1).
+ * dsa_topk -- stage 2, per-row top-k selection ("Learned Token Selection" §3.1).
  *
  * For each row (b, i), t = q_pos0 + i, reads scores[b,i,0..t] and writes the
  * positions of the k largest values to idx[b,i,:] in ascending order, then -1
@@ -146,8 +147,9 @@ typedef struct dsa_attn_shape {
 } dsa_attn_shape;
 
 /*
- * dsa_sparse_attn -- stage 3, attention over the selected rows (first page
- * §3.3, §10.1; one selection shared by all heads, §4.1-4.2).
+ * dsa_sparse_attn -- stage 3, attention over the selected rows
+ * ("Learned Token Selection" §3.3, §10.1; one selection shared by all heads,
+ * §4.1-4.2).
  *
  *   out[b,i,h,:] = sum_{s in S} softmax_s(scale * q[b,i,h,:] . K[b,s,g,:]) * V[b,s,g,:]
  *   with g = h / (Hq / Hkv) and S = { idx[b,i,j] : idx[b,i,j] >= 0 }.

@@ -16,13 +16,16 @@ bf16 bit patterns for bf16 data. Every function takes the rows to evaluate as
 sample of query rows.
 
 Parity status per function (what pins it, independently of this code):
-  indexer_rows : hand-traced t=10 example (first page §2.3-2.5), ReLU(q.k)
+  indexer_rows : hand-traced t=10 example ("Learned Token Selection" §2.3-2.5), ReLU(q.k)
                  against numpy matmul for H=1, exact integer arithmetic.
-  topk_rows    : the page's S_10 = {3, 8, 9} and rank order (first page §3.2),
+  topk_rows    : the page's S_10 = {3, 8, 9} and rank order ("Learned Token Selection" §3.2),
                  Python's sort on tiny rows, the closed-form count of
-                 selected entries (first page §7.2-7.3).
+                 selected entries ("Learned Token Selection" §7.2-7.3);
+                 with include_self (§3.4): S_10 = {3, 9, 10} from the
+                 page's trace, t always kept, the rest equal to Python's
+                 sort of positions 0..t-1.
   attn_rows    : torch's dense causal scaled_dot_product_attention when the
-                 budget covers every candidate (first page §7.6 note, §9.3),
+                 budget covers every candidate ("Learned Token Selection" §7.6 note, §9.3),
                  |S|=1 and equal-score special cases, permutation invariance.
 """
 from __future__ import annotations
@@ -71,6 +74,8 @@ def _load():
     lib.oracle_indexer_rows.restype = None
     lib.oracle_topk_rows.argtypes = [ci, i32p, f32p, ci, ci, i32p, ci]
     lib.oracle_topk_rows.restype = None
+    lib.oracle_topk_self_rows.argtypes = [ci, i32p, f32p, ci, ci, i32p, ci]
+    lib.oracle_topk_self_rows.restype = None
     lib.oracle_attn_rows.argtypes = [ci, i32p, vp, vp, vp, ci,
                                      i64, i64, i64, i64, i64, i64,
                                      i32p, ci, ci, ci, ci, ci, ctypes.c_double,
@@ -107,7 +112,7 @@ def _rows(row_b, row_t):
 
 
 def indexer_rows(q_rows, w_rows, k_cache, row_b, row_t, nthreads: int = 0):
-    """I[t, s] for each requested row (first page §2.1).
+    """I[t, s] for each requested row ("Learned Token Selection" §2.1).
 
     q_rows [n, H, d], w_rows [n, H] float32, k_cache [B, L, d].
     Returns float32 [n, L] with -inf at s > t.
@@ -134,10 +139,12 @@ def indexer_rows(q_rows, w_rows, k_cache, row_b, row_t, nthreads: int = 0):
     return out
 
 
-def topk_rows(scores, row_t, k: int, nthreads: int = 0):
-    """S_t for each row (first page §3.1): ascending positions, -1 padded.
+def topk_rows(scores, row_t, k: int, nthreads: int = 0, include_self: bool = False):
+    """S_t for each row ("Learned Token Selection" §3.1): ascending positions, -1 padded.
 
-    scores [n, L] float32; only entries 0..row_t[r] are read.
+    scores [n, L] float32; only entries 0..row_t[r] are read. With
+    include_self, S_t = {t} plus the k-1 best of positions 0..t-1 (§3.4:
+    the current token is always included).
     """
     lib = _load()
     scores = np.ascontiguousarray(scores, dtype=np.float32)
@@ -146,15 +153,15 @@ def topk_rows(scores, row_t, k: int, nthreads: int = 0):
     if row_t.shape != (n,) or k < 1 or (n and (row_t.min() < 0 or row_t.max() >= L)):
         raise ValueError("topk_rows: bad arguments")
     idx = np.empty((n, k), dtype=np.int32)
-    lib.oracle_topk_rows(n, _ptr(row_t, ctypes.c_int32), _ptr(scores, ctypes.c_float),
-                         L, k, _ptr(idx, ctypes.c_int32), nthreads)
+    fn = lib.oracle_topk_self_rows if include_self else lib.oracle_topk_rows
+    fn(n, _ptr(row_t, ctypes.c_int32), _ptr(scores, ctypes.c_float), L, k, _ptr(idx, ctypes.c_int32), nthreads)
     return idx
 
 
 def attn_rows(q_rows, k_cache, v_cache, idx, row_b, scale: float,
               k_strides=None, v_strides=None, Hkv: int | None = None,
               Dv: int | None = None, nthreads: int = 0, want_lse: bool = False):
-    """u[t, h] for each row (first page §3.3, §10.1), fp64.
+    """u[t, h] for each row ("Learned Token Selection" §3.3, §10.1), fp64.
 
     q_rows [n, Hq, Dqk]. k_cache / v_cache are either 4-D [B, L, Hkv, D]
     contiguous arrays, or flat buffers with explicit element strides
@@ -198,13 +205,13 @@ def attn_rows(q_rows, k_cache, v_cache, idx, row_b, scale: float,
 
 def forward_rows(q_idx_rows, w_rows, k_idx_cache, q_rows, k_cache, v_cache,
                  row_b, row_t, k: int, scale: float, k_strides=None, v_strides=None,
-                 Hkv=None, Dv=None, nthreads: int = 0):
+                 Hkv=None, Dv=None, nthreads: int = 0, include_self: bool = False):
     """The three stages back to back for the requested rows.
 
     Returns (scores [n, L] float32, idx [n, k] int32, out [n, Hq, Dv] fp64).
     """
     scores = indexer_rows(q_idx_rows, w_rows, k_idx_cache, row_b, row_t, nthreads)
-    idx = topk_rows(scores, row_t, k, nthreads)
+    idx = topk_rows(scores, row_t, k, nthreads, include_self)
     out = attn_rows(q_rows, k_cache, v_cache, idx, row_b, scale, k_strides, v_strides,
                     Hkv, Dv, nthreads)
     return scores, idx, out

@@ -14,6 +14,7 @@
  *   "DeepSeek Sparse Attention: Learned Token Selection from Scratch"
  *     §2.1, boxed equation for I_{t,s}     -> oracle_indexer_rows
  *     §3.1, boxed equation for S_t         -> oracle_topk_rows
+ *     §3.4, always including the current token -> oracle_topk_self_rows
  *     §3.3, equations for alpha and u_t;
  *     §10.1, the common attention form     -> oracle_attn_rows
  *     §4.1-4.2, one selected set shared by every head (MQA mode of MLA)
@@ -35,7 +36,7 @@
  *   - positions s > t are written as -inf in the score rows.
  *
  * Parity pins: the fp64 results are checked, independently of this file,
- * against the hand-traced t=10 example of the first page, brute-force
+ * against the hand-traced t=10 example of "Learned Token Selection", brute-force
  * sorting, closed-form counts and library dense attention (see tests/).
  */
 #include <math.h>
@@ -81,7 +82,7 @@ int oracle_max_threads(void)
 }
 
 /*
- * Lightning-indexer scores, first page §2.1:
+ * Lightning-indexer scores, "Learned Token Selection" §2.1:
  *   I[t,s] = sum_{j=1..H} w[t,j] * ReLU( q[t,j] . k[s] )
  * for s = 0..t; s > t is not a candidate and is written as -inf.
  *
@@ -154,7 +155,7 @@ static int ascending_int(const void *pa, const void *pb)
 }
 
 /*
- * Top-k selection, first page §3.1: S_t holds the positions of the k largest
+ * Top-k selection, "Learned Token Selection" §3.1: S_t holds the positions of the k largest
  * I[t,s] over the candidates s = 0..t. Brute force: sort every candidate by
  * (descending score, ascending position) and keep the first min(t+1, k).
  *   scores: [nrows, L] fp32 (only entries 0..row_t[r] are read)
@@ -183,10 +184,44 @@ void oracle_topk_rows(int nrows, const int32_t *row_t, const float *scores,
 }
 
 /*
- * Attention restricted to the selected set, first page §3.3 and §10.1:
+ * Top-k selection that always keeps the query's own position
+ * ("Learned Token Selection" §3.4: a token whose own score does not reach
+ * the top k is kept by always including the current token):
+ *
+ *   S_t = {t} united with the min(t, k-1) highest-scoring positions of 0..t-1
+ *
+ * with the same order and tie rule as oracle_topk_rows. When t+1 <= k this is
+ * every candidate, as without the rule.
+ */
+void oracle_topk_self_rows(int nrows, const int32_t *row_t, const float *scores,
+                           int L, int k, int32_t *idx, int nthreads)
+{
+    set_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int r = 0; r < nrows; ++r) {
+        const int t = row_t[r];
+        /* the candidates other than t itself */
+        candidate *c = (candidate *)malloc(sizeof(candidate) * (size_t)(t > 0 ? t : 1));
+        for (int s = 0; s < t; ++s) {
+            c[s].score = scores[(size_t)r * L + s];
+            c[s].pos = s;
+        }
+        qsort(c, (size_t)t, sizeof(candidate), by_score_then_pos);
+        const int others = t < k - 1 ? t : k - 1;
+        int32_t *out = idx + (size_t)r * k;
+        for (int j = 0; j < others; ++j) out[j] = c[j].pos;
+        out[others] = t;
+        qsort(out, (size_t)others + 1, sizeof(int32_t), ascending_int);
+        for (int j = others + 1; j < k; ++j) out[j] = -1;
+        free(c);
+    }
+}
+
+/*
+ * Attention restricted to the selected set, "Learned Token Selection" §3.3 and §10.1:
  *   alpha[t,h,s] = exp(q[t,h].k[s,g]*scale) / sum_{s' in S_t} exp(q[t,h].k[s',g]*scale)
  *   u[t,h]       = sum_{s in S_t} alpha[t,h,s] * v[s,g]
- * Every query head h uses the same S_t (first page §4.1-4.2); head h reads
+ * Every query head h uses the same S_t ("Learned Token Selection" §4.1-4.2); head h reads
  * KV head g = h / (Hq / Hkv). idx entries of -1 are padding and skipped.
  * The max is subtracted before exp (the result is unchanged).
  *   q_rows : [nrows, Hq, Dqk] (dtype)

@@ -41,7 +41,7 @@ def cache_strides(t: torch.Tensor):
     return t.stride(0), t.stride(1), t.stride(2)
 
 
-def oracle_forward(wl, inp, flat_rows, nthreads=0, idx_override=None, want_lse=False):
+def oracle_forward(wl, inp, flat_rows, nthreads=0, idx_override=None, want_lse=False, include_self=False):
     """Run the oracle on the given rows of a make_inputs() dict (CPU tensors).
 
     Returns (scores, idx, out), plus the log-sum-exp per (row, head) when
@@ -51,7 +51,7 @@ def oracle_forward(wl, inp, flat_rows, nthreads=0, idx_override=None, want_lse=F
     w = inp["w"][row_b, row_i]
     q = inp["q"][row_b, row_i]
     scores = oracle.indexer_rows(bits(q_idx), w.numpy(), bits(inp["k_idx"]), row_b, row_t, nthreads)
-    idx = oracle.topk_rows(scores, row_t, wl.k, nthreads) if idx_override is None else idx_override
+    idx = oracle.topk_rows(scores, row_t, wl.k, nthreads, include_self) if idx_override is None else idx_override
     kc = inp["k_cache"]
     vc = inp["v_cache"]
     kbuf = bits(kc)

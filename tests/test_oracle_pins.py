@@ -353,3 +353,45 @@ def test_forward_rows_subset_equals_full():
         assert np.array_equal(a[rows], b)
     # count invariant on the worked-example workload itself (§7.3: 45)
     assert int((full[1] >= 0).sum()) == 45
+
+
+# ---------------------------------------------------------------- top-k, current token always kept
+
+def test_trace_include_self_keeps_token_10():
+    """§3.4: token 10 misses the top 3 of its own row (I_10 = 0 with
+    k^I_10 = [-1, -1]); keeping the current token gives {3, 9, 10}: 10 plus
+    the two best of positions 0..9 (2.9 at 3, 2.2 at 9 in §2.5)."""
+    row, t = _scores(extra_key=[-1.0, -1.0])
+    assert t == 10
+    plain = oracle.topk_rows(row[None], [t], 3)[0].tolist()
+    kept = oracle.topk_rows(row[None], [t], 3, include_self=True)[0].tolist()
+    assert plain == [3, 8, 9]
+    assert kept == [3, 9, 10]
+
+
+def _brute_topk_self(row, t, k):
+    if t + 1 <= k:
+        return list(range(t + 1)) + [-1] * (k - t - 1)
+    order = sorted(range(t), key=lambda s: (-float(row[s]), s))
+    sel = sorted(order[: k - 1] + [t])
+    return sel + [-1] * (k - len(sel))
+
+
+@pytest.mark.parametrize("kind", ["int", "equal", "normal", "neg", "mixed"])
+def test_topk_include_self_brute_force(kind):
+    from learned_sparse_attention_dsa_b200.inputs import random_score_rows
+    gen = torch.Generator().manual_seed(11)
+    L = 41
+    rows = random_score_rows(gen, 60, L, kind).numpy()
+    rng = np.random.default_rng(5)
+    row_t = rng.integers(0, L, size=60).astype(np.int32)
+    row_t[:3] = [0, 1, L - 1]
+    for k in (1, 2, 5, 17, 40, 64):
+        got = oracle.topk_rows(rows, row_t, k, include_self=True)
+        plain = oracle.topk_rows(rows, row_t, k)
+        for r in range(60):
+            t = int(row_t[r])
+            assert got[r].tolist() == _brute_topk_self(rows[r], t, k), (kind, k, r)
+            assert t in got[r].tolist()
+            if t in plain[r].tolist():  # already selected: the rule changes nothing
+                assert got[r].tolist() == plain[r].tolist()
