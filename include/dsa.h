@@ -131,6 +131,20 @@ dsa_status dsa_indexer_scores(const void *q_idx, const void *k_idx, const float 
 dsa_status dsa_topk(const float *scores, int B, int Tq, int L, int q_pos0, int k,
                     int32_t *idx, void *ws, size_t ws_bytes, dsa_stream_t stream);
 
+/* Selection options (dsa_topk_ex flags, dsa_forward_args.flags). */
+typedef enum {
+    /* Keep the query's own position: S_t = {t} and the min(t, k-1) best of
+     * positions 0..t-1, same order and tie rule ("Learned Token Selection"
+     * §3.4: a token that misses its own top k is kept by always including
+     * the current token). Without it S_t is the plain top k of 0..t. */
+    DSA_FLAG_INCLUDE_SELF = 1
+} dsa_flags;
+
+/* dsa_topk with options: flags is 0 or DSA_FLAG_INCLUDE_SELF; any other bit
+ * gives DSA_ERR_INVALID_ARG. Otherwise as dsa_topk (same workspace). */
+dsa_status dsa_topk_ex(const float *scores, int B, int Tq, int L, int q_pos0, int k, unsigned flags,
+                       int32_t *idx, void *ws, size_t ws_bytes, dsa_stream_t stream);
+
 size_t dsa_topk_workspace_bytes(int B, int Tq, int L, int q_pos0, int k);
 
 /* Shape of the attention stage. */
@@ -223,12 +237,21 @@ typedef struct dsa_forward_args {
     int32_t *idx_out;         /* [B, Tq, k] or NULL: the selected positions */
     float *scores_out;        /* [B, Tq, L] or NULL: the indexer scores (then
                                  filled with -inf above the diagonal) */
+    unsigned flags;           /* 0 or DSA_FLAG_INCLUDE_SELF */
 } dsa_forward_args;
 
 /*
  * dsa_forward -- stages 1-3 back to back on one stream.
  * Scores and indices go to caller memory when scores_out / idx_out are set,
- * otherwise to the workspace. Results equal those of the three stage calls.
+ * otherwise to the workspace. Results equal those of the three stage calls
+ * (dsa_topk_ex with a->flags).
+ * Short context: when every query row has t + 1 <= k (q_pos0 + Tq <= k), the
+ * selection is all of 0..t by definition, so the top-k is skipped and the
+ * dense selections are written directly; the indexer runs only if
+ * scores_out asks for its scores. The attention then covers every causal
+ * position ("Learned Token Selection" §9.3: short sequences use plain masked
+ * attention). The outputs are the same as those of the full path.
+ * a->flags: 0 or DSA_FLAG_INCLUDE_SELF (anything else: DSA_ERR_INVALID_ARG).
  * ws: at least dsa_forward_workspace_bytes(a) bytes.
  */
 dsa_status dsa_forward(const dsa_forward_args *a, void *ws, size_t ws_bytes,

@@ -17,6 +17,7 @@ LIB_PATH = os.path.join(_PKG, "libdsa.so")
 
 DSA_F32 = 0
 DSA_BF16 = 1
+DSA_FLAG_INCLUDE_SELF = 1
 
 STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED",
                 3: "DSA_ERR_WORKSPACE", 4: "DSA_ERR_CUDA", 5: "DSA_ERR_TIMEOUT"}
@@ -24,7 +25,7 @@ STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED",
 # Symbols declared in include/dsa.h.
 EXPORTED = ("dsa_version", "dsa_kernel_launch_count", "dsa_status_string", "dsa_indexer_scores", "dsa_topk",
             "dsa_topk_workspace_bytes", "dsa_sparse_attn", "dsa_sparse_attn_workspace_bytes",
-            "dsa_forward", "dsa_forward_workspace_bytes", "dsa_device_error")
+            "dsa_forward", "dsa_forward_workspace_bytes", "dsa_device_error", "dsa_topk_ex")
 
 
 class DSAError(RuntimeError):
@@ -53,7 +54,7 @@ class ForwardArgs(ctypes.Structure):
                 ("v_stride_b", ctypes.c_int64), ("v_stride_s", ctypes.c_int64), ("v_stride_h", ctypes.c_int64),
                 ("attn_dtype", ctypes.c_int),
                 ("out", ctypes.c_void_p), ("lse", ctypes.c_void_p), ("idx_out", ctypes.c_void_p),
-                ("scores_out", ctypes.c_void_p)]
+                ("scores_out", ctypes.c_void_p), ("flags", ctypes.c_uint)]
 
 
 _lib = None
@@ -76,6 +77,8 @@ def load_library(path: str = LIB_PATH):
     lib.dsa_indexer_scores.restype = ci
     lib.dsa_topk.argtypes = [vp, ci, ci, ci, ci, ci, vp, vp, sz, vp]
     lib.dsa_topk.restype = ci
+    lib.dsa_topk_ex.argtypes = [vp, ci, ci, ci, ci, ci, ctypes.c_uint, vp, vp, sz, vp]
+    lib.dsa_topk_ex.restype = ci
     lib.dsa_topk_workspace_bytes.argtypes = [ci, ci, ci, ci, ci]
     lib.dsa_topk_workspace_bytes.restype = sz
     lib.dsa_sparse_attn.argtypes = [vp, vp, vp, vp, ctypes.POINTER(AttnShape), ci, vp, vp, vp, sz, vp]
@@ -160,8 +163,9 @@ def indexer_scores(q_idx, k_idx, w, q_pos0: int = 0, scores=None, stream=None):
     return scores
 
 
-def topk(scores, k: int, q_pos0: int = 0, idx=None, ws=None, stream=None):
-    """dsa_topk: int32 [B, Tq, k], ascending positions then -1."""
+def topk(scores, k: int, q_pos0: int = 0, idx=None, ws=None, stream=None, include_self: bool = False):
+    """dsa_topk_ex: int32 [B, Tq, k], ascending positions then -1 (with
+    include_self, S_t always holds t)."""
     lib = load_library()
     _need_cuda(scores, idx)
     B, Tq, L = scores.shape
@@ -169,8 +173,9 @@ def topk(scores, k: int, q_pos0: int = 0, idx=None, ws=None, stream=None):
         idx = torch.empty((B, Tq, k), dtype=torch.int32, device=scores.device)
     nbytes = lib.dsa_topk_workspace_bytes(B, Tq, L, q_pos0, k)
     ws = _workspace(nbytes, scores.device, ws)
-    st = lib.dsa_topk(_p(scores), B, Tq, L, q_pos0, k, _p(idx), _p(ws), nbytes, _stream(stream))
-    _check(st, "dsa_topk")
+    flags = DSA_FLAG_INCLUDE_SELF if include_self else 0
+    st = lib.dsa_topk_ex(_p(scores), B, Tq, L, q_pos0, k, flags, _p(idx), _p(ws), nbytes, _stream(stream))
+    _check(st, "dsa_topk_ex")
     return idx
 
 
@@ -202,7 +207,7 @@ def sparse_attn(q, k_cache, v_cache, idx, scale=None, out=None, lse=None, want_l
 
 
 def forward_args(q_idx, k_idx, w, q, k_cache, v_cache, k: int, q_pos0: int = 0, scale=None,
-                 out=None, lse=None, idx_out=None, scores_out=None) -> ForwardArgs:
+                 out=None, lse=None, idx_out=None, scores_out=None, include_self: bool = False) -> ForwardArgs:
     B, Tq, H, d = q_idx.shape
     sh = attn_shape(q, k_cache, v_cache, k, scale)
     return ForwardArgs(B, Tq, k_idx.shape[1], q_pos0, k,
@@ -214,7 +219,8 @@ def forward_args(q_idx, k_idx, w, q, k_cache, v_cache, k: int, q_pos0: int = 0, 
                        out.data_ptr() if out is not None else None,
                        lse.data_ptr() if lse is not None else None,
                        idx_out.data_ptr() if idx_out is not None else None,
-                       scores_out.data_ptr() if scores_out is not None else None)
+                       scores_out.data_ptr() if scores_out is not None else None,
+                       DSA_FLAG_INCLUDE_SELF if include_self else 0)
 
 
 def forward_workspace_bytes(args: ForwardArgs) -> int:
@@ -222,7 +228,8 @@ def forward_workspace_bytes(args: ForwardArgs) -> int:
 
 
 def forward(q_idx, k_idx, w, q, k_cache, v_cache, k: int, q_pos0: int = 0, scale=None,
-            out=None, lse=None, idx_out=None, scores_out=None, ws=None, stream=None):
+            out=None, lse=None, idx_out=None, scores_out=None, ws=None, stream=None,
+            include_self: bool = False):
     """dsa_forward: all three stages; returns out (and fills lse/idx_out/scores_out if given)."""
     lib = load_library()
     _need_cuda(q_idx, k_idx, w, q, k_cache, v_cache, out, lse, idx_out, scores_out)
@@ -230,7 +237,7 @@ def forward(q_idx, k_idx, w, q, k_cache, v_cache, k: int, q_pos0: int = 0, scale
         out = torch.empty((q.shape[0], q.shape[1], q.shape[2], v_cache.shape[3]), dtype=q.dtype,
                           device=q.device)
     args = forward_args(q_idx, k_idx, w, q, k_cache, v_cache, k, q_pos0, scale, out, lse, idx_out,
-                        scores_out)
+                        scores_out, include_self)
     nbytes = lib.dsa_forward_workspace_bytes(ctypes.byref(args))
     ws = _workspace(nbytes, q.device, ws)
     st = lib.dsa_forward(ctypes.byref(args), _p(ws), nbytes, _stream(stream))

@@ -182,6 +182,7 @@ dsa_status check_forward(const dsa_forward_args *a) {
                                   a->idx_dtype, a->scores_out ? a->scores_out : a->w);
     if (st != DSA_OK) return st;
     if (a->k < 1) return DSA_ERR_INVALID_ARG;
+    if (a->flags & ~(unsigned)DSA_FLAG_INCLUDE_SELF) return DSA_ERR_INVALID_ARG;
     if (a->idx_out && !aligned(a->idx_out, 4)) return DSA_ERR_INVALID_ARG;
     dsa_attn_shape sh = forward_attn_shape(a);
     // idx is produced internally: pass a non-null placeholder to the check
@@ -233,14 +234,21 @@ size_t dsa_topk_workspace_bytes(int B, int Tq, int L, int q_pos0, int k) {
     return topk_workspace_bytes(B, Tq, L, q_pos0, k);
 }
 
-dsa_status dsa_topk(const float *scores, int B, int Tq, int L, int q_pos0, int k, int32_t *idx, void *ws,
-                    size_t ws_bytes, dsa_stream_t stream) {
+dsa_status dsa_topk_ex(const float *scores, int B, int Tq, int L, int q_pos0, int k, unsigned flags, int32_t *idx,
+                       void *ws, size_t ws_bytes, dsa_stream_t stream) {
     dsa_status st = check_topk(scores, B, Tq, L, q_pos0, k, idx);
     if (st != DSA_OK) return st;
+    if (flags & ~(unsigned)DSA_FLAG_INCLUDE_SELF) return DSA_ERR_INVALID_ARG;
     const size_t need = topk_workspace_bytes(B, Tq, L, q_pos0, k);
     if (need > 0 && (!ws || ws_bytes < need || !aligned(ws, 16))) return DSA_ERR_WORKSPACE;
     TopkProblem p{scores, B, Tq, L, q_pos0, k, idx, ws, ws_bytes};
+    p.include_self = (flags & DSA_FLAG_INCLUDE_SELF) != 0;
     return from_cuda(launch_topk(p, static_cast<cudaStream_t>(stream)));
+}
+
+dsa_status dsa_topk(const float *scores, int B, int Tq, int L, int q_pos0, int k, int32_t *idx, void *ws,
+                    size_t ws_bytes, dsa_stream_t stream) {
+    return dsa_topk_ex(scores, B, Tq, L, q_pos0, k, 0u, idx, ws, ws_bytes, stream);
 }
 
 size_t dsa_sparse_attn_workspace_bytes(const dsa_attn_shape *sh, dsa_dtype dt) {
@@ -275,14 +283,21 @@ dsa_status dsa_forward(const dsa_forward_args *a, void *ws, size_t ws_bytes, dsa
     int32_t *idx = a->idx_out ? a->idx_out : reinterpret_cast<int32_t *>(base + lay.idx);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
 
-    IndexerProblem ip{a->q_idx, a->k_idx, a->w, a->B, a->Tq, a->L, a->q_pos0, a->H_I, a->d_I,
-                      a->idx_dtype, scores, a->scores_out != nullptr};
-    cudaError_t err = launch_indexer(ip, s);
-    if (err != cudaSuccess) return DSA_ERR_CUDA;
+    // Every row keeping all of its candidates (t + 1 <= k): the selection is
+    // known without scores; the indexer runs only when they are asked for.
+    const bool short_context = (long long)a->q_pos0 + a->Tq <= a->k;
+    cudaError_t err = cudaSuccess;
+    if (!short_context || a->scores_out != nullptr) {
+        IndexerProblem ip{a->q_idx, a->k_idx, a->w, a->B, a->Tq, a->L, a->q_pos0, a->H_I, a->d_I,
+                          a->idx_dtype, scores, a->scores_out != nullptr};
+        if ((err = launch_indexer(ip, s)) != cudaSuccess) return DSA_ERR_CUDA;
+    }
 
     TopkProblem tp{scores, a->B, a->Tq, a->L, a->q_pos0, a->k, idx,
                    lay.topk_bytes ? base + lay.topk : nullptr, lay.topk_bytes};
-    if ((err = launch_topk(tp, s)) != cudaSuccess) return DSA_ERR_CUDA;
+    tp.include_self = (a->flags & DSA_FLAG_INCLUDE_SELF) != 0;
+    err = short_context ? launch_dense_selection(tp, s) : launch_topk(tp, s);
+    if (err != cudaSuccess) return DSA_ERR_CUDA;
 
     dsa_attn_shape sh = forward_attn_shape(a);
     AttnProblem ap = make_attn_problem(a->q, a->k_cache, a->v_cache, idx, &sh, a->attn_dtype, a->out, a->lse,

@@ -123,12 +123,6 @@ struct Args {
     float *part_o, *part_ml;  // split partials (splits > 1)
 };
 
-// 2^x with the hardware approximation (relative error below 2^-22; 2^-inf = 0).
-__device__ __forceinline__ float ex2_approx(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);

@@ -255,14 +255,15 @@ attn_mma_kernel(const Args a) {
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
             const float m_new = fmaxf(m_r[hh], mx);
-            const float corr = m_new == -INFINITY ? 1.0f : exp2f(m_r[hh] - m_new);
+            const float corr = m_new == -INFINITY ? 1.0f : ex2_approx(m_r[hh] - m_new);
+            const float mr = m_new == -INFINITY ? 0.0f : m_new;  // masked entries: 2^-inf = 0
             float sum = 0.0f;
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                     const float v = s[nt][2 * hh + e];
-                    const float pv = v == -INFINITY ? 0.0f : exp2f(v - m_new);
+                    const float pv = ex2_approx(v - mr);
                     p[nt][2 * hh + e] = pv;
                     sum += pv;
                 }

@@ -47,9 +47,13 @@ struct TopkProblem {
     int32_t *idx;         // [B, Tq, k]
     void *ws;
     size_t ws_bytes;
+    bool include_self = false;  // S_t = {t} and the k-1 best of 0..t-1
 };
 size_t topk_workspace_bytes(int B, int Tq, int L, int q_pos0, int k);
 cudaError_t launch_topk(const TopkProblem &p, cudaStream_t stream);
+// The selection when every row keeps all of its candidates (q_pos0 + Tq <= k):
+// idx[b, i, :] = 0 .. t, then -1. Reads no scores.
+cudaError_t launch_dense_selection(const TopkProblem &p, cudaStream_t stream);
 
 // ----------------------------------------------------------------- attention
 struct AttnProblem {

@@ -174,7 +174,16 @@ struct Slice {
     const float *src;  // first score of this CTA's slice
     int cnt;           // scores in the slice
     int w_lo, w_hi;    // this warp's segment [w_lo, w_hi) of the slice
+    int self_s;        // slice position forced into the selection, or -1
 };
+
+// Key of slice position s: the order-preserving key of its score, or (SELF:
+// keep the row's own position) the largest key, above every finite score.
+template <bool SELF>
+__device__ __forceinline__ uint32_t slice_key(const Slice &sl, int s, float v) {
+    if constexpr (SELF) return s == sl.self_s ? 0xFFFFFFFFu : order_key(v);
+    return order_key(v);
+}
 
 template <int KPT>
 struct RegKeys {
@@ -185,7 +194,7 @@ struct RegKeys {
 // consecutive positions per step. KPT > 0: the keys are the registers loaded
 // by load_keys; KPT == 0: streamed from global memory, four steps' loads in
 // flight.
-template <int KPT, typename F>
+template <int KPT, bool SELF, typename F>
 __device__ __forceinline__ void sweep(const Slice &sl, const RegKeys<KPT> &rk, F fn) {
     const int lane = threadIdx.x & 31;
     if constexpr (KPT > 0) {
@@ -205,13 +214,13 @@ __device__ __forceinline__ void sweep(const Slice &sl, const RegKeys<KPT> &rk, F
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const int s = base + u * kWarp + lane;
-                fn(s, order_key(v[u]), s < sl.w_hi);
+                fn(s, slice_key<SELF>(sl, s, v[u]), s < sl.w_hi);
             }
         }
     }
 }
 
-template <int KPT>
+template <int KPT, bool SELF>
 __global__ void __launch_bounds__(kThreads, 2)  // two CTAs per SM: at most 64 registers
 topk_kernel(const float *__restrict__ scores, int Tq, int L, int q_pos0, int k, int32_t *__restrict__ idx) {
     __shared__ __align__(16) int hist[3][kBins];
@@ -247,6 +256,8 @@ topk_kernel(const float *__restrict__ scores, int Tq, int L, int q_pos0, int k, 
     const int seg = KPT > 0 ? KPT * kWarp : ((sl.cnt + kWarps - 1) / kWarps + 31) & ~31;
     sl.w_lo = min(sl.cnt, warp * seg);
     sl.w_hi = min(sl.cnt, sl.w_lo + seg);
+    // the row's own position t = n - 1 sits at the end of the last slice
+    sl.self_s = (SELF && t >= lo && t < lo + sl.cnt) ? t - lo : -1;
 
     for (int b = threadIdx.x; b < kBins; b += kThreads) {
         hist[0][b] = 0;
@@ -270,10 +281,10 @@ topk_kernel(const float *__restrict__ scores, int Tq, int L, int q_pos0, int k, 
         for (int i = 0; i < KPT; ++i) {
             const int s = sl.w_lo + i * kWarp + lane;
             const float v = s < sl.w_hi ? __ldg(sl.src + s) : 0.0f;
-            rk.k[i] = order_key(v);
+            rk.k[i] = slice_key<SELF>(sl, s, v);
         }
     }
-    sweep<KPT>(sl, rk, [&](int, uint32_t key, bool ok) {
+    sweep<KPT, SELF>(sl, rk, [&](int, uint32_t key, bool ok) {
         if (ok) atomicAdd(&hist[0][key >> 21], 1);
     });
     __syncthreads();
@@ -285,7 +296,7 @@ topk_kernel(const float *__restrict__ scores, int Tq, int L, int q_pos0, int k, 
 
     // ---- compact the threshold bucket; count keys in higher buckets per warp
     int gt1 = 0;
-    sweep<KPT>(sl, rk, [&](int s, uint32_t key, bool ok) {
+    sweep<KPT, SELF>(sl, rk, [&](int s, uint32_t key, bool ok) {
         const bool cand = ok && (key >> 21) == d1;
         gt1 += ok && (key >> 21) > d1;
         const unsigned m = __ballot_sync(0xffffffffu, cand);
@@ -404,7 +415,7 @@ topk_kernel(const float *__restrict__ scores, int Tq, int L, int q_pos0, int k, 
         for (int j = threadIdx.x; j < n_list; j += kThreads)
             atomicAdd(&hist[1][(list_key[j] >> 10) & 2047u], 1);
     } else {
-        sweep<KPT>(sl, rk, [&](int, uint32_t key, bool ok) {
+        sweep<KPT, SELF>(sl, rk, [&](int, uint32_t key, bool ok) {
             if (ok && (key >> 21) == d1) atomicAdd(&hist[1][(key >> 10) & 2047u], 1);
         });
     }
@@ -421,7 +432,7 @@ topk_kernel(const float *__restrict__ scores, int Tq, int L, int q_pos0, int k, 
             if ((key >> 10) == p2) atomicAdd(&hist[2][key & 1023u], 1);
         }
     } else {
-        sweep<KPT>(sl, rk, [&](int, uint32_t key, bool ok) {
+        sweep<KPT, SELF>(sl, rk, [&](int, uint32_t key, bool ok) {
             if (ok && (key >> 10) == p2) atomicAdd(&hist[2][key & 1023u], 1);
         });
     }
@@ -442,7 +453,7 @@ topk_kernel(const float *__restrict__ scores, int Tq, int L, int q_pos0, int k, 
         }
     } else {
         int gt = 0, eq = 0;
-        sweep<KPT>(sl, rk, [&](int, uint32_t key, bool ok) {
+        sweep<KPT, SELF>(sl, rk, [&](int, uint32_t key, bool ok) {
             gt += ok && key > T;
             eq += ok && key == T;
         });
@@ -481,7 +492,7 @@ topk_kernel(const float *__restrict__ scores, int Tq, int L, int q_pos0, int k, 
     gt_b += w_gt[warp];
     eq_b += w_eq[warp];
     const unsigned lt = lanemask_lt();
-    sweep<KPT>(sl, rk, [&](int s, uint32_t key, bool ok) {
+    sweep<KPT, SELF>(sl, rk, [&](int s, uint32_t key, bool ok) {
         const bool gt = ok && key > T;
         const bool eq = ok && key == T;
         const unsigned gm = __ballot_sync(0xffffffffu, gt);
@@ -503,6 +514,26 @@ constexpr size_t kDynSmem = 8 * (size_t)kListCap + sizeof(FindScratch) + 4 * (si
 
 size_t topk_workspace_bytes(int, int, int, int, int) { return 0; }
 
+namespace {
+
+__global__ void dense_selection_kernel(int Tq, int q_pos0, int k, int32_t *__restrict__ idx) {
+    const int row = blockIdx.x;
+    const int t = q_pos0 + row % Tq;
+    int32_t *out = idx + (size_t)row * k;
+    for (int j = threadIdx.x; j < k; j += blockDim.x) out[j] = j <= t ? j : -1;
+}
+
+}  // namespace
+
+cudaError_t launch_dense_selection(const TopkProblem &p, cudaStream_t stream) {
+    const long long rows = (long long)p.B * p.Tq;
+    if (rows == 0) return cudaSuccess;
+    if (rows > 0x7fffffffLL) return cudaErrorInvalidValue;
+    dense_selection_kernel<<<(unsigned)rows, 256, 0, stream>>>(p.Tq, p.q_pos0, p.k, p.idx);
+    count_launch();
+    return cudaGetLastError();
+}
+
 // CTAs per row: enough to cover the SMs when rows are few (at most 16).
 static int cluster_parts(int rows, int sm_count) {
     int P = 1;
@@ -510,9 +541,9 @@ static int cluster_parts(int rows, int sm_count) {
     return P;
 }
 
-template <int KPT>
+template <int KPT, bool SELF>
 static cudaError_t launch_parts(const TopkProblem &p, int P, cudaStream_t stream) {
-    auto kern = topk_kernel<KPT>;
+    auto kern = topk_kernel<KPT, SELF>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDynSmem);
     if (err != cudaSuccess) return err;
     if (P > 8) {
@@ -548,9 +579,14 @@ static cudaError_t launch_parts(const TopkProblem &p, int P, cudaStream_t stream
 static cudaError_t launch_with(const TopkProblem &p, int P, cudaStream_t stream) {
     const int n_max = p.q_pos0 + p.Tq;
     const int per = (n_max + P - 1) / P;
-    if (per <= kThreads * 8) return launch_parts<8>(p, P, stream);
-    if (per <= kThreads * 16) return launch_parts<16>(p, P, stream);
-    return launch_parts<0>(p, P, stream);
+    if (p.include_self) {
+        if (per <= kThreads * 8) return launch_parts<8, true>(p, P, stream);
+        if (per <= kThreads * 16) return launch_parts<16, true>(p, P, stream);
+        return launch_parts<0, true>(p, P, stream);
+    }
+    if (per <= kThreads * 8) return launch_parts<8, false>(p, P, stream);
+    if (per <= kThreads * 16) return launch_parts<16, false>(p, P, stream);
+    return launch_parts<0, false>(p, P, stream);
 }
 
 cudaError_t launch_topk(const TopkProblem &p, cudaStream_t stream) {

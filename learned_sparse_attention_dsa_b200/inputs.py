@@ -92,6 +92,10 @@ WORKLOADS = {
     "decode128k": Workload("decode128k", B=8, Tq=1, L=131072, q_pos0=131071, H_I=64,
                            d_I=128, k=2048, Hq=128, Hkv=1, Dqk=576, Dv=512,
                            kv_alias=True, seed=1239),
+    # a context no longer than the budget: every row keeps all of its
+    # candidates, so the forward skips the indexer and the top-k
+    "prefill2k": Workload("prefill2k", B=1, Tq=2048, L=2048, q_pos0=0, H_I=64,
+                          d_I=128, k=2048, Hq=16, Hkv=1, Dqk=192, Dv=128, seed=1240),
 }
 
 

@@ -83,3 +83,12 @@ def test_binding_fails_loudly_without_library(tmp_path):
             binding.load_library(str(tmp_path / "missing.so"))
     finally:
         binding._lib = saved
+
+
+def test_unknown_flags_rejected(dsa_lib):
+    fake = ctypes.c_void_p(0x1000)  # never dereferenced: the checks fail first
+    dsa_lib.dsa_topk_ex.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                    ctypes.c_int, ctypes.c_uint, ctypes.c_void_p, ctypes.c_void_p,
+                                    ctypes.c_size_t, ctypes.c_void_p]
+    assert dsa_lib.dsa_topk_ex(fake, 1, 1, 3, 0, 2, 2, fake, None, 0, None) == 1
+    assert dsa_lib.dsa_topk_ex(fake, 1, 1, 3, 0, 2, 0x80000000, fake, None, 0, None) == 1

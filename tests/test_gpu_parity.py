@@ -204,3 +204,61 @@ def test_invalid_arguments_enqueue_nothing(cuda):
     with pytest.raises(binding.DSAError):
         binding.topk(torch.zeros((1, 2, 8), device="cuda"), 0)
     torch.cuda.synchronize()
+
+
+# ---------------------------------------------------------------- current token always kept
+
+@pytest.mark.parametrize("kind", ["int", "normal", "mixed"])
+@pytest.mark.parametrize("L,Tq,q_pos0,k", [(37, 37, 0, 5), (5000, 3, 4997, 2048), (3000, 2, 2998, 1),
+                                           (140000, 1, 139999, 2048), (2100, 2100, 0, 2048)])
+def test_topk_stage_include_self(cuda, kind, L, Tq, q_pos0, k):
+    gen = torch.Generator().manual_seed(L + Tq + k + 1)
+    scores = random_score_rows(gen, Tq, L, kind)[None]
+    got = binding.topk(scores.cuda(), k, q_pos0=q_pos0, include_self=True).cpu().numpy()[0]
+    row_t = q_pos0 + np.arange(Tq)
+    ref = oracle.topk_rows(scores[0].numpy(), row_t, k, include_self=True)
+    assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("name", ["prefill_mqa_700", "chunked_prefill", "decode_5000"])
+def test_forward_include_self(cuda, name):
+    wl = MEDIUM[name]
+    cpu, dev = _inputs(wl)
+    out = torch.empty((wl.B, wl.Tq, wl.Hq, wl.Dv), dtype=dev["q"].dtype, device="cuda")
+    idx = torch.empty((wl.B, wl.Tq, wl.k), dtype=torch.int32, device="cuda")
+    binding.forward(dev["q_idx"], dev["k_idx"], dev["w"], dev["q"], dev["k_cache"], dev["v_cache"],
+                    wl.k, wl.q_pos0, wl.scale, out=out, idx_out=idx, include_self=True)
+    binding.device_error()
+    flat = np.arange(wl.B * wl.Tq)
+    _, o_idx, o_out = oracle_forward(wl, cpu, flat, include_self=True)
+    assert np.array_equal(idx.cpu().numpy().reshape(-1, wl.k), o_idx)
+    assert_attn_close(out.float().cpu().numpy().reshape(-1, wl.Hq, wl.Dv), o_out, name)
+
+
+# ---------------------------------------------------------------- short context: no top-k
+
+@pytest.mark.parametrize("name", ["short_context", "latent_short"])
+def test_short_context_forward_without_scores(cuda, name):
+    """q_pos0 + Tq <= k: the selection is every causal position; without
+    scores_out the forward skips the indexer and the top-k. Same outputs as
+    the path that computes the scores, and as the oracle."""
+    wl = MEDIUM[name]
+    assert wl.q_pos0 + wl.Tq <= wl.k
+    cpu, dev = _inputs(wl)
+    out = torch.empty((wl.B, wl.Tq, wl.Hq, wl.Dv), dtype=dev["q"].dtype, device="cuda")
+    idx = torch.empty((wl.B, wl.Tq, wl.k), dtype=torch.int32, device="cuda")
+    n0 = binding.kernel_launch_count()
+    binding.forward(dev["q_idx"], dev["k_idx"], dev["w"], dev["q"], dev["k_cache"], dev["v_cache"],
+                    wl.k, wl.q_pos0, wl.scale, out=out, idx_out=idx)
+    launches_short = binding.kernel_launch_count() - n0
+    binding.device_error()
+    _, idx_full, out_full = _gpu_forward(wl, dev)          # with scores_out: the indexer runs
+    assert torch.equal(idx, idx_full)
+    assert torch.equal(out, out_full)
+    n0 = binding.kernel_launch_count()
+    _gpu_forward(wl, dev)
+    assert launches_short < binding.kernel_launch_count() - n0
+    flat = np.arange(wl.B * wl.Tq)
+    _, o_idx, o_out = oracle_forward(wl, cpu, flat)
+    assert np.array_equal(idx.cpu().numpy().reshape(-1, wl.k), o_idx)
+    assert_attn_close(out.float().cpu().numpy().reshape(-1, wl.Hq, wl.Dv), o_out, name)
