@@ -10,8 +10,9 @@ time; see that file's header for the page passages each function follows and
 the readings taken where the pages are silent). This module compiles it with
 gcc, and marshals numpy arrays into it.
 
-Inputs are numpy arrays: ``float32`` for fp32 data, or ``uint16`` holding raw
-bf16 bit patterns for bf16 data. Every function takes the rows to evaluate as
+Inputs are numpy arrays: ``float32`` for fp32 data, ``uint16`` holding raw
+bf16 bit patterns for bf16 data, or ``uint8`` holding e4m3 codes (indexer
+inputs only). Every function takes the rows to evaluate as
 ``(row_b, row_t)`` arrays so that a full-size problem can be checked on a
 sample of query rows.
 
@@ -43,6 +44,7 @@ _LIB_PATH = os.path.join(_HERE, "liboracle.so")
 
 F32 = 0
 BF16 = 1
+E4M3 = 2
 
 _lib = None
 
@@ -83,6 +85,8 @@ def _load():
     lib.oracle_attn_rows.restype = None
     lib.oracle_max_threads.argtypes = []
     lib.oracle_max_threads.restype = ci
+    lib.oracle_e4m3_decode.argtypes = [ci, ctypes.POINTER(ctypes.c_uint8), ctypes.POINTER(ctypes.c_double)]
+    lib.oracle_e4m3_decode.restype = None
     _lib = lib
     return lib
 
@@ -96,7 +100,18 @@ def _dtype_code(a: np.ndarray) -> int:
         return F32
     if a.dtype == np.uint16:
         return BF16
-    raise TypeError(f"oracle inputs must be float32 or uint16 (bf16 bits), got {a.dtype}")
+    if a.dtype == np.uint8:
+        return E4M3
+    raise TypeError(f"oracle inputs must be float32, uint16 (bf16 bits) or uint8 (e4m3 codes), got {a.dtype}")
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """float64 values of e4m3 codes (uint8), as the oracle reads them."""
+    lib = _load()
+    codes = np.ascontiguousarray(codes, dtype=np.uint8).ravel()
+    out = np.empty(codes.shape, dtype=np.float64)
+    lib.oracle_e4m3_decode(codes.size, _ptr(codes, ctypes.c_uint8), _ptr(out, ctypes.c_double))
+    return out
 
 
 def _ptr(a: np.ndarray, ctype):

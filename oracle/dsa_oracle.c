@@ -47,20 +47,46 @@
 #include <omp.h>
 #endif
 
-enum { ORACLE_F32 = 0, ORACLE_BF16 = 1 };
+enum { ORACLE_F32 = 0, ORACLE_BF16 = 1, ORACLE_E4M3 = 2 };
 
-/* Read element i of an array stored as fp32 or as raw bf16 bits.
- * A bf16 value is the top half of an fp32 bit pattern, so the widening is
- * exact. */
+/* Value of an 8-bit e4m3 code (the FP8 format the pages suggest for the
+ * indexer, "Learned Token Selection" §7.4): 1 sign bit, 4 exponent bits with
+ * bias 7, 3 mantissa bits; exponent 0 holds the subnormals m/8 * 2^-6; the
+ * one non-finite pattern per sign, exponent 15 with mantissa 7, is NaN (the
+ * format has no infinities). */
+static double e4m3_value(uint8_t code)
+{
+    const int sign = code >> 7;
+    const int e = (code >> 3) & 15;
+    const int m = code & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m / 8.0, -6);
+    else v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sign ? -v : v;
+}
+
+/* Read element i of an array stored as fp32, as raw bf16 bits, or as e4m3
+ * codes. A bf16 value is the top half of an fp32 bit pattern, so the widening
+ * is exact; every e4m3 value is exact in a double. */
 static double load_value(const void *base, size_t i, int dtype)
 {
     if (dtype == ORACLE_F32) {
         return (double)((const float *)base)[i];
     }
+    if (dtype == ORACLE_E4M3) {
+        return e4m3_value(((const uint8_t *)base)[i]);
+    }
     uint32_t bits = (uint32_t)((const uint16_t *)base)[i] << 16;
     float f;
     memcpy(&f, &bits, sizeof f);
     return (double)f;
+}
+
+/* The decoded values of n e4m3 codes (for the pins of the decoding). */
+void oracle_e4m3_decode(int n, const uint8_t *codes, double *out)
+{
+    for (int i = 0; i < n; ++i) out[i] = e4m3_value(codes[i]);
 }
 
 static void set_threads(int nthreads)

@@ -20,12 +20,14 @@ LSE_ATOL = 2e-3
 
 
 def bits(t: torch.Tensor) -> np.ndarray:
-    """A CPU tensor as the oracle's numpy input (fp32, or raw bf16 bits)."""
+    """A CPU tensor as the oracle's numpy input (fp32, raw bf16 bits, or e4m3 codes)."""
     t = t.detach().cpu().contiguous()
     if t.dtype == torch.float32:
         return t.numpy()
     if t.dtype == torch.bfloat16:
         return t.view(torch.int16).numpy().view(np.uint16)
+    if t.dtype == torch.float8_e4m3fn:
+        return t.view(torch.uint8).numpy()
     raise TypeError(t.dtype)
 
 

@@ -395,3 +395,34 @@ def test_topk_include_self_brute_force(kind):
             assert t in got[r].tolist()
             if t in plain[r].tolist():  # already selected: the rule changes nothing
                 assert got[r].tolist() == plain[r].tolist()
+
+
+# ---------------------------------------------------------------- e4m3 indexer inputs
+
+def test_e4m3_decode_matches_torch_for_every_code():
+    """The oracle's e4m3 decoding (written from the format's definition)
+    against torch's float8_e4m3fn conversion, all 256 codes."""
+    codes = np.arange(256, dtype=np.uint8)
+    got = oracle.e4m3_decode(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+    assert nan.sum() == 2                                  # 0x7f and 0xff
+    assert got[0x7e] == 448.0 and got[0x01] == 2.0 ** -9   # largest finite, smallest subnormal
+
+
+def test_e4m3_indexer_equals_fp32_on_integers():
+    """Integers in [-8, 8] are exact in e4m3, and their products sum exactly:
+    the e4m3 indexer equals the fp32 one on the same values."""
+    rng = np.random.default_rng(12)
+    n, H, d = 23, 4, 32
+    qf = rng.integers(-8, 9, size=(n, H, d)).astype(np.float32)
+    kf = rng.integers(-8, 9, size=(1, n, d)).astype(np.float32)
+    w = (2.0 ** rng.integers(-3, 1, size=(n, H)) * rng.choice([-1, 1], size=(n, H))).astype(np.float32)
+    q8 = torch.from_numpy(qf).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    k8 = torch.from_numpy(kf).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(oracle.e4m3_decode(q8).reshape(qf.shape), qf)
+    got = oracle.indexer_rows(q8, w, k8, np.zeros(n), np.arange(n))
+    ref = oracle.indexer_rows(qf, w, kf, np.zeros(n), np.arange(n))
+    assert np.array_equal(got, ref)
