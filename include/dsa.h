@@ -64,7 +64,11 @@ typedef enum {
 
 typedef enum {
     DSA_F32 = 0,   /* IEEE fp32 */
-    DSA_BF16 = 1   /* bfloat16 */
+    DSA_BF16 = 1,  /* bfloat16 */
+    DSA_E4M3 = 2   /* 8-bit e4m3 codes (1 sign, 4 exponent bits with bias 7,
+                      3 mantissa bits): indexer inputs only (q_idx, k_idx of
+                      dsa_indexer_scores and dsa_forward_args.idx_dtype), the
+                      FP8 indexer of "Learned Token Selection" §7.4 */
 } dsa_dtype;
 
 /* Library version, e.g. 100 for 0.1.0. */

@@ -17,6 +17,7 @@ LIB_PATH = os.path.join(_PKG, "libdsa.so")
 
 DSA_F32 = 0
 DSA_BF16 = 1
+DSA_E4M3 = 2
 DSA_FLAG_INCLUDE_SELF = 1
 
 STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED",
@@ -114,6 +115,8 @@ def _dt(t: torch.Tensor) -> int:
         return DSA_F32
     if t.dtype == torch.bfloat16:
         return DSA_BF16
+    if t.dtype == torch.float8_e4m3fn:
+        return DSA_E4M3
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 

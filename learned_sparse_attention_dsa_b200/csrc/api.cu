@@ -56,8 +56,9 @@ namespace {
 constexpr size_t kWsAlign = 256;
 
 bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
-size_t dtype_bytes(dsa_dtype dt) { return dt == DSA_F32 ? 4 : 2; }
+size_t dtype_bytes(dsa_dtype dt) { return dt == DSA_F32 ? 4 : (dt == DSA_E4M3 ? 1 : 2); }
 bool valid_dtype(dsa_dtype dt) { return dt == DSA_F32 || dt == DSA_BF16; }
+bool valid_indexer_dtype(dsa_dtype dt) { return valid_dtype(dt) || dt == DSA_E4M3; }
 
 dsa_status from_cuda(cudaError_t err) { return err == cudaSuccess ? DSA_OK : DSA_ERR_CUDA; }
 
@@ -79,7 +80,7 @@ dsa_status check_indexer(const void *q_idx, const void *k_idx, const float *w, i
     dsa_status st = check_rows(B, Tq, L, q_pos0);
     if (st != DSA_OK) return st;
     if (H_I < 1 || d_I < 1) return DSA_ERR_INVALID_ARG;
-    if (!valid_dtype(dt)) return DSA_ERR_UNSUPPORTED;
+    if (!valid_indexer_dtype(dt)) return DSA_ERR_UNSUPPORTED;
     const size_t eb = dtype_bytes(dt);
     if (!aligned(q_idx, eb) || !aligned(k_idx, eb) || !aligned(w, 4) || !aligned(scores, 4))
         return DSA_ERR_INVALID_ARG;

@@ -3,6 +3,7 @@
 
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <stdint.h>
 
 #include "dsa.h"
@@ -17,6 +18,11 @@ template <typename T> struct Elem;
 template <> struct Elem<float> {
     static __device__ __forceinline__ float load(const float *p, size_t i) { return p[i]; }
     static __device__ __forceinline__ void store(float *p, size_t i, float v) { p[i] = v; }
+};
+template <> struct Elem<__nv_fp8_e4m3> {  // indexer inputs only: loads
+    static __device__ __forceinline__ float load(const __nv_fp8_e4m3 *p, size_t i) {
+        return static_cast<float>(p[i]);
+    }
 };
 template <> struct Elem<__nv_bfloat16> {
     static __device__ __forceinline__ float load(const __nv_bfloat16 *p, size_t i) {

@@ -1,4 +1,4 @@
-// Lightning-indexer scores on CUDA cores (any H, d, fp32 or bf16).
+// Lightning-indexer scores on CUDA cores (any H, d; fp32, bf16 or e4m3 inputs).
 //
 //   I[t,s] = sum_j w[t,j] * ReLU(q[t,j] . k[s]),  s <= t
 // ("DeepSeek Sparse Attention: Learned Token Selection from Scratch" §2.1).
@@ -103,8 +103,9 @@ size_t indexer_cuda_core_smem_bytes(int H, int d) {
 }
 
 cudaError_t launch_indexer_cuda_core(const IndexerProblem &p, cudaStream_t stream) {
-    return p.dt == DSA_F32 ? launch_cuda_core<float>(p, stream)
-                           : launch_cuda_core<__nv_bfloat16>(p, stream);
+    if (p.dt == DSA_F32) return launch_cuda_core<float>(p, stream);
+    if (p.dt == DSA_E4M3) return launch_cuda_core<__nv_fp8_e4m3>(p, stream);
+    return launch_cuda_core<__nv_bfloat16>(p, stream);
 }
 
 cudaError_t launch_indexer(const IndexerProblem &p, cudaStream_t stream) {

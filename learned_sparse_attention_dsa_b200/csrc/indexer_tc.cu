@@ -17,9 +17,10 @@
 //   warp 1      allocates TMEM; one thread issues tcgen05.mma (bf16 in, fp32
 //               accumulate) into one of two TMEM accumulators.
 //   warps 2-9   epilogue, two warps per TMEM lane quarter (each takes every
-//               other query of the tile): tcgen05.ld of the accumulator, ReLU,
-//               weight and head sum with packed fp32x2 FMAs, one fp32 score
-//               per (query, key), causal mask.
+//               other query of the tile; with one query per tile, as in
+//               decode, every other tile): tcgen05.ld of the accumulator,
+//               ReLU, weight and head sum with packed fp32x2 FMAs, one fp32
+//               score per (query, key), causal mask.
 // The two accumulators let the epilogue of tile n overlap the MMAs of tile
 // n+1. A work unit is (batch entry, query group, chunk of at most C key
 // tiles); units are spread over the CTAs round-robin. Causal: a query group
@@ -91,16 +92,18 @@ __device__ __forceinline__ bool decode_unit(int u, const Params &p, Unit &un) {
     return true;
 }
 
-template <int D, int N_TILE>
+template <int D, int N_TILE, bool FP8>
 struct Cfg {
-    static constexpr int kHalves = D / 64;                          // 64-element (128-byte) K slices
+    static constexpr int kBoxElems = FP8 ? 128 : 64;                 // elements per 128-byte K slice
+    static constexpr int kHalves = D / kBoxElems;                    // 128-byte K slices per row
     static constexpr uint32_t kQHalf = N_TILE * 128;
     static constexpr uint32_t kQBytes = kQHalf * kHalves;
     static constexpr uint32_t kKHalf = kBlockM * 128;
     static constexpr uint32_t kKBytes = kKHalf * kHalves;
     static constexpr int kQBufs = 2;
     static constexpr int kStagesRaw = (int)((kSmemBudget - kQBufs * kQBytes) / kKBytes);
-    static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
+    // as many key stages as fit: with 16 KB e4m3 stages, 13 keep ~200 KB in flight
+    static constexpr int kStages = kStagesRaw > 16 ? 16 : kStagesRaw;
     static constexpr uint32_t kTmemCols = 2 * N_TILE;
     static constexpr int kBars = 2 * kStages + 2 * kQBufs + 4;
     static constexpr size_t kSmem = 1024 + (size_t)kQBufs * kQBytes + (size_t)kStages * kKBytes + kBars * 8 + 16;
@@ -108,11 +111,11 @@ struct Cfg {
     static_assert(kTmemCols == 128 || kTmemCols == 256 || kTmemCols == 512, "TMEM columns");
 };
 
-template <int D, int N_TILE>
+template <int D, int N_TILE, bool FP8>
 __global__ void __launch_bounds__(kThreads, 1)
 indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const Params p) {
-    using C = Cfg<D, N_TILE>;
+    using C = Cfg<D, N_TILE, FP8>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *q_sm = smem;
@@ -138,9 +141,12 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             mbar_init(&q_full[s], 1);
             mbar_init(&q_empty[s], 1);
         }
+        // one query per tile (decode): the two warps of a TMEM lane quarter
+        // take alternate tiles (accumulators), else alternate queries
+        const int releasers = p.QPT == 1 ? kEpilogueThreads / 2 : kEpilogueThreads;
         for (int s = 0; s < 2; ++s) {
             mbar_init(&acc_full[s], 1);
-            mbar_init(&acc_empty[s], kEpilogueThreads);
+            mbar_init(&acc_empty[s], releasers);
         }
         fence_barrier_init();
     }
@@ -169,7 +175,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 const int qrow = (un.b * p.Tq + un.i0) * p.H;
 #pragma unroll
                 for (int h = 0; h < C::kHalves; ++h)
-                    tma_load_2d(q_sm + qb * C::kQBytes + h * C::kQHalf, &tm_q, &q_full[qb], h * 64, qrow);
+                    tma_load_2d(q_sm + qb * C::kQBytes + h * C::kQHalf, &tm_q, &q_full[qb], h * C::kBoxElems, qrow);
                 if (++qb == C::kQBufs) { qb = 0; qph ^= 1u; }
                 for (int kt = un.kt0; kt < un.kt1; ++kt) {
                     if (!mbar_wait(&k_empty[ks], kph ^ 1u)) { ok = false; break; }
@@ -177,7 +183,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     const int krow = un.b * p.L + kt * kBlockM;
 #pragma unroll
                     for (int h = 0; h < C::kHalves; ++h)
-                        tma_load_2d(k_sm + ks * C::kKBytes + h * C::kKHalf, &tm_k, &k_full[ks], h * 64, krow);
+                        tma_load_2d(k_sm + ks * C::kKBytes + h * C::kKHalf, &tm_k, &k_full[ks], h * C::kBoxElems, krow);
                     if (++ks == C::kStages) { ks = 0; kph ^= 1u; }
                 }
             }
@@ -192,7 +198,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 if (!decode_unit(u, p, un)) continue;
                 if (!mbar_wait(&q_full[qb], qph)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t idesc = idesc_bf16_f32(kBlockM, un.qcount * p.H);
+                const uint32_t idesc = FP8 ? idesc_e4m3_f32(kBlockM, un.qcount * p.H)
+                                           : idesc_bf16_f32(kBlockM, un.qcount * p.H);
                 const uint32_t q_base = smem_addr(q_sm + qb * C::kQBytes);
                 for (int kt = un.kt0; kt < un.kt1; ++kt) {
                     if (!mbar_wait(&k_full[ks], kph)) { ok = false; break; }
@@ -203,10 +210,13 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 #pragma unroll
                     for (int h = 0; h < C::kHalves; ++h) {
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {  // 4 x K=16 per 128-byte swizzle row
+                        for (int kk = 0; kk < 4; ++kk) {  // 4 MMAs of 32 bytes of K per 128-byte swizzle row
                             const uint64_t a = smem_desc_k_sw128(k_base + h * C::kKHalf + kk * 32);
                             const uint64_t b = smem_desc_k_sw128(q_base + h * C::kQHalf + kk * 32);
-                            mma_f16_ss(d_tmem, a, b, idesc, (h | kk) != 0);
+                            if constexpr (FP8)
+                                mma_f8_ss(d_tmem, a, b, idesc, (h | kk) != 0);
+                            else
+                                mma_f16_ss(d_tmem, a, b, idesc, (h | kk) != 0);
                         }
                     }
                     mma_commit(&k_empty[ks]);   // key stage free once these MMAs finish
@@ -222,7 +232,10 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     } else {
         // ---------------------------------------------------- epilogue
         const int quarter = warp & 3;                 // TMEM lanes this warp may read
-        const int q_first = (warp - 2) >> 2;          // 0 or 1: this warp takes queries q_first, q_first+2, ...
+        const int half = (warp - 2) >> 2;             // 0 or 1: the warp's share of the tiles' work
+        const bool by_tile = p.QPT == 1;              // decode: accumulator `half` only, its one query
+        const int q_first = by_tile ? 0 : half;       // else queries half, half + 2, ...
+        const int q_step = by_tile ? 1 : 2;
         const int key_in_tile = quarter * 32 + lane;  // TMEM lane = key
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
         int ab = 0;
@@ -233,11 +246,15 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             const size_t row0 = (size_t)un.b * p.Tq + un.i0;
             const float4 *w4 = reinterpret_cast<const float4 *>(p.w + row0 * p.H);
             for (int kt = un.kt0; kt < un.kt1; ++kt) {
+                if (by_tile && ab != half) {  // the other warp of the quarter takes this tile
+                    if (++ab == 2) { ab = 0; aph ^= 1u; }
+                    continue;
+                }
                 if (!mbar_wait(&acc_full[ab], aph)) { ok = false; break; }
                 tc_fence_after();
                 const int s = kt * kBlockM + key_in_tile;
                 const uint32_t tbase = tmem_base + lane_addr + (uint32_t)(ab * N_TILE);
-                for (int q = q_first; q < un.qcount; q += 2) {
+                for (int q = q_first; q < un.qcount; q += q_step) {
                     // four independent packed (f32x2) partial sums
                     uint64_t part[4] = {0ull, 0ull, 0ull, 0ull};
                     for (int c = 0; c < p.H; c += 32) {
@@ -294,13 +311,15 @@ __global__ void fill_beyond_tiles_kernel(float *__restrict__ scores, int Tq, int
     for (int s = start + threadIdx.x; s < L; s += blockDim.x) out[s] = -INFINITY;
 }
 
-template <int D, int N_TILE>
+template <int D, int N_TILE, bool FP8>
 cudaError_t launch_tc(const IndexerProblem &pr, const DeviceInfo &info, cudaStream_t stream) {
-    using C = Cfg<D, N_TILE>;
+    using C = Cfg<D, N_TILE, FP8>;
     if ((size_t)info.max_smem_optin < C::kSmem) return cudaErrorInvalidValue;
     CUtensorMap tm_q, tm_k;
-    if (!make_map_bf16_sw128(&tm_q, pr.q_idx, (uint64_t)pr.B * pr.Tq * pr.H, (uint64_t)D, (uint64_t)D * 2, N_TILE) ||
-        !make_map_bf16_sw128(&tm_k, pr.k_idx, (uint64_t)pr.B * pr.L, (uint64_t)D, (uint64_t)D * 2, kBlockM))
+    auto make = FP8 ? make_map_u8_sw128 : make_map_bf16_sw128;
+    const uint64_t pitch = (uint64_t)D * (FP8 ? 1 : 2);
+    if (!make(&tm_q, pr.q_idx, (uint64_t)pr.B * pr.Tq * pr.H, (uint64_t)D, pitch, N_TILE) ||
+        !make(&tm_k, pr.k_idx, (uint64_t)pr.B * pr.L, (uint64_t)D, pitch, kBlockM))
         return cudaErrorInvalidValue;
 
     Params p;
@@ -331,7 +350,7 @@ cudaError_t launch_tc(const IndexerProblem &pr, const DeviceInfo &info, cudaStre
     if (units > 0x7fffffffLL) return cudaErrorInvalidValue;
     p.units = (int)units;
 
-    auto kern = indexer_tc_kernel<D, N_TILE>;
+    auto kern = indexer_tc_kernel<D, N_TILE, FP8>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
     if (err != cudaSuccess) return err;
     const int grid = p.units < info.sm_count ? p.units : info.sm_count;
@@ -357,8 +376,10 @@ unsigned int indexer_take_device_error() {
 
 cudaError_t launch_indexer_tc(const IndexerProblem &p, cudaStream_t stream, bool *taken) {
     *taken = false;
-    if (p.dt != DSA_BF16) return cudaSuccess;
-    if (!(p.d == 64 || p.d == 128)) return cudaSuccess;
+    // bf16 rows of 64 or 128 elements; e4m3 rows of 128 (one 128-byte slice)
+    const bool fp8 = p.dt == DSA_E4M3;
+    if (p.dt != DSA_BF16 && !fp8) return cudaSuccess;
+    if (!(p.d == 128 || (p.d == 64 && !fp8))) return cudaSuccess;
     if (!(p.H == 32 || p.H == 64 || p.H == 128)) return cudaSuccess;
     if (((uintptr_t)p.q_idx | (uintptr_t)p.k_idx | (uintptr_t)p.w) % 16 != 0) return cudaSuccess;
     DeviceInfo info;
@@ -373,14 +394,19 @@ cudaError_t launch_indexer_tc(const IndexerProblem &p, cudaStream_t stream, bool
     // a TMA box may not be taller than the tensor it reads
     if ((long long)p.B * p.Tq * p.H < n_tile || (long long)p.B * p.L < kBlockM) return cudaSuccess;
     *taken = true;
-    if (p.d == 128) {
-        if (n_tile == 64) return launch_tc<128, 64>(p, info, stream);
-        if (n_tile == 128) return launch_tc<128, 128>(p, info, stream);
-        return launch_tc<128, 256>(p, info, stream);
+    if (fp8) {
+        if (n_tile == 64) return launch_tc<128, 64, true>(p, info, stream);
+        if (n_tile == 128) return launch_tc<128, 128, true>(p, info, stream);
+        return launch_tc<128, 256, true>(p, info, stream);
     }
-    if (n_tile == 64) return launch_tc<64, 64>(p, info, stream);
-    if (n_tile == 128) return launch_tc<64, 128>(p, info, stream);
-    return launch_tc<64, 256>(p, info, stream);
+    if (p.d == 128) {
+        if (n_tile == 64) return launch_tc<128, 64, false>(p, info, stream);
+        if (n_tile == 128) return launch_tc<128, 128, false>(p, info, stream);
+        return launch_tc<128, 256, false>(p, info, stream);
+    }
+    if (n_tile == 64) return launch_tc<64, 64, false>(p, info, stream);
+    if (n_tile == 128) return launch_tc<64, 128, false>(p, info, stream);
+    return launch_tc<64, 256, false>(p, info, stream);
 }
 
 }  // namespace dsa

@@ -27,6 +27,9 @@ void count_launch(int n = 1);
 // columns (128 bytes) with the 128-byte swizzle. False if the driver rejects it.
 bool make_map_bf16_sw128(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint64_t pitch_bytes,
                          uint32_t box_rows);
+// The same over 8-bit elements (e4m3 codes): boxes of box_rows x 128 columns.
+bool make_map_u8_sw128(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint64_t pitch_bytes,
+                       uint32_t box_rows);
 
 // ----------------------------------------------------------------- indexer
 struct IndexerProblem {

@@ -52,6 +52,7 @@ class Workload:
     idx_range: int = 8         # indexer integers uniform in [-idx_range, idx_range]
     w_kind: str = "pow2"       # "pow2": +-2^j, j in -3..0; "set": {0.5, 1, 2}
     kv_alias: bool = False     # V = first Dv columns of each K row
+    idx_dtype: str = ""        # q^I/k^I storage: "" = as dtype, "e4m3" = 8-bit FP8 codes
     seed: int = 1234
 
     @property
@@ -94,6 +95,9 @@ WORKLOADS = {
                            kv_alias=True, seed=1239),
     # a context no longer than the budget: every row keeps all of its
     # candidates, so the forward skips the indexer and the top-k
+    # decode32k with the indexer inputs in e4m3 (half the key bytes)
+    "decode32k_fp8": Workload("decode32k_fp8", B=32, Tq=1, L=32768, q_pos0=32767, H_I=64,
+                              d_I=128, k=2048, Hq=16, Hkv=1, Dqk=128, Dv=128, idx_dtype="e4m3", seed=1236),
     "prefill2k": Workload("prefill2k", B=1, Tq=2048, L=2048, q_pos0=0, H_I=64,
                           d_I=128, k=2048, Hq=16, Hkv=1, Dqk=192, Dv=128, seed=1240),
 }
@@ -142,6 +146,9 @@ def make_inputs(wl: Workload, seed: int | None = None) -> dict:
     dt = _dtype(wl)
     q_idx = _ints(gen, (wl.B, wl.Tq, wl.H_I, wl.d_I), wl.idx_range, dt)
     k_idx = _ints(gen, (wl.B, wl.L, wl.d_I), wl.idx_range, dt)
+    if wl.idx_dtype == "e4m3":  # the same integers, exact in e4m3 up to 16
+        q_idx = q_idx.to(torch.float8_e4m3fn)
+        k_idx = k_idx.to(torch.float8_e4m3fn)
     w = _weights(gen, (wl.B, wl.Tq, wl.H_I), wl.w_kind)
     q = _normal(gen, (wl.B, wl.Tq, wl.Hq, wl.Dqk), dt)
     k_cache = _normal(gen, (wl.B, wl.L, wl.Hkv, wl.Dqk), dt)

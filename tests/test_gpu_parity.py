@@ -56,6 +56,7 @@ FULL_ROWS = {
     "prefill8k": [0, 1, 2046, 2047, 2048, 5000, 8191],
     "prefill32k": [0, 2047, 2048, 20000, 32767],
     "decode128k": [0, 5],
+    "decode32k_fp8": [0, 13, 31],
 }
 
 _cache = {}
@@ -262,3 +263,35 @@ def test_short_context_forward_without_scores(cuda, name):
     _, o_idx, o_out = oracle_forward(wl, cpu, flat)
     assert np.array_equal(idx.cpu().numpy().reshape(-1, wl.k), o_idx)
     assert_attn_close(out.float().cpu().numpy().reshape(-1, wl.Hq, wl.Dv), o_out, name)
+
+
+# ---------------------------------------------------------------- e4m3 indexer inputs
+
+@pytest.mark.parametrize("name", ["prefill_mqa_700", "decode_5000", "odd_heads", "tiny_f32"])
+def test_indexer_stage_e4m3(cuda, name):
+    """The same integers in e4m3: scores bit-exact against the oracle reading
+    the 8-bit codes (tensor-core kernel for d = 128, CUDA cores otherwise)."""
+    wl = MEDIUM[name].replace(idx_dtype="e4m3")
+    cpu = make_inputs(wl)
+    q8, k8 = cpu["q_idx"].cuda(), cpu["k_idx"].cuda()
+    assert q8.dtype == torch.float8_e4m3fn
+    scores = binding.indexer_scores(q8, k8, cpu["w"].cuda(), wl.q_pos0).cpu().numpy()
+    flat = np.arange(wl.B * wl.Tq)
+    row_b, row_i, row_t = rows_of(wl, flat)
+    ref = oracle.indexer_rows(bits(cpu["q_idx"][row_b, row_i]), cpu["w"][row_b, row_i].numpy(),
+                              bits(cpu["k_idx"]), row_b, row_t)
+    assert np.array_equal(scores.reshape(-1, wl.L), ref)
+
+
+@pytest.mark.parametrize("name", ["decode_5000", "chunked_prefill"])
+def test_forward_e4m3_equals_bf16(cuda, name):
+    """Integer indexer inputs are exact in both formats, so the e4m3 forward
+    gives the bf16 forward's scores, selections and outputs bit for bit."""
+    wl = MEDIUM[name]
+    cpu, dev = _inputs(wl)
+    s16, i16, o16 = _gpu_forward(wl, dev)
+    dev8 = dict(dev, q_idx=dev["q_idx"].to(torch.float8_e4m3fn), k_idx=dev["k_idx"].to(torch.float8_e4m3fn))
+    s8, i8, o8 = _gpu_forward(wl, dev8)
+    assert torch.equal(s8, s16)
+    assert torch.equal(i8, i16)
+    assert torch.equal(o8, o16)
