@@ -589,9 +589,15 @@ static cudaError_t launch_with(const TopkProblem &p, int P, cudaStream_t stream)
     return launch_parts<0, false>(p, P, stream);
 }
 
+cudaError_t launch_topk_block(const TopkProblem &p, cudaStream_t stream, bool *taken);
+
 cudaError_t launch_topk(const TopkProblem &p, cudaStream_t stream) {
+    // rows of at most 32,768 scores: one CTA per row, the row in registers
+    bool taken = false;
+    cudaError_t err = launch_topk_block(p, stream, &taken);
+    if (taken || err != cudaSuccess) return err;
     DeviceInfo info;
-    cudaError_t err = device_info(&info);
+    err = device_info(&info);
     if (err != cudaSuccess) return err;
     const long long rows = (long long)p.B * p.Tq;
     if (rows == 0) return cudaSuccess;

@@ -136,8 +136,9 @@ def test_indexer_stage_all_rows(cuda, name):
 
 @pytest.mark.parametrize("kind", ["int", "equal", "normal", "neg", "mixed"])
 @pytest.mark.parametrize("L,Tq,q_pos0,k", [(37, 37, 0, 5), (5000, 3, 4997, 2048), (3000, 2, 2998, 1),
-                                           (70000, 2, 69998, 2048), (140000, 1, 139999, 2048),
-                                           (2100, 2100, 0, 2048)])
+                                           (12000, 3, 11997, 2048), (32768, 2, 32766, 2048),
+                                           (32768, 3, 32765, 1000), (70000, 2, 69998, 2048),
+                                           (140000, 1, 139999, 2048), (2100, 2100, 0, 2048)])
 def test_topk_stage(cuda, kind, L, Tq, q_pos0, k):
     gen = torch.Generator().manual_seed(L + Tq + k)
     scores = random_score_rows(gen, Tq, L, kind)[None]            # [1, Tq, L]
