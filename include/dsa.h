@@ -264,6 +264,75 @@ dsa_status dsa_forward(const dsa_forward_args *a, void *ws, size_t ws_bytes,
 /* Workspace needed by dsa_forward; 0 when the arguments are invalid. */
 size_t dsa_forward_workspace_bytes(const dsa_forward_args *a);
 
+/* ------------------------------------------------------------------------
+ * The indexer's training loss and its backward pass ("Learned Token
+ * Selection" §5 dense warm-up and §6 sparse training; "DeepSeek NSA and DSA"
+ * §3.3). The target is supplied by the caller; the main model's attention
+ * that would produce it in training lies outside this library.
+ * ------------------------------------------------------------------------ */
+
+/*
+ * dsa_indexer_kl -- per query row, loss_t = KL(p_t || Softmax(I_t)) over the
+ * row's set, and the gradient of sum_t loss_t with respect to I.
+ *   scores   [B, Tq, L] fp32: indexer scores I (dsa_indexer_scores). Only
+ *            the entries of each row's set are read.
+ *   idx      NULL: the dense warm-up loss ("Learned Token Selection" §5.4);
+ *            the set of row t is s = 0..t and target is [B, Tq, L] (entries
+ *            s > t are not read).
+ *            Otherwise [B, Tq, k] int32, e.g. from dsa_topk: the loss of the
+ *            sparse stage, restricted to S_t (§6.2). The set is the entries
+ *            with 0 <= s <= t (the -1 padding and anything else outside that
+ *            range is skipped); entries must be distinct. target is then
+ *            [B, Tq, k], aligned with idx.
+ *   target   non-negative fp32 weights a of the target distribution, such as
+ *            the head sums of the main attention's weights (§5.2, step 1).
+ *            Each row is L1-normalised over its set (§5.2, step 2), so an
+ *            already normalised p may be passed too. A row whose weights sum
+ *            to 0 has loss 0 and a zero gradient; 0 * log 0 counts as 0.
+ *   loss_rows [B * Tq] fp32 (required): loss_t of every row.
+ *   loss_sum  [1] fp32 or NULL: the sum of loss_rows, accumulated in fp64 in
+ *            a fixed order (the same value on every call).
+ *   grad     [B, Tq, L] fp32 or NULL: softmax(I_t)_s - p_t[s] on the set, 0
+ *            everywhere else (every entry is written). Must not overlap
+ *            scores or target.
+ * Arithmetic: fp32 with expf/logf; the loss is formed from the row sums
+ * sum(a), sum(a I), sum(a log a) and the log-sum-exp of I over the set.
+ * Errors: DSA_ERR_INVALID_ARG for a null scores, target or loss_rows, bad
+ * sizes (as dsa_topk; k >= 1 when idx is given) or pointers not 4-byte
+ * aligned.
+ */
+dsa_status dsa_indexer_kl(const float *scores, const float *target, const int32_t *idx,
+                          int B, int Tq, int L, int q_pos0, int k,
+                          float *loss_rows, float *loss_sum, float *grad,
+                          dsa_stream_t stream);
+
+/*
+ * dsa_indexer_backward -- gradients of the indexer's inputs for an incoming
+ * gradient g = d loss / d I (e.g. dsa_indexer_kl's grad). Differentiating
+ * I[t,s] = sum_j w[t,j] ReLU(x[t,j,s]), x[t,j,s] = q^I[t,j] . k^I[s]
+ * ("Learned Token Selection" §2.1; by §6.4 the loss reaches only the
+ * indexer), with ReLU'(0) = 0 and G[t,j,s] = g[t,s] w[t,j] [x[t,j,s] > 0]:
+ *   dw[t,j] = sum_{s<=t} g[t,s] ReLU(x[t,j,s])
+ *   dq[t,j] = sum_{s<=t} G[t,j,s] k^I[s]
+ *   dk[s]   = sum over this call's query rows t >= s of sum_j G[t,j,s] q^I[t,j]
+ *   q_idx, k_idx, w, B, Tq, L, q_pos0, H_I, d_I, dt: as dsa_indexer_scores;
+ *            dt is DSA_BF16 or DSA_F32 (DSA_E4M3: DSA_ERR_UNSUPPORTED).
+ *   grad     [B, Tq, L] fp32; entries s > t are not read.
+ *   dq       [B, Tq, H_I, d_I] fp32 or NULL (then not computed).
+ *   dk       [B, L, d_I] fp32 or NULL; keys that no query row of the call
+ *            reaches (s > q_pos0 + Tq - 1) get 0. Every entry is written.
+ *   dw       [B, Tq, H_I] fp32 or NULL.
+ * Arithmetic: bf16 inputs with H_I * d_I on the tensor-core path (d_I = 128,
+ * H_I = 64) multiply x exactly (bf16 products, fp32 sums) and round G to
+ * bf16 for the second product; sums are fp32. Elsewhere every step is fp32.
+ * Errors: DSA_ERR_INVALID_ARG as dsa_indexer_scores, or a null grad;
+ * DSA_ERR_UNSUPPORTED when the fallback's staging does not fit.
+ */
+dsa_status dsa_indexer_backward(const void *q_idx, const void *k_idx, const float *w,
+                                const float *grad, int B, int Tq, int L, int q_pos0,
+                                int H_I, int d_I, dsa_dtype dt,
+                                float *dq, float *dk, float *dw, dsa_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

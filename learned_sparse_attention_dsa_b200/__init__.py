@@ -7,6 +7,9 @@ declared in ``include/dsa.h``):
   topk             S_t = the k largest I[t,s], ties to the lower s
   sparse_attn      softmax attention of every query head over S_t
   forward          the three back to back on one stream
+  indexer_kl       the indexer's training loss KL(p_t || Softmax(I_t)) and
+                   its gradient with respect to the scores
+  indexer_backward dq, dk, dw of the indexer inputs for that gradient
 
 The Python functions are argument marshalling only; every step runs in the
 CUDA library, which is loaded on first use and raises if it is missing.
@@ -16,7 +19,7 @@ from .inputs import WORKLOADS, Workload, make_inputs, to_device  # noqa: F401
 
 _BINDING_NAMES = ("indexer_scores", "topk", "sparse_attn", "forward", "forward_args",
                   "forward_workspace_bytes", "attn_shape", "load_library", "DSAError", "device_error",
-                  "kernel_launch_count")
+                  "kernel_launch_count", "indexer_kl", "indexer_backward")
 
 
 def __getattr__(name):

@@ -26,7 +26,8 @@ STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED",
 # Symbols declared in include/dsa.h.
 EXPORTED = ("dsa_version", "dsa_kernel_launch_count", "dsa_status_string", "dsa_indexer_scores", "dsa_topk",
             "dsa_topk_workspace_bytes", "dsa_sparse_attn", "dsa_sparse_attn_workspace_bytes",
-            "dsa_forward", "dsa_forward_workspace_bytes", "dsa_device_error", "dsa_topk_ex")
+            "dsa_forward", "dsa_forward_workspace_bytes", "dsa_device_error", "dsa_topk_ex",
+            "dsa_indexer_kl", "dsa_indexer_backward")
 
 
 class DSAError(RuntimeError):
@@ -91,6 +92,10 @@ def load_library(path: str = LIB_PATH):
     lib.dsa_forward_workspace_bytes.argtypes = [ctypes.POINTER(ForwardArgs)]
     lib.dsa_forward_workspace_bytes.restype = sz
     lib.dsa_device_error.argtypes, lib.dsa_device_error.restype = [vp], ci
+    lib.dsa_indexer_kl.argtypes = [vp, vp, vp, ci, ci, ci, ci, ci, vp, vp, vp, vp]
+    lib.dsa_indexer_kl.restype = ci
+    lib.dsa_indexer_backward.argtypes = [vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, vp, vp, vp, vp]
+    lib.dsa_indexer_backward.restype = ci
     _lib = lib
     return lib
 
@@ -180,6 +185,50 @@ def topk(scores, k: int, q_pos0: int = 0, idx=None, ws=None, stream=None, includ
     st = lib.dsa_topk_ex(_p(scores), B, Tq, L, q_pos0, k, flags, _p(idx), _p(ws), nbytes, _stream(stream))
     _check(st, "dsa_topk_ex")
     return idx
+
+
+def indexer_kl(scores, target, q_pos0: int = 0, idx=None, loss_rows=None, loss_sum=None, grad=None,
+               want_grad: bool = True, want_sum: bool = True, stream=None):
+    """dsa_indexer_kl: per-row KL(p_t || softmax(I_t)) over s <= t (idx None)
+    or over the selected set (idx [B, Tq, k], target aligned with it).
+    Returns (loss_rows [B*Tq], loss_sum [1] or None, grad [B, Tq, L] or None)."""
+    lib = load_library()
+    _need_cuda(scores, target, idx, loss_rows, loss_sum, grad)
+    B, Tq, L = scores.shape
+    k = 0 if idx is None else idx.shape[-1]
+    dev = scores.device
+    if loss_rows is None:
+        loss_rows = torch.empty(B * Tq, dtype=torch.float32, device=dev)
+    if loss_sum is None and want_sum:
+        loss_sum = torch.empty(1, dtype=torch.float32, device=dev)
+    if grad is None and want_grad:
+        grad = torch.empty((B, Tq, L), dtype=torch.float32, device=dev)
+    st = lib.dsa_indexer_kl(_p(scores), _p(target), _p(idx), B, Tq, L, q_pos0, k, _p(loss_rows), _p(loss_sum),
+                            _p(grad), _stream(stream))
+    _check(st, "dsa_indexer_kl")
+    return loss_rows, loss_sum, grad
+
+
+def indexer_backward(q_idx, k_idx, w, grad, q_pos0: int = 0, dq=None, dk=None, dw=None,
+                     want=("dq", "dk", "dw"), stream=None):
+    """dsa_indexer_backward: fp32 dq [B, Tq, H, d], dk [B, L, d], dw [B, Tq, H]
+    for the incoming gradient grad = d loss / d I (outputs not in `want` and
+    not given are skipped and returned as None)."""
+    lib = load_library()
+    _need_cuda(q_idx, k_idx, w, grad, dq, dk, dw)
+    B, Tq, H, d = q_idx.shape
+    L = k_idx.shape[1]
+    dev = q_idx.device
+    if dq is None and "dq" in want:
+        dq = torch.empty((B, Tq, H, d), dtype=torch.float32, device=dev)
+    if dk is None and "dk" in want:
+        dk = torch.empty((B, L, d), dtype=torch.float32, device=dev)
+    if dw is None and "dw" in want:
+        dw = torch.empty((B, Tq, H), dtype=torch.float32, device=dev)
+    st = lib.dsa_indexer_backward(_p(q_idx), _p(k_idx), _p(w), _p(grad), B, Tq, L, q_pos0, H, d, _dt(q_idx),
+                                  _p(dq), _p(dk), _p(dw), _stream(stream))
+    _check(st, "dsa_indexer_backward")
+    return dq, dk, dw
 
 
 def attn_shape(q, k_cache, v_cache, k: int, scale=None) -> AttnShape:

@@ -306,4 +306,37 @@ dsa_status dsa_forward(const dsa_forward_args *a, void *ws, size_t ws_bytes, dsa
     return from_cuda(launch_attn(ap, s));
 }
 
+dsa_status dsa_indexer_kl(const float *scores, const float *target, const int32_t *idx, int B, int Tq, int L,
+                          int q_pos0, int k, float *loss_rows, float *loss_sum, float *grad, dsa_stream_t stream) {
+    if (!scores || !target || !loss_rows) return DSA_ERR_INVALID_ARG;
+    dsa_status st = check_rows(B, Tq, L, q_pos0);
+    if (st != DSA_OK) return st;
+    if (idx && k < 1) return DSA_ERR_INVALID_ARG;
+    if (!aligned(scores, 4) || !aligned(target, 4) || !aligned(loss_rows, 4) || (idx && !aligned(idx, 4)) ||
+        (loss_sum && !aligned(loss_sum, 4)) || (grad && !aligned(grad, 4)))
+        return DSA_ERR_INVALID_ARG;
+    KlProblem p{scores, target, idx, B, Tq, L, q_pos0, idx ? k : 0, loss_rows, loss_sum, grad};
+    return from_cuda(launch_indexer_kl(p, static_cast<cudaStream_t>(stream)));
+}
+
+dsa_status dsa_indexer_backward(const void *q_idx, const void *k_idx, const float *w, const float *grad, int B,
+                                int Tq, int L, int q_pos0, int H_I, int d_I, dsa_dtype dt, float *dq, float *dk,
+                                float *dw, dsa_stream_t stream) {
+    if (!q_idx || !k_idx || !w || !grad) return DSA_ERR_INVALID_ARG;
+    dsa_status st = check_rows(B, Tq, L, q_pos0);
+    if (st != DSA_OK) return st;
+    if (H_I < 1 || d_I < 1) return DSA_ERR_INVALID_ARG;
+    if (!valid_dtype(dt)) return DSA_ERR_UNSUPPORTED;
+    const size_t eb = dtype_bytes(dt);
+    if (!aligned(q_idx, eb) || !aligned(k_idx, eb) || !aligned(w, 4) || !aligned(grad, 4) ||
+        (dq && !aligned(dq, 4)) || (dk && !aligned(dk, 4)) || (dw && !aligned(dw, 4)))
+        return DSA_ERR_INVALID_ARG;
+    const int lim = smem_limit();
+    if (lim == 0) return DSA_ERR_CUDA;
+    if (indexer_bwd_cuda_core_smem_bytes(H_I, d_I) > (size_t)lim) return DSA_ERR_UNSUPPORTED;
+    if (!dq && !dk && !dw) return DSA_OK;
+    IndexerBwdProblem p{q_idx, k_idx, w, grad, B, Tq, L, q_pos0, H_I, d_I, dt, dq, dk, dw};
+    return from_cuda(launch_indexer_bwd(p, static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

@@ -76,6 +76,33 @@ struct AttnProblem {
 size_t attn_workspace_bytes(const AttnProblem &p);
 cudaError_t launch_attn(const AttnProblem &p, cudaStream_t stream);
 
+// ----------------------------------------------------------------- indexer loss
+struct KlProblem {
+    const float *scores;    // [B, Tq, L]
+    const float *target;    // dense: [B, Tq, L]; restricted: [B, Tq, k]
+    const int32_t *idx;     // null (dense loss) or [B, Tq, k]
+    int B, Tq, L, q_pos0, k;
+    float *loss_rows;       // [B * Tq]
+    float *loss_sum;        // [1] or null
+    float *grad;            // [B, Tq, L] or null
+};
+cudaError_t launch_indexer_kl(const KlProblem &p, cudaStream_t stream);
+
+// ----------------------------------------------------------------- indexer backward
+struct IndexerBwdProblem {
+    const void *q_idx;      // [B, Tq, H, d]
+    const void *k_idx;      // [B, L, d]
+    const float *w;         // [B, Tq, H]
+    const float *grad;      // [B, Tq, L]: d loss / d I
+    int B, Tq, L, q_pos0, H, d;
+    dsa_dtype dt;
+    float *dq;              // [B, Tq, H, d] or null
+    float *dk;              // [B, L, d] or null
+    float *dw;              // [B, Tq, H] or null
+};
+cudaError_t launch_indexer_bwd(const IndexerBwdProblem &p, cudaStream_t stream);
+size_t indexer_bwd_cuda_core_smem_bytes(int H, int d);
+
 // Read and clear the error word of a kernel family with bounded waits
 // (non-zero: some launch gave up on a wait).
 unsigned int indexer_take_device_error();

@@ -174,6 +174,16 @@ def to_device(inputs: dict, device) -> dict:
     return out
 
 
+def target_weights(gen: torch.Generator, shape, sigma: float = 2.0, zero_frac: float = 0.1) -> torch.Tensor:
+    """Non-negative fp32 target weights a[t, s] for the indexer's training
+    loss: log-normal exp(sigma * N(0, 1)), a peaked spread like that of
+    attention weights summed over heads, with a fraction of exact zeros.
+    The loss normalises them itself."""
+    a = torch.exp(sigma * torch.randn(shape, generator=gen, dtype=torch.float32))
+    a[torch.rand(shape, generator=gen) < zero_frac] = 0.0
+    return a
+
+
 def random_score_rows(gen: torch.Generator, n_rows: int, L: int, kind: str) -> torch.Tensor:
     """fp32 score rows for exercising the selector on its own.
 
