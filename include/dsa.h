@@ -322,16 +322,30 @@ dsa_status dsa_indexer_kl(const float *scores, const float *target, const int32_
  *   dk       [B, L, d_I] fp32 or NULL; keys that no query row of the call
  *            reaches (s > q_pos0 + Tq - 1) get 0. Every entry is written.
  *   dw       [B, Tq, H_I] fp32 or NULL.
- * Arithmetic: bf16 inputs with H_I * d_I on the tensor-core path (d_I = 128,
- * H_I = 64) multiply x exactly (bf16 products, fp32 sums) and round G to
- * bf16 for the second product; sums are fp32. Elsewhere every step is fp32.
+ *   ws       at least dsa_indexer_backward_workspace_bytes(...) bytes when dk
+ *            is requested (may be NULL when that is 0).
+ * Paths: bf16 inputs with d_I = 128, H_I in {32, 64, 128}, L a multiple of 4,
+ * 16-byte aligned pointers and at least 128 rows of q_idx and of k_idx run on
+ * the tensor cores: x is exact there (bf16 products, fp32 sums), G is rounded
+ * to bf16 for the second product, sums are fp32. Every other shape runs on
+ * CUDA cores in fp32.
  * Errors: DSA_ERR_INVALID_ARG as dsa_indexer_scores, or a null grad;
- * DSA_ERR_UNSUPPORTED when the fallback's staging does not fit.
+ * DSA_ERR_WORKSPACE when dk is requested and ws is missing or too small;
+ * DSA_ERR_UNSUPPORTED when the CUDA-core path's staging does not fit.
  */
 dsa_status dsa_indexer_backward(const void *q_idx, const void *k_idx, const float *w,
                                 const float *grad, int B, int Tq, int L, int q_pos0,
                                 int H_I, int d_I, dsa_dtype dt,
-                                float *dq, float *dk, float *dw, dsa_stream_t stream);
+                                float *dq, float *dk, float *dw,
+                                void *ws, size_t ws_bytes, dsa_stream_t stream);
+
+/* Workspace dsa_indexer_backward needs when dk is requested (16-byte aligned;
+ * 0 when the shape takes the CUDA-core path or the arguments are invalid).
+ * It holds fp32 partial sums of dk, 64 KB per (128-key tile, chunk of query
+ * rows); the chunks of a tile are summed in a fixed order, so dk is the same
+ * on every call. */
+size_t dsa_indexer_backward_workspace_bytes(int B, int Tq, int L, int q_pos0, int H_I, int d_I,
+                                            dsa_dtype dt);
 
 #ifdef __cplusplus
 }

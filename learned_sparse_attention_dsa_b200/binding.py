@@ -27,7 +27,7 @@ STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED",
 EXPORTED = ("dsa_version", "dsa_kernel_launch_count", "dsa_status_string", "dsa_indexer_scores", "dsa_topk",
             "dsa_topk_workspace_bytes", "dsa_sparse_attn", "dsa_sparse_attn_workspace_bytes",
             "dsa_forward", "dsa_forward_workspace_bytes", "dsa_device_error", "dsa_topk_ex",
-            "dsa_indexer_kl", "dsa_indexer_backward")
+            "dsa_indexer_kl", "dsa_indexer_backward", "dsa_indexer_backward_workspace_bytes")
 
 
 class DSAError(RuntimeError):
@@ -94,8 +94,10 @@ def load_library(path: str = LIB_PATH):
     lib.dsa_device_error.argtypes, lib.dsa_device_error.restype = [vp], ci
     lib.dsa_indexer_kl.argtypes = [vp, vp, vp, ci, ci, ci, ci, ci, vp, vp, vp, vp]
     lib.dsa_indexer_kl.restype = ci
-    lib.dsa_indexer_backward.argtypes = [vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, vp, vp, vp, vp]
+    lib.dsa_indexer_backward.argtypes = [vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, vp, vp, vp, vp, sz, vp]
     lib.dsa_indexer_backward.restype = ci
+    lib.dsa_indexer_backward_workspace_bytes.argtypes = [ci, ci, ci, ci, ci, ci, ci]
+    lib.dsa_indexer_backward_workspace_bytes.restype = sz
     _lib = lib
     return lib
 
@@ -209,8 +211,14 @@ def indexer_kl(scores, target, q_pos0: int = 0, idx=None, loss_rows=None, loss_s
     return loss_rows, loss_sum, grad
 
 
+def indexer_backward_workspace_bytes(q_idx, k_idx, q_pos0: int = 0) -> int:
+    B, Tq, H, d = q_idx.shape
+    return int(load_library().dsa_indexer_backward_workspace_bytes(B, Tq, k_idx.shape[1], q_pos0, H, d,
+                                                                   _dt(q_idx)))
+
+
 def indexer_backward(q_idx, k_idx, w, grad, q_pos0: int = 0, dq=None, dk=None, dw=None,
-                     want=("dq", "dk", "dw"), stream=None):
+                     want=("dq", "dk", "dw"), ws=None, stream=None):
     """dsa_indexer_backward: fp32 dq [B, Tq, H, d], dk [B, L, d], dw [B, Tq, H]
     for the incoming gradient grad = d loss / d I (outputs not in `want` and
     not given are skipped and returned as None)."""
@@ -225,8 +233,10 @@ def indexer_backward(q_idx, k_idx, w, grad, q_pos0: int = 0, dq=None, dk=None, d
         dk = torch.empty((B, L, d), dtype=torch.float32, device=dev)
     if dw is None and "dw" in want:
         dw = torch.empty((B, Tq, H), dtype=torch.float32, device=dev)
+    nbytes = indexer_backward_workspace_bytes(q_idx, k_idx, q_pos0) if dk is not None else 0
+    ws = _workspace(nbytes, dev, ws)
     st = lib.dsa_indexer_backward(_p(q_idx), _p(k_idx), _p(w), _p(grad), B, Tq, L, q_pos0, H, d, _dt(q_idx),
-                                  _p(dq), _p(dk), _p(dw), _stream(stream))
+                                  _p(dq), _p(dk), _p(dw), _p(ws), nbytes, _stream(stream))
     _check(st, "dsa_indexer_backward")
     return dq, dk, dw
 

@@ -203,7 +203,8 @@ uint64_t dsa_kernel_launch_count(void) { return g_launches.load(std::memory_orde
 
 dsa_status dsa_device_error(dsa_stream_t stream) {
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return DSA_ERR_CUDA;
-    unsigned int words = dsa::indexer_take_device_error() | dsa::attn_mla_tc_take_device_error();
+    unsigned int words = dsa::indexer_take_device_error() | dsa::attn_mla_tc_take_device_error() |
+                         dsa::indexer_bwd_take_device_error();
     if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
     return words ? DSA_ERR_TIMEOUT : DSA_OK;
 }
@@ -319,9 +320,19 @@ dsa_status dsa_indexer_kl(const float *scores, const float *target, const int32_
     return from_cuda(launch_indexer_kl(p, static_cast<cudaStream_t>(stream)));
 }
 
+size_t dsa_indexer_backward_workspace_bytes(int B, int Tq, int L, int q_pos0, int H_I, int d_I, dsa_dtype dt) {
+    if (check_rows(B, Tq, L, q_pos0) != DSA_OK || H_I < 1 || d_I < 1 || !valid_dtype(dt)) return 0;
+    // aligned placeholder pointers: the plan depends only on shapes and alignment
+    const void *fake = reinterpret_cast<const void *>(uintptr_t(256));
+    IndexerBwdProblem p{fake, fake, static_cast<const float *>(fake), static_cast<const float *>(fake), B, Tq, L,
+                        q_pos0, H_I, d_I, dt, nullptr, reinterpret_cast<float *>(uintptr_t(256)), nullptr,
+                        nullptr, 0};
+    return indexer_bwd_tc_workspace_bytes(p);
+}
+
 dsa_status dsa_indexer_backward(const void *q_idx, const void *k_idx, const float *w, const float *grad, int B,
                                 int Tq, int L, int q_pos0, int H_I, int d_I, dsa_dtype dt, float *dq, float *dk,
-                                float *dw, dsa_stream_t stream) {
+                                float *dw, void *ws, size_t ws_bytes, dsa_stream_t stream) {
     if (!q_idx || !k_idx || !w || !grad) return DSA_ERR_INVALID_ARG;
     dsa_status st = check_rows(B, Tq, L, q_pos0);
     if (st != DSA_OK) return st;
@@ -334,8 +345,12 @@ dsa_status dsa_indexer_backward(const void *q_idx, const void *k_idx, const floa
     const int lim = smem_limit();
     if (lim == 0) return DSA_ERR_CUDA;
     if (indexer_bwd_cuda_core_smem_bytes(H_I, d_I) > (size_t)lim) return DSA_ERR_UNSUPPORTED;
+    IndexerBwdProblem p{q_idx, k_idx, w, grad, B, Tq, L, q_pos0, H_I, d_I, dt, dq, dk, dw, ws, ws_bytes};
+    if (dk) {
+        const size_t need = indexer_bwd_tc_workspace_bytes(p);
+        if (need > 0 && (!ws || ws_bytes < need || !aligned(ws, 16))) return DSA_ERR_WORKSPACE;
+    }
     if (!dq && !dk && !dw) return DSA_OK;
-    IndexerBwdProblem p{q_idx, k_idx, w, grad, B, Tq, L, q_pos0, H_I, d_I, dt, dq, dk, dw};
     return from_cuda(launch_indexer_bwd(p, static_cast<cudaStream_t>(stream)));
 }
 

@@ -1,13 +1,571 @@
-// Backward pass of the lightning indexer on the tensor cores (tcgen05).
+// Backward pass of the lightning indexer on the 5th-generation tensor cores.
+//
+// For the incoming gradient g = d loss / d I of the indexer's training loss
+// ("DeepSeek Sparse Attention: Learned Token Selection from Scratch" §5.4,
+// §6.2; §6.4: it reaches only the indexer) and the score of §2.1,
+// I[t,s] = sum_j w[t,j] ReLU(x[t,j,s]), x[t,j,s] = q[t,j] . k[s]:
+//   G[t,j,s] = g[t,s] w[t,j] [x[t,j,s] > 0]
+//   dq[t,j]  = sum_{s<=t} G[t,j,s] k[s]           dw[t,j] = sum_{s<=t} g[t,s] ReLU(x[t,j,s])
+//   dk[s]    = sum_{t>=s} sum_j G[t,j,s] q[t,j]
+//
+// Both products are GEMMs around an elementwise step, so one kernel serves
+// both sides with the roles of the operands swapped:
+//   query side (dq, dw): a group of 128 / H queries (128 rows (t, j)) stays
+//       resident; 128-key tiles stream past it.
+//       MMA 1  X[(t,j), s]  = Q[(t,j), :] . K[s, :]        M=128 N=128 K=128
+//       epilogue  G = g w [X > 0] in bf16 into TMEM, dw += g ReLU(X) in fp32
+//       MMA 2  dQ[(t,j), :] += G[(t,j), s] K[s, :]          M=128 N=128 K=128
+//   key side (dk): a 128-key tile stays resident; query groups stream past.
+//       MMA 1  X[s, (t,j)]  = K[s, :] . Q[(t,j), :]
+//       epilogue  G[s, (t,j)] as above
+//       MMA 2  dK[s, :] += G[s, (t,j)] Q[(t,j), :]
+// MMA 2 reads G from TMEM (A operand) and the streamed tile a second time, as
+// an MN-major B operand: a 128-row tile of 128-byte swizzled rows is K-major
+// for MMA 1 (rows along N) and MN-major for MMA 2 (rows along K), so one copy
+// in shared memory feeds both. x is exact (integer-valued bf16, fp32 sums);
+// G is rounded to bf16 for MMA 2; sums are fp32.
+//
+// Warp roles (320 threads, one CTA per SM, persistent over work units):
+//   warp 0     TMA: the resident tile of each unit (two buffers), streamed
+//              tiles through a 4-stage ring.
+//   warp 1     TMEM owner; one thread issues the MMAs: MMA 1 of tile n+1
+//              before MMA 2 of tile n, so the epilogue of one tile overlaps
+//              the tensor core's work on its neighbours.
+//   warps 2-9  epilogue: two warps per TMEM lane quarter, each taking 64 of
+//              the 128 columns of X and of the accumulator.
+// TMEM: X in two buffers [0, 256), G in two buffers [256, 384) (two bf16 per
+// column), the accumulator [384, 512).
+// Work: query side, one unit per query group (longest causal range first);
+// key side, one unit per (key tile, chunk of query groups), each chunk's
+// partial dK written to a workspace slot and the slots of a key tile summed
+// in a fixed order by indexer_bwd_reduce_kernel (the same result every call).
+// Every mbarrier wait is bounded; on a timeout the CTA records an error word,
+// waits for its own MMAs and copies, frees TMEM and returns.
+#include <math.h>
+
+#include <cuda.h>
+
 #include "common.cuh"
 #include "internal.h"
+#include "sm100.cuh"
 
 namespace dsa {
 
-cudaError_t launch_indexer_bwd_tc(const IndexerBwdProblem &p, cudaStream_t stream, bool *taken) {
-    (void)p;
-    (void)stream;
+namespace {
+
+using namespace sm100;
+
+constexpr int kRows = 128;                  // MMA M and rows of every tile
+constexpr int kD = 128;                     // d_I
+constexpr uint32_t kBox = kRows * 128;      // 128 rows x 64 bf16 columns (128-byte swizzle)
+constexpr uint32_t kTile = 2 * kBox;        // 128 rows x 128 columns
+constexpr int kStages = 4;
+constexpr int kResBufs = 2;
+constexpr int kEpiThreads = 256;
+constexpr int kThreads = 64 + kEpiThreads;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColX = 0;               // 2 x 128
+constexpr uint32_t kColG = 256;             // 2 x 64
+constexpr uint32_t kColAcc = 384;           // 128
+constexpr uint32_t kIdescMnMajorB = 1u << 16;
+// barriers: res_full/empty[2], st_full/empty[4], x_full/empty[2], g_full/empty[2], acc_full, acc_empty, drain
+constexpr int kNumBars = 2 * kResBufs + 2 * kStages + 4 + 4 + 3;
+constexpr size_t kSmem = 1024 + (size_t)kResBufs * kTile + (size_t)kStages * kTile + kNumBars * 8 + 16;
+static_assert(kSmem <= 232448, "shared memory budget");
+
+__device__ unsigned int g_indexer_bwd_error = 0;  // 1 = a bounded wait gave up
+
+struct Params {
+    const float *w, *grad;
+    int B, Tq, L, q_pos0, H, QPG;  // QPG = 128 / H queries per group
+    int ngroups;                    // query groups per batch entry
+    int nkt;                        // key tiles per batch entry
+    int nchunks, C;                 // key side: chunks of C groups
+    int units;
+    float *dq, *dw;                 // query side
+    float *part;                    // key side: [B * nchunks * nkt][128][128]
+};
+
+struct Unit {
+    int b;
+    int g0, g1;    // query groups [g0, g1) (query side: one group)
+    int kt0, kt1;  // key tiles [kt0, kt1) (key side: one tile)
+    int slot;      // key side: partial slot
+};
+
+__device__ __forceinline__ int first_group(const Params &p, int kt) {
+    // first query group holding a query at t >= kt * 128
+    const int i = kt * kRows - p.q_pos0;
+    return i <= 0 ? 0 : i / p.QPG;
+}
+
+template <bool KEY_SIDE>
+__device__ __forceinline__ bool decode_unit(int u, const Params &p, Unit &un) {
+    if (!KEY_SIDE) {
+        const int b = u % p.B;
+        const int g = p.ngroups - 1 - u / p.B;
+        const int i0 = g * p.QPG;
+        const int qcount = min(p.QPG, p.Tq - i0);
+        const int t_last = p.q_pos0 + i0 + qcount - 1;
+        un.b = b;
+        un.g0 = g;
+        un.g1 = g + 1;
+        un.kt0 = 0;
+        un.kt1 = t_last / kRows + 1;
+        un.slot = 0;
+        return true;
+    }
+    const int kt = u % p.nkt;
+    const int rest = u / p.nkt;
+    const int c = rest % p.nchunks;
+    const int b = rest / p.nchunks;
+    const int gf = first_group(p, kt);
+    const int g0 = max(gf, c * p.C);
+    const int g1 = min(p.ngroups, (c + 1) * p.C);
+    if (g0 >= g1) return false;
+    un.b = b;
+    un.g0 = g0;
+    un.g1 = g1;
+    un.kt0 = kt;
+    un.kt1 = kt + 1;
+    un.slot = u;
+    return true;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+template <bool KEY_SIDE>
+__global__ void __launch_bounds__(kThreads, 1)
+indexer_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                      const Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *res_sm = smem;
+    uint8_t *st_sm = res_sm + kResBufs * kTile;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(st_sm + kStages * kTile);
+    uint64_t *res_full = bars;
+    uint64_t *res_empty = res_full + kResBufs;
+    uint64_t *st_full = res_empty + kResBufs;
+    uint64_t *st_empty = st_full + kStages;
+    uint64_t *x_full = st_empty + kStages;
+    uint64_t *x_empty = x_full + 2;
+    uint64_t *g_full = x_empty + 2;
+    uint64_t *g_empty = g_full + 2;
+    uint64_t *acc_full = g_empty + 2;
+    uint64_t *acc_empty = acc_full + 1;
+    uint64_t *drain = acc_empty + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    // the resident tile comes from K on the key side, from Q on the query side
+    const CUtensorMap *tm_res = KEY_SIDE ? &tm_k : &tm_q;
+    const CUtensorMap *tm_str = KEY_SIDE ? &tm_q : &tm_k;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kResBufs; ++s) {
+            mbar_init(&res_full[s], 1);
+            mbar_init(&res_empty[s], 1);
+        }
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&st_full[s], 1);
+            mbar_init(&st_empty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&x_full[s], 1);
+            mbar_init(&x_empty[s], kEpiThreads);
+            mbar_init(&g_full[s], kEpiThreads);
+            mbar_init(&g_empty[s], 1);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, kEpiThreads);
+        mbar_init(drain, 1);
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    bool ok = true;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------------ TMA producer
+            prefetch_tensor_map(&tm_q);
+            prefetch_tensor_map(&tm_k);
+            int sb = 0, rb = 0;
+            uint32_t sph = 0, rph = 0;
+            int st_armed[kStages], res_armed[kResBufs];  // parity of each buffer's last armed phase, or -1
+            for (int s = 0; s < kStages; ++s) st_armed[s] = -1;
+            for (int s = 0; s < kResBufs; ++s) res_armed[s] = -1;
+            for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
+                Unit un;
+                if (!decode_unit<KEY_SIDE>(u, p, un)) continue;
+                if (!mbar_wait(&res_empty[rb], rph ^ 1u)) { ok = false; break; }
+                mbar_arrive_expect_tx(&res_full[rb], kTile);
+                res_armed[rb] = (int)rph;
+                const int rrow = KEY_SIDE ? un.b * p.L + un.kt0 * kRows : (un.b * p.Tq + un.g0 * p.QPG) * p.H;
+                tma_load_2d(res_sm + rb * kTile, tm_res, &res_full[rb], 0, rrow);
+                tma_load_2d(res_sm + rb * kTile + kBox, tm_res, &res_full[rb], 64, rrow);
+                if (++rb == kResBufs) { rb = 0; rph ^= 1u; }
+                const int n0 = KEY_SIDE ? un.g0 : un.kt0, n1 = KEY_SIDE ? un.g1 : un.kt1;
+                for (int n = n0; n < n1; ++n) {
+                    if (!mbar_wait(&st_empty[sb], sph ^ 1u)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&st_full[sb], kTile);
+                    st_armed[sb] = (int)sph;
+                    const int srow = KEY_SIDE ? (un.b * p.Tq + n * p.QPG) * p.H : un.b * p.L + n * kRows;
+                    tma_load_2d(st_sm + sb * kTile, tm_str, &st_full[sb], 0, srow);
+                    tma_load_2d(st_sm + sb * kTile + kBox, tm_str, &st_full[sb], 64, srow);
+                    if (++sb == kStages) { sb = 0; sph ^= 1u; }
+                }
+            }
+            // no copy may still be landing when the CTA exits
+            for (int s = 0; s < kStages; ++s)
+                if (st_armed[s] >= 0 && !mbar_wait(&st_full[s], (uint32_t)st_armed[s])) ok = false;
+            for (int s = 0; s < kResBufs; ++s)
+                if (res_armed[s] >= 0 && !mbar_wait(&res_full[s], (uint32_t)res_armed[s])) ok = false;
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ------------------------------------------------ MMA issuer
+            const uint32_t idesc1 = idesc_bf16_f32(kRows, kRows);
+            const uint32_t idesc2 = idesc_bf16_f32(kRows, kD) | kIdescMnMajorB;
+            int sb = 0, rb = 0, xb = 0;
+            uint32_t sph = 0, rph = 0, xph = 0, aph = 0;
+            for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
+                Unit un;
+                if (!decode_unit<KEY_SIDE>(u, p, un)) continue;
+                if (!mbar_wait(&res_full[rb], rph)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t a_base = smem_addr(res_sm + rb * kTile);
+                const int ntiles = KEY_SIDE ? un.g1 - un.g0 : un.kt1 - un.kt0;
+                int prev_sb = -1, prev_xb = 0;
+                uint32_t prev_xph = 0;
+                for (int n = 0; n <= ntiles && ok; ++n) {
+                    if (n < ntiles) {
+                        // MMA 1 of tile n: X = A . B^T
+                        if (!mbar_wait(&st_full[sb], sph)) { ok = false; break; }
+                        if (!mbar_wait(&x_empty[xb], xph ^ 1u)) { ok = false; break; }
+                        tc_fence_after();
+                        const uint32_t b_base = smem_addr(st_sm + sb * kTile);
+                        const uint32_t d = tmem + kColX + (uint32_t)(xb * 128);
+#pragma unroll
+                        for (int h = 0; h < 2; ++h)
+#pragma unroll
+                            for (int kk = 0; kk < 4; ++kk)
+                                mma_f16_ss(d, smem_desc_k_sw128(a_base + h * kBox + kk * 32),
+                                           smem_desc_k_sw128(b_base + h * kBox + kk * 32), idesc1, (h | kk) != 0);
+                        mma_commit(&x_full[xb]);
+                    }
+                    if (n > 0) {
+                        // MMA 2 of tile n-1: acc += G (TMEM) . B (MN-major)
+                        if (!mbar_wait(&g_full[prev_xb], prev_xph)) { ok = false; break; }
+                        if (n == 1 && !mbar_wait(acc_empty, aph ^ 1u)) { ok = false; break; }
+                        tc_fence_after();
+                        const uint32_t b_base = smem_addr(st_sm + prev_sb * kTile);
+                        const uint32_t a_tm = tmem + kColG + (uint32_t)(prev_xb * 64);
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk)
+                            mma_f16_ts(tmem + kColAcc, a_tm + (uint32_t)(kk * 8),
+                                       smem_desc_mn_sw128(b_base + kk * 2048, kBox), idesc2,
+                                       (n > 1 || kk > 0) ? 1u : 0u);
+                        mma_commit(&st_empty[prev_sb]);  // the streamed tile is no longer read
+                        mma_commit(&g_empty[prev_xb]);
+                    }
+                    if (n < ntiles) {
+                        prev_sb = sb;
+                        prev_xb = xb;
+                        prev_xph = xph;
+                        if (++sb == kStages) { sb = 0; sph ^= 1u; }
+                        if (++xb == 2) { xb = 0; xph ^= 1u; }
+                    }
+                }
+                if (!ok) break;
+                mma_commit(acc_full);
+                aph ^= 1u;
+                mma_commit(&res_empty[rb]);
+                if (++rb == kResBufs) { rb = 0; rph ^= 1u; }
+            }
+            // every MMA issued here has finished before TMEM is freed
+            mma_commit(drain);
+            if (!mbar_wait(drain, 0)) ok = false;
+        }
+    } else {
+        // ---------------------------------------------------- epilogue
+        const int quarter = warp & 3;
+        const int half = (warp - 2) >> 2;          // columns [64 half, 64 half + 64)
+        const int r = quarter * 32 + lane;         // TMEM lane: resident row
+        const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+        int xb = 0;
+        uint32_t xph = 0, aph = 0;
+        for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
+            Unit un;
+            if (!decode_unit<KEY_SIDE>(u, p, un)) continue;
+            const int ntiles = KEY_SIDE ? un.g1 - un.g0 : un.kt1 - un.kt0;
+            // query side: this lane's (query, head) and its weight
+            int qi = 0, t_row = 0, row = 0;
+            float w_r = 0.f, dw_acc = 0.f;
+            if (!KEY_SIDE) {
+                qi = r / p.H;
+                const int i = un.g0 * p.QPG + qi;
+                row = un.b * p.Tq + i;
+                t_row = p.q_pos0 + i;
+                if (i < p.Tq) {
+                    w_r = p.w[(size_t)row * p.H + (r - qi * p.H)];
+                } else {
+                    t_row = -1;  // no such query: G = 0
+                }
+            }
+            for (int n = 0; n < ntiles && ok; ++n) {
+                if (!mbar_wait(&x_full[xb], xph)) { ok = false; break; }
+                tc_fence_after();
+                uint32_t xr[64];
+                const uint32_t xaddr = tmem + lane_addr + kColX + (uint32_t)(xb * 128 + half * 64);
+                tmem_ld_32x32b_x32(xaddr, xr);
+                tmem_ld_32x32b_x32(xaddr + 32, xr + 32);
+                tmem_ld_wait();
+                tc_fence_before();
+                mbar_arrive(&x_empty[xb]);
+                uint32_t gp[32];
+                if (!KEY_SIDE) {
+                    // columns = keys s0 + 64 half + c; g[t, s] shared by the warp's lanes
+                    const int s_base = (un.kt0 + n) * kRows + half * 64;
+                    const float *grow = p.grad + (size_t)(row < p.B * p.Tq ? row : 0) * p.L;
+#pragma unroll
+                    for (int c4 = 0; c4 < 16; ++c4) {
+                        const int s = s_base + 4 * c4;
+                        float4 gv = make_float4(0.f, 0.f, 0.f, 0.f);
+                        if (s <= t_row) gv = __ldg(reinterpret_cast<const float4 *>(grow + s));
+                        const float gs[4] = {s <= t_row ? gv.x : 0.f, s + 1 <= t_row ? gv.y : 0.f,
+                                             s + 2 <= t_row ? gv.z : 0.f, s + 3 <= t_row ? gv.w : 0.f};
+                        float G[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float x = __uint_as_float(xr[4 * c4 + e]);
+                            G[e] = x > 0.f ? gs[e] * w_r : 0.f;
+                            dw_acc = fmaf(gs[e], fmaxf(x, 0.f), dw_acc);
+                        }
+                        gp[2 * c4] = pack_bf16x2(G[0], G[1]);
+                        gp[2 * c4 + 1] = pack_bf16x2(G[2], G[3]);
+                    }
+                } else {
+                    // lanes = keys s; columns = (query, head) pairs of group g
+                    const int g = un.g0 + n;
+                    const int s = un.kt0 * kRows + r;
+                    const int c_base = half * 64;
+                    // the (at most two) queries of this half's columns
+                    const int qa = c_base / p.H, qb = (c_base + 63) / p.H;
+                    float g_q[2] = {0.f, 0.f};
+#pragma unroll
+                    for (int z = 0; z < 2; ++z) {
+                        const int qz = z == 0 ? qa : qb;
+                        const int i = g * p.QPG + qz;
+                        if (i < p.Tq && s <= p.q_pos0 + i)
+                            g_q[z] = p.grad[(size_t)(un.b * p.Tq + i) * p.L + s];
+                    }
+#pragma unroll
+                    for (int c4 = 0; c4 < 16; ++c4) {
+                        const int cc = c_base + 4 * c4;  // 4 columns of one query (H is a multiple of 4)
+                        const int qz = cc / p.H;
+                        const int i = g * p.QPG + qz;
+                        const float gq = qz == qa ? g_q[0] : g_q[1];
+                        float4 wv = make_float4(0.f, 0.f, 0.f, 0.f);
+                        if (i < p.Tq)
+                            wv = __ldg(reinterpret_cast<const float4 *>(p.w + (size_t)(un.b * p.Tq + i) * p.H +
+                                                                        (cc - qz * p.H)));
+                        const float ws[4] = {wv.x, wv.y, wv.z, wv.w};
+                        float G[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float x = __uint_as_float(xr[4 * c4 + e]);
+                            G[e] = x > 0.f ? gq * ws[e] : 0.f;
+                        }
+                        gp[2 * c4] = pack_bf16x2(G[0], G[1]);
+                        gp[2 * c4 + 1] = pack_bf16x2(G[2], G[3]);
+                    }
+                }
+                if (!mbar_wait(&g_empty[xb], xph ^ 1u)) { ok = false; break; }
+                tc_fence_after();
+                tmem_st_32x32b_x32(tmem + lane_addr + kColG + (uint32_t)(xb * 64 + half * 32), gp);
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(&g_full[xb]);
+                if (++xb == 2) { xb = 0; xph ^= 1u; }
+            }
+            if (!ok) break;
+            // ---- the unit's accumulator
+            if (!mbar_wait(acc_full, aph)) { ok = false; break; }
+            tc_fence_after();
+            uint32_t ar[64];
+            const uint32_t aaddr = tmem + lane_addr + kColAcc + (uint32_t)(half * 64);
+            tmem_ld_32x32b_x32(aaddr, ar);
+            tmem_ld_32x32b_x32(aaddr + 32, ar + 32);
+            tmem_ld_wait();
+            tc_fence_before();
+            mbar_arrive(acc_empty);
+            aph ^= 1u;
+            float *dst = nullptr;
+            if (KEY_SIDE) {
+                dst = p.part + ((size_t)un.slot * kRows + r) * kD + half * 64;
+            } else if (t_row >= 0) {
+                if (p.dq) dst = p.dq + ((size_t)row * p.H + (r - qi * p.H)) * kD + half * 64;
+                // the two halves' sums land on a zeroed word: (0 + a) + b == (0 + b) + a
+                if (p.dw) atomicAdd(p.dw + (size_t)row * p.H + (r - qi * p.H), dw_acc);
+            }
+            if (dst) {
+                float4 *d4 = reinterpret_cast<float4 *>(dst);
+#pragma unroll
+                for (int c4 = 0; c4 < 16; ++c4)
+                    d4[c4] = make_float4(__uint_as_float(ar[4 * c4]), __uint_as_float(ar[4 * c4 + 1]),
+                                         __uint_as_float(ar[4 * c4 + 2]), __uint_as_float(ar[4 * c4 + 3]));
+            }
+        }
+    }
+
+    if (!ok) atomicOr(&g_indexer_bwd_error, 1u);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// dk[b, kt * 128 + r, :] = sum over the key tile's chunks, in chunk order.
+__global__ void __launch_bounds__(256)
+indexer_bwd_reduce_kernel(const float *__restrict__ part, const Params p, float *__restrict__ dk) {
+    const int kt = blockIdx.x, b = blockIdx.y;
+    const int gf = first_group(p, kt);
+    const int c0 = gf >= p.ngroups ? p.nchunks : gf / p.C;
+    const int rows = min(kRows, p.L - kt * kRows);
+    for (int v = threadIdx.x; v < rows * (kD / 4); v += blockDim.x) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int c = c0; c < p.nchunks; ++c) {
+            const size_t slot = ((size_t)b * p.nchunks + c) * p.nkt + kt;
+            const float4 x = reinterpret_cast<const float4 *>(part + slot * kRows * kD)[v];
+            acc.x += x.x;
+            acc.y += x.y;
+            acc.z += x.z;
+            acc.w += x.w;
+        }
+        reinterpret_cast<float4 *>(dk + ((size_t)b * p.L + (size_t)kt * kRows) * kD)[v] = acc;
+    }
+}
+
+// The problem shapes this path takes, and its parameters.
+bool plan(const IndexerBwdProblem &pr, const DeviceInfo &info, Params &p) {
+    if (pr.dt != DSA_BF16 || pr.d != kD) return false;
+    if (!(pr.H == 32 || pr.H == 64 || pr.H == 128)) return false;
+    if (info.cc_major != 10 || (size_t)info.max_smem_optin < kSmem) return false;
+    if (((uintptr_t)pr.q_idx | (uintptr_t)pr.k_idx | (uintptr_t)pr.w | (uintptr_t)pr.grad) % 16 != 0) return false;
+    if ((pr.dq && (uintptr_t)pr.dq % 16) || (pr.dk && (uintptr_t)pr.dk % 16)) return false;
+    if (pr.L % 4 != 0) return false;  // 16-byte rows of g
+    // a TMA box may not be taller than the tensor it reads
+    if ((long long)pr.B * pr.Tq * pr.H < kRows || (long long)pr.B * pr.L < kRows) return false;
+    p.w = pr.w;
+    p.grad = pr.grad;
+    p.B = pr.B;
+    p.Tq = pr.Tq;
+    p.L = pr.L;
+    p.q_pos0 = pr.q_pos0;
+    p.H = pr.H;
+    p.QPG = kRows / pr.H;
+    p.ngroups = ceil_div(pr.Tq, p.QPG);
+    p.nkt = ceil_div(pr.L, kRows);
+    p.dq = pr.dq;
+    p.dw = pr.dw;
+    p.part = nullptr;
+    // key side: chunks of C groups, about three units per SM in total
+    long long visits = 0;  // (key tile, group) pairs per batch entry
+    for (int kt = 0; kt < p.nkt; ++kt) {
+        const int i = kt * kRows - pr.q_pos0;
+        const int gf = i <= 0 ? 0 : i / p.QPG;
+        if (gf < p.ngroups) visits += p.ngroups - gf;
+    }
+    long long C = (visits * pr.B + 3LL * info.sm_count - 1) / (3LL * info.sm_count);
+    if (C < 8) C = 8;
+    if (C > p.ngroups) C = p.ngroups;
+    p.C = (int)C;
+    p.nchunks = ceil_div(p.ngroups, p.C);
+    return true;
+}
+
+size_t part_bytes(const Params &p) {
+    return (size_t)p.B * p.nchunks * p.nkt * kRows * kD * sizeof(float);
+}
+
+}  // namespace
+
+unsigned int indexer_bwd_take_device_error() {
+    unsigned int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_indexer_bwd_error, sizeof(v)) != cudaSuccess) return 0;
+    cudaMemcpyToSymbol(g_indexer_bwd_error, &zero, sizeof(zero));
+    return v;
+}
+
+size_t indexer_bwd_tc_workspace_bytes(const IndexerBwdProblem &pr) {
+    DeviceInfo info;
+    if (device_info(&info) != cudaSuccess) return 0;
+    Params p;
+    if (!plan(pr, info, p)) return 0;
+    return part_bytes(p);
+}
+
+cudaError_t launch_indexer_bwd_tc(const IndexerBwdProblem &pr, cudaStream_t stream, bool *taken) {
     *taken = false;
+    DeviceInfo info;
+    cudaError_t err = device_info(&info);
+    if (err != cudaSuccess) return err;
+    Params p;
+    if (!plan(pr, info, p)) return cudaSuccess;
+    if (pr.dk && (pr.ws == nullptr || pr.ws_bytes < part_bytes(p) || (uintptr_t)pr.ws % 16 != 0))
+        return cudaSuccess;  // no room for the key side's partials: the CUDA-core path takes the call
+    CUtensorMap tm_q, tm_k;
+    if (!make_map_bf16_sw128(&tm_q, pr.q_idx, (uint64_t)pr.B * pr.Tq * pr.H, kD, kD * 2, kRows) ||
+        !make_map_bf16_sw128(&tm_k, pr.k_idx, (uint64_t)pr.B * pr.L, kD, kD * 2, kRows))
+        return cudaSuccess;
+    *taken = true;
+    if (pr.dq || pr.dw) {
+        if (pr.dw && (err = cudaMemsetAsync(pr.dw, 0, (size_t)pr.B * pr.Tq * pr.H * sizeof(float), stream)) !=
+                         cudaSuccess)
+            return err;
+        Params q = p;
+        q.units = p.B * p.ngroups;
+        auto kern = indexer_bwd_tc_kernel<false>;
+        if ((err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem)) !=
+            cudaSuccess)
+            return err;
+        const int grid = q.units < info.sm_count ? q.units : info.sm_count;
+        kern<<<grid, kThreads, kSmem, stream>>>(tm_q, tm_k, q);
+        count_launch();
+        if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    }
+    if (pr.dk) {
+        Params k = p;
+        k.part = static_cast<float *>(pr.ws);
+        const long long units = (long long)p.B * p.nchunks * p.nkt;
+        if (units > 0x7fffffffLL) return cudaErrorInvalidValue;
+        k.units = (int)units;
+        auto kern = indexer_bwd_tc_kernel<true>;
+        if ((err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem)) !=
+            cudaSuccess)
+            return err;
+        const int grid = k.units < info.sm_count ? k.units : info.sm_count;
+        kern<<<grid, kThreads, kSmem, stream>>>(tm_q, tm_k, k);
+        count_launch();
+        if ((err = cudaGetLastError()) != cudaSuccess) return err;
+        indexer_bwd_reduce_kernel<<<dim3(p.nkt, p.B), 256, 0, stream>>>(k.part, k, pr.dk);
+        count_launch();
+        if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    }
     return cudaSuccess;
 }
 

@@ -99,13 +99,18 @@ struct IndexerBwdProblem {
     float *dq;              // [B, Tq, H, d] or null
     float *dk;              // [B, L, d] or null
     float *dw;              // [B, Tq, H] or null
+    void *ws;               // tensor-core path: partial dk sums
+    size_t ws_bytes;
 };
 cudaError_t launch_indexer_bwd(const IndexerBwdProblem &p, cudaStream_t stream);
 size_t indexer_bwd_cuda_core_smem_bytes(int H, int d);
+// Workspace the tensor-core path needs for this problem (0: it does not take it).
+size_t indexer_bwd_tc_workspace_bytes(const IndexerBwdProblem &p);
 
 // Read and clear the error word of a kernel family with bounded waits
 // (non-zero: some launch gave up on a wait).
 unsigned int indexer_take_device_error();
 unsigned int attn_mla_tc_take_device_error();
+unsigned int indexer_bwd_take_device_error();
 
 }  // namespace dsa

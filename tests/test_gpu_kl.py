@@ -242,3 +242,30 @@ def test_indexer_backward_partial_outputs(cuda):
     assert torch.equal(dk, dk2) and torch.equal(dq, dq2) and torch.equal(dw, dw2)
     # keys after the last query row receive nothing
     assert not dk[:, wl.q_pos0 + wl.Tq:].any()
+
+
+@pytest.mark.parametrize("name", ["prefill8k"])
+def test_indexer_backward_full_size_sampled(cuda, name):
+    """The training step's backward at full size (dense warm-up loss on the
+    indexer's own scores, then dq, dk, dw on the tensor cores), checked on
+    sampled query rows and keys against the oracle (G rounded to bf16:
+    2^-8 of the absolute sums)."""
+    wl = WORKLOADS[name]
+    cpu = make_inputs(wl)
+    dev = to_device(cpu, "cuda")
+    scores = binding.indexer_scores(dev["q_idx"], dev["k_idx"], dev["w"], wl.q_pos0)
+    gen = torch.Generator().manual_seed(77)
+    target = target_weights(gen, (wl.B, wl.Tq, wl.L)).cuda()
+    _, _, grad = binding.indexer_kl(scores, target, wl.q_pos0, want_sum=False)
+    del scores, target
+    dq, dk, dw = binding.indexer_backward(dev["q_idx"], dev["k_idx"], dev["w"], grad, wl.q_pos0)
+    binding.device_error()
+    n = wl.Tq
+    rows = np.array([0, 1, 127, 128, n // 2 + 3, n - 2, n - 1])
+    keys = np.array([0, 5, 127, 128, n // 3, n - 129, n - 1])
+    g_rows = grad[0, torch.from_numpy(rows)].cpu().numpy()
+    # the oracle needs g only on the sampled rows (dq, dw) and columns (dk)
+    g = np.zeros((1, wl.Tq, wl.L), dtype=np.float32)
+    g[0, rows] = g_rows
+    g[0][:, keys] = grad[0][:, torch.from_numpy(keys)].cpu().numpy()
+    _check_backward(wl, cpu, g, dq, dk, dw, rows=rows, keys=keys, rel=2.0 ** -8)
