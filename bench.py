@@ -566,6 +566,256 @@ def run_stage(args, wl):
                       "ms_per_call": e0.elapsed_time(e1) / args.steps}))
 
 
+# ------------------------------------------------------------------ training side
+
+TRAIN_METRIC = ("indexer training tokens/s (scores, dense KL loss and backward); "
+                "% tensor/HBM roofline per stage")
+
+
+def train_work(wl):
+    """Algorithmic bytes and flops per training step, per stage.
+
+    scores:   as the forward indexer stage (2 H d flops per causal pair).
+    kl:       reads one fp32 score and one fp32 target weight per causal pair,
+              writes the fp32 gradient of every (row, key) entry (zeros above
+              the diagonal) and one loss per row.
+    backward: two products per side (x recomputed, then G times the other
+              operand) on the query side (dq, dw) and on the key side (dk):
+              8 H d flops per causal pair; reads q, k, w and one fp32
+              gradient per causal pair, writes dq, dk, dw in fp32.
+    """
+    rows = wl.B * wl.Tq
+    pairs = wl.causal_pairs()
+    eb = 2
+    idx_bytes = (wl.B * wl.L * wl.d_I * eb + rows * wl.H_I * wl.d_I * eb + rows * wl.H_I * 4 + pairs * 4)
+    kl_bytes = pairs * 8 + rows * wl.L * 4 + rows * 4
+    bwd_bytes = (wl.B * wl.L * wl.d_I * eb + rows * wl.H_I * wl.d_I * eb + rows * wl.H_I * 4 + pairs * 4
+                 + rows * wl.H_I * wl.d_I * 4 + wl.B * wl.L * wl.d_I * 4 + rows * wl.H_I * 4)
+    return {"scores": (idx_bytes, 2.0 * wl.H_I * wl.d_I * pairs), "kl": (kl_bytes, 0.0),
+            "backward": (bwd_bytes, 8.0 * wl.H_I * wl.d_I * pairs)}
+
+
+def _train_buffers(wl, dev, binding):
+    device = dev["q_idx"].device
+    f32 = dict(dtype=torch.float32, device=device)
+    bufs = {
+        "scores": torch.empty((wl.B, wl.Tq, wl.L), **f32),
+        "grad": torch.empty((wl.B, wl.Tq, wl.L), **f32),
+        "loss_rows": torch.empty(wl.B * wl.Tq, **f32),
+        "loss_sum": torch.empty(1, **f32),
+        "dq": torch.empty((wl.B, wl.Tq, wl.H_I, wl.d_I), **f32),
+        "dk": torch.empty((wl.B, wl.L, wl.d_I), **f32),
+        "dw": torch.empty((wl.B, wl.Tq, wl.H_I), **f32),
+    }
+    nbytes = binding.indexer_backward_workspace_bytes(dev["q_idx"], dev["k_idx"], wl.q_pos0)
+    bufs["ws"] = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=device)
+    return bufs
+
+
+def _train_calls(wl, dev, target, bufs, binding):
+    def scores():
+        binding.indexer_scores(dev["q_idx"], dev["k_idx"], dev["w"], wl.q_pos0, scores=bufs["scores"])
+
+    def kl():
+        binding.indexer_kl(bufs["scores"], target, wl.q_pos0, loss_rows=bufs["loss_rows"],
+                           loss_sum=bufs["loss_sum"], grad=bufs["grad"])
+
+    def backward():
+        binding.indexer_backward(dev["q_idx"], dev["k_idx"], dev["w"], bufs["grad"], wl.q_pos0, dq=bufs["dq"],
+                                 dk=bufs["dk"], dw=bufs["dw"], ws=bufs["ws"])
+
+    return {"scores": scores, "kl": kl, "backward": backward}
+
+
+def time_train_oracle(wl, cpu, target, n_rows: int, nthreads: int = 0):
+    """The oracle on a sample: scores, loss and dq/dw of n_rows query rows,
+    dk of n_rows keys (rows and keys spread evenly). Returns (seconds, rows,
+    keys); a full step is rows_total / rows times the row part plus
+    keys_total / keys times the key part, both already in the seconds."""
+    import oracle
+    from oracle import kl as okl
+
+    def bits(t):
+        t = t.contiguous()
+        return t.view(torch.int16).numpy().view(np.uint16) if t.dtype == torch.bfloat16 else t.numpy()
+
+    total = wl.B * wl.Tq
+    flat = np.linspace(0, total - 1, num=min(n_rows, total)).round().astype(np.int64)
+    rb, ri = (flat // wl.Tq).astype(np.int32), (flat % wl.Tq).astype(np.int32)
+    rt = ri + wl.q_pos0
+    q_all, k_all, w_all = bits(cpu["q_idx"]), bits(cpu["k_idx"]), cpu["w"].numpy()
+    tg = target.numpy()
+    t0 = time.perf_counter()
+    sc = oracle.indexer_rows(q_all[rb, ri], w_all[rb, ri], k_all, rb, rt, nthreads)
+    _, g = okl.kl_rows(sc, tg[rb, ri], rt)
+    grad = np.zeros((wl.B, wl.Tq, wl.L), dtype=np.float64) if total * wl.L <= 1 << 26 else None
+    if grad is not None:
+        grad[rb, ri] = g
+        okl.indexer_backward_rows(q_all, k_all, w_all, grad, rb, rt, ri)
+    t_rows = time.perf_counter() - t0
+    # key part: dk of sampled keys needs g[t, s] for every t >= s of those keys
+    keys = np.linspace(0, wl.B * wl.L - 1, num=min(n_rows, wl.B * wl.L)).round().astype(np.int64)
+    kb, ks = keys // wl.L, keys % wl.L
+    t1 = time.perf_counter()
+    gk = np.zeros((wl.B, wl.Tq, wl.L), dtype=np.float64) if total * wl.L <= 1 << 26 else None
+    if gk is not None:
+        okl.indexer_backward_keys(q_all, k_all, w_all, gk, kb, ks, wl.q_pos0)
+    t_keys = time.perf_counter() - t1
+    sec = t_rows * total / len(flat) + t_keys * (wl.B * wl.L) / len(keys)
+    return sec, len(flat), len(keys), t_rows + t_keys
+
+
+def run_train(args, wl):
+    from learned_sparse_attention_dsa_b200 import binding
+    from learned_sparse_attention_dsa_b200.inputs import target_weights
+
+    world, rank, local = _dist()
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    binding.load_library()
+    cpu = make_inputs(wl, seed=wl.seed + rank)
+    target_cpu = target_weights(torch.Generator().manual_seed(wl.seed + 7 + rank), (wl.B, wl.Tq, wl.L))
+    dev = to_device(cpu, device)
+    target = target_cpu.to(device)
+    bufs = _train_buffers(wl, dev, binding)
+    calls = _train_calls(wl, dev, target, bufs, binding)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        calls["scores"]()
+        calls["kl"]()
+        calls["backward"]()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    graph, launches_per_step = _capture(step, binding, device)
+    run = graph.replay if graph is not None else step
+    for _ in range(args.warmup):
+        run()
+    torch.cuda.synchronize(device)
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    _barrier(world)
+    torch.cuda.synchronize(device)
+    launches0 = binding.kernel_launch_count()
+    h0 = time.perf_counter()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        run()
+    ev1.record(stream)
+    torch.cuda.synchronize(device)
+    h1 = time.perf_counter()
+    launches = (launches_per_step * args.steps if graph is not None
+                else binding.kernel_launch_count() - launches0)
+    _barrier(world)
+    sampler.stop()
+    sec_max = _max_over_ranks(ev0.elapsed_time(ev1) / 1000.0, world, device)
+    units = float(args.steps * wl.B * wl.Tq)
+    unit = "training tokens/s"
+    value = units * world / sec_max
+    clocks = sampler.summary(h0, h1)
+
+    # ---- per-stage timing for the roofline (graph replays, launching stream)
+    peaks = _peaks()
+    work = train_work(wl)
+    iters = max(3, min(args.steps, 20))
+    stage_report = {}
+    for name, fn in calls.items():
+        g, _ = _capture(fn, binding, device)
+        r = g.replay if g is not None else fn
+        for _ in range(3):
+            r()
+        torch.cuda.synchronize(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(iters):
+            r()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        ms = e0.elapsed_time(e1) / iters
+        nbytes, flops = work[name]
+        entry = {"ms": ms, "GB/s": nbytes / (ms / 1e3) / 1e9, "algorithmic_bytes": nbytes,
+                 "algorithmic_flops": flops}
+        entry["hbm_frac"] = entry["GB/s"] / peaks["hbm_gbs"]
+        if flops:
+            entry["TFLOP/s"] = flops / (ms / 1e3) / 1e12
+            entry["tensor_frac"] = entry["TFLOP/s"] / peaks["bf16_tflops"]
+        stage_report[name] = entry
+    dominant = max(stage_report, key=lambda n: stage_report[n]["ms"])
+    d = stage_report[dominant]
+    if d["algorithmic_flops"]:
+        roofline = {"bound": "tensor", "kernel": dominant, "achieved": d["TFLOP/s"], "peak": peaks["bf16_tflops"],
+                    "unit": "TFLOP/s", "frac": d["tensor_frac"], "traffic": None, "peak_source": peaks["source"]}
+    else:
+        roofline = {"bound": "hbm", "kernel": dominant, "achieved": d["GB/s"], "peak": peaks["hbm_gbs"],
+                    "unit": "GB/s", "frac": d["hbm_frac"], "traffic": None, "peak_source": peaks["source"]}
+
+    # ---- end to end: inputs and target from pinned host memory, loss read back
+    host = {"q_idx": cpu["q_idx"].contiguous().pin_memory(), "k_idx": cpu["k_idx"].contiguous().pin_memory(),
+            "w": cpu["w"].contiguous().pin_memory(), "target": target_cpu.contiguous().pin_memory()}
+    dst = {"q_idx": dev["q_idx"], "k_idx": dev["k_idx"], "w": dev["w"], "target": target}
+    loss_host = torch.empty(1, dtype=torch.float32).pin_memory()
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+
+    def e2e_step():
+        for k2, v in host.items():
+            dst[k2].copy_(v, non_blocking=True)
+        step()
+        loss_host.copy_(bufs["loss_sum"], non_blocking=True)
+
+    e2e_step()
+    _barrier(world)
+    torch.cuda.synchronize(device)
+    ev0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    ev1.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_sec = _max_over_ranks(ev0.elapsed_time(ev1) / 1000.0, world, device)
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    e2e = {"value": e2e_steps * wl.B * wl.Tq * world / e2e_sec, "unit": unit, "h2d_bytes_per_step": int(h2d),
+           "d2h_bytes_per_step": 4, "steps": e2e_steps,
+           "note": "indexer inputs and the target copied from pinned host memory, the summed loss read back, "
+                   "every step"}
+
+    cpu_baseline = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        nthreads = oracle.max_threads()
+        _, _, _, probe = time_train_oracle(wl, cpu, target_cpu, 4, nthreads)
+        n = int(min(256, max(4, 4 * args.cpu_budget / max(probe, 1e-6))))
+        sec, r, k, _ = time_train_oracle(wl, cpu, target_cpu, n, nthreads)
+        cpu_baseline = {"value": wl.B * wl.Tq / sec, "unit": unit, "cores": nthreads, "kind": "oracle",
+                        "sample": f"{r} query rows (scores, loss, dq, dw) and {k} keys (dk), scaled to a full "
+                                  f"step ({sec:.1f} s extrapolated)"}
+
+    if rank == 0:
+        line = {
+            "metric": TRAIN_METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1000.0 * sec_max / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": dict(_config(wl, world), **{"pass": "train", "target": "log-normal weights, 10% zeros"}),
+            "roofline": roofline, "stages": stage_report, "cpu_baseline": cpu_baseline, "e2e": e2e,
+            "gpu_launches": int(launches), "clocks": clocks,
+            "timing": "CUDA-graph replay of one training step" if graph is not None else "eager calls",
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--stage", choices=["indexer", "topk", "attn"], default=None,
@@ -573,15 +823,22 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default="decode32k", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default=None, choices=sorted(WORKLOADS),
+                    help="default: decode32k (forward), prefill8k (train)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle wall time")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--pass", dest="pass_", default="forward", choices=["forward", "train"],
+                    help="train: indexer scores, dense KL loss and indexer backward per step")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)  # at least three untimed warm-up steps
+    if args.workload is None:
+        args.workload = "prefill8k" if args.pass_ == "train" else "decode32k"
     wl = WORKLOADS[args.workload]
-    if args.stage is not None:
+    if args.pass_ == "train" and args.impl == "ours" and args.stage is None:
+        run_train(args, wl)
+    elif args.stage is not None:
         run_stage(args, wl)
     elif args.impl == "reference":
         run_reference(args, wl)

@@ -132,12 +132,30 @@ __device__ __forceinline__ bool decode_unit(int u, const Params &p, Unit &un) {
     return true;
 }
 
+// acc(lo, hi) += (a_lo * b_lo, a_hi * b_hi): two IEEE fp32 FMAs in one instruction
+__device__ __forceinline__ void fma2(uint64_t &acc, float a_lo, float a_hi, float b_lo, float b_hi) {
+    uint64_t a, b;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(a_lo), "f"(a_hi));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(b) : "f"(b_lo), "f"(b_hi));
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(a), "l"(b));
+}
+// (lo, hi) = (a_lo * b_lo, a_hi * b_hi)
+__device__ __forceinline__ void mul2(float &lo, float &hi, float a_lo, float a_hi, float b_lo, float b_hi) {
+    uint64_t a, b, d;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(a_lo), "f"(a_hi));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(b) : "f"(b_lo), "f"(b_hi));
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(d));
+}
+__device__ __forceinline__ float lo_f32(uint64_t v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float hi_f32(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
-template <bool KEY_SIDE>
+template <bool KEY_SIDE, int H>
 __global__ void __launch_bounds__(kThreads, 1)
 indexer_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const Params p) {
@@ -159,6 +177,7 @@ indexer_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     uint64_t *drain = acc_empty + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
 
+    constexpr int QPG = kRows / H;  // queries per group
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     // the resident tile comes from K on the key side, from Q on the query side
@@ -299,6 +318,11 @@ indexer_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         }
     } else {
         // ---------------------------------------------------- epilogue
+        // Query side: w[t,j] is constant along a TMEM lane, so MMA 2 takes
+        // M = g [X > 0] and the accumulator is multiplied by w once per unit
+        // (G = w M; for the power-of-two weights the rounding of M and of G
+        // to bf16 is the same). Key side: G = (g w)[X > 0], with g constant
+        // per (lane, query) and w per column.
         const int quarter = warp & 3;
         const int half = (warp - 2) >> 2;          // columns [64 half, 64 half + 64)
         const int r = quarter * 32 + lane;         // TMEM lane: resident row
@@ -309,20 +333,13 @@ indexer_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             Unit un;
             if (!decode_unit<KEY_SIDE>(u, p, un)) continue;
             const int ntiles = KEY_SIDE ? un.g1 - un.g0 : un.kt1 - un.kt0;
-            // query side: this lane's (query, head) and its weight
-            int qi = 0, t_row = 0, row = 0;
-            float w_r = 0.f, dw_acc = 0.f;
-            if (!KEY_SIDE) {
-                qi = r / p.H;
-                const int i = un.g0 * p.QPG + qi;
-                row = un.b * p.Tq + i;
-                t_row = p.q_pos0 + i;
-                if (i < p.Tq) {
-                    w_r = p.w[(size_t)row * p.H + (r - qi * p.H)];
-                } else {
-                    t_row = -1;  // no such query: G = 0
-                }
-            }
+            // query side: this lane's (query, head)
+            const int qi = r / H, j = r % H;
+            const int i_row = un.g0 * QPG + qi;
+            const bool row_ok = !KEY_SIDE && i_row < p.Tq;
+            const int row = un.b * p.Tq + i_row;
+            const int t_row = row_ok ? p.q_pos0 + i_row : -1;  // no such query: nothing passes
+            uint64_t dw2 = 0ull;                                // two partial sums of g ReLU(x)
             for (int n = 0; n < ntiles && ok; ++n) {
                 if (!mbar_wait(&x_full[xb], xph)) { ok = false; break; }
                 tc_fence_after();
@@ -335,60 +352,62 @@ indexer_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 mbar_arrive(&x_empty[xb]);
                 uint32_t gp[32];
                 if (!KEY_SIDE) {
-                    // columns = keys s0 + 64 half + c; g[t, s] shared by the warp's lanes
+                    // columns = keys s_base + c; g[t, s] is the same for the warp's lanes
                     const int s_base = (un.kt0 + n) * kRows + half * 64;
-                    const float *grow = p.grad + (size_t)(row < p.B * p.Tq ? row : 0) * p.L;
+                    if (t_row < s_base) {  // every key of this half lies after t (or no query)
 #pragma unroll
-                    for (int c4 = 0; c4 < 16; ++c4) {
-                        const int s = s_base + 4 * c4;
-                        float4 gv = make_float4(0.f, 0.f, 0.f, 0.f);
-                        if (s <= t_row) gv = __ldg(reinterpret_cast<const float4 *>(grow + s));
-                        const float gs[4] = {s <= t_row ? gv.x : 0.f, s + 1 <= t_row ? gv.y : 0.f,
-                                             s + 2 <= t_row ? gv.z : 0.f, s + 3 <= t_row ? gv.w : 0.f};
-                        float G[4];
+                        for (int c = 0; c < 32; ++c) gp[c] = 0u;
+                    } else {
+                        const float4 *g4 = reinterpret_cast<const float4 *>(p.grad + (size_t)row * p.L + s_base);
+                        const bool full = s_base + 63 <= t_row;  // no key of this half after t
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float x = __uint_as_float(xr[4 * c4 + e]);
-                            G[e] = x > 0.f ? gs[e] * w_r : 0.f;
-                            dw_acc = fmaf(gs[e], fmaxf(x, 0.f), dw_acc);
+                        for (int c4 = 0; c4 < 16; ++c4) {
+                            float4 gv = make_float4(0.f, 0.f, 0.f, 0.f);
+                            if (full || s_base + 4 * c4 <= t_row) gv = __ldg(g4 + c4);
+                            if (!full) {
+                                const int s = s_base + 4 * c4;
+                                if (s + 1 > t_row) gv.y = 0.f;
+                                if (s + 2 > t_row) gv.z = 0.f;
+                                if (s + 3 > t_row) gv.w = 0.f;
+                            }
+                            const float x0 = __uint_as_float(xr[4 * c4]), x1 = __uint_as_float(xr[4 * c4 + 1]);
+                            const float x2 = __uint_as_float(xr[4 * c4 + 2]), x3 = __uint_as_float(xr[4 * c4 + 3]);
+                            const float m0 = x0 > 0.f ? gv.x : 0.f, m1 = x1 > 0.f ? gv.y : 0.f;
+                            const float m2 = x2 > 0.f ? gv.z : 0.f, m3 = x3 > 0.f ? gv.w : 0.f;
+                            fma2(dw2, m0, m1, x0, x1);
+                            fma2(dw2, m2, m3, x2, x3);
+                            gp[2 * c4] = pack_bf16x2(m0, m1);
+                            gp[2 * c4 + 1] = pack_bf16x2(m2, m3);
                         }
-                        gp[2 * c4] = pack_bf16x2(G[0], G[1]);
-                        gp[2 * c4 + 1] = pack_bf16x2(G[2], G[3]);
                     }
                 } else {
-                    // lanes = keys s; columns = (query, head) pairs of group g
+                    // lanes = keys s; columns = (query, head) pairs of group g;
+                    // half h holds queries [h * 64 / H, (h * 64 + 63) / H]
                     const int g = un.g0 + n;
                     const int s = un.kt0 * kRows + r;
-                    const int c_base = half * 64;
-                    // the (at most two) queries of this half's columns
-                    const int qa = c_base / p.H, qb = (c_base + 63) / p.H;
-                    float g_q[2] = {0.f, 0.f};
+                    constexpr int QPH = 64 / H > 0 ? 64 / H : 1;  // queries per half
 #pragma unroll
-                    for (int z = 0; z < 2; ++z) {
-                        const int qz = z == 0 ? qa : qb;
-                        const int i = g * p.QPG + qz;
-                        if (i < p.Tq && s <= p.q_pos0 + i)
-                            g_q[z] = p.grad[(size_t)(un.b * p.Tq + i) * p.L + s];
-                    }
+                    for (int z = 0; z < QPH; ++z) {
+                        const int qz = (half * 64) / H + z;
+                        const int i = g * QPG + qz;
+                        float gq = 0.f;
+                        if (i < p.Tq && s <= p.q_pos0 + i) gq = p.grad[(size_t)(un.b * p.Tq + i) * p.L + s];
+                        const float4 *w4 =
+                            reinterpret_cast<const float4 *>(p.w + (size_t)(un.b * p.Tq + (i < p.Tq ? i : 0)) * H +
+                                                             ((half * 64) % H));
+                        constexpr int C4 = (H < 64 ? H : 64) / 4;  // float4s of this query in the half
 #pragma unroll
-                    for (int c4 = 0; c4 < 16; ++c4) {
-                        const int cc = c_base + 4 * c4;  // 4 columns of one query (H is a multiple of 4)
-                        const int qz = cc / p.H;
-                        const int i = g * p.QPG + qz;
-                        const float gq = qz == qa ? g_q[0] : g_q[1];
-                        float4 wv = make_float4(0.f, 0.f, 0.f, 0.f);
-                        if (i < p.Tq)
-                            wv = __ldg(reinterpret_cast<const float4 *>(p.w + (size_t)(un.b * p.Tq + i) * p.H +
-                                                                        (cc - qz * p.H)));
-                        const float ws[4] = {wv.x, wv.y, wv.z, wv.w};
-                        float G[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float x = __uint_as_float(xr[4 * c4 + e]);
-                            G[e] = x > 0.f ? gq * ws[e] : 0.f;
+                        for (int c4 = 0; c4 < C4; ++c4) {
+                            const int cc = z * (C4 * 4) + 4 * c4;  // column within the half
+                            const float4 wv = __ldg(w4 + c4);
+                            float gw0, gw1, gw2, gw3;
+                            mul2(gw0, gw1, gq, gq, wv.x, wv.y);
+                            mul2(gw2, gw3, gq, gq, wv.z, wv.w);
+                            const float x0 = __uint_as_float(xr[cc]), x1 = __uint_as_float(xr[cc + 1]);
+                            const float x2 = __uint_as_float(xr[cc + 2]), x3 = __uint_as_float(xr[cc + 3]);
+                            gp[cc / 2] = pack_bf16x2(x0 > 0.f ? gw0 : 0.f, x1 > 0.f ? gw1 : 0.f);
+                            gp[cc / 2 + 1] = pack_bf16x2(x2 > 0.f ? gw2 : 0.f, x3 > 0.f ? gw3 : 0.f);
                         }
-                        gp[2 * c4] = pack_bf16x2(G[0], G[1]);
-                        gp[2 * c4 + 1] = pack_bf16x2(G[2], G[3]);
                     }
                 }
                 if (!mbar_wait(&g_empty[xb], xph ^ 1u)) { ok = false; break; }
@@ -412,19 +431,22 @@ indexer_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             mbar_arrive(acc_empty);
             aph ^= 1u;
             float *dst = nullptr;
+            float scale = 1.f;
             if (KEY_SIDE) {
                 dst = p.part + ((size_t)un.slot * kRows + r) * kD + half * 64;
-            } else if (t_row >= 0) {
-                if (p.dq) dst = p.dq + ((size_t)row * p.H + (r - qi * p.H)) * kD + half * 64;
+            } else if (row_ok) {
+                scale = p.w[(size_t)row * H + j];
+                if (p.dq) dst = p.dq + ((size_t)row * H + j) * kD + half * 64;
                 // the two halves' sums land on a zeroed word: (0 + a) + b == (0 + b) + a
-                if (p.dw) atomicAdd(p.dw + (size_t)row * p.H + (r - qi * p.H), dw_acc);
+                if (p.dw) atomicAdd(p.dw + (size_t)row * H + j, lo_f32(dw2) + hi_f32(dw2));
             }
             if (dst) {
                 float4 *d4 = reinterpret_cast<float4 *>(dst);
 #pragma unroll
                 for (int c4 = 0; c4 < 16; ++c4)
-                    d4[c4] = make_float4(__uint_as_float(ar[4 * c4]), __uint_as_float(ar[4 * c4 + 1]),
-                                         __uint_as_float(ar[4 * c4 + 2]), __uint_as_float(ar[4 * c4 + 3]));
+                    d4[c4] = make_float4(__uint_as_float(ar[4 * c4]) * scale, __uint_as_float(ar[4 * c4 + 1]) * scale,
+                                         __uint_as_float(ar[4 * c4 + 2]) * scale,
+                                         __uint_as_float(ar[4 * c4 + 3]) * scale);
             }
         }
     }
@@ -539,7 +561,8 @@ cudaError_t launch_indexer_bwd_tc(const IndexerBwdProblem &pr, cudaStream_t stre
             return err;
         Params q = p;
         q.units = p.B * p.ngroups;
-        auto kern = indexer_bwd_tc_kernel<false>;
+        auto kern = pr.H == 32 ? indexer_bwd_tc_kernel<false, 32>
+                               : (pr.H == 64 ? indexer_bwd_tc_kernel<false, 64> : indexer_bwd_tc_kernel<false, 128>);
         if ((err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem)) !=
             cudaSuccess)
             return err;
@@ -554,7 +577,8 @@ cudaError_t launch_indexer_bwd_tc(const IndexerBwdProblem &pr, cudaStream_t stre
         const long long units = (long long)p.B * p.nchunks * p.nkt;
         if (units > 0x7fffffffLL) return cudaErrorInvalidValue;
         k.units = (int)units;
-        auto kern = indexer_bwd_tc_kernel<true>;
+        auto kern = pr.H == 32 ? indexer_bwd_tc_kernel<true, 32>
+                               : (pr.H == 64 ? indexer_bwd_tc_kernel<true, 64> : indexer_bwd_tc_kernel<true, 128>);
         if ((err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem)) !=
             cudaSuccess)
             return err;
