@@ -325,10 +325,13 @@ dsa_status dsa_indexer_kl(const float *scores, const float *target, const int32_
  *   ws       at least dsa_indexer_backward_workspace_bytes(...) bytes when dk
  *            is requested (may be NULL when that is 0).
  * Paths: bf16 inputs with d_I = 128, H_I in {32, 64, 128}, L a multiple of 4,
- * 16-byte aligned pointers and at least 128 rows of q_idx and of k_idx run on
- * the tensor cores: x is exact there (bf16 products, fp32 sums), G is rounded
- * to bf16 for the second product, sums are fp32. Every other shape runs on
- * CUDA cores in fp32.
+ * 16-byte aligned pointers, L >= 128 and at least 128 rows of q_idx run on
+ * the tensor cores: x is exact there (bf16 products, fp32 sums); the products
+ * with k and q take g [x > 0] (times w on the key side) rounded to bf16, so
+ * dq and dk carry a relative error of at most 2^-8 of the sums of absolute
+ * terms; dw is formed as q . sum_s g [x > 0] k[s] (the same value, since
+ * x = q . k[s]) and carries the same bound against sum_s |g| ReLU(x). Every
+ * other shape runs on CUDA cores in fp32.
  * Errors: DSA_ERR_INVALID_ARG as dsa_indexer_scores, or a null grad;
  * DSA_ERR_WORKSPACE when dk is requested and ws is missing or too small;
  * DSA_ERR_UNSUPPORTED when the CUDA-core path's staging does not fit.

@@ -13,8 +13,11 @@
 //   query side (dq, dw): a group of 128 / H queries (128 rows (t, j)) stays
 //       resident; 128-key tiles stream past it.
 //       MMA 1  X[(t,j), s]  = Q[(t,j), :] . K[s, :]        M=128 N=128 K=128
-//       epilogue  G = g w [X > 0] in bf16 into TMEM, dw += g ReLU(X) in fp32
-//       MMA 2  dQ[(t,j), :] += G[(t,j), s] K[s, :]          M=128 N=128 K=128
+//       epilogue  M = g [X > 0] in bf16 into TMEM (w[t,j] is constant along
+//                 a row, so G = w M is applied to the result)
+//       MMA 2  acc[(t,j), :] += M[(t,j), s] K[s, :]          M=128 N=128 K=128
+//       dq = w acc, and dw = q . acc, since sum_s g ReLU(x) = sum_s M x and
+//       x = q . k[s] (one dot product per row and unit, no per-element work)
 //   key side (dk): a 128-key tile stays resident; query groups stream past.
 //       MMA 1  X[s, (t,j)]  = K[s, :] . Q[(t,j), :]
 //       epilogue  G[s, (t,j)] as above
@@ -25,13 +28,13 @@
 // in shared memory feeds both. x is exact (integer-valued bf16, fp32 sums);
 // G is rounded to bf16 for MMA 2; sums are fp32.
 //
-// Warp roles (320 threads, one CTA per SM, persistent over work units):
+// Warp roles (576 threads, one CTA per SM, persistent over work units):
 //   warp 0     TMA: the resident tile of each unit (two buffers), streamed
 //              tiles through a 4-stage ring.
-//   warp 1     TMEM owner; one thread issues the MMAs: MMA 1 of tile n+1
-//              before MMA 2 of tile n, so the epilogue of one tile overlaps
-//              the tensor core's work on its neighbours.
-//   warps 2-9  epilogue: two warps per TMEM lane quarter, each taking 64 of
+//   warp 1     TMEM owner; one thread issues two streams of MMAs, each as
+//              soon as its inputs are ready: MMA 1 runs up to two tiles ahead
+//              of the epilogue, MMA 2 follows it.
+//   warps 2-17 epilogue: four warps per TMEM lane quarter, each taking 32 of
 //              the 128 columns of X and of the accumulator.
 // TMEM: X in two buffers [0, 256), G in two buffers [256, 384) (two bf16 per
 // column), the accumulator [384, 512).
@@ -61,16 +64,24 @@ constexpr uint32_t kBox = kRows * 128;      // 128 rows x 64 bf16 columns (128-b
 constexpr uint32_t kTile = 2 * kBox;        // 128 rows x 128 columns
 constexpr int kStages = 4;
 constexpr int kResBufs = 2;
-constexpr int kEpiThreads = 256;
+constexpr int kEpiWarps = 16;               // four per TMEM lane quarter
+constexpr int kEpiThreads = kEpiWarps * 32;
+constexpr int kParts = kEpiWarps / 4;         // column parts of a tile
+constexpr int kCW = 128 / kParts;             // columns per epilogue warp
 constexpr int kThreads = 64 + kEpiThreads;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColX = 0;               // 2 x 128
 constexpr uint32_t kColG = 256;             // 2 x 64
 constexpr uint32_t kColAcc = 384;           // 128
 constexpr uint32_t kIdescMnMajorB = 1u << 16;
-// barriers: res_full/empty[2], st_full/empty[4], x_full/empty[2], g_full/empty[2], acc_full, acc_empty, drain
-constexpr int kNumBars = 2 * kResBufs + 2 * kStages + 4 + 4 + 3;
-constexpr size_t kSmem = 1024 + (size_t)kResBufs * kTile + (size_t)kStages * kTile + kNumBars * 8 + 16;
+// barriers: res_full/empty[2], st_full/empty[4], x_full/empty[2], g_full/empty[2], acc_full, acc_empty,
+// drain, dw_bar
+constexpr int kNumBars = 2 * kResBufs + 2 * kStages + 4 + 4 + 4;
+constexpr uint32_t kDwBytes = 2 * kParts * kRows * 4;  // dw partial sums, two buffers
+constexpr uint32_t kGBytes = 4 * kRows * 4;            // per stage: g of up to 4 queries x 128 keys
+constexpr uint32_t kWBytes = kRows * 4;                // per stage: w of one query group (key side)
+constexpr size_t kSmem = 1024 + (size_t)kResBufs * kTile + (size_t)kStages * (kTile + kGBytes + kWBytes) + kDwBytes +
+                         kNumBars * 8 + 16;
 static_assert(kSmem <= 232448, "shared memory budget");
 
 __device__ unsigned int g_indexer_bwd_error = 0;  // 1 = a bounded wait gave up
@@ -132,13 +143,6 @@ __device__ __forceinline__ bool decode_unit(int u, const Params &p, Unit &un) {
     return true;
 }
 
-// acc(lo, hi) += (a_lo * b_lo, a_hi * b_hi): two IEEE fp32 FMAs in one instruction
-__device__ __forceinline__ void fma2(uint64_t &acc, float a_lo, float a_hi, float b_lo, float b_hi) {
-    uint64_t a, b;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(a_lo), "f"(a_hi));
-    asm("mov.b64 %0, {%1, %2};" : "=l"(b) : "f"(b_lo), "f"(b_hi));
-    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(a), "l"(b));
-}
 // (lo, hi) = (a_lo * b_lo, a_hi * b_hi)
 __device__ __forceinline__ void mul2(float &lo, float &hi, float a_lo, float a_hi, float b_lo, float b_hi) {
     uint64_t a, b, d;
@@ -147,8 +151,6 @@ __device__ __forceinline__ void mul2(float &lo, float &hi, float a_lo, float a_h
     asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(d));
 }
-__device__ __forceinline__ float lo_f32(uint64_t v) { return __uint_as_float((uint32_t)v); }
-__device__ __forceinline__ float hi_f32(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -158,12 +160,16 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 template <bool KEY_SIDE, int H>
 __global__ void __launch_bounds__(kThreads, 1)
 indexer_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_w,
                       const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *res_sm = smem;
     uint8_t *st_sm = res_sm + kResBufs * kTile;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(st_sm + kStages * kTile);
+    float *g_sm = reinterpret_cast<float *>(st_sm + kStages * kTile);      // [stage][query][128 keys]
+    float *w_sm = g_sm + kStages * (kGBytes / 4);                          // [stage][128 (query, head)]
+    float *dw_sm = w_sm + kStages * (kWBytes / 4);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(dw_sm) + kDwBytes);
     uint64_t *res_full = bars;
     uint64_t *res_empty = res_full + kResBufs;
     uint64_t *st_full = res_empty + kResBufs;
@@ -175,9 +181,13 @@ indexer_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     uint64_t *acc_full = g_empty + 2;
     uint64_t *acc_empty = acc_full + 1;
     uint64_t *drain = acc_empty + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    uint64_t *dw_bar = drain + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(dw_bar + 1);
 
     constexpr int QPG = kRows / H;  // queries per group
+    // bytes each streamed tile brings: the tile, g of the group's queries over
+    // the 128 keys, and (key side) w of the group
+    constexpr uint32_t kStageTx = kTile + QPG * kRows * 4 + (KEY_SIDE ? kRows * 4 : 0);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     // the resident tile comes from K on the key side, from Q on the query side
@@ -187,7 +197,7 @@ indexer_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     if (threadIdx.x == 0) {
         for (int s = 0; s < kResBufs; ++s) {
             mbar_init(&res_full[s], 1);
-            mbar_init(&res_empty[s], 1);
+            mbar_init(&res_empty[s], 1 + kEpiThreads);  // the MMAs and the epilogue's last reads
         }
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&st_full[s], 1);
@@ -202,6 +212,7 @@ indexer_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, kEpiThreads);
         mbar_init(drain, 1);
+        mbar_init(dw_bar, kEpiThreads);
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -219,6 +230,8 @@ indexer_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             // ------------------------------------------------ TMA producer
             prefetch_tensor_map(&tm_q);
             prefetch_tensor_map(&tm_k);
+            prefetch_tensor_map(&tm_g);
+            if (KEY_SIDE) prefetch_tensor_map(&tm_w);
             int sb = 0, rb = 0;
             uint32_t sph = 0, rph = 0;
             int st_armed[kStages], res_armed[kResBufs];  // parity of each buffer's last armed phase, or -1
@@ -237,11 +250,16 @@ indexer_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 const int n0 = KEY_SIDE ? un.g0 : un.kt0, n1 = KEY_SIDE ? un.g1 : un.kt1;
                 for (int n = n0; n < n1; ++n) {
                     if (!mbar_wait(&st_empty[sb], sph ^ 1u)) { ok = false; break; }
-                    mbar_arrive_expect_tx(&st_full[sb], kTile);
+                    mbar_arrive_expect_tx(&st_full[sb], kStageTx);
                     st_armed[sb] = (int)sph;
-                    const int srow = KEY_SIDE ? (un.b * p.Tq + n * p.QPG) * p.H : un.b * p.L + n * kRows;
+                    const int srow = KEY_SIDE ? (un.b * p.Tq + n * QPG) * H : un.b * p.L + n * kRows;
                     tma_load_2d(st_sm + sb * kTile, tm_str, &st_full[sb], 0, srow);
                     tma_load_2d(st_sm + sb * kTile + kBox, tm_str, &st_full[sb], 64, srow);
+                    // g[t, s] for the (group, key tile) pair of this step
+                    const int grow = un.b * p.Tq + (KEY_SIDE ? n : un.g0) * QPG;
+                    const int gcol = (KEY_SIDE ? un.kt0 : n) * kRows;
+                    tma_load_2d(g_sm + sb * (kGBytes / 4), &tm_g, &st_full[sb], gcol, grow);
+                    if (KEY_SIDE) tma_load_2d(w_sm + sb * (kWBytes / 4), &tm_w, &st_full[sb], 0, grow);
                     if (++sb == kStages) { sb = 0; sph ^= 1u; }
                 }
             }
@@ -254,56 +272,68 @@ indexer_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     } else if (warp == 1) {
         if (lane == 0) {
             // ------------------------------------------------ MMA issuer
+            // Two streams of MMAs, each issued as soon as its inputs are
+            // ready: MMA 1 of the next tile (a stage landed, an X buffer
+            // free) and MMA 2 of the oldest tile whose G is in TMEM. MMA 1
+            // thus runs up to two tiles ahead of the epilogue.
             const uint32_t idesc1 = idesc_bf16_f32(kRows, kRows);
             const uint32_t idesc2 = idesc_bf16_f32(kRows, kD) | kIdescMnMajorB;
-            int sb = 0, rb = 0, xb = 0;
-            uint32_t sph = 0, rph = 0, xph = 0, aph = 0;
+            int sb1 = 0, xb1 = 0, sb2 = 0, xb2 = 0, rb = 0;
+            uint32_t sph1 = 0, xph1 = 0, xph2 = 0, rph = 0, aph = 0;
             for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
                 Unit un;
                 if (!decode_unit<KEY_SIDE>(u, p, un)) continue;
                 if (!mbar_wait(&res_full[rb], rph)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t a_base = smem_addr(res_sm + rb * kTile);
+                const uint64_t a_desc = smem_desc_k_sw128(smem_addr(res_sm + rb * kTile));
                 const int ntiles = KEY_SIDE ? un.g1 - un.g0 : un.kt1 - un.kt0;
-                int prev_sb = -1, prev_xb = 0;
-                uint32_t prev_xph = 0;
-                for (int n = 0; n <= ntiles && ok; ++n) {
-                    if (n < ntiles) {
-                        // MMA 1 of tile n: X = A . B^T
-                        if (!mbar_wait(&st_full[sb], sph)) { ok = false; break; }
-                        if (!mbar_wait(&x_empty[xb], xph ^ 1u)) { ok = false; break; }
+                int n1 = 0, n2 = 0;
+                uint32_t idle = 0;
+                uint64_t t_idle = 0;
+                while (n2 < ntiles) {
+                    bool progress = false;
+                    if (n1 < ntiles && mbar_test_wait(&st_full[sb1], sph1) && mbar_test_wait(&x_empty[xb1], xph1 ^ 1u)) {
+                        // MMA 1: X = A . B^T, both K-major
                         tc_fence_after();
-                        const uint32_t b_base = smem_addr(st_sm + sb * kTile);
-                        const uint32_t d = tmem + kColX + (uint32_t)(xb * 128);
+                        const uint64_t b_desc = smem_desc_k_sw128(smem_addr(st_sm + sb1 * kTile));
+                        const uint32_t d = tmem + kColX + (uint32_t)(xb1 * 128);
 #pragma unroll
                         for (int h = 0; h < 2; ++h)
 #pragma unroll
-                            for (int kk = 0; kk < 4; ++kk)
-                                mma_f16_ss(d, smem_desc_k_sw128(a_base + h * kBox + kk * 32),
-                                           smem_desc_k_sw128(b_base + h * kBox + kk * 32), idesc1, (h | kk) != 0);
-                        mma_commit(&x_full[xb]);
+                            for (int kk = 0; kk < 4; ++kk) {
+                                const uint64_t off = (uint64_t)((h * kBox + kk * 32) >> 4);
+                                mma_f16_ss(d, a_desc + off, b_desc + off, idesc1, (h | kk) != 0);
+                            }
+                        mma_commit(&x_full[xb1]);
+                        ++n1;
+                        if (++sb1 == kStages) { sb1 = 0; sph1 ^= 1u; }
+                        if (++xb1 == 2) { xb1 = 0; xph1 ^= 1u; }
+                        progress = true;
                     }
-                    if (n > 0) {
-                        // MMA 2 of tile n-1: acc += G (TMEM) . B (MN-major)
-                        if (!mbar_wait(&g_full[prev_xb], prev_xph)) { ok = false; break; }
-                        if (n == 1 && !mbar_wait(acc_empty, aph ^ 1u)) { ok = false; break; }
+                    if (n2 < n1 && mbar_test_wait(&g_full[xb2], xph2) &&
+                        (n2 > 0 || mbar_test_wait(acc_empty, aph ^ 1u))) {
+                        // MMA 2: acc += G (TMEM) . B (the same stage, MN-major)
                         tc_fence_after();
-                        const uint32_t b_base = smem_addr(st_sm + prev_sb * kTile);
-                        const uint32_t a_tm = tmem + kColG + (uint32_t)(prev_xb * 64);
+                        const uint64_t b_desc = smem_desc_mn_sw128(smem_addr(st_sm + sb2 * kTile), kBox);
+                        const uint32_t a_tm = tmem + kColG + (uint32_t)(xb2 * 64);
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk)
-                            mma_f16_ts(tmem + kColAcc, a_tm + (uint32_t)(kk * 8),
-                                       smem_desc_mn_sw128(b_base + kk * 2048, kBox), idesc2,
-                                       (n > 1 || kk > 0) ? 1u : 0u);
-                        mma_commit(&st_empty[prev_sb]);  // the streamed tile is no longer read
-                        mma_commit(&g_empty[prev_xb]);
+                            mma_f16_ts(tmem + kColAcc, a_tm + (uint32_t)(kk * 8), b_desc + (uint64_t)((kk * 2048) >> 4),
+                                       idesc2, (n2 > 0 || kk > 0) ? 1u : 0u);
+                        mma_commit(&st_empty[sb2]);  // the streamed tile is no longer read
+                        mma_commit(&g_empty[xb2]);
+                        ++n2;
+                        if (++sb2 == kStages) sb2 = 0;
+                        if (++xb2 == 2) { xb2 = 0; xph2 ^= 1u; }
+                        progress = true;
                     }
-                    if (n < ntiles) {
-                        prev_sb = sb;
-                        prev_xb = xb;
-                        prev_xph = xph;
-                        if (++sb == kStages) { sb = 0; sph ^= 1u; }
-                        if (++xb == 2) { xb = 0; xph ^= 1u; }
+                    if (progress) {
+                        idle = 0;
+                    } else {
+                        // bounded: give up after the wait limit without progress
+                        if (idle == 0) t_idle = global_timer_ns();
+                        if ((++idle & 63u) == 0u && global_timer_ns() - t_idle > kWaitTimeoutNs) { ok = false; break; }
+                        __nanosleep(20);
                     }
                 }
                 if (!ok) break;
@@ -324,11 +354,12 @@ indexer_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         // to bf16 is the same). Key side: G = (g w)[X > 0], with g constant
         // per (lane, query) and w per column.
         const int quarter = warp & 3;
-        const int half = (warp - 2) >> 2;          // columns [64 half, 64 half + 64)
+        const int part = (warp - 2) >> 2;          // columns [kCW part, kCW part + kCW)
+        const int col0 = part * kCW;
         const int r = quarter * 32 + lane;         // TMEM lane: resident row
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-        int xb = 0;
-        uint32_t xph = 0, aph = 0;
+        int xb = 0, unit_n = 0, sb = 0, rb = 0;
+        uint32_t xph = 0, aph = 0, sph = 0, rph = 0;
         for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
             Unit un;
             if (!decode_unit<KEY_SIDE>(u, p, un)) continue;
@@ -339,67 +370,65 @@ indexer_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             const bool row_ok = !KEY_SIDE && i_row < p.Tq;
             const int row = un.b * p.Tq + i_row;
             const int t_row = row_ok ? p.q_pos0 + i_row : -1;  // no such query: nothing passes
-            uint64_t dw2 = 0ull;                                // two partial sums of g ReLU(x)
             for (int n = 0; n < ntiles && ok; ++n) {
                 if (!mbar_wait(&x_full[xb], xph)) { ok = false; break; }
+                // (complete already: MMA 1 read this stage) makes the TMA writes of g and w visible here
+                if (!mbar_wait(&st_full[sb], sph)) { ok = false; break; }
                 tc_fence_after();
-                uint32_t xr[64];
-                const uint32_t xaddr = tmem + lane_addr + kColX + (uint32_t)(xb * 128 + half * 64);
-                tmem_ld_32x32b_x32(xaddr, xr);
-                tmem_ld_32x32b_x32(xaddr + 32, xr + 32);
+                const float *gs = g_sm + sb * (kGBytes / 4);
+                const float *wsm = w_sm + sb * (kWBytes / 4);
+                uint32_t xr[kCW];
+                tmem_ld_32x32b_x32(tmem + lane_addr + kColX + (uint32_t)(xb * 128 + col0), xr);
                 tmem_ld_wait();
                 tc_fence_before();
                 mbar_arrive(&x_empty[xb]);
-                uint32_t gp[32];
+                uint32_t gp[kCW / 2];
                 if (!KEY_SIDE) {
                     // columns = keys s_base + c; g[t, s] is the same for the warp's lanes
-                    const int s_base = (un.kt0 + n) * kRows + half * 64;
-                    if (t_row < s_base) {  // every key of this half lies after t (or no query)
+                    const int s_base = (un.kt0 + n) * kRows + col0;
+                    const float4 *g4 = reinterpret_cast<const float4 *>(gs + qi * kRows + col0);
+                    if (t_row < s_base) {  // every key of this part lies after t (or no query)
 #pragma unroll
-                        for (int c = 0; c < 32; ++c) gp[c] = 0u;
-                    } else {
-                        const float4 *g4 = reinterpret_cast<const float4 *>(p.grad + (size_t)row * p.L + s_base);
-                        const bool full = s_base + 63 <= t_row;  // no key of this half after t
+                        for (int c = 0; c < kCW / 2; ++c) gp[c] = 0u;
+                    } else if (s_base + kCW - 1 <= t_row) {  // no key of this part after t
 #pragma unroll
-                        for (int c4 = 0; c4 < 16; ++c4) {
-                            float4 gv = make_float4(0.f, 0.f, 0.f, 0.f);
-                            if (full || s_base + 4 * c4 <= t_row) gv = __ldg(g4 + c4);
-                            if (!full) {
-                                const int s = s_base + 4 * c4;
-                                if (s + 1 > t_row) gv.y = 0.f;
-                                if (s + 2 > t_row) gv.z = 0.f;
-                                if (s + 3 > t_row) gv.w = 0.f;
-                            }
-                            const float x0 = __uint_as_float(xr[4 * c4]), x1 = __uint_as_float(xr[4 * c4 + 1]);
-                            const float x2 = __uint_as_float(xr[4 * c4 + 2]), x3 = __uint_as_float(xr[4 * c4 + 3]);
-                            const float m0 = x0 > 0.f ? gv.x : 0.f, m1 = x1 > 0.f ? gv.y : 0.f;
-                            const float m2 = x2 > 0.f ? gv.z : 0.f, m3 = x3 > 0.f ? gv.w : 0.f;
-                            fma2(dw2, m0, m1, x0, x1);
-                            fma2(dw2, m2, m3, x2, x3);
+                        for (int c4 = 0; c4 < kCW / 4; ++c4) {
+                            const float4 gv = g4[c4];
+                            gp[2 * c4] = pack_bf16x2(__uint_as_float(xr[4 * c4]) > 0.f ? gv.x : 0.f,
+                                                     __uint_as_float(xr[4 * c4 + 1]) > 0.f ? gv.y : 0.f);
+                            gp[2 * c4 + 1] = pack_bf16x2(__uint_as_float(xr[4 * c4 + 2]) > 0.f ? gv.z : 0.f,
+                                                         __uint_as_float(xr[4 * c4 + 3]) > 0.f ? gv.w : 0.f);
+                        }
+                    } else {  // the diagonal: keys after t pass nothing
+#pragma unroll
+                        for (int c4 = 0; c4 < kCW / 4; ++c4) {
+                            const float4 gv = g4[c4];
+                            const int s = s_base + 4 * c4;
+                            const float m0 = (__uint_as_float(xr[4 * c4]) > 0.f && s <= t_row) ? gv.x : 0.f;
+                            const float m1 = (__uint_as_float(xr[4 * c4 + 1]) > 0.f && s + 1 <= t_row) ? gv.y : 0.f;
+                            const float m2 = (__uint_as_float(xr[4 * c4 + 2]) > 0.f && s + 2 <= t_row) ? gv.z : 0.f;
+                            const float m3 = (__uint_as_float(xr[4 * c4 + 3]) > 0.f && s + 3 <= t_row) ? gv.w : 0.f;
                             gp[2 * c4] = pack_bf16x2(m0, m1);
                             gp[2 * c4 + 1] = pack_bf16x2(m2, m3);
                         }
                     }
                 } else {
-                    // lanes = keys s; columns = (query, head) pairs of group g;
-                    // half h holds queries [h * 64 / H, (h * 64 + 63) / H]
+                    // lanes = keys s; columns = (query, head) pairs of group g
                     const int g = un.g0 + n;
                     const int s = un.kt0 * kRows + r;
-                    constexpr int QPH = 64 / H > 0 ? 64 / H : 1;  // queries per half
+                    constexpr int QPP = kCW / H > 0 ? kCW / H : 1;  // queries in this part
+                    constexpr int C4 = (H < kCW ? H : kCW) / 4;     // float4s of one query in the part
 #pragma unroll
-                    for (int z = 0; z < QPH; ++z) {
-                        const int qz = (half * 64) / H + z;
+                    for (int z = 0; z < QPP; ++z) {
+                        const int qz = col0 / H + z;
                         const int i = g * QPG + qz;
                         float gq = 0.f;
-                        if (i < p.Tq && s <= p.q_pos0 + i) gq = p.grad[(size_t)(un.b * p.Tq + i) * p.L + s];
-                        const float4 *w4 =
-                            reinterpret_cast<const float4 *>(p.w + (size_t)(un.b * p.Tq + (i < p.Tq ? i : 0)) * H +
-                                                             ((half * 64) % H));
-                        constexpr int C4 = (H < 64 ? H : 64) / 4;  // float4s of this query in the half
+                        if (i < p.Tq && s <= p.q_pos0 + i) gq = gs[qz * kRows + r];
+                        const float4 *w4 = reinterpret_cast<const float4 *>(wsm + qz * H + (col0 % H));
 #pragma unroll
                         for (int c4 = 0; c4 < C4; ++c4) {
-                            const int cc = z * (C4 * 4) + 4 * c4;  // column within the half
-                            const float4 wv = __ldg(w4 + c4);
+                            const int cc = z * (C4 * 4) + 4 * c4;  // column within the part
+                            const float4 wv = w4[c4];
                             float gw0, gw1, gw2, gw3;
                             mul2(gw0, gw1, gq, gq, wv.x, wv.y);
                             mul2(gw2, gw3, gq, gq, wv.z, wv.w);
@@ -412,20 +441,19 @@ indexer_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 }
                 if (!mbar_wait(&g_empty[xb], xph ^ 1u)) { ok = false; break; }
                 tc_fence_after();
-                tmem_st_32x32b_x32(tmem + lane_addr + kColG + (uint32_t)(xb * 64 + half * 32), gp);
+                tmem_st_32x32b_x16(tmem + lane_addr + kColG + (uint32_t)(xb * 64 + col0 / 2), gp);
                 tmem_st_wait();
                 tc_fence_before();
                 mbar_arrive(&g_full[xb]);
                 if (++xb == 2) { xb = 0; xph ^= 1u; }
+                if (++sb == kStages) { sb = 0; sph ^= 1u; }
             }
             if (!ok) break;
             // ---- the unit's accumulator
             if (!mbar_wait(acc_full, aph)) { ok = false; break; }
             tc_fence_after();
-            uint32_t ar[64];
-            const uint32_t aaddr = tmem + lane_addr + kColAcc + (uint32_t)(half * 64);
-            tmem_ld_32x32b_x32(aaddr, ar);
-            tmem_ld_32x32b_x32(aaddr + 32, ar + 32);
+            uint32_t ar[kCW];
+            tmem_ld_32x32b_x32(tmem + lane_addr + kColAcc + (uint32_t)col0, ar);
             tmem_ld_wait();
             tc_fence_before();
             mbar_arrive(acc_empty);
@@ -433,21 +461,56 @@ indexer_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             float *dst = nullptr;
             float scale = 1.f;
             if (KEY_SIDE) {
-                dst = p.part + ((size_t)un.slot * kRows + r) * kD + half * 64;
-            } else if (row_ok) {
-                scale = p.w[(size_t)row * H + j];
-                if (p.dq) dst = p.dq + ((size_t)row * H + j) * kD + half * 64;
-                // the two halves' sums land on a zeroed word: (0 + a) + b == (0 + b) + a
-                if (p.dw) atomicAdd(p.dw + (size_t)row * H + j, lo_f32(dw2) + hi_f32(dw2));
+                tc_fence_before();
+                mbar_arrive(&res_empty[rb]);  // nothing here reads the resident tile
+                dst = p.part + ((size_t)un.slot * kRows + r) * kD + col0;
+            } else {
+                // dw[t,j] = sum_s g ReLU(x) = sum_s M[s] x[s] = q[t,j] . (sum_s M[s] k[s]):
+                // this lane's resident q row (bf16, 128-byte swizzle) against the
+                // unscaled accumulator, over this part's 32 columns
+                // (complete already: MMA 1 read this tile) makes the TMA writes visible here
+                if (!mbar_wait(&res_full[rb], rph)) { ok = false; break; }
+                const uint8_t *qrow = res_sm + rb * kTile + (col0 >> 6) * kBox + r * 128;
+                float dwp = 0.f;
+#pragma unroll
+                for (int c = 0; c < kCW / 8; ++c) {
+                    const int chunk = ((col0 & 63) >> 3) + c;
+                    const uint4 v = *reinterpret_cast<const uint4 *>(qrow + ((chunk ^ (r & 7)) << 4));
+                    const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        dwp = fmaf(__uint_as_float(wv[e] << 16), __uint_as_float(ar[8 * c + 2 * e]), dwp);
+                        dwp = fmaf(__uint_as_float(wv[e] & 0xffff0000u), __uint_as_float(ar[8 * c + 2 * e + 1]), dwp);
+                    }
+                }
+                mbar_arrive(&res_empty[rb]);
+                // the parts' partial sums meet in shared memory (two buffers, by
+                // unit parity) and part 0 adds them in a fixed order
+                float *dws = dw_sm + (unit_n & 1) * (kParts * kRows);
+                dws[part * kRows + r] = dwp;
+                mbar_arrive(dw_bar);
+                if (part == 0) {
+                    if (!mbar_wait(dw_bar, (uint32_t)(unit_n & 1))) { ok = false; break; }
+                    float sum = dws[r];
+#pragma unroll
+                    for (int q = 1; q < kParts; ++q) sum += dws[q * kRows + r];
+                    if (row_ok && p.dw) p.dw[(size_t)row * H + j] = sum;
+                }
+                if (row_ok) {
+                    scale = p.w[(size_t)row * H + j];
+                    if (p.dq) dst = p.dq + ((size_t)row * H + j) * kD + col0;
+                }
             }
             if (dst) {
                 float4 *d4 = reinterpret_cast<float4 *>(dst);
 #pragma unroll
-                for (int c4 = 0; c4 < 16; ++c4)
+                for (int c4 = 0; c4 < kCW / 4; ++c4)
                     d4[c4] = make_float4(__uint_as_float(ar[4 * c4]) * scale, __uint_as_float(ar[4 * c4 + 1]) * scale,
                                          __uint_as_float(ar[4 * c4 + 2]) * scale,
                                          __uint_as_float(ar[4 * c4 + 3]) * scale);
             }
+            if (++rb == kResBufs) { rb = 0; rph ^= 1u; }
+            ++unit_n;
         }
     }
 
@@ -489,7 +552,8 @@ bool plan(const IndexerBwdProblem &pr, const DeviceInfo &info, Params &p) {
     if (info.cc_major != 10 || (size_t)info.max_smem_optin < kSmem) return false;
     if (((uintptr_t)pr.q_idx | (uintptr_t)pr.k_idx | (uintptr_t)pr.w | (uintptr_t)pr.grad) % 16 != 0) return false;
     if ((pr.dq && (uintptr_t)pr.dq % 16) || (pr.dk && (uintptr_t)pr.dk % 16)) return false;
-    if (pr.L % 4 != 0) return false;  // 16-byte rows of g
+    // 16-byte rows of g, and TMA boxes no larger than the tensors they read
+    if (pr.L % 4 != 0 || pr.L < kRows) return false;
     // a TMA box may not be taller than the tensor it reads
     if ((long long)pr.B * pr.Tq * pr.H < kRows || (long long)pr.B * pr.L < kRows) return false;
     p.w = pr.w;
@@ -550,15 +614,15 @@ cudaError_t launch_indexer_bwd_tc(const IndexerBwdProblem &pr, cudaStream_t stre
     if (!plan(pr, info, p)) return cudaSuccess;
     if (pr.dk && (pr.ws == nullptr || pr.ws_bytes < part_bytes(p) || (uintptr_t)pr.ws % 16 != 0))
         return cudaSuccess;  // no room for the key side's partials: the CUDA-core path takes the call
-    CUtensorMap tm_q, tm_k;
-    if (!make_map_bf16_sw128(&tm_q, pr.q_idx, (uint64_t)pr.B * pr.Tq * pr.H, kD, kD * 2, kRows) ||
-        !make_map_bf16_sw128(&tm_k, pr.k_idx, (uint64_t)pr.B * pr.L, kD, kD * 2, kRows))
+    CUtensorMap tm_q, tm_k, tm_g, tm_w;
+    const uint64_t rows = (uint64_t)pr.B * pr.Tq;
+    if (!make_map_bf16_sw128(&tm_q, pr.q_idx, rows * pr.H, kD, kD * 2, kRows) ||
+        !make_map_bf16_sw128(&tm_k, pr.k_idx, (uint64_t)pr.B * pr.L, kD, kD * 2, kRows) ||
+        !make_map_f32(&tm_g, pr.grad, rows, (uint64_t)pr.L, (uint64_t)pr.L * 4, (uint32_t)p.QPG, kRows) ||
+        !make_map_f32(&tm_w, pr.w, rows, (uint64_t)pr.H, (uint64_t)pr.H * 4, (uint32_t)p.QPG, (uint32_t)pr.H))
         return cudaSuccess;
     *taken = true;
     if (pr.dq || pr.dw) {
-        if (pr.dw && (err = cudaMemsetAsync(pr.dw, 0, (size_t)pr.B * pr.Tq * pr.H * sizeof(float), stream)) !=
-                         cudaSuccess)
-            return err;
         Params q = p;
         q.units = p.B * p.ngroups;
         auto kern = pr.H == 32 ? indexer_bwd_tc_kernel<false, 32>
@@ -567,7 +631,7 @@ cudaError_t launch_indexer_bwd_tc(const IndexerBwdProblem &pr, cudaStream_t stre
             cudaSuccess)
             return err;
         const int grid = q.units < info.sm_count ? q.units : info.sm_count;
-        kern<<<grid, kThreads, kSmem, stream>>>(tm_q, tm_k, q);
+        kern<<<grid, kThreads, kSmem, stream>>>(tm_q, tm_k, tm_g, tm_w, q);
         count_launch();
         if ((err = cudaGetLastError()) != cudaSuccess) return err;
     }
@@ -583,7 +647,7 @@ cudaError_t launch_indexer_bwd_tc(const IndexerBwdProblem &pr, cudaStream_t stre
             cudaSuccess)
             return err;
         const int grid = k.units < info.sm_count ? k.units : info.sm_count;
-        kern<<<grid, kThreads, kSmem, stream>>>(tm_q, tm_k, k);
+        kern<<<grid, kThreads, kSmem, stream>>>(tm_q, tm_k, tm_g, tm_w, k);
         count_launch();
         if ((err = cudaGetLastError()) != cudaSuccess) return err;
         indexer_bwd_reduce_kernel<<<dim3(p.nkt, p.B), 256, 0, stream>>>(k.part, k, pr.dk);

@@ -31,6 +31,11 @@ bool make_map_bf16_sw128(CUtensorMap *map, const void *base, uint64_t rows, uint
 bool make_map_u8_sw128(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint64_t pitch_bytes,
                        uint32_t box_rows);
 
+// The same over fp32 elements without swizzle: boxes of box_rows x box_cols
+// (box_cols * 4 a multiple of 16), rows of the box consecutive in shared memory.
+bool make_map_f32(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint64_t pitch_bytes,
+                  uint32_t box_rows, uint32_t box_cols);
+
 // ----------------------------------------------------------------- indexer
 struct IndexerProblem {
     const void *q_idx;   // [B, Tq, H, d]

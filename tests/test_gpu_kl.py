@@ -190,7 +190,13 @@ def _check_backward(wl, cpu, grad, dq, dk, dw, rows=None, keys=None, rel=1e-5):
     got_dq = dq.cpu().numpy()[rb, ri].astype(np.float64)
     got_dw = dw.cpu().numpy()[rb, ri].astype(np.float64)
     assert np.all(np.abs(got_dq - ref["dq"]) <= rel * ref["dq_abs"] + 1e-6), "dq"
-    assert np.all(np.abs(got_dw - ref["dw"]) <= 1e-5 * ref["dw_abs"] + 1e-6), "dw"
+    # the tensor-core path forms dw as q . sum_s M k with M = g [x > 0] in bf16:
+    # rel of sum |g| ReLU(x), plus fp32 rounding of the 128-term dot product
+    from oracle.kl import to_f64
+    qa = np.abs(to_f64(q)[rb, ri])
+    wa = np.abs(w[rb, ri]).astype(np.float64)
+    dot_abs = (qa * ref["dq_abs"]).sum(axis=-1) / np.where(wa > 0, wa, 1.0)
+    assert np.all(np.abs(got_dw - ref["dw"]) <= rel * ref["dw_abs"] + 1e-6 * dot_abs + 1e-6), "dw"
     kb, ks = keys // wl.L, keys % wl.L
     refk = kl.indexer_backward_keys(q, k, w, g, kb, ks, wl.q_pos0)
     got_dk = dk.cpu().numpy()[kb, ks].astype(np.float64)
