@@ -34,10 +34,12 @@
 //   warp 1     TMEM owner; one thread issues two streams of MMAs, each as
 //              soon as its inputs are ready: MMA 1 runs up to two tiles ahead
 //              of the epilogue, MMA 2 follows it.
-//   warps 2-17 epilogue: four warps per TMEM lane quarter, each taking 32 of
-//              the 128 columns of X and of the accumulator.
-// TMEM: X in two buffers [0, 256), G in two buffers [256, 384) (two bf16 per
-// column), the accumulator [384, 512).
+//   warps 2-17 epilogue: two groups of eight warps taking alternate tiles
+//              (two tiles in flight), two warps per TMEM lane quarter in a
+//              group, 64 columns each; at the end of a unit all sixteen read
+//              the accumulator, 32 columns each.
+// TMEM: X in two buffers [0, 256) and G in two [256, 384) (two bf16 per
+// column), one pair per epilogue group; the accumulator [384, 512).
 // Work: query side, one unit per query group (longest causal range first);
 // key side, one unit per (key tile, chunk of query groups), each chunk's
 // partial dK written to a workspace slot and the slots of a key tile summed
@@ -70,9 +72,9 @@ constexpr int kParts = kEpiWarps / 4;         // column parts of a tile
 constexpr int kCW = 128 / kParts;             // columns per epilogue warp
 constexpr int kThreads = 64 + kEpiThreads;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColX = 0;               // 2 x 128
-constexpr uint32_t kColG = 256;             // 2 x 64
-constexpr uint32_t kColAcc = 384;           // 128
+constexpr uint32_t kColX = 0;               // 2 x 128: X
+constexpr uint32_t kColG = 256;             // 2 x 64: G (bf16 pairs), A of MMA 2
+constexpr uint32_t kColAcc = 384;           // 128: the accumulator
 constexpr uint32_t kIdescMnMajorB = 1u << 16;
 // barriers: res_full/empty[2], st_full/empty[4], x_full/empty[2], g_full/empty[2], acc_full, acc_empty,
 // drain, dw_bar
@@ -203,10 +205,10 @@ indexer_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             mbar_init(&st_full[s], 1);
             mbar_init(&st_empty[s], 1);
         }
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < 2; ++s) {  // buffer s serves the tiles of epilogue group s
             mbar_init(&x_full[s], 1);
-            mbar_init(&x_empty[s], kEpiThreads);
-            mbar_init(&g_full[s], kEpiThreads);
+            mbar_init(&x_empty[s], kEpiThreads / 2);
+            mbar_init(&g_full[s], kEpiThreads / 2);
             mbar_init(&g_empty[s], 1);
         }
         mbar_init(acc_full, 1);
@@ -278,8 +280,9 @@ indexer_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             // thus runs up to two tiles ahead of the epilogue.
             const uint32_t idesc1 = idesc_bf16_f32(kRows, kRows);
             const uint32_t idesc2 = idesc_bf16_f32(kRows, kD) | kIdescMnMajorB;
-            int sb1 = 0, xb1 = 0, sb2 = 0, xb2 = 0, rb = 0;
+            int sb1 = 0, xb1 = 0, sb2 = 0, rb = 0;
             uint32_t sph1 = 0, xph1 = 0, xph2 = 0, rph = 0, aph = 0;
+            int xb2 = 0;
             for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
                 Unit un;
                 if (!decode_unit<KEY_SIDE>(u, p, un)) continue;
@@ -298,12 +301,10 @@ indexer_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                         const uint64_t b_desc = smem_desc_k_sw128(smem_addr(st_sm + sb1 * kTile));
                         const uint32_t d = tmem + kColX + (uint32_t)(xb1 * 128);
 #pragma unroll
-                        for (int h = 0; h < 2; ++h)
-#pragma unroll
-                            for (int kk = 0; kk < 4; ++kk) {
-                                const uint64_t off = (uint64_t)((h * kBox + kk * 32) >> 4);
-                                mma_f16_ss(d, a_desc + off, b_desc + off, idesc1, (h | kk) != 0);
-                            }
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const uint64_t off = (uint64_t)(((kk >> 2) * kBox + (kk & 3) * 32) >> 4);
+                            mma_f16_ss(d, a_desc + off, b_desc + off, idesc1, kk != 0);
+                        }
                         mma_commit(&x_full[xb1]);
                         ++n1;
                         if (++sb1 == kStages) { sb1 = 0; sph1 ^= 1u; }
@@ -353,13 +354,20 @@ indexer_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         // (G = w M; for the power-of-two weights the rounding of M and of G
         // to bf16 is the same). Key side: G = (g w)[X > 0], with g constant
         // per (lane, query) and w per column.
+        // Tiles alternate between two groups of eight warps (grp), so that two
+        // tiles are in the epilogue at once; within a group, the two warps of
+        // a lane quarter (sub) take 64 columns each, in two chunks of kCW.
+        // At the end of a unit all sixteen warps read the accumulator, kCW
+        // columns each (part).
         const int quarter = warp & 3;
-        const int part = (warp - 2) >> 2;          // columns [kCW part, kCW part + kCW)
+        const int part = (warp - 2) >> 2;          // 0..3
+        const int grp = part >> 1, sub = part & 1;
         const int col0 = part * kCW;
         const int r = quarter * 32 + lane;         // TMEM lane: resident row
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-        int xb = 0, unit_n = 0, sb = 0, rb = 0;
-        uint32_t xph = 0, aph = 0, sph = 0, rph = 0;
+        int unit_n = 0, rb = 0;
+        uint32_t aph = 0, rph = 0;
+        uint32_t gt = 0;                           // streamed tiles seen so far (all units)
         for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
             Unit un;
             if (!decode_unit<KEY_SIDE>(u, p, un)) continue;
@@ -370,83 +378,95 @@ indexer_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             const bool row_ok = !KEY_SIDE && i_row < p.Tq;
             const int row = un.b * p.Tq + i_row;
             const int t_row = row_ok ? p.q_pos0 + i_row : -1;  // no such query: nothing passes
-            for (int n = 0; n < ntiles && ok; ++n) {
-                if (!mbar_wait(&x_full[xb], xph)) { ok = false; break; }
+            for (int n = 0; n < ntiles && ok; ++n, ++gt) {
+                const int xbuf = (int)(gt & 1u);
+                if (xbuf != grp) continue;  // the other group takes this tile
+                const uint32_t xphase = (gt >> 1) & 1u;
+                const int sbuf = (int)(gt % kStages);
+                const uint32_t sphase = (gt / kStages) & 1u;
+                if (!mbar_wait(&x_full[xbuf], xphase)) { ok = false; break; }
                 // (complete already: MMA 1 read this stage) makes the TMA writes of g and w visible here
-                if (!mbar_wait(&st_full[sb], sph)) { ok = false; break; }
+                if (!mbar_wait(&st_full[sbuf], sphase)) { ok = false; break; }
                 tc_fence_after();
-                const float *gs = g_sm + sb * (kGBytes / 4);
-                const float *wsm = w_sm + sb * (kWBytes / 4);
-                uint32_t xr[kCW];
-                tmem_ld_32x32b_x32(tmem + lane_addr + kColX + (uint32_t)(xb * 128 + col0), xr);
+                const float *gs = g_sm + sbuf * (kGBytes / 4);
+                const float *wsm = w_sm + sbuf * (kWBytes / 4);
+                // G of kCW columns starting at c0 from X in xr
+                auto chunk = [&](const uint32_t *xr, int c0, uint32_t *gp) {
+                    if (!KEY_SIDE) {
+                        // columns = keys s_base + c; g[t, s] is the same for the warp's lanes
+                        const int s_base = (un.kt0 + n) * kRows + c0;
+                        const float4 *g4 = reinterpret_cast<const float4 *>(gs + qi * kRows + c0);
+                        if (t_row < s_base) {  // every key of this part lies after t (or no query)
+    #pragma unroll
+                            for (int c = 0; c < kCW / 2; ++c) gp[c] = 0u;
+                        } else if (s_base + kCW - 1 <= t_row) {  // no key of this part after t
+    #pragma unroll
+                            for (int c4 = 0; c4 < kCW / 4; ++c4) {
+                                const float4 gv = g4[c4];
+                                gp[2 * c4] = pack_bf16x2(__uint_as_float(xr[4 * c4]) > 0.f ? gv.x : 0.f,
+                                                         __uint_as_float(xr[4 * c4 + 1]) > 0.f ? gv.y : 0.f);
+                                gp[2 * c4 + 1] = pack_bf16x2(__uint_as_float(xr[4 * c4 + 2]) > 0.f ? gv.z : 0.f,
+                                                             __uint_as_float(xr[4 * c4 + 3]) > 0.f ? gv.w : 0.f);
+                            }
+                        } else {  // the diagonal: keys after t pass nothing
+    #pragma unroll
+                            for (int c4 = 0; c4 < kCW / 4; ++c4) {
+                                const float4 gv = g4[c4];
+                                const int s = s_base + 4 * c4;
+                                const float m0 = (__uint_as_float(xr[4 * c4]) > 0.f && s <= t_row) ? gv.x : 0.f;
+                                const float m1 = (__uint_as_float(xr[4 * c4 + 1]) > 0.f && s + 1 <= t_row) ? gv.y : 0.f;
+                                const float m2 = (__uint_as_float(xr[4 * c4 + 2]) > 0.f && s + 2 <= t_row) ? gv.z : 0.f;
+                                const float m3 = (__uint_as_float(xr[4 * c4 + 3]) > 0.f && s + 3 <= t_row) ? gv.w : 0.f;
+                                gp[2 * c4] = pack_bf16x2(m0, m1);
+                                gp[2 * c4 + 1] = pack_bf16x2(m2, m3);
+                            }
+                        }
+                    } else {
+                        // lanes = keys s; columns = (query, head) pairs of group g
+                        const int g = un.g0 + n;
+                        const int s = un.kt0 * kRows + r;
+                        constexpr int QPP = kCW / H > 0 ? kCW / H : 1;  // queries in this part
+                        constexpr int C4 = (H < kCW ? H : kCW) / 4;     // float4s of one query in the part
+    #pragma unroll
+                        for (int z = 0; z < QPP; ++z) {
+                            const int qz = c0 / H + z;
+                            const int i = g * QPG + qz;
+                            float gq = 0.f;
+                            if (i < p.Tq && s <= p.q_pos0 + i) gq = gs[qz * kRows + r];
+                            const float4 *w4 = reinterpret_cast<const float4 *>(wsm + qz * H + (c0 % H));
+    #pragma unroll
+                            for (int c4 = 0; c4 < C4; ++c4) {
+                                const int cc = z * (C4 * 4) + 4 * c4;  // column within the part
+                                const float4 wv = w4[c4];
+                                float gw0, gw1, gw2, gw3;
+                                mul2(gw0, gw1, gq, gq, wv.x, wv.y);
+                                mul2(gw2, gw3, gq, gq, wv.z, wv.w);
+                                const float x0 = __uint_as_float(xr[cc]), x1 = __uint_as_float(xr[cc + 1]);
+                                const float x2 = __uint_as_float(xr[cc + 2]), x3 = __uint_as_float(xr[cc + 3]);
+                                gp[cc / 2] = pack_bf16x2(x0 > 0.f ? gw0 : 0.f, x1 > 0.f ? gw1 : 0.f);
+                                gp[cc / 2 + 1] = pack_bf16x2(x2 > 0.f ? gw2 : 0.f, x3 > 0.f ? gw3 : 0.f);
+                            }
+                        }
+                    }
+                };
+                uint32_t xr[kCW], gpa[kCW / 2], gpb[kCW / 2];
+                const int c0a = sub * (2 * kCW), c0b = c0a + kCW;
+                tmem_ld_32x32b_x32(tmem + lane_addr + kColX + (uint32_t)(xbuf * 128 + c0a), xr);
+                tmem_ld_wait();
+                chunk(xr, c0a, gpa);
+                tmem_ld_32x32b_x32(tmem + lane_addr + kColX + (uint32_t)(xbuf * 128 + c0b), xr);
                 tmem_ld_wait();
                 tc_fence_before();
-                mbar_arrive(&x_empty[xb]);
-                uint32_t gp[kCW / 2];
-                if (!KEY_SIDE) {
-                    // columns = keys s_base + c; g[t, s] is the same for the warp's lanes
-                    const int s_base = (un.kt0 + n) * kRows + col0;
-                    const float4 *g4 = reinterpret_cast<const float4 *>(gs + qi * kRows + col0);
-                    if (t_row < s_base) {  // every key of this part lies after t (or no query)
-#pragma unroll
-                        for (int c = 0; c < kCW / 2; ++c) gp[c] = 0u;
-                    } else if (s_base + kCW - 1 <= t_row) {  // no key of this part after t
-#pragma unroll
-                        for (int c4 = 0; c4 < kCW / 4; ++c4) {
-                            const float4 gv = g4[c4];
-                            gp[2 * c4] = pack_bf16x2(__uint_as_float(xr[4 * c4]) > 0.f ? gv.x : 0.f,
-                                                     __uint_as_float(xr[4 * c4 + 1]) > 0.f ? gv.y : 0.f);
-                            gp[2 * c4 + 1] = pack_bf16x2(__uint_as_float(xr[4 * c4 + 2]) > 0.f ? gv.z : 0.f,
-                                                         __uint_as_float(xr[4 * c4 + 3]) > 0.f ? gv.w : 0.f);
-                        }
-                    } else {  // the diagonal: keys after t pass nothing
-#pragma unroll
-                        for (int c4 = 0; c4 < kCW / 4; ++c4) {
-                            const float4 gv = g4[c4];
-                            const int s = s_base + 4 * c4;
-                            const float m0 = (__uint_as_float(xr[4 * c4]) > 0.f && s <= t_row) ? gv.x : 0.f;
-                            const float m1 = (__uint_as_float(xr[4 * c4 + 1]) > 0.f && s + 1 <= t_row) ? gv.y : 0.f;
-                            const float m2 = (__uint_as_float(xr[4 * c4 + 2]) > 0.f && s + 2 <= t_row) ? gv.z : 0.f;
-                            const float m3 = (__uint_as_float(xr[4 * c4 + 3]) > 0.f && s + 3 <= t_row) ? gv.w : 0.f;
-                            gp[2 * c4] = pack_bf16x2(m0, m1);
-                            gp[2 * c4 + 1] = pack_bf16x2(m2, m3);
-                        }
-                    }
-                } else {
-                    // lanes = keys s; columns = (query, head) pairs of group g
-                    const int g = un.g0 + n;
-                    const int s = un.kt0 * kRows + r;
-                    constexpr int QPP = kCW / H > 0 ? kCW / H : 1;  // queries in this part
-                    constexpr int C4 = (H < kCW ? H : kCW) / 4;     // float4s of one query in the part
-#pragma unroll
-                    for (int z = 0; z < QPP; ++z) {
-                        const int qz = col0 / H + z;
-                        const int i = g * QPG + qz;
-                        float gq = 0.f;
-                        if (i < p.Tq && s <= p.q_pos0 + i) gq = gs[qz * kRows + r];
-                        const float4 *w4 = reinterpret_cast<const float4 *>(wsm + qz * H + (col0 % H));
-#pragma unroll
-                        for (int c4 = 0; c4 < C4; ++c4) {
-                            const int cc = z * (C4 * 4) + 4 * c4;  // column within the part
-                            const float4 wv = w4[c4];
-                            float gw0, gw1, gw2, gw3;
-                            mul2(gw0, gw1, gq, gq, wv.x, wv.y);
-                            mul2(gw2, gw3, gq, gq, wv.z, wv.w);
-                            const float x0 = __uint_as_float(xr[cc]), x1 = __uint_as_float(xr[cc + 1]);
-                            const float x2 = __uint_as_float(xr[cc + 2]), x3 = __uint_as_float(xr[cc + 3]);
-                            gp[cc / 2] = pack_bf16x2(x0 > 0.f ? gw0 : 0.f, x1 > 0.f ? gw1 : 0.f);
-                            gp[cc / 2 + 1] = pack_bf16x2(x2 > 0.f ? gw2 : 0.f, x3 > 0.f ? gw3 : 0.f);
-                        }
-                    }
-                }
-                if (!mbar_wait(&g_empty[xb], xph ^ 1u)) { ok = false; break; }
+                mbar_arrive(&x_empty[xbuf]);
+                chunk(xr, c0b, gpb);
+                // this group's G buffer: MMA 2 of its previous tile has read it
+                if (!mbar_wait(&g_empty[xbuf], xphase ^ 1u)) { ok = false; break; }
                 tc_fence_after();
-                tmem_st_32x32b_x16(tmem + lane_addr + kColG + (uint32_t)(xb * 64 + col0 / 2), gp);
+                tmem_st_32x32b_x16(tmem + lane_addr + kColG + (uint32_t)(xbuf * 64 + c0a / 2), gpa);
+                tmem_st_32x32b_x16(tmem + lane_addr + kColG + (uint32_t)(xbuf * 64 + c0b / 2), gpb);
                 tmem_st_wait();
                 tc_fence_before();
-                mbar_arrive(&g_full[xb]);
-                if (++xb == 2) { xb = 0; xph ^= 1u; }
-                if (++sb == kStages) { sb = 0; sph ^= 1u; }
+                mbar_arrive(&g_full[xbuf]);
             }
             if (!ok) break;
             // ---- the unit's accumulator
