@@ -295,8 +295,9 @@ size_t dsa_forward_workspace_bytes(const dsa_forward_args *a);
  *   grad     [B, Tq, L] fp32 or NULL: softmax(I_t)_s - p_t[s] on the set, 0
  *            everywhere else (every entry is written). Must not overlap
  *            scores or target.
- * Arithmetic: fp32 with expf/logf; the loss is formed from the row sums
- * sum(a), sum(a I), sum(a log a) and the log-sum-exp of I over the set.
+ * Arithmetic: fp32, exp and log through the hardware base-2 approximations
+ * (relative error below 2^-21); the loss is formed from the row sums sum(a),
+ * sum(a I), sum(a log a) and the log-sum-exp of I over the set.
  * Errors: DSA_ERR_INVALID_ARG for a null scores, target or loss_rows, bad
  * sizes (as dsa_topk; k >= 1 when idx is given) or pointers not 4-byte
  * aligned.

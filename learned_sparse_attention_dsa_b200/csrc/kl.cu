@@ -13,6 +13,8 @@
 // needs no second pass. Pass 2 (only when the gradient is wanted) reads the
 // row again, from L2, and writes exp(I - LSE) - a / S. HBM-bound: 8 bytes
 // read per causal pair (score and target) plus 4 written for the gradient.
+// exp and log use the hardware base-2 approximations: with the library
+// functions the kernel was bound by instruction issue, not by memory.
 #include <math.h>
 
 #include "common.cuh"
@@ -24,6 +26,17 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+// exp(x) and log(x) through the hardware base-2 approximations (relative
+// error below 2^-21 after the scaling); ex2 of -inf is 0.
+__device__ __forceinline__ float fast_exp(float x) { return ex2_approx(x * kLog2e); }
+__device__ __forceinline__ float fast_log(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y * kLn2;
+}
 
 struct Acc {
     float m, z, S, aI, alna;
@@ -41,15 +54,15 @@ __device__ __forceinline__ void acc_add(Acc &c, float I, float a) {
     if (I == -INFINITY) {
         // exp(-inf) adds nothing to z
     } else if (I > c.m) {
-        c.z = c.z * expf(c.m - I) + 1.f;  // exp(-inf) = 0 for the first element
+        c.z = c.z * fast_exp(c.m - I) + 1.f;  // exp(-inf) = 0 for the first element
         c.m = I;
     } else {
-        c.z += expf(I - c.m);
+        c.z += fast_exp(I - c.m);
     }
     c.S += a;
     if (a > 0.f) {
         c.aI += a * I;
-        c.alna += a * logf(a);
+        c.alna += a * fast_log(a);
     }
 }
 
@@ -58,7 +71,7 @@ __device__ __forceinline__ void acc_merge(Acc &c, const Acc &o) {
     if (m == -INFINITY) {
         c.z = 0.f;
     } else {
-        c.z = c.z * expf(c.m - m) + o.z * expf(o.m - m);
+        c.z = c.z * fast_exp(c.m - m) + o.z * fast_exp(o.m - m);
     }
     c.m = m;
     c.S += o.S;
@@ -156,7 +169,7 @@ indexer_kl_kernel(const KlParams p) {
         const float *a = p.target + (size_t)row * p.k;
         for (int j = tid; j < p.k; j += kThreads) {
             const int s = sel[j];
-            if (s >= 0 && s <= t) g[s] = expf(I[s] - lse) - a[j] * inv_S;
+            if (s >= 0 && s <= t) g[s] = fast_exp(I[s] - lse) - a[j] * inv_S;
         }
     } else {
         const float *a = p.target + (size_t)row * p.L;
@@ -171,16 +184,16 @@ indexer_kl_kernel(const KlParams p) {
                 float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (s < n) {
                     const float4 x = I4[v], y = a4[v];
-                    o.x = expf(x.x - lse) - y.x * inv_S;
-                    if (s + 1 < n) o.y = expf(x.y - lse) - y.y * inv_S;
-                    if (s + 2 < n) o.z = expf(x.z - lse) - y.z * inv_S;
-                    if (s + 3 < n) o.w = expf(x.w - lse) - y.w * inv_S;
+                    o.x = fast_exp(x.x - lse) - y.x * inv_S;
+                    if (s + 1 < n) o.y = fast_exp(x.y - lse) - y.y * inv_S;
+                    if (s + 2 < n) o.z = fast_exp(x.z - lse) - y.z * inv_S;
+                    if (s + 3 < n) o.w = fast_exp(x.w - lse) - y.w * inv_S;
                 }
                 g4[v] = o;
             }
             s0 = p.L & ~3;
         }
-        for (int s = s0 + tid; s < p.L; s += kThreads) g[s] = s < n ? expf(I[s] - lse) - a[s] * inv_S : 0.f;
+        for (int s = s0 + tid; s < p.L; s += kThreads) g[s] = s < n ? fast_exp(I[s] - lse) - a[s] * inv_S : 0.f;
     }
 }
 

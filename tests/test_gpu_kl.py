@@ -131,7 +131,8 @@ def test_kl_degenerate_rows(cuda):
     assert loss[0].item() == 0.0 and not grad[0].any()
     # a single candidate: position 0 of a one-row prefill
     l1, _, g1 = binding.indexer_kl(scores[:1, :, :1].contiguous().cuda(), target[1:2, :, :1].contiguous().cuda(), 0)
-    assert l1.item() == 0.0 and g1.item() == 0.0
+    # exactly 0 up to the hardware exp/log approximations (relative 2^-21)
+    assert abs(l1.item()) <= 1e-6 and abs(g1.item()) <= 1e-6
     # shuffled selection with padding in the middle; no gradient requested
     idx = torch.tensor([[[9, -1, 2, 15, 0, -1]]], dtype=torch.int32).repeat(4, 1, 1)
     tsel = torch.rand(4, 1, 6, generator=torch.Generator().manual_seed(9))
