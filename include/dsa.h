@@ -351,6 +351,63 @@ dsa_status dsa_indexer_backward(const void *q_idx, const void *k_idx, const floa
 size_t dsa_indexer_backward_workspace_bytes(int B, int Tq, int L, int q_pos0, int H_I, int d_I,
                                             dsa_dtype dt);
 
+/* ------------------------------------------------------------------------
+ * Context parallelism: the indexer keys and the KV cache split by position
+ * over P ranks (rank r holds positions [key_pos0_r, key_pos0_r + L_r)), every
+ * rank holding all the query rows. Every member of the global selection S_t
+ * ("Learned Token Selection" §3.1) is among the k best of its own shard, so
+ * the shards' selections merge into S_t exactly; the attention over S_t
+ * (§3.3) is a log-sum-exp merge of the shards' partial attentions. A step:
+ * dsa_indexer_scores + dsa_topk on the local keys, dsa_cp_select_candidates,
+ * an all-gather of the candidates (k scores and k positions per row and
+ * rank), dsa_cp_merge, dsa_cp_localize, dsa_sparse_attn with lse on the local
+ * cache, an all-gather of (output, lse), dsa_cp_combine. The collectives are
+ * the caller's (NCCL through torch.distributed in the Python package).
+ * ------------------------------------------------------------------------ */
+
+/*
+ * dsa_cp_select_candidates -- a shard's selection as merge candidates.
+ *   scores      [rows, L] fp32 local scores; idx [rows, k] int32 local
+ *               positions (dsa_topk), -1 padded.
+ *   cand_scores [rows, k] fp32: scores[row, idx], -inf for padding.
+ *   cand_idx    [rows, k] int32: idx + key_pos0 (global positions), -1 for
+ *               padding (and for any entry outside [0, L)).
+ */
+dsa_status dsa_cp_select_candidates(const float *scores, const int32_t *idx, int rows, int L, int k,
+                                    int key_pos0, float *cand_scores, int32_t *cand_idx,
+                                    dsa_stream_t stream);
+
+/*
+ * dsa_cp_merge -- the global selection from P shards' candidates.
+ *   cand_scores, cand_idx  [P, rows, kc] (rank-major, as an all-gather of the
+ *               ranks' [rows, kc] arrays leaves them), ranks in ascending
+ *               position order, each rank's list ascending (dsa_topk order),
+ *               cand_idx -1 for no candidate.
+ *   idx         [rows, k] int32: the k best candidates by score, equal scores
+ *               to the lower position, as ascending global positions, then
+ *               -1 (all valid candidates when there are at most k).
+ * Errors: DSA_ERR_UNSUPPORTED when P * kc > 16384 (one CTA holds a row).
+ */
+dsa_status dsa_cp_merge(const float *cand_scores, const int32_t *cand_idx, int P, int rows, int kc, int k,
+                        int32_t *idx, dsa_stream_t stream);
+
+/* dsa_cp_localize -- idx_local = idx - key_pos0 where key_pos0 <= idx <
+ * key_pos0 + L_local, else -1 ([rows, k] int32 both). */
+dsa_status dsa_cp_localize(const int32_t *idx, int rows, int k, int key_pos0, int L_local,
+                           int32_t *idx_local, dsa_stream_t stream);
+
+/*
+ * dsa_cp_combine -- merge P partial attentions over disjoint key sets.
+ *   parts     [P, rows, Hq, Dv] in dt (DSA_BF16 or DSA_F32); parts_lse
+ *             [P, rows, Hq] fp32, -inf where a part selected nothing (its
+ *             output is then ignored).
+ *   out       [rows, Hq, Dv] in dt: sum_p exp(lse_p - LSE) parts[p], with
+ *             LSE = log sum_p exp(lse_p); lse [rows, Hq] fp32 or NULL: LSE.
+ *             A pair with no part: out 0, LSE -inf.
+ */
+dsa_status dsa_cp_combine(const void *parts, const float *parts_lse, int P, int rows, int Hq, int Dv,
+                          dsa_dtype dt, void *out, float *lse, dsa_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

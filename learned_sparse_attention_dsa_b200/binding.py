@@ -27,7 +27,8 @@ STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED",
 EXPORTED = ("dsa_version", "dsa_kernel_launch_count", "dsa_status_string", "dsa_indexer_scores", "dsa_topk",
             "dsa_topk_workspace_bytes", "dsa_sparse_attn", "dsa_sparse_attn_workspace_bytes",
             "dsa_forward", "dsa_forward_workspace_bytes", "dsa_device_error", "dsa_topk_ex",
-            "dsa_indexer_kl", "dsa_indexer_backward", "dsa_indexer_backward_workspace_bytes")
+            "dsa_indexer_kl", "dsa_indexer_backward", "dsa_indexer_backward_workspace_bytes",
+            "dsa_cp_select_candidates", "dsa_cp_merge", "dsa_cp_localize", "dsa_cp_combine")
 
 
 class DSAError(RuntimeError):
@@ -98,6 +99,14 @@ def load_library(path: str = LIB_PATH):
     lib.dsa_indexer_backward.restype = ci
     lib.dsa_indexer_backward_workspace_bytes.argtypes = [ci, ci, ci, ci, ci, ci, ci]
     lib.dsa_indexer_backward_workspace_bytes.restype = sz
+    lib.dsa_cp_select_candidates.argtypes = [vp, vp, ci, ci, ci, ci, vp, vp, vp]
+    lib.dsa_cp_select_candidates.restype = ci
+    lib.dsa_cp_merge.argtypes = [vp, vp, ci, ci, ci, ci, vp, vp]
+    lib.dsa_cp_merge.restype = ci
+    lib.dsa_cp_localize.argtypes = [vp, ci, ci, ci, ci, vp, vp]
+    lib.dsa_cp_localize.restype = ci
+    lib.dsa_cp_combine.argtypes = [vp, vp, ci, ci, ci, ci, ci, vp, vp, vp]
+    lib.dsa_cp_combine.restype = ci
     _lib = lib
     return lib
 
@@ -239,6 +248,66 @@ def indexer_backward(q_idx, k_idx, w, grad, q_pos0: int = 0, dq=None, dk=None, d
                                   _p(dq), _p(dk), _p(dw), _p(ws), nbytes, _stream(stream))
     _check(st, "dsa_indexer_backward")
     return dq, dk, dw
+
+
+def cp_select_candidates(scores, idx, key_pos0: int, cand_scores=None, cand_idx=None, stream=None):
+    """dsa_cp_select_candidates: ([..., k] fp32 scores, [..., k] int32 global
+    positions) of a shard's selection (scores [..., L], idx [..., k])."""
+    lib = load_library()
+    _need_cuda(scores, idx, cand_scores, cand_idx)
+    L, k = scores.shape[-1], idx.shape[-1]
+    rows = idx.numel() // k
+    if cand_scores is None:
+        cand_scores = torch.empty(idx.shape, dtype=torch.float32, device=idx.device)
+    if cand_idx is None:
+        cand_idx = torch.empty(idx.shape, dtype=torch.int32, device=idx.device)
+    st = lib.dsa_cp_select_candidates(_p(scores), _p(idx), rows, L, k, key_pos0, _p(cand_scores), _p(cand_idx),
+                                      _stream(stream))
+    _check(st, "dsa_cp_select_candidates")
+    return cand_scores, cand_idx
+
+
+def cp_merge(cand_scores, cand_idx, k: int, idx=None, stream=None):
+    """dsa_cp_merge: candidates [P, rows..., kc] -> global selection
+    [rows..., k] (ascending positions, -1 padded)."""
+    lib = load_library()
+    _need_cuda(cand_scores, cand_idx, idx)
+    P, kc = cand_scores.shape[0], cand_scores.shape[-1]
+    rows = cand_scores.numel() // (P * kc)
+    if idx is None:
+        idx = torch.empty(tuple(cand_scores.shape[1:-1]) + (k,), dtype=torch.int32, device=cand_scores.device)
+    st = lib.dsa_cp_merge(_p(cand_scores), _p(cand_idx), P, rows, kc, k, _p(idx), _stream(stream))
+    _check(st, "dsa_cp_merge")
+    return idx
+
+
+def cp_localize(idx, key_pos0: int, L_local: int, out=None, stream=None):
+    """dsa_cp_localize: global positions -> this shard's positions (or -1)."""
+    lib = load_library()
+    _need_cuda(idx, out)
+    k = idx.shape[-1]
+    if out is None:
+        out = torch.empty_like(idx)
+    st = lib.dsa_cp_localize(_p(idx), idx.numel() // k, k, key_pos0, L_local, _p(out), _stream(stream))
+    _check(st, "dsa_cp_localize")
+    return out
+
+
+def cp_combine(parts, parts_lse, out=None, lse=None, want_lse=False, stream=None):
+    """dsa_cp_combine: parts [P, rows..., Hq, Dv], parts_lse [P, rows..., Hq]
+    -> out [rows..., Hq, Dv] (and the merged lse)."""
+    lib = load_library()
+    _need_cuda(parts, parts_lse, out, lse)
+    P, Hq, Dv = parts.shape[0], parts.shape[-2], parts.shape[-1]
+    rows = parts.numel() // (P * Hq * Dv)
+    if out is None:
+        out = torch.empty(parts.shape[1:], dtype=parts.dtype, device=parts.device)
+    if lse is None and want_lse:
+        lse = torch.empty(parts_lse.shape[1:], dtype=torch.float32, device=parts.device)
+    st = lib.dsa_cp_combine(_p(parts), _p(parts_lse), P, rows, Hq, Dv, _dt(parts), _p(out), _p(lse),
+                            _stream(stream))
+    _check(st, "dsa_cp_combine")
+    return (out, lse) if want_lse else out
 
 
 def attn_shape(q, k_cache, v_cache, k: int, scale=None) -> AttnShape:

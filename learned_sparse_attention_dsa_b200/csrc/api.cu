@@ -354,4 +354,43 @@ dsa_status dsa_indexer_backward(const void *q_idx, const void *k_idx, const floa
     return from_cuda(launch_indexer_bwd(p, static_cast<cudaStream_t>(stream)));
 }
 
+dsa_status dsa_cp_select_candidates(const float *scores, const int32_t *idx, int rows, int L, int k, int key_pos0,
+                                    float *cand_scores, int32_t *cand_idx, dsa_stream_t stream) {
+    if (!scores || !idx || !cand_scores || !cand_idx) return DSA_ERR_INVALID_ARG;
+    if (rows < 1 || L < 1 || k < 1 || key_pos0 < 0) return DSA_ERR_INVALID_ARG;
+    if (!aligned(scores, 4) || !aligned(idx, 4) || !aligned(cand_scores, 4) || !aligned(cand_idx, 4))
+        return DSA_ERR_INVALID_ARG;
+    return from_cuda(launch_select_candidates(scores, idx, rows, L, k, key_pos0, cand_scores, cand_idx,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
+dsa_status dsa_cp_merge(const float *cand_scores, const int32_t *cand_idx, int P, int rows, int kc, int k,
+                        int32_t *idx, dsa_stream_t stream) {
+    if (!cand_scores || !cand_idx || !idx) return DSA_ERR_INVALID_ARG;
+    if (P < 1 || rows < 1 || kc < 1 || k < 1) return DSA_ERR_INVALID_ARG;
+    if ((long long)P * kc > 16384) return DSA_ERR_UNSUPPORTED;
+    if (!aligned(cand_scores, 4) || !aligned(cand_idx, 4) || !aligned(idx, 4)) return DSA_ERR_INVALID_ARG;
+    return from_cuda(launch_topk_merge(cand_scores, cand_idx, P, rows, kc, k, idx, static_cast<cudaStream_t>(stream)));
+}
+
+dsa_status dsa_cp_localize(const int32_t *idx, int rows, int k, int key_pos0, int L_local, int32_t *idx_local,
+                           dsa_stream_t stream) {
+    if (!idx || !idx_local || rows < 1 || k < 1 || key_pos0 < 0 || L_local < 1) return DSA_ERR_INVALID_ARG;
+    if (!aligned(idx, 4) || !aligned(idx_local, 4)) return DSA_ERR_INVALID_ARG;
+    return from_cuda(launch_localize(idx, (long long)rows * k, key_pos0, L_local, idx_local,
+                                     static_cast<cudaStream_t>(stream)));
+}
+
+dsa_status dsa_cp_combine(const void *parts, const float *parts_lse, int P, int rows, int Hq, int Dv, dsa_dtype dt,
+                          void *out, float *lse, dsa_stream_t stream) {
+    if (!parts || !parts_lse || !out) return DSA_ERR_INVALID_ARG;
+    if (P < 1 || rows < 1 || Hq < 1 || Dv < 1) return DSA_ERR_INVALID_ARG;
+    if (!valid_dtype(dt)) return DSA_ERR_UNSUPPORTED;
+    const size_t eb = dtype_bytes(dt);
+    if (!aligned(parts, eb) || !aligned(out, eb) || !aligned(parts_lse, 4) || (lse && !aligned(lse, 4)))
+        return DSA_ERR_INVALID_ARG;
+    return from_cuda(launch_combine_parts(parts, parts_lse, P, (long long)rows * Hq, Dv, dt, out, lse,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

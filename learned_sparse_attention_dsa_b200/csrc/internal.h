@@ -112,6 +112,16 @@ size_t indexer_bwd_cuda_core_smem_bytes(int H, int d);
 // Workspace the tensor-core path needs for this problem (0: it does not take it).
 size_t indexer_bwd_tc_workspace_bytes(const IndexerBwdProblem &p);
 
+// ----------------------------------------------------------------- context parallelism
+cudaError_t launch_select_candidates(const float *scores, const int32_t *idx, long long rows, int L, int k,
+                                     int key_pos0, float *cand_score, int32_t *cand_idx, cudaStream_t stream);
+cudaError_t launch_topk_merge(const float *cand_score, const int32_t *cand_idx, int P, int rows, int kc, int k,
+                              int32_t *idx, cudaStream_t stream);
+cudaError_t launch_localize(const int32_t *idx, long long n, int key_pos0, int L_local, int32_t *out,
+                            cudaStream_t stream);
+cudaError_t launch_combine_parts(const void *parts, const float *parts_lse, int P, long long pairs, int Dv,
+                                 dsa_dtype dt, void *out, float *lse, cudaStream_t stream);
+
 // Read and clear the error word of a kernel family with bounded waits
 // (non-zero: some launch gave up on a wait).
 unsigned int indexer_take_device_error();

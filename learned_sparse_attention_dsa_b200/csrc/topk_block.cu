@@ -178,7 +178,130 @@ cudaError_t launch_block(const TopkProblem &p, cudaStream_t stream) {
     return cudaGetLastError();
 }
 
+// Merge of per-shard selections (context parallelism): row `row` has P * kc
+// candidates, candidate c = p * kc + j at cand_*[(p * rows + row) * kc + j],
+// ordered by ascending global position (shards in position order, each list
+// ascending). The k best valid candidates (cand_idx >= 0) by score, ties to
+// the lower position (= the lower candidate number), are written as global
+// positions in ascending order, then -1. Same radix select as above, with the
+// invalid candidates given key 0, below every score.
+template <int KPT>
+__global__ void __launch_bounds__(kBlockThreads, 1)
+topk_merge_kernel(const float *__restrict__ cand_score, const int32_t *__restrict__ cand_idx, int P, int rows,
+                  int kc, int k, int32_t *__restrict__ idx) {
+    __shared__ int hist[kBins];
+    __shared__ int warp_sum[kBlockWarps];
+    __shared__ int warp_gt[kBlockWarps], warp_eq[kBlockWarps];
+    __shared__ int s_digit, s_above;
+
+    const int row = blockIdx.x;
+    const int n = P * kc;
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    int32_t *out = idx + (size_t)row * k;
+    for (int b = tid; b < kBins; b += kBlockThreads) hist[b] = 0;
+
+    const int base = warp * 32 * KPT + lane;
+    uint32_t key[KPT];
+    int nvalid = 0;
+#pragma unroll
+    for (int j = 0; j < KPT; ++j) {
+        const int c = base + 32 * j;
+        key[j] = 0u;
+        if (c < n) {
+            const int p = c / kc, jj = c - p * kc;
+            const size_t off = ((size_t)p * rows + row) * kc + jj;
+            if (cand_idx[off] >= 0) {
+                key[j] = block_order_key(cand_score[off]);
+                ++nvalid;
+            }
+        }
+    }
+    nvalid = warp_sum_int(nvalid);
+    if (lane == 0) warp_gt[warp] = nvalid;
+    __syncthreads();
+    int total = 0;
+    for (int w = 0; w < kBlockWarps; ++w) total += warp_gt[w];
+    __syncthreads();
+
+    uint32_t T = 0u;  // every valid key is above 0
+    int r = 0;
+    if (total > k) {
+#pragma unroll
+        for (int j = 0; j < KPT; ++j)
+            if (base + 32 * j < n) atomicAdd(&hist[key[j] >> 21], 1);
+        __syncthreads();
+        int want = k;
+        const uint32_t d1 = (uint32_t)find_digit(hist, want, warp_sum, &s_digit, &s_above);
+        want -= s_above;
+#pragma unroll
+        for (int j = 0; j < KPT; ++j)
+            if (base + 32 * j < n && (key[j] >> 21) == d1) atomicAdd(&hist[(key[j] >> 10) & 2047u], 1);
+        __syncthreads();
+        const uint32_t d2 = (uint32_t)find_digit(hist, want, warp_sum, &s_digit, &s_above);
+        want -= s_above;
+        const uint32_t hi2 = (d1 << 11) | d2;
+#pragma unroll
+        for (int j = 0; j < KPT; ++j)
+            if (base + 32 * j < n && (key[j] >> 10) == hi2) atomicAdd(&hist[key[j] & 1023u], 1);
+        __syncthreads();
+        const uint32_t d3 = (uint32_t)find_digit(hist, want, warp_sum, &s_digit, &s_above);
+        want -= s_above;
+        T = (hi2 << 10) | d3;
+        r = want;
+    }
+
+    int gt = 0, eq = 0;
+#pragma unroll
+    for (int j = 0; j < KPT; ++j) {
+        gt += __popc(__ballot_sync(0xffffffffu, key[j] > T));
+        eq += __popc(__ballot_sync(0xffffffffu, key[j] == T));
+    }
+    if (lane == 0) {
+        warp_gt[warp] = gt;
+        warp_eq[warp] = eq;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const int g = warp_gt[lane], e = warp_eq[lane];
+        const int gi = warp_inclusive_scan(g), ei = warp_inclusive_scan(e);
+        warp_gt[lane] = gi - g;
+        warp_eq[lane] = ei - e;
+    }
+    __syncthreads();
+    int gt_b = warp_gt[warp], eq_b = warp_eq[warp];
+    const unsigned lt = lanemask_lt_block();
+#pragma unroll
+    for (int j = 0; j < KPT; ++j) {
+        const bool g = key[j] > T, e = key[j] == T && T != 0u;
+        const unsigned gm = __ballot_sync(0xffffffffu, g);
+        const unsigned em = __ballot_sync(0xffffffffu, e);
+        const int eq_rank = eq_b + __popc(em & lt);
+        if (g || (e && eq_rank < r)) {
+            const int c = base + 32 * j;
+            const int p = c / kc, jj = c - p * kc;
+            out[gt_b + __popc(gm & lt) + min(r, eq_rank)] = cand_idx[((size_t)p * rows + row) * kc + jj];
+        }
+        gt_b += __popc(gm);
+        eq_b += __popc(em);
+    }
+    const int kept = total < k ? total : k;
+    for (int j = kept + tid; j < k; j += kBlockThreads) out[j] = -1;
+}
+
 }  // namespace
+
+cudaError_t launch_topk_merge(const float *cand_score, const int32_t *cand_idx, int P, int rows, int kc, int k,
+                              int32_t *idx, cudaStream_t stream) {
+    const long long n = (long long)P * kc;
+    if (n > (long long)kBlockThreads * 16 || rows < 1) return cudaErrorInvalidValue;
+    if (n <= (long long)kBlockThreads * 8)
+        topk_merge_kernel<8><<<rows, kBlockThreads, 0, stream>>>(cand_score, cand_idx, P, rows, kc, k, idx);
+    else
+        topk_merge_kernel<16><<<rows, kBlockThreads, 0, stream>>>(cand_score, cand_idx, P, rows, kc, k, idx);
+    count_launch();
+    return cudaGetLastError();
+}
 
 // One CTA per row for many rows of at most 16,384 scores (measured on B200:
 // prefill8k 0.41 -> 0.27 ms; with 32 keys per thread the kernel spills and is
