@@ -816,6 +816,96 @@ def run_train(args, wl):
         dist.destroy_process_group()
 
 
+# ------------------------------------------------------------------ context parallelism
+
+def run_cp(args, wl):
+    """The context-parallel decode step with its P shards emulated one after
+    another on one GPU: every shard's indexer, top-k and candidate gather,
+    the merge, every shard's attention over its part of the selection, and
+    the log-sum-exp combine. Each shard writes into its slot of the buffers an
+    all-gather would fill, so the step runs the library's kernels only (no
+    collective: one GPU)."""
+    from learned_sparse_attention_dsa_b200 import binding
+
+    world, rank, _ = _dist()
+    if world > 1:
+        raise SystemExit("--pass cp emulates the shards on one GPU; run it with --gpus 1")
+    if not wl.is_decode:
+        raise SystemExit("--pass cp is a decode step (one query row per batch entry)")
+    P = args.shards
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    binding.load_library()
+    cpu = make_inputs(wl)
+    dev = to_device(cpu, device)
+    step_len = -(-wl.L // P)
+    bounds = [(a, min(wl.L, a + step_len)) for a in range(0, wl.L, step_len)]
+    P = len(bounds)
+    shards = []
+    for a, b in bounds:
+        kc = dev["k_cache"][:, a:b].contiguous()
+        shards.append({"a": a, "L": b - a, "k_idx": dev["k_idx"][:, a:b].contiguous(), "k": kc,
+                       "v": kc[..., : wl.Dv] if wl.kv_alias else dev["v_cache"][:, a:b].contiguous(),
+                       "scores": torch.empty((wl.B, 1, b - a), dtype=torch.float32, device=device),
+                       "idx": torch.empty((wl.B, 1, wl.k), dtype=torch.int32, device=device),
+                       "idx_local": torch.empty((wl.B, 1, wl.k), dtype=torch.int32, device=device)})
+    del dev["k_cache"], dev["v_cache"], dev["k_idx"]
+    f32 = dict(dtype=torch.float32, device=device)
+    cand_s = torch.empty((P, wl.B, 1, wl.k), **f32)
+    cand_i = torch.empty((P, wl.B, 1, wl.k), dtype=torch.int32, device=device)
+    idx = torch.empty((wl.B, 1, wl.k), dtype=torch.int32, device=device)
+    parts = torch.empty((P, wl.B, 1, wl.Hq, wl.Dv), dtype=dev["q"].dtype, device=device)
+    lses = torch.empty((P, wl.B, 1, wl.Hq), **f32)
+    out = torch.empty((wl.B, 1, wl.Hq, wl.Dv), dtype=dev["q"].dtype, device=device)
+    t = wl.L - 1
+
+    def step():
+        for r, sh in enumerate(shards):
+            q0 = min(t - sh["a"], sh["L"] - 1)
+            binding.indexer_scores(dev["q_idx"], sh["k_idx"], dev["w"], q0, scores=sh["scores"])
+            binding.topk(sh["scores"], wl.k, q0, idx=sh["idx"])
+            binding.cp_select_candidates(sh["scores"], sh["idx"], sh["a"], cand_scores=cand_s[r],
+                                         cand_idx=cand_i[r])
+        binding.cp_merge(cand_s, cand_i, wl.k, idx=idx)
+        for r, sh in enumerate(shards):
+            binding.cp_localize(idx, sh["a"], sh["L"], out=sh["idx_local"])
+            binding.sparse_attn(dev["q"], sh["k"], sh["v"], sh["idx_local"], wl.scale, out=parts[r], lse=lses[r])
+        binding.cp_combine(parts, lses, out=out)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    graph, launches_per_step = _capture(step, binding, device)
+    run = graph.replay if graph is not None else step
+    for _ in range(args.warmup):
+        run()
+    stream = torch.cuda.current_stream(device)
+    sampler = ClockSampler(0)
+    sampler.start()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(device)
+    h0 = time.perf_counter()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        run()
+    ev1.record(stream)
+    torch.cuda.synchronize(device)
+    h1 = time.perf_counter()
+    sampler.stop()
+    sec = ev0.elapsed_time(ev1) / 1000.0
+    line = {
+        "metric": "context-parallel decode steps/s (shards emulated on one GPU)", "value": args.steps / sec,
+        "unit": "decode steps/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * sec / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(_config(wl, 1), **{"pass": "cp", "shards": P, "shard_len": step_len}),
+        "gpu_launches": int(launches_per_step * args.steps) if graph is not None else None,
+        "clocks": sampler.summary(h0, h1),
+        "timing": "CUDA-graph replay of one emulated step" if graph is not None else "eager calls",
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--stage", choices=["indexer", "topk", "attn"], default=None,
@@ -829,8 +919,10 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle wall time")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--pass", dest="pass_", default="forward", choices=["forward", "train"],
-                    help="train: indexer scores, dense KL loss and indexer backward per step")
+    ap.add_argument("--pass", dest="pass_", default="forward", choices=["forward", "train", "cp"],
+                    help="train: indexer scores, dense KL loss and indexer backward per step; "
+                         "cp: the context-parallel decode step with its shards emulated on one GPU")
+    ap.add_argument("--shards", type=int, default=8, help="--pass cp: number of context shards")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)  # at least three untimed warm-up steps
     if args.workload is None:
@@ -838,6 +930,8 @@ def main():
     wl = WORKLOADS[args.workload]
     if args.pass_ == "train" and args.impl == "ours" and args.stage is None:
         run_train(args, wl)
+    elif args.pass_ == "cp" and args.impl == "ours" and args.stage is None:
+        run_cp(args, wl)
     elif args.stage is not None:
         run_stage(args, wl)
     elif args.impl == "reference":
