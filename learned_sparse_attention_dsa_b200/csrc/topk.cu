@@ -590,11 +590,15 @@ static cudaError_t launch_with(const TopkProblem &p, int P, cudaStream_t stream)
 }
 
 cudaError_t launch_topk_block(const TopkProblem &p, cudaStream_t stream, bool *taken);
+cudaError_t launch_topk_smem(const TopkProblem &p, cudaStream_t stream, bool *taken);
 
 cudaError_t launch_topk(const TopkProblem &p, cudaStream_t stream) {
-    // rows of at most 32,768 scores: one CTA per row, the row in registers
+    // many rows of at most 16,384 scores: one CTA per row, the row in registers
     bool taken = false;
     cudaError_t err = launch_topk_block(p, stream, &taken);
+    if (taken || err != cudaSuccess) return err;
+    // many rows of at most 49,152 scores: one CTA per row, the row in shared memory
+    err = launch_topk_smem(p, stream, &taken);
     if (taken || err != cudaSuccess) return err;
     DeviceInfo info;
     err = device_info(&info);

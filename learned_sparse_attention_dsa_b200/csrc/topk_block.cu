@@ -178,6 +178,119 @@ cudaError_t launch_block(const TopkProblem &p, cudaStream_t stream) {
     return cudaGetLastError();
 }
 
+// One CTA per row with the row's keys in shared memory (rows of up to
+// kSmemMaxN scores): the scores are read once with 16-byte loads, turned
+// into keys in shared memory, and the three radix passes and the output run
+// from there, with no cluster synchronisation. Positions are dealt to the
+// warps in contiguous segments (lane l of a warp takes every 32nd position of
+// its segment: conflict-free shared-memory reads), so that per-warp ballots
+// and one block scan give each kept position its slot in ascending order.
+constexpr int kSmemMaxN = 49152;
+
+__global__ void __launch_bounds__(kBlockThreads, 1)
+topk_smem_kernel(const float *__restrict__ scores, int Tq, int L, int q_pos0, int k, int include_self,
+                 int32_t *__restrict__ idx) {
+    extern __shared__ uint32_t keys[];
+    __shared__ int hist[kBins];
+    __shared__ int warp_sum[kBlockWarps];
+    __shared__ int warp_gt[kBlockWarps], warp_eq[kBlockWarps];
+    __shared__ int s_digit, s_above;
+
+    const int row = blockIdx.x;
+    const int t = q_pos0 + row % Tq;
+    const int n = t + 1;
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    int32_t *out = idx + (size_t)row * k;
+
+    if (n <= k) {  // every candidate is kept
+        for (int j = tid; j < k; j += kBlockThreads) out[j] = j < n ? j : -1;
+        return;
+    }
+    for (int b = tid; b < kBins; b += kBlockThreads) hist[b] = 0;
+
+    // ---- keys into shared memory: 16-byte loads from the first aligned element
+    const float *src = scores + (size_t)row * L;
+    const int head = (int)((4 - (((uintptr_t)src >> 2) & 3)) & 3);  // scalars before 16-byte alignment
+    const int h = head < n ? head : n;
+    for (int s = tid; s < h; s += kBlockThreads) keys[s] = block_order_key(src[s]);
+    const int n4 = (n - h) >> 2;
+    const float4 *src4 = reinterpret_cast<const float4 *>(src + h);
+#pragma unroll 4
+    for (int v = tid; v < n4; v += kBlockThreads) {
+        const float4 x = src4[v];
+        const int s = h + 4 * v;
+        keys[s] = block_order_key(x.x);
+        keys[s + 1] = block_order_key(x.y);
+        keys[s + 2] = block_order_key(x.z);
+        keys[s + 3] = block_order_key(x.w);
+    }
+    for (int s = h + 4 * n4 + tid; s < n; s += kBlockThreads) keys[s] = block_order_key(src[s]);
+    __syncthreads();
+    if (include_self && tid == 0) keys[t] = 0xFFFFFFFFu;  // the row's own position is always kept
+    __syncthreads();
+
+    // ---- pass 1: bits 31-21
+    for (int s = tid; s < n; s += kBlockThreads) atomicAdd(&hist[keys[s] >> 21], 1);
+    __syncthreads();
+    int want = k;
+    const uint32_t d1 = (uint32_t)find_digit(hist, want, warp_sum, &s_digit, &s_above);
+    want -= s_above;
+    // ---- pass 2: bits 20-10 of the keys whose bits 31-21 are d1
+    for (int s = tid; s < n; s += kBlockThreads) {
+        const uint32_t x = keys[s];
+        if ((x >> 21) == d1) atomicAdd(&hist[(x >> 10) & 2047u], 1);
+    }
+    __syncthreads();
+    const uint32_t d2 = (uint32_t)find_digit(hist, want, warp_sum, &s_digit, &s_above);
+    want -= s_above;
+    const uint32_t hi2 = (d1 << 11) | d2;
+    // ---- pass 3: bits 9-0 of the keys whose bits 31-10 are (d1, d2)
+    for (int s = tid; s < n; s += kBlockThreads) {
+        const uint32_t x = keys[s];
+        if ((x >> 10) == hi2) atomicAdd(&hist[x & 1023u], 1);
+    }
+    __syncthreads();
+    const uint32_t d3 = (uint32_t)find_digit(hist, want, warp_sum, &s_digit, &s_above);
+    want -= s_above;
+    const uint32_t T = (hi2 << 10) | d3;  // the k-th largest key
+    const int r = want;                   // keys equal to T that are kept (the first r by position)
+
+    // ---- output: warp w takes positions [w * seg, (w + 1) * seg)
+    const int seg = ((n + kBlockWarps - 1) / kBlockWarps + 31) & ~31;
+    const int s0 = warp * seg, s1 = min(n, s0 + seg);
+    int gt = 0, eq = 0;
+    for (int s = s0 + lane; s < s0 + seg; s += 32) {
+        const uint32_t x = s < s1 ? keys[s] : 0u;
+        gt += __popc(__ballot_sync(0xffffffffu, x > T));
+        eq += __popc(__ballot_sync(0xffffffffu, x == T && s < s1));
+    }
+    if (lane == 0) {
+        warp_gt[warp] = gt;
+        warp_eq[warp] = eq;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const int g = warp_gt[lane], e = warp_eq[lane];
+        const int gi = warp_inclusive_scan(g), ei = warp_inclusive_scan(e);
+        warp_gt[lane] = gi - g;
+        warp_eq[lane] = ei - e;
+    }
+    __syncthreads();
+    int gt_b = warp_gt[warp], eq_b = warp_eq[warp];
+    const unsigned lt = lanemask_lt_block();
+    for (int s = s0 + lane; s < s0 + seg; s += 32) {
+        const uint32_t x = s < s1 ? keys[s] : 0u;
+        const bool g = x > T, e = x == T && s < s1;
+        const unsigned gm = __ballot_sync(0xffffffffu, g);
+        const unsigned em = __ballot_sync(0xffffffffu, e);
+        const int eq_rank = eq_b + __popc(em & lt);
+        if (g || (e && eq_rank < r)) out[gt_b + __popc(gm & lt) + min(r, eq_rank)] = s;
+        gt_b += __popc(gm);
+        eq_b += __popc(em);
+    }
+}
+
 // Merge of per-shard selections (context parallelism): row `row` has P * kc
 // candidates, candidate c = p * kc + j at cand_*[(p * rows + row) * kc + j],
 // ordered by ascending global position (shards in position order, each list
@@ -299,6 +412,27 @@ cudaError_t launch_topk_merge(const float *cand_score, const int32_t *cand_idx, 
         topk_merge_kernel<8><<<rows, kBlockThreads, 0, stream>>>(cand_score, cand_idx, P, rows, kc, k, idx);
     else
         topk_merge_kernel<16><<<rows, kBlockThreads, 0, stream>>>(cand_score, cand_idx, P, rows, kc, k, idx);
+    count_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_topk_smem(const TopkProblem &p, cudaStream_t stream, bool *taken) {
+    *taken = false;
+    const long long rows = p.B * (long long)p.Tq;
+    const long long n_max = (long long)p.q_pos0 + p.Tq;
+    if (rows == 0 || rows > 0x7fffffffLL || n_max > kSmemMaxN) return cudaSuccess;
+    // with fewer rows than SMs the row is better split over a cluster (decode32k:
+    // 16.5 us with eight CTAs per row, 20.5 us with one)
+    DeviceInfo info;
+    cudaError_t err = device_info(&info);
+    if (err != cudaSuccess) return err;
+    if (rows < info.sm_count) return cudaSuccess;
+    const size_t smem = (size_t)n_max * sizeof(uint32_t);
+    err = cudaFuncSetAttribute(topk_smem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    *taken = true;
+    topk_smem_kernel<<<(unsigned)rows, kBlockThreads, smem, stream>>>(p.scores, p.Tq, p.L, p.q_pos0, p.k,
+                                                                      p.include_self ? 1 : 0, p.idx);
     count_launch();
     return cudaGetLastError();
 }
