@@ -51,10 +51,35 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
+// ldmatrix of four 8x8 bf16 matrices (rows of 16 bytes, one row address per lane)
+__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t *r) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t *r) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+// d += A (16x16, row) . B (16x8, col), bf16 in, fp32 accumulate
+__device__ __forceinline__ void mma_bf16_16816(float *d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
 // Stage layout: K then V, each [kRows][H * D] bf16; 16-byte chunk c of row r
 // is stored at chunk position c ^ (r & 7).
 template <int D, int STAGES>
-__global__ void __launch_bounds__(D == 64 ? 512 : 256)
+__global__ void __launch_bounds__(D == 64 ? 512 : 256, 1)
 attn_perhead_kernel(const Args a) {
     extern __shared__ __align__(128) uint8_t smem[];
     constexpr int kChunksPerHead = D / 8;
@@ -98,47 +123,51 @@ attn_perhead_kernel(const Args a) {
     const __nv_bfloat16 *kb = a.k_cache + b * a.k_sb;
     const __nv_bfloat16 *vb = a.v_cache + b * a.v_sb;
 
+    // Copies: thread i always moves 16-byte chunk x = i % row_chunks of a
+    // position's row (fixed head and column offsets), for rows r0, r0 + step, ...
+    // of the tile, K and V alike (row_chunks divides the thread count).
+    const int cstep = nthreads / row_chunks;  // rows per pass: 4 (D = 64) or 2 (D = 128)
+    const int cx = threadIdx.x % row_chunks, cr0 = threadIdx.x / row_chunks;
+    const int64_t koff = (int64_t)(cx / kChunksPerHead) * a.k_sh + (cx % kChunksPerHead) * 8;
+    const int64_t voff = (int64_t)(cx / kChunksPerHead) * a.v_sh + (cx % kChunksPerHead) * 8;
+    const uint32_t vstage_off = kRows * row_chunks * 16;
     auto issue = [&](int tile, int stage) {
         const uint32_t kdst = smem_base + stage * stage_bytes;
-        const uint32_t vdst = kdst + kRows * row_chunks * 16;
-        const int total = 2 * kRows * row_chunks;
-        const int half_total = kRows * row_chunks;
-        for (int c = threadIdx.x; c < total; c += nthreads) {
-            const bool is_v = c >= half_total;
-            const int cc = c & (half_total - 1);
-            const int r = cc >> a.rc_shift;
-            const int x = cc & (row_chunks - 1);  // chunk within the position's row
-            const int h = x / kChunksPerHead, ch = x % kChunksPerHead;
+#pragma unroll 4
+        for (int r = cr0; r < kRows; r += cstep) {
             const int jj = tile * kRows + r;
             const bool valid = jj < n_sel;
             const int s = valid ? sel[jj] : 0;
-            const __nv_bfloat16 *src = is_v ? vb + (int64_t)s * a.v_ss + h * a.v_sh + ch * 8
-                                            : kb + (int64_t)s * a.k_ss + h * a.k_sh + ch * 8;
-            const uint32_t dst = (is_v ? vdst : kdst) + (r * row_chunks + (x ^ (r & 7))) * 16;
-            cp_async16(dst, src, valid);
+            const uint32_t dst = kdst + (r * row_chunks + (cx ^ (r & 7))) * 16;
+            cp_async16(dst, kb + (int64_t)s * a.k_ss + koff, valid);
+            cp_async16(dst + vstage_off, vb + (int64_t)s * a.v_ss + voff, valid);
         }
     };
 
-    // this warp's head: lane half hf (= lane / 16) holds query columns
-    // [hf * D/2, hf * D/2 + D/2), pre-scaled into log2 units
+    // ---- this warp's head h: both products on the tensor cores (mma.sync
+    // m16n8k16, bf16 in, fp32 accumulate). Every row of the A operand is the
+    // same query (logits) or the same probabilities (weighted sum), so every
+    // accumulator row holds the same values; lane (g, t) = (lane / 4, lane % 4)
+    // holds positions 8 nb + 2t, 8 nb + 2t + 1 of each 8-position block nb.
     const int h = warp;
-    const int hf = lane >> 4;
-    float qreg[D / 2];
+    const int t4 = lane & 3, g8 = lane >> 2;
+    constexpr int kKSteps = D / 16;  // 16-wide slices of the head
+    constexpr int kNBlk = D / 8;     // 8-wide output column blocks
+    uint32_t qa[kKSteps][2];         // A fragments: q pairs (2t, 2t+1) and (2t+8, 2t+9) of each slice
     {
-        const __nv_bfloat16 *qh = a.q + ((size_t)row * a.H + h) * D + hf * (D / 2);
+        const __nv_bfloat16 *qh = a.q + ((size_t)row * a.H + h) * D;
 #pragma unroll
-        for (int c = 0; c < D / 16; ++c) {
-            float f[8];
-            bf16x8_to_f32(*reinterpret_cast<const uint4 *>(qh + c * 8), f);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) qreg[c * 8 + u] = f[u] * a.scale_log2;
+        for (int ks = 0; ks < kKSteps; ++ks) {
+            qa[ks][0] = *reinterpret_cast<const uint32_t *>(qh + ks * 16 + 2 * t4);
+            qa[ks][1] = *reinterpret_cast<const uint32_t *>(qh + ks * 16 + 8 + 2 * t4);
         }
     }
-    constexpr int kCols = D / 32;  // output columns per lane: lane*kCols ...
-    float acc[kCols];
+    float acc[kNBlk][2];
 #pragma unroll
-    for (int c = 0; c < kCols; ++c) acc[c] = 0.0f;
+    for (int j = 0; j < kNBlk; ++j) acc[j][0] = acc[j][1] = 0.0f;
     float m = -INFINITY, l = 0.0f;
+    const int hx = h * kChunksPerHead;  // the head's first 16-byte chunk in a position row
+    const int row_bytes = row_chunks * 16;
 
 #pragma unroll
     for (int st = 0; st < STAGES - 1; ++st) {
@@ -152,61 +181,86 @@ attn_perhead_kernel(const Args a) {
         cp_async_wait<STAGES - 1>();
         __syncthreads();
 
-        const uint8_t *kt = smem + stage * stage_bytes;
-        const uint8_t *vt = kt + kRows * row_chunks * 16;
-        // half hf of the logit of position r (lanes r and r + 16)
-        const int r = lane & (kRows - 1);
-        float z = -INFINITY;
-        {
-            const uint8_t *krow = kt + r * row_chunks * 16;
-            float dot[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // independent chains
+        const uint32_t kt = smem_base + stage * stage_bytes;
+        const uint32_t vt = kt + kRows * row_bytes;
+        // logits of the 16 positions: S = q . K^T, two 8-position blocks
+        float sc[2][2];
 #pragma unroll
-            for (int c = 0; c < kChunksPerHead / 2; ++c) {
-                const int x = h * kChunksPerHead + hf * (kChunksPerHead / 2) + c;
-                float f[8];
-                bf16x8_to_f32(*reinterpret_cast<const uint4 *>(krow + (x ^ (r & 7)) * 16), f);
+        for (int nb = 0; nb < 2; ++nb) {
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int u = 0; u < 8; ++u) dot[u & 3] = fmaf(qreg[c * 8 + u], f[u], dot[u & 3]);
+            for (int c = 0; c < kChunksPerHead; c += 4) {
+                // matrices: positions 8 nb .. 8 nb + 7, chunks c .. c + 3 of the head
+                const int p = nb * 8 + (lane & 7);
+                const int x = hx + c + (lane >> 3);
+                uint32_t b[4];
+                ldmatrix_x4(kt + p * row_bytes + ((x ^ (p & 7)) << 4), b);
+                mma_bf16_16816(d, qa[c / 2][0], qa[c / 2][0], qa[c / 2][1], qa[c / 2][1], b[0], b[1]);
+                mma_bf16_16816(d, qa[c / 2 + 1][0], qa[c / 2 + 1][0], qa[c / 2 + 1][1], qa[c / 2 + 1][1], b[2],
+                               b[3]);
             }
-            float zp = (dot[0] + dot[1]) + (dot[2] + dot[3]);
-            zp += __shfl_xor_sync(0xffffffffu, zp, 16);  // both halves hold the full logit
-            if (tile * kRows + r < n_sel) z = zp;
+            const int p0 = tile * kRows + nb * 8 + 2 * t4;
+            sc[nb][0] = p0 < n_sel ? d[0] * a.scale_log2 : -INFINITY;
+            sc[nb][1] = p0 + 1 < n_sel ? d[1] * a.scale_log2 : -INFINITY;
         }
-        const float zmax = warp_max(z);
+        // online softmax over the tile (lanes sharing t hold the same values)
+        float zmax = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
+        zmax = fmaxf(zmax, __shfl_xor_sync(0xffffffffu, zmax, 1));
+        zmax = fmaxf(zmax, __shfl_xor_sync(0xffffffffu, zmax, 2));
         const float m_new = fmaxf(m, zmax);
-        const float corr = m_new == -INFINITY ? 1.0f : ex2_approx(m - m_new);
-        const float p = z == -INFINITY ? 0.0f : ex2_approx(z - m_new);
-        l = l * corr + warp_sum(hf == 0 ? p : 0.0f);  // each position counted once
-        m = m_new;
+        const float mr = m_new == -INFINITY ? 0.0f : m_new;  // masked entries: 2^-inf = 0
+        float pr[2][2], psum = 0.0f;
 #pragma unroll
-        for (int c = 0; c < kCols; ++c) acc[c] *= corr;
-        // weighted value rows: lane owns columns [lane*kCols, lane*kCols + kCols)
-        const int valid_rows = min(kRows, n_sel - tile * kRows);
-        for (int rr = 0; rr < valid_rows; ++rr) {
-            const float pr = __shfl_sync(0xffffffffu, p, rr);
-            const int x = h * kChunksPerHead + (lane * kCols) / 8;
-            const uint8_t *vrow = vt + rr * row_chunks * 16 + (x ^ (rr & 7)) * 16 + ((lane * kCols) % 8) * 2;
-            if constexpr (kCols == 2) {
-                const __nv_bfloat162 v2 = *reinterpret_cast<const __nv_bfloat162 *>(vrow);
-                acc[0] = fmaf(pr, __low2float(v2), acc[0]);
-                acc[1] = fmaf(pr, __high2float(v2), acc[1]);
-            } else {
-                const uint2 v4 = *reinterpret_cast<const uint2 *>(vrow);
-                acc[0] = fmaf(pr, __uint_as_float(v4.x << 16), acc[0]);
-                acc[1] = fmaf(pr, __uint_as_float(v4.x & 0xffff0000u), acc[1]);
-                acc[2] = fmaf(pr, __uint_as_float(v4.y << 16), acc[2]);
-                acc[3] = fmaf(pr, __uint_as_float(v4.y & 0xffff0000u), acc[3]);
+        for (int nb = 0; nb < 2; ++nb)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                pr[nb][e] = ex2_approx(sc[nb][e] - mr);
+                psum += pr[nb][e];
             }
+        psum += __shfl_xor_sync(0xffffffffu, psum, 1);
+        psum += __shfl_xor_sync(0xffffffffu, psum, 2);
+        if (m_new != m) {  // warp-uniform
+            const float corr = ex2_approx(m - mr);
+            l *= corr;
+#pragma unroll
+            for (int j = 0; j < kNBlk; ++j) {
+                acc[j][0] *= corr;
+                acc[j][1] *= corr;
+            }
+            m = m_new;
+        }
+        l += psum;
+        // weighted value rows: acc += P . V (P in bf16; positions are the K dimension)
+        const uint32_t pa0 = pack_bf16x2(pr[0][0], pr[0][1]), pa2 = pack_bf16x2(pr[1][0], pr[1][1]);
+#pragma unroll
+        for (int j = 0; j < kNBlk; j += 2) {
+            // matrices: positions 0-7 and 8-15 of chunks j and j + 1, transposed
+            const int mi = lane >> 3;
+            const int p = (mi & 1) * 8 + (lane & 7);
+            const int x = hx + j + (mi >> 1);
+            uint32_t b[4];
+            ldmatrix_x4_trans(vt + p * row_bytes + ((x ^ (p & 7)) << 4), b);
+            float d0[4] = {acc[j][0], acc[j][1], acc[j][0], acc[j][1]};
+            mma_bf16_16816(d0, pa0, pa0, pa2, pa2, b[0], b[1]);
+            acc[j][0] = d0[0];
+            acc[j][1] = d0[1];
+            float d1[4] = {acc[j + 1][0], acc[j + 1][1], acc[j + 1][0], acc[j + 1][1]};
+            mma_bf16_16816(d1, pa0, pa0, pa2, pa2, b[2], b[3]);
+            acc[j + 1][0] = d1[0];
+            acc[j + 1][1] = d1[1];
         }
         __syncthreads();  // the stage is refilled by a later iteration's issue
     }
     cp_async_wait<0>();
 
+    // lane (g, t) writes output columns 8 j + 2t, 8 j + 2t + 1 for j = g, g + 4, ...
     const float inv = l > 0.0f ? 1.0f / l : 0.0f;
-    __nv_bfloat16 *dst = a.out + ((size_t)row * a.H + h) * D + lane * kCols;
+    __nv_bfloat16 *dst = a.out + ((size_t)row * a.H + h) * D;
 #pragma unroll
-    for (int c = 0; c < kCols; c += 2)
-        *reinterpret_cast<__nv_bfloat162 *>(dst + c) = __floats2bfloat162_rn(acc[c] * inv, acc[c + 1] * inv);
+    for (int j = 0; j < kNBlk; ++j)
+        if ((j & 7) == g8)
+            *reinterpret_cast<__nv_bfloat162 *>(dst + j * 8 + 2 * t4) =
+                __floats2bfloat162_rn(acc[j][0] * inv, acc[j][1] * inv);
     if (a.lse != nullptr && lane == 0)
         a.lse[(size_t)row * a.H + h] = l > 0.0f ? (m + log2f(l)) / kLog2e : -INFINITY;
 }
