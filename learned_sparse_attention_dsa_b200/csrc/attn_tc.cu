@@ -19,6 +19,7 @@
 #include <math.h>
 
 #include <cooperative_groups.h>
+#include <type_traits>
 
 #include "common.cuh"
 #include "internal.h"
@@ -175,25 +176,27 @@ attn_mma_kernel(const Args a) {
     const __nv_bfloat16 *vbase = a.v_cache + b * a.v_sb + g * a.v_sh;
     const uint32_t smem_base = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
 
-    auto issue_tile = [&](int tile, int stage) {
-        const uint32_t kdst = smem_base + stage * C::kStageBytes;
-        const uint32_t vdst = kdst + C::kKBytes;
-        constexpr int kChunks = kRowsPerTile * (C::kKChunks + C::kVChunks);
-        for (int c = threadIdx.x; c < kChunks; c += kThreads) {
-            const int r = c / (C::kKChunks + C::kVChunks);
-            const int ch = c - r * (C::kKChunks + C::kVChunks);
+    // Copies: K rows, then V rows; for each, thread i moves the fixed 16-byte
+    // chunk column i % C of rows r0, r0 + R, ... (C chunks per row, R =
+    // kThreads / C rows per pass; threads beyond R * C idle for that part).
+    auto issue_rows = [&](uint32_t dst0, const __nv_bfloat16 *base, int64_t ss, int tile, auto chunks_c) {
+        constexpr int CH = decltype(chunks_c)::value;
+        constexpr int R = kThreads / CH;
+        const int ch = threadIdx.x % CH, r0 = threadIdx.x / CH;
+        if (r0 >= R) return;
+        const __nv_bfloat16 *src0 = base + ch * 8;
+#pragma unroll 4
+        for (int r = r0; r < kRowsPerTile; r += R) {
             const int jj = tile * kRowsPerTile + r;
             const bool valid = jj < n_sel;
             const int s = valid ? sel[jj] : 0;
-            if (ch < C::kKChunks) {
-                const uint32_t dst = kdst + r * (DQK * 2) + ((ch ^ (r & 7)) << 4);
-                cp_async16(dst, kbase + (int64_t)s * a.k_ss + ch * 8, valid);
-            } else {
-                const int cv = ch - C::kKChunks;
-                const uint32_t dst = vdst + r * (DV * 2) + ((cv ^ (r & 7)) << 4);
-                cp_async16(dst, vbase + (int64_t)s * a.v_ss + cv * 8, valid);
-            }
+            cp_async16(dst0 + r * (CH * 16) + ((ch ^ (r & 7)) << 4), src0 + (int64_t)s * ss, valid);
         }
+    };
+    auto issue_tile = [&](int tile, int stage) {
+        const uint32_t kdst = smem_base + stage * C::kStageBytes;
+        issue_rows(kdst, kbase, a.k_ss, tile, std::integral_constant<int, C::kKChunks>{});
+        issue_rows(kdst + C::kKBytes, vbase, a.v_ss, tile, std::integral_constant<int, C::kVChunks>{});
     };
 
     float o[DV / 8][4];
