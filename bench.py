@@ -536,8 +536,13 @@ def run_e2e(wl, cpu, binding, device, stream, steps, world):
 
 def run_stage(args, wl):
     """Eager launches of one stage only (for profiler captures): W warm-up
-    calls then K timed calls; prints the average device time per call."""
+    calls then K timed calls; prints the average device time per call.
+    --tail-rows R keeps only the last R query rows of the workload (a small
+    case of the same kernel for full profiler captures)."""
     from learned_sparse_attention_dsa_b200 import binding
+    if args.tail_rows:
+        R = min(args.tail_rows, wl.Tq)
+        wl = wl.replace(name=f"{wl.name}_tail{R}", Tq=R, q_pos0=wl.q_pos0 + wl.Tq - R)
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
     dev = to_device(make_inputs(wl), device)
@@ -923,6 +928,8 @@ def main():
                     help="train: indexer scores, dense KL loss and indexer backward per step; "
                          "cp: the context-parallel decode step with its shards emulated on one GPU")
     ap.add_argument("--shards", type=int, default=8, help="--pass cp: number of context shards")
+    ap.add_argument("--tail-rows", type=int, default=0,
+                    help="--stage: keep only the last R query rows (small profiler cases)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)  # at least three untimed warm-up steps
     if args.workload is None:
