@@ -11,12 +11,12 @@
 // of a query in its own registers, so the ReLU, the weights and the head sum
 // need no cross-thread reduction, and the per-head scores never leave the SM.
 //
-// Warp roles (320 threads, one CTA per SM, persistent over work units):
+// Warp roles (64 + 32 EPI threads, one CTA per SM, persistent over work units):
 //   warp 0      TMA producer: Q tile of the unit once, then key tiles through
 //               a K_STAGES-deep ring (128-byte swizzle, K-major).
 //   warp 1      allocates TMEM; one thread issues tcgen05.mma (bf16 in, fp32
 //               accumulate) into one of two TMEM accumulators.
-//   warps 2-9   epilogue, two warps per TMEM lane quarter (each takes every
+//   warps 2..   epilogue, EPI = 8 or 16 warps, EPI / 4 per TMEM lane quarter (each takes every
 //               other query of the tile; with one query per tile, as in
 //               decode, every other tile): tcgen05.ld of the accumulator,
 //               ReLU, weight and head sum with packed fp32x2 FMAs, one fp32
@@ -44,8 +44,14 @@ namespace {
 using namespace sm100;
 
 constexpr int kBlockM = 128;       // keys per tile (TMEM lanes)
-constexpr int kEpilogueThreads = 256;            // 8 warps: two per TMEM lane quarter
-constexpr int kThreads = 64 + kEpilogueThreads;  // + the TMA and MMA warps
+// Epilogue warps: EPI = 16 (four per TMEM lane quarter) when a tile holds
+// several queries (prefill), 8 (two per quarter, taking alternate tiles) for
+// one query per tile (decode, where more warps only cost registers).
+template <int EPI>
+struct Threads {
+    static constexpr int kEpilogue = EPI * 32;
+    static constexpr int kAll = 64 + kEpilogue;  // + the TMA and MMA warps
+};
 
 // acc(lo, hi) += (a_lo * b_lo, a_hi * b_hi), two independent IEEE fp32 FMAs
 __device__ __forceinline__ void fma2(uint64_t &acc, float a_lo, float a_hi, float b_lo, float b_hi) {
@@ -111,8 +117,8 @@ struct Cfg {
     static_assert(kTmemCols == 128 || kTmemCols == 256 || kTmemCols == 512, "TMEM columns");
 };
 
-template <int D, int N_TILE, bool FP8>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int D, int N_TILE, bool FP8, int EPI>
+__global__ void __launch_bounds__(Threads<EPI>::kAll, 1)
 indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const Params p) {
     using C = Cfg<D, N_TILE, FP8>;
@@ -143,7 +149,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
         // one query per tile (decode): the two warps of a TMEM lane quarter
         // take alternate tiles (accumulators), else alternate queries
-        const int releasers = p.QPT == 1 ? kEpilogueThreads / 2 : kEpilogueThreads;
+        // decode: each tile is taken by one group of four warps (one per lane quarter)
+        const int releasers = p.QPT == 1 ? 128 : Threads<EPI>::kEpilogue;
         for (int s = 0; s < 2; ++s) {
             mbar_init(&acc_full[s], 1);
             mbar_init(&acc_empty[s], releasers);
@@ -232,10 +239,10 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     } else {
         // ---------------------------------------------------- epilogue
         const int quarter = warp & 3;                 // TMEM lanes this warp may read
-        const int half = (warp - 2) >> 2;             // 0 or 1: the warp's share of the tiles' work
-        const bool by_tile = p.QPT == 1;              // decode: accumulator `half` only, its one query
-        const int q_first = by_tile ? 0 : half;       // else queries half, half + 2, ...
-        const int q_step = by_tile ? 1 : 2;
+        const int half = (warp - 2) >> 2;             // the warp's group: its share of the tiles' work
+        const bool by_tile = p.QPT == 1;              // decode: accumulator `half` only (groups 0, 1)
+        const int q_first = by_tile ? 0 : half;       // else queries half, half + EPI / 4, ...
+        const int q_step = by_tile ? 1 : EPI / 4;
         const int key_in_tile = quarter * 32 + lane;  // TMEM lane = key
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
         int ab = 0;
@@ -311,7 +318,7 @@ __global__ void fill_beyond_tiles_kernel(float *__restrict__ scores, int Tq, int
     for (int s = start + threadIdx.x; s < L; s += blockDim.x) out[s] = -INFINITY;
 }
 
-template <int D, int N_TILE, bool FP8>
+template <int D, int N_TILE, bool FP8, int EPI>
 cudaError_t launch_tc(const IndexerProblem &pr, const DeviceInfo &info, cudaStream_t stream) {
     using C = Cfg<D, N_TILE, FP8>;
     if ((size_t)info.max_smem_optin < C::kSmem) return cudaErrorInvalidValue;
@@ -350,11 +357,11 @@ cudaError_t launch_tc(const IndexerProblem &pr, const DeviceInfo &info, cudaStre
     if (units > 0x7fffffffLL) return cudaErrorInvalidValue;
     p.units = (int)units;
 
-    auto kern = indexer_tc_kernel<D, N_TILE, FP8>;
+    auto kern = indexer_tc_kernel<D, N_TILE, FP8, EPI>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
     if (err != cudaSuccess) return err;
     const int grid = p.units < info.sm_count ? p.units : info.sm_count;
-    kern<<<grid, kThreads, C::kSmem, stream>>>(tm_q, tm_k, p);
+    kern<<<grid, Threads<EPI>::kAll, C::kSmem, stream>>>(tm_q, tm_k, p);
     count_launch();
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     if (pr.fill_masked) {
@@ -363,6 +370,23 @@ cudaError_t launch_tc(const IndexerProblem &pr, const DeviceInfo &info, cudaStre
         err = cudaGetLastError();
     }
     return err;
+}
+
+template <int EPI>
+cudaError_t dispatch_tc(const IndexerProblem &p, const DeviceInfo &info, cudaStream_t stream, bool fp8, int n_tile) {
+    if (fp8) {
+        if (n_tile == 64) return launch_tc<128, 64, true, EPI>(p, info, stream);
+        if (n_tile == 128) return launch_tc<128, 128, true, EPI>(p, info, stream);
+        return launch_tc<128, 256, true, EPI>(p, info, stream);
+    }
+    if (p.d == 128) {
+        if (n_tile == 64) return launch_tc<128, 64, false, EPI>(p, info, stream);
+        if (n_tile == 128) return launch_tc<128, 128, false, EPI>(p, info, stream);
+        return launch_tc<128, 256, false, EPI>(p, info, stream);
+    }
+    if (n_tile == 64) return launch_tc<64, 64, false, EPI>(p, info, stream);
+    if (n_tile == 128) return launch_tc<64, 128, false, EPI>(p, info, stream);
+    return launch_tc<64, 256, false, EPI>(p, info, stream);
 }
 
 }  // namespace
@@ -394,19 +418,9 @@ cudaError_t launch_indexer_tc(const IndexerProblem &p, cudaStream_t stream, bool
     // a TMA box may not be taller than the tensor it reads
     if ((long long)p.B * p.Tq * p.H < n_tile || (long long)p.B * p.L < kBlockM) return cudaSuccess;
     *taken = true;
-    if (fp8) {
-        if (n_tile == 64) return launch_tc<128, 64, true>(p, info, stream);
-        if (n_tile == 128) return launch_tc<128, 128, true>(p, info, stream);
-        return launch_tc<128, 256, true>(p, info, stream);
-    }
-    if (p.d == 128) {
-        if (n_tile == 64) return launch_tc<128, 64, false>(p, info, stream);
-        if (n_tile == 128) return launch_tc<128, 128, false>(p, info, stream);
-        return launch_tc<128, 256, false>(p, info, stream);
-    }
-    if (n_tile == 64) return launch_tc<64, 64, false>(p, info, stream);
-    if (n_tile == 128) return launch_tc<64, 128, false>(p, info, stream);
-    return launch_tc<64, 256, false>(p, info, stream);
+    // one query per tile (decode): 8 epilogue warps, else 16
+    if (qpt == 1) return dispatch_tc<8>(p, info, stream, fp8, n_tile);
+    return dispatch_tc<16>(p, info, stream, fp8, n_tile);
 }
 
 }  // namespace dsa
