@@ -49,7 +49,7 @@ struct Cfg {
     static constexpr int kMaxSel = 2048;  // selected entries one CTA handles
     // four warps' (O, m, l), then the CTA's merged (O, m, l) for the cluster merge
     // (plus one merge weight per split and head)
-    static constexpr int kMergeBytes = (kWarps + 1) * kHeads * (DV + 2) * 4 + 8 * kHeads * 4;
+    static constexpr int kMergeBytes = (kWarps + 1) * kHeads * (DV + 10) * 4 + 8 * kHeads * 4;
     static constexpr int kPipeBytes = kStages * kStageBytes;
     static constexpr size_t kSmem =
         (size_t)(kPipeBytes > kMergeBytes ? kPipeBytes : kMergeBytes) + kMaxSel * 4 + 64;
@@ -309,18 +309,19 @@ attn_mma_kernel(const Args a) {
         l_r[hh] += __shfl_xor_sync(0xffffffffu, l_r[hh], 1);
         l_r[hh] += __shfl_xor_sync(0xffffffffu, l_r[hh], 2);
     }
-    float *mrg_o = reinterpret_cast<float *>(smem);                    // [warp][16][DV]
-    float *mrg_ml = mrg_o + kWarps * kHeads * DV;                      // [warp][16][2]
+    // rows of DV + 8 floats: the float2 stores below and the column reads
+    // after them hit distinct banks
+    constexpr int kRowF = DV + 8;
+    float *mrg_o = reinterpret_cast<float *>(smem);                    // [warp][16][kRowF]
+    float *mrg_ml = mrg_o + kWarps * kHeads * kRowF;                   // [warp][16][2]
     {
         const int hr = lane >> 2, cc = (lane & 3) * 2;
 #pragma unroll
         for (int n = 0; n < DV / 8; ++n) {
-            float *d0 = mrg_o + ((warp * kHeads + hr) * DV) + n * 8 + cc;
-            float *d8 = mrg_o + ((warp * kHeads + hr + 8) * DV) + n * 8 + cc;
-            d0[0] = o[n][0];
-            d0[1] = o[n][1];
-            d8[0] = o[n][2];
-            d8[1] = o[n][3];
+            *reinterpret_cast<float2 *>(mrg_o + ((warp * kHeads + hr) * kRowF) + n * 8 + cc) =
+                make_float2(o[n][0], o[n][1]);
+            *reinterpret_cast<float2 *>(mrg_o + ((warp * kHeads + hr + 8) * kRowF) + n * 8 + cc) =
+                make_float2(o[n][2], o[n][3]);
         }
         if ((lane & 3) == 0) {
             mrg_ml[(warp * kHeads + hr) * 2 + 0] = m_r[0];
@@ -342,7 +343,7 @@ attn_mma_kernel(const Args a) {
     float fw[kWarps], l_all = 0.0f;
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) {
-        fw[w] = m_all == -INFINITY ? 0.0f : exp2f(mw[w] - m_all);
+        fw[w] = m_all == -INFINITY ? 0.0f : ex2_approx(mw[w] - m_all);
         l_all += fw[w] * mrg_ml[(w * kHeads + hh) * 2 + 1];
     }
     const int h = h0 + hh;
@@ -352,7 +353,7 @@ attn_mma_kernel(const Args a) {
         for (int c = c0; c < DV; c += 8) {
             float acc = 0.0f;
 #pragma unroll
-            for (int w = 0; w < kWarps; ++w) acc += fw[w] * mrg_o[(w * kHeads + hh) * DV + c];
+            for (int w = 0; w < kWarps; ++w) acc += fw[w] * mrg_o[(w * kHeads + hh) * kRowF + c];
             dst[c] = __float2bfloat16_rn(acc * inv);
         }
         if (a.lse != nullptr && c0 == 0)
@@ -367,7 +368,7 @@ attn_mma_kernel(const Args a) {
         for (int c = c0; c < DV; c += 8) {
             float acc = 0.0f;
 #pragma unroll
-            for (int w = 0; w < kWarps; ++w) acc += fw[w] * mrg_o[(w * kHeads + hh) * DV + c];
+            for (int w = 0; w < kWarps; ++w) acc += fw[w] * mrg_o[(w * kHeads + hh) * kRowF + c];
             cta_o[hh * DV + c] = acc;
         }
         if (c0 == 0) {
@@ -397,7 +398,7 @@ attn_mma_kernel(const Args a) {
             float l_x = 0.0f;
 #pragma unroll
             for (int r = 0; r < 8; ++r) {
-                ms[r] = (r < P && m_x != -INFINITY) ? exp2f(ms[r] - m_x) : 0.0f;
+                ms[r] = (r < P && m_x != -INFINITY) ? ex2_approx(ms[r] - m_x) : 0.0f;
                 l_x += ms[r] * ls[r];
             }
             const float inv = l_x > 0.0f ? 1.0f / l_x : 0.0f;
@@ -439,7 +440,7 @@ attn_mma_kernel(const Args a) {
         for (int c = c0; c < DV; c += 8) {
             float acc = 0.0f;
 #pragma unroll
-            for (int w = 0; w < kWarps; ++w) acc += fw[w] * mrg_o[(w * kHeads + hh) * DV + c];
+            for (int w = 0; w < kWarps; ++w) acc += fw[w] * mrg_o[(w * kHeads + hh) * kRowF + c];
             dst[c] = acc;
         }
         if (c0 == 0) {
