@@ -538,13 +538,18 @@ attn_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Args a) {
     }
 }
 
-// Merge the split partials of one (row, head): one warp; lane j holds the
-// (max, sum) of split j; every lane then owns float4 columns and sums the
-// splits' partials for them, undoing the rotation of the half rows.
+// Merge the split partials of one (row, head): lane j of each warp holds the
+// (max, sum) of split j; the pair's 128 output float4s are spread over four
+// warps, and every lane sums the splits' partials for its float4, undoing the
+// rotation of the half rows.
 __global__ void attn_mla_combine_kernel(const float4 *__restrict__ part_o, const float *__restrict__ part_ml,
                                         int n_pairs, int splits, __nv_bfloat16 *__restrict__ out,
                                         float *__restrict__ lse) {
-    const int pair = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    // four warps per (row, head): warp quarter qt owns output float4s
+    // [32 qt, 32 qt + 32), one per lane, and loads every split's value for it
+    // independently (all in flight at once)
+    const int gw = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int pair = gw >> 2, qt = gw & 3;
     const int lane = threadIdx.x & 31;
     if (pair >= n_pairs) return;
     const int h = pair % kHeads;
@@ -552,31 +557,29 @@ __global__ void attn_mla_combine_kernel(const float4 *__restrict__ part_o, const
     const float m_s = lane < splits ? ml[2 * lane] : -INFINITY;
     const float l_s = lane < splits ? ml[2 * lane + 1] : 0.0f;
     const float m_all = warp_max(m_s);
-    const float f_s = (m_all == -INFINITY || lane >= splits) ? 0.0f : exp2f(m_s - m_all);
+    const float f_s = (m_all == -INFINITY || lane >= splits) ? 0.0f : ex2_approx(m_s - m_all);
     const float l_all = warp_sum(f_s * l_s);
     const float inv = l_all > 0.0f ? 1.0f / l_all : 0.0f;
     const float4 *po = part_o + (size_t)pair * splits * (DV / 4);
-#pragma unroll
-    for (int it = 0; it < DV / 4 / 32; ++it) {  // 4 float4 per lane
-        const int c4 = it * 32 + lane;            // output float4 index in [0, 128)
-        const int hf = c4 / (kHalfDv / 4), q = c4 % (kHalfDv / 4);
-        const int pos = hf * (kHalfDv / 4) + rot_q(h, q);
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-        for (int sp = 0; sp < splits; ++sp) {
-            const float f = __shfl_sync(0xffffffffu, f_s, sp);
-            const float4 v = po[(size_t)sp * (DV / 4) + pos];
-            acc.x = fmaf(f, v.x, acc.x);
-            acc.y = fmaf(f, v.y, acc.y);
-            acc.z = fmaf(f, v.z, acc.z);
-            acc.w = fmaf(f, v.w, acc.w);
-        }
-        uint2 w;
-        w.x = pack_bf16x2(acc.x * inv, acc.y * inv);
-        w.y = pack_bf16x2(acc.z * inv, acc.w * inv);
-        *reinterpret_cast<uint2 *>(out + (size_t)pair * DV + 4 * c4) = w;
+    const int c4 = qt * 32 + lane;  // output float4 index in [0, 128)
+    const int hf = c4 / (kHalfDv / 4), q = c4 % (kHalfDv / 4);
+    const int pos = hf * (kHalfDv / 4) + rot_q(h, q);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+    for (int sp = 0; sp < splits; ++sp) {
+        const float f = __shfl_sync(0xffffffffu, f_s, sp);
+        const float4 v = po[(size_t)sp * (DV / 4) + pos];
+        acc.x = fmaf(f, v.x, acc.x);
+        acc.y = fmaf(f, v.y, acc.y);
+        acc.z = fmaf(f, v.z, acc.z);
+        acc.w = fmaf(f, v.w, acc.w);
     }
-    if (lse != nullptr && lane == 0) lse[pair] = l_all > 0.0f ? (m_all + log2f(l_all)) / kLog2e : -INFINITY;
+    uint2 w;
+    w.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+    w.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+    *reinterpret_cast<uint2 *>(out + (size_t)pair * DV + 4 * c4) = w;
+    if (lse != nullptr && qt == 0 && lane == 0)
+        lse[pair] = l_all > 0.0f ? (m_all + log2f(l_all)) / kLog2e : -INFINITY;
 }
 
 // Splits per row: one CTA per SM over (row, split, part), at most kMaxTiles
@@ -658,8 +661,8 @@ cudaError_t launch_attn_mla_tc(const AttnProblem &p, const DeviceInfo &info, cud
     count_launch();
     if (err != cudaSuccess) return err;
     if (splits > 1) {
-        const int warps_per_block = 8;
-        const int blocks = (int)((n_pairs + warps_per_block - 1) / warps_per_block);
+        const int warps_per_block = 8;  // four warps per (row, head) pair
+        const int blocks = (int)((4 * n_pairs + warps_per_block - 1) / warps_per_block);
         attn_mla_combine_kernel<<<blocks, warps_per_block * 32, 0, stream>>>(
             reinterpret_cast<const float4 *>(a.part_o), a.part_ml, (int)n_pairs, splits, a.out, a.lse);
         count_launch();
