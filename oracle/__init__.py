@@ -5,10 +5,12 @@ legs of ``bench.py`` may import this package. The product (the CUDA library
 under ``learned_sparse_attention_dsa_b200`` and its binding) never imports it,
 and it imports nothing from the product.
 
-The arithmetic lives in ``dsa_oracle.c`` (plain C, fp64, one query row at a
-time; see that file's header for the page passages each function follows and
-the readings taken where the pages are silent). This module compiles it with
-gcc, and marshals numpy arrays into it.
+The arithmetic of the forward path lives in ``dsa_oracle.c`` (plain C, fp64,
+one query row at a time; see that file's header for the page passages each
+function follows and the readings taken where the pages are silent). This
+module compiles it with gcc, and marshals numpy arrays into it. The indexer's
+training loss and its backward pass are in ``kl.py`` (numpy, fp64; its header
+lists its sources, readings and pins).
 
 Inputs are numpy arrays: ``float32`` for fp32 data, ``uint16`` holding raw
 bf16 bit patterns for bf16 data, or ``uint8`` holding e4m3 codes (indexer
@@ -25,6 +27,9 @@ Parity status per function (what pins it, independently of this code):
                  with include_self (§3.4): S_10 = {3, 9, 10} from the
                  page's trace, t always kept, the rest equal to Python's
                  sort of positions 0..t-1.
+  kl.kl_rows, kl.indexer_backward_* : see kl.py (the warm-up target example
+                 of "Learned Token Selection" §5.3, KL closed forms, torch's
+                 kl_div and autograd, central differences).
   attn_rows    : torch's dense causal scaled_dot_product_attention when the
                  budget covers every candidate ("Learned Token Selection" §7.6 note, §9.3),
                  |S|=1 and equal-score special cases, permutation invariance.
