@@ -212,6 +212,10 @@ BWD_SHAPES = {
                                                   seed=41),
     "bwd_prefill_300": WORKLOADS["prefill8k"].replace(name="bwd_prefill_300", Tq=300, L=300, seed=42),
     "bwd_odd": WORKLOADS["prefill8k"].replace(name="bwd_odd", Tq=150, L=150, H_I=32, d_I=64, seed=43),
+    # the tensor-core path with 32 and 128 heads (four and one queries per group)
+    "bwd_heads32": WORKLOADS["prefill8k"].replace(name="bwd_heads32", Tq=260, L=260, H_I=32, seed=44),
+    "bwd_heads128": WORKLOADS["prefill8k"].replace(name="bwd_heads128", B=2, Tq=131, L=200, q_pos0=69, H_I=128,
+                                                   seed=45),
 }
 
 

@@ -48,6 +48,14 @@ MEDIUM = {
                          Dqk=20, Dv=12, dtype="f32", idx_range=4, seed=18),
     "single_position": Workload("single_position", B=2, Tq=1, L=1, q_pos0=0, H_I=64, d_I=128, k=1,
                                 Hq=16, Hkv=1, Dqk=128, Dv=128, seed=19),
+    # indexer heads other than 64 on the tensor cores: 128 heads (two queries
+    # per tile, half the epilogue groups idle) and 32 heads of width 128
+    "heads128_prefill": Workload("heads128_prefill", B=2, Tq=260, L=260, q_pos0=0, H_I=128, d_I=128, k=40,
+                                 Hq=16, Hkv=1, Dqk=128, Dv=128, seed=23),
+    "heads32_prefill": Workload("heads32_prefill", B=1, Tq=333, L=333, q_pos0=0, H_I=32, d_I=128, k=40,
+                                Hq=16, Hkv=1, Dqk=128, Dv=128, seed=24),
+    "heads128_decode": Workload("heads128_decode", B=3, Tq=1, L=3000, q_pos0=2999, H_I=128, d_I=128, k=256,
+                                Hq=16, Hkv=1, Dqk=128, Dv=128, seed=25),
 }
 
 FULL_ROWS = {
@@ -122,7 +130,7 @@ def test_hand_trace_on_gpu(cuda):
 
 
 @pytest.mark.parametrize("name", ["prefill_mqa_700", "chunked_prefill", "decode_5000", "odd_heads",
-                                  "tiny_f32"])
+                                  "tiny_f32", "heads128_prefill", "heads32_prefill", "heads128_decode"])
 def test_indexer_stage_all_rows(cuda, name):
     wl = MEDIUM[name]
     cpu, dev = _inputs(wl)
