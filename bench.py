@@ -229,7 +229,7 @@ def _oracle_rate(wl, seconds: float, rows: int) -> float:
 
 def _sample_rows_for(wl, budget_s: float, nthreads: int, cpu) -> int:
     """Rows of the oracle that fit a wall-clock budget (probe with a few rows)."""
-    probe = max(1, min(wl.B * wl.Tq, max(1, nthreads)))
+    probe = max(1, min(wl.B * wl.Tq, max(8, nthreads)))
     sec, rows = time_oracle(wl, cpu, probe, nthreads)
     per_row = sec / rows
     return int(max(1, min(wl.B * wl.Tq, budget_s / per_row)))
@@ -414,6 +414,11 @@ def run_ours(args, wl):
                         "kind": "oracle",
                         "sample": f"{rows} of {wl.B * wl.Tq} query rows (all three stages), {reps} "
                                   f"repetition(s), {total_s:.1f} s in total, scaled to a full step"}
+        # the same oracle on one core, on a smaller sample of the same rows
+        rows1 = _sample_rows_for(wl, args.cpu_budget / 4, 1, cpu)
+        secs1, r1 = time_oracle(wl, cpu, rows1, 1)
+        cpu_baseline["single_core"] = {"value": _oracle_rate(wl, secs1, r1), "unit": unit, "cores": 1,
+                                       "sample": f"{r1} query rows, {secs1:.1f} s, scaled to a full step"}
 
     if rank == 0:
         line = {
