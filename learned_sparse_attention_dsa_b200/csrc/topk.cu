@@ -11,15 +11,25 @@
 // k-th largest score and the number r of T-valued positions that still fit.
 //
 // A row is handled by a cluster of P CTAs (P = 1..16; P > 1 when there are
-// fewer rows than SMs, as in decode), each owning a contiguous slice. Digit
-// histograms are summed across the cluster through distributed shared memory
-// so every CTA derives the same threshold. A slice of at most 512 * KPT keys
-// is held in registers (KPT keys per thread); longer slices are streamed from
-// global memory (L2 after the first read), so several CTAs fit on an SM.
-// After the first pass the keys of the threshold bucket -- usually a few
-// percent of the row -- are compacted into shared memory with their
-// positions; the later passes and the per-warp counts run on that list only
-// (slices with more candidates than the list holds are swept again).
+// fewer rows than SMs, as in decode), each owning a contiguous slice. A slice
+// of at most 512 * KPT keys is held in registers (KPT keys per thread);
+// longer slices are streamed from global memory (L2 after the first read), so
+// two CTAs fit on an SM. The exchange is built from few cluster barriers,
+// each preceded by fire-and-forget writes into the other CTAs' shared memory:
+//  1. every CTA adds the non-empty bins of its first-digit histogram into
+//     every CTA's copy of the row histogram (distributed shared memory
+//     atomics); after one barrier each CTA picks the same first digit d1
+//     locally;
+//  2. every CTA compacts the keys of bucket d1 -- usually a few percent of
+//     the row -- into a list in position order and stores it, 16 bytes at a
+//     time, into its own region of every CTA's gather buffer, with its
+//     candidate count and its count of keys above d1; after a second barrier
+//     each CTA runs passes 2 and 3 alone on the gathered keys (warp c walks
+//     the region of CTA c) and touches no other CTA's memory again.
+// When some CTA has more candidates than its region holds (heavy ties),
+// passes 2 and 3 run cluster-wide instead: each CTA reduces one segment of
+// the digit histograms over the cluster and the digit is found from the
+// segment totals (the lists, or sweeps when a list overflows, feed them).
 // Output: each warp owns a contiguous segment of its CTA's slice; with the
 // number of keys > T and = T before the segment (from the list, the warps
 // before it and the CTAs before it) every kept position's output slot is
@@ -41,7 +51,7 @@ constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / kWarp;
 constexpr int kBins = 2048;
 constexpr int kListCap = 4096;    // candidate keys + positions of this CTA, in shared memory
-constexpr int kGatherCap = 4096;  // candidate keys of the whole row gathered by every CTA
+constexpr int kGatherCap = 8192;  // candidate keys of the whole row gathered by every CTA
 // (list + gather buffer + scratch + histograms stay under half the shared
 // memory of an SM, so two 512-thread CTAs fit)
 constexpr int kMaxCluster = 16;
@@ -66,9 +76,11 @@ __device__ __forceinline__ void cluster_wait() {
 }
 
 struct FindScratch {
-    int local[kThreads];     // bucket total per thread (descending digit order)
-    int red[kBins];          // this CTA's segment of the cluster-summed histogram
+    int local[kWarps];       // per-warp totals of the digit search
+    int red[kBins];          // the cluster-summed first-digit histogram; later (passes 2
+                             // and 3 of the slow path) this CTA's segment of a summed one
     int seg_total;           // sum of that segment
+    int pad_[3];             // keeps the gather buffer after this struct 16-byte aligned
 };
 
 __device__ __forceinline__ void pick_in_segment(const int *seg_bins, int seg, int first_digit, int base_above,
@@ -128,43 +140,34 @@ __device__ __forceinline__ void find_digit_rs(const cg::cluster_group &cluster, 
 
 // Bins seg_bins[0..seg) hold the counts of digits first_digit .. first_digit +
 // seg - 1; base_above keys lie in higher digits. Find the digit whose bucket
-// holds the remaining-th largest key: each thread sums (seg / kThreads, at
-// least one) consecutive bins from the top, warp 0 scans the totals. Sets
-// s_digit / s_above. Two block barriers.
+// holds the remaining-th largest key: thread i sums the per = max(1, seg /
+// kThreads) consecutive bins below seg - 1 - i * per (descending digits), a
+// block-wide scan of those sums finds the one thread whose range crosses
+// `remaining`, and that thread walks its own bins. Sets s_digit / s_above.
+// Two block barriers.
 __device__ __forceinline__ void pick_in_segment(const int *seg_bins, int seg, int first_digit, int base_above,
                                                 int remaining, FindScratch &fs, int *s_digit, int *s_above) {
     const int per = seg >= kThreads ? seg / kThreads : 1;
+    const int top = seg - 1 - (int)threadIdx.x * per;  // this thread's highest bin
     int local = 0;
-    if (threadIdx.x * per < seg) {
-        for (int j = 0; j < per; ++j) local += seg_bins[seg - 1 - (threadIdx.x * per + j)];  // descending
-    }
-    fs.local[threadIdx.x] = local;
+    if (top >= 0)
+        for (int j = 0; j < per; ++j) local += seg_bins[top - j];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int incl = warp_inclusive_scan(local);
+    if (lane == kWarp - 1) fs.local[warp] = incl;  // warp totals
     __syncthreads();
-    if (threadIdx.x < kWarp) {
-        const int lane = threadIdx.x;
-        constexpr int kPerLane = kThreads / kWarp;
-        int sum = 0;
-#pragma unroll
-        for (int i = 0; i < kPerLane; ++i) sum += fs.local[lane * kPerLane + i];
-        const int incl = warp_inclusive_scan(sum);
-        int run = base_above + incl - sum;
-        if (run < remaining && base_above + incl >= remaining) {
-            for (int i = 0; i < kPerLane; ++i) {
-                const int t = lane * kPerLane + i;
-                if (run + fs.local[t] >= remaining) {
-                    for (int j = 0; j < per; ++j) {
-                        const int cj = seg_bins[seg - 1 - (t * per + j)];
-                        if (run + cj >= remaining) {
-                            *s_digit = first_digit + seg - 1 - (t * per + j);
-                            *s_above = run;
-                            break;
-                        }
-                        run += cj;
-                    }
-                    break;
-                }
-                run += fs.local[t];
+    const int before = warp_sum_int(lane < warp ? fs.local[lane] : 0);  // kWarps <= 32
+    const int upto = base_above + before + incl;  // keys in this thread's bins and above
+    int run = upto - local;                       // keys above this thread's bins
+    if (run < remaining && upto >= remaining) {
+        for (int j = 0; j < per; ++j) {
+            const int c = seg_bins[top - j];
+            if (run + c >= remaining) {
+                *s_digit = first_digit + top - j;
+                *s_above = run;
+                break;
             }
+            run += c;
         }
     }
     __syncthreads();
@@ -229,10 +232,12 @@ topk_kernel(const float *__restrict__ scores, int Tq, int L, int q_pos0, int k, 
     int32_t *list_pos = reinterpret_cast<int32_t *>(dyn_smem + 4 * kListCap);   // [kListCap]
     FindScratch &fs = *reinterpret_cast<FindScratch *>(dyn_smem + 8 * kListCap);
     uint32_t *gkey = reinterpret_cast<uint32_t *>(dyn_smem + 8 * kListCap + sizeof(FindScratch));  // [kGatherCap]
-    __shared__ int w_gt[kWarps], w_eq[kWarps];
-    __shared__ int s_digit, s_above, s_nlist, s_seg, s_gather;
-    __shared__ int s_counts[2], s_pub[2], s_before[2];
-    __shared__ int g_n[kMaxCluster], g_gt1[kMaxCluster], g_off[kMaxCluster + 1];
+    // per warp: candidates in bucket d1, keys above it, and (gathered path)
+    // candidates > T and = T
+    __shared__ int w_cnt[kWarps], w_gt[kWarps], w_eq[kWarps], w_gtT[kWarps];
+    __shared__ int s_digit, s_above, s_seg;
+    __shared__ int s_counts[2], s_before[2];
+    __shared__ int g_n[kMaxCluster], g_gt1[kMaxCluster];  // per CTA of the cluster
 
     cg::cluster_group cluster = cg::this_cluster();
     const int P = (int)cluster.num_blocks();
@@ -259,13 +264,15 @@ topk_kernel(const float *__restrict__ scores, int Tq, int L, int q_pos0, int k, 
     // the row's own position t = n - 1 sits at the end of the last slice
     sl.self_s = (SELF && t >= lo && t < lo + sl.cnt) ? t - lo : -1;
 
-    for (int b = threadIdx.x; b < kBins; b += kThreads) {
-        hist[0][b] = 0;
-        hist[1][b] = 0;
-        hist[2][b] = 0;
+    // zero the three local histograms and fs.red, which receives the
+    // cluster-wide sum of the first-digit histograms
+    {
+        int4 *h4 = reinterpret_cast<int4 *>(&hist[0][0]);
+        for (int i = threadIdx.x; i < 3 * kBins / 4; i += kThreads) h4[i] = make_int4(0, 0, 0, 0);
+        int4 *r4 = reinterpret_cast<int4 *>(fs.red);
+        for (int i = threadIdx.x; i < kBins / 4; i += kThreads) r4[i] = make_int4(0, 0, 0, 0);
     }
     if (threadIdx.x == 0) {
-        s_nlist = 0;
         s_seg = 0;  // always a valid cluster rank, even if a search found nothing
         s_digit = 0;
         s_above = 0;
@@ -273,6 +280,7 @@ topk_kernel(const float *__restrict__ scores, int Tq, int L, int q_pos0, int k, 
         s_before[1] = 0;
     }
     __syncthreads();
+    cluster_arrive();  // (1) this CTA's sum is zeroed; waited on after pass 1
 
     // ---- pass 1: bits 31..21 of every key (the keys land in registers)
     RegKeys<KPT> rk;
@@ -288,84 +296,90 @@ topk_kernel(const float *__restrict__ scores, int Tq, int L, int q_pos0, int k, 
         if (ok) atomicAdd(&hist[0][key >> 21], 1);
     });
     __syncthreads();
-    cluster.sync();
-    int remaining = k;
-    find_digit_rs<kBins>(cluster, hist[0], P, part, remaining, fs, &s_digit, &s_above, &s_seg);
+    cluster_wait();  // (1) every CTA of the cluster has zeroed its sum
+    // add this CTA's non-empty bins into every CTA's sum
+    for (int b = threadIdx.x; b < kBins; b += kThreads) {
+        const int c = hist[0][b];
+        if (c)
+            for (int r = 0; r < P; ++r) atomicAdd(cluster.map_shared_rank(fs.red, r) + b, c);
+    }
+    cluster.sync();  // (2) the row's first-digit histogram is complete everywhere
+    pick_in_segment(fs.red, kBins, 0, 0, k, fs, &s_digit, &s_above);
     const uint32_t d1 = (uint32_t)s_digit;
-    remaining -= s_above;
+    int remaining = k - s_above;
 
-    // ---- compact the threshold bucket; count keys in higher buckets per warp
-    int gt1 = 0;
-    sweep<KPT, SELF>(sl, rk, [&](int s, uint32_t key, bool ok) {
-        const bool cand = ok && (key >> 21) == d1;
-        gt1 += ok && (key >> 21) > d1;
-        const unsigned m = __ballot_sync(0xffffffffu, cand);
-        if (m) {
-            int slot0 = 0;
-            if (lane == 0) slot0 = atomicAdd(&s_nlist, __popc(m));
-            slot0 = __shfl_sync(0xffffffffu, slot0, 0);
-            const int slot = slot0 + __popc(m & lanemask_lt());
-            if (cand && slot < kListCap) {
-                list_key[slot] = key;
-                list_pos[slot] = s;
-            }
+    // ---- per warp: keys in bucket d1 (candidates) and above it
+    {
+        int cnt = 0, gt1 = 0;
+        sweep<KPT, SELF>(sl, rk, [&](int, uint32_t key, bool ok) {
+            cnt += ok && (key >> 21) == d1;
+            gt1 += ok && (key >> 21) > d1;
+        });
+        cnt = warp_sum_int(cnt);
+        gt1 = warp_sum_int(gt1);
+        if (lane == 0) {
+            w_cnt[warp] = cnt;
+            w_gt[warp] = gt1;
+            w_eq[warp] = 0;
         }
-    });
-    gt1 = warp_sum_int(gt1);
-    if (lane == 0) {
-        w_gt[warp] = gt1;
-        w_eq[warp] = 0;
     }
     __syncthreads();
-    const int n_list = s_nlist;
+    // first slot of this warp's candidates among the CTA's, and their number (kWarps <= 32)
+    const int wbase = warp_sum_int(lane < warp ? w_cnt[lane] : 0);
+    const int n_list = warp_sum_int(lane < kWarps ? w_cnt[lane] : 0);
     const bool use_list = n_list <= kListCap;
+    const int cap = kGatherCap / P;  // gather-buffer region of each CTA (a multiple of four keys)
 
-    // ---- publish (candidates, keys above the bucket) and read everyone's
-    if (threadIdx.x == 0) {
+    // ---- this CTA's candidates into its list, in position order
+    if (use_list) {
+        int slot = wbase;
+        sweep<KPT, SELF>(sl, rk, [&](int s, uint32_t key, bool ok) {
+            const bool cand = ok && (key >> 21) == d1;
+            const unsigned m = __ballot_sync(0xffffffffu, cand);
+            if (cand) {
+                const int j = slot + __popc(m & lanemask_lt());
+                list_key[j] = key;
+                list_pos[j] = s;
+            }
+            slot += __popc(m);
+        });
+    }
+    // the number of candidates and of keys above bucket d1, to every CTA
+    if (threadIdx.x < P) {
         int g = 0;
         for (int w = 0; w < kWarps; ++w) g += w_gt[w];
-        s_pub[0] = n_list;
-        s_pub[1] = g;
+        cluster.map_shared_rank(g_n, threadIdx.x)[part] = n_list;
+        cluster.map_shared_rank(g_gt1, threadIdx.x)[part] = g;
     }
-    __syncthreads();
-    cluster.sync();
-    if (threadIdx.x < P) {
-        const int *rc = cluster.map_shared_rank(s_pub, threadIdx.x);
-        g_n[threadIdx.x] = rc[0];
-        g_gt1[threadIdx.x] = rc[1];
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        int off = 0, ok = 1;
-        for (int c = 0; c < P; ++c) {
-            g_off[c] = off;
-            off += g_n[c];
-            ok &= g_n[c] <= kListCap;
+    if (n_list <= cap) {
+        // the list into this CTA's region of every CTA's gather buffer, 16 bytes at a time
+        __syncthreads();
+        const int n4 = (n_list + 3) >> 2;
+        const uint4 *src = reinterpret_cast<const uint4 *>(list_key);
+        for (int i = threadIdx.x; i < P * n4; i += kThreads) {
+            const int r = i / n4, q = i - r * n4;
+            reinterpret_cast<uint4 *>(cluster.map_shared_rank(gkey, r) + part * cap)[q] = src[q];
         }
-        g_off[P] = off;
-        s_gather = ok && off <= kGatherCap;
     }
-    __syncthreads();
+    cluster.sync();  // (3) candidates and counts delivered; no remote access after this on the gathered path
+    // the gathered path when every CTA's candidates fit its region (the same decision everywhere)
+    const bool gather = __syncthreads_and(threadIdx.x >= P || g_n[threadIdx.x] <= cap);
 
     uint32_t T;
     int r, gt_b = 0, eq_b = 0;
-    if (s_gather) {
-        // ---- every CTA gathers all candidate keys of the row and finishes
-        // the selection alone: no more cluster-wide rounds
-        const int total = g_off[P];
-        for (int c = 0; c < P; ++c) {
-            const uint32_t *src = cluster.map_shared_rank(list_key, c);
-            for (int j = threadIdx.x; j < g_n[c]; j += kThreads) gkey[g_off[c] + j] = src[j];
-        }
-        cluster_arrive();  // done with the other CTAs' shared memory
-        __syncthreads();
-        for (int j = threadIdx.x; j < total; j += kThreads) atomicAdd(&hist[1][(gkey[j] >> 10) & 2047u], 1);
+    if (gather) {
+        // ---- every CTA holds all candidate keys of the row, CTA c's in
+        // region c in position order, and finishes the selection alone;
+        // warp c walks region c
+        const uint32_t *reg = gkey + warp * cap;
+        const int n_reg = warp < P ? g_n[warp] : 0;
+        for (int j = lane; j < n_reg; j += kWarp) atomicAdd(&hist[1][(reg[j] >> 10) & 2047u], 1);
         __syncthreads();
         pick_in_segment(hist[1], kBins, 0, 0, remaining, fs, &s_digit, &s_above);
         const uint32_t p2 = (d1 << 11) | (uint32_t)s_digit;
         remaining -= s_above;
-        for (int j = threadIdx.x; j < total; j += kThreads) {
-            const uint32_t key = gkey[j];
+        for (int j = lane; j < n_reg; j += kWarp) {
+            const uint32_t key = reg[j];
             if ((key >> 10) == p2) atomicAdd(&hist[2][key & 1023u], 1);
         }
         __syncthreads();
@@ -373,43 +387,40 @@ topk_kernel(const float *__restrict__ scores, int Tq, int L, int q_pos0, int k, 
         T = (p2 << 10) | (uint32_t)s_digit;
         remaining -= s_above;
         r = remaining;
-        // keys > T and = T before this CTA (gathered), and per warp of this CTA (own list)
-        int gb = 0, eb = 0;
-        for (int j = threadIdx.x; j < g_off[part]; j += kThreads) {
-            gb += gkey[j] > T;
-            eb += gkey[j] == T;
-        }
-        for (int j = threadIdx.x; j < n_list; j += kThreads) {
-            const uint32_t key = list_key[j];
-            const int w = list_pos[j] / seg;
-            if (key > T) atomicAdd(&w_gt[w], 1);
-            else if (key == T) atomicAdd(&w_eq[w], 1);
-        }
-        gb = warp_sum_int(gb);
-        eb = warp_sum_int(eb);
-        if (lane == 0) {
-            atomicAdd(&s_before[0], gb);
-            atomicAdd(&s_before[1], eb);
-        }
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            int g = 0, e = 0;
-            for (int w = 0; w < kWarps; ++w) {
-                const int gw = w_gt[w], ew = w_eq[w];
-                w_gt[w] = g;
-                w_eq[w] = e;
-                g += gw;
-                e += ew;
+        // candidates > T and = T in the CTAs before this one (warp c: region c)
+        if (warp < part) {
+            int gb = 0, eb = 0;
+            for (int j = lane; j < n_reg; j += kWarp) {
+                const uint32_t key = reg[j];
+                gb += key > T;
+                eb += key == T;
+            }
+            gb = warp_sum_int(gb);
+            eb = warp_sum_int(eb);
+            if (lane == 0) {
+                atomicAdd(&s_before[0], gb);
+                atomicAdd(&s_before[1], eb);
             }
         }
+        // ... and in this warp's own range of this CTA's region
+        int wg = 0, we = 0;
+        for (int j = lane; j < w_cnt[warp]; j += kWarp) {
+            const uint32_t key = gkey[part * cap + wbase + j];
+            wg += key > T;
+            we += key == T;
+        }
+        wg = warp_sum_int(wg);
+        we = warp_sum_int(we);
+        if (lane == 0) {
+            w_gtT[warp] = wg;
+            w_eq[warp] = we;
+        }
         __syncthreads();
-        gt_b = s_before[0];
-        eq_b = s_before[1];
+        gt_b = s_before[0] + warp_sum_int(lane < warp ? w_gt[lane] + w_gtT[lane] : 0);
+        eq_b = s_before[1] + warp_sum_int(lane < warp ? w_eq[lane] : 0);
         for (int c = 0; c < part; ++c) gt_b += g_gt1[c];
     } else {
         // ---- too many candidates (heavy ties): cluster-wide passes 2 and 3
-        uint32_t p2;
-        {
     // ---- pass 2: bits 20..10 of the keys in bucket d1
     if (use_list) {
         for (int j = threadIdx.x; j < n_list; j += kThreads)
@@ -422,7 +433,7 @@ topk_kernel(const float *__restrict__ scores, int Tq, int L, int q_pos0, int k, 
     __syncthreads();
     cluster.sync();
     find_digit_rs<kBins>(cluster, hist[1], P, part, remaining, fs, &s_digit, &s_above, &s_seg);
-    p2 = (d1 << 11) | (uint32_t)s_digit;
+    const uint32_t p2 = (d1 << 11) | (uint32_t)s_digit;
     remaining -= s_above;
 
     // ---- pass 3: bits 9..0 of the keys whose top 22 bits are p2
@@ -485,12 +496,11 @@ topk_kernel(const float *__restrict__ scores, int Tq, int L, int q_pos0, int k, 
         eq_b += rc[1];
     }
     cluster_arrive();  // done with the other CTAs' shared memory
-        }
+    gt_b += w_gt[warp];
+    eq_b += w_eq[warp];
     }
 
     // ---- write the kept positions of this warp's segment in order
-    gt_b += w_gt[warp];
-    eq_b += w_eq[warp];
     const unsigned lt = lanemask_lt();
     sweep<KPT, SELF>(sl, rk, [&](int s, uint32_t key, bool ok) {
         const bool gt = ok && key > T;
@@ -505,7 +515,7 @@ topk_kernel(const float *__restrict__ scores, int Tq, int L, int q_pos0, int k, 
         gt_b += __popc(gm);
         eq_b += __popc(em);
     });
-    cluster_wait();  // no CTA leaves while another may still read its shared memory
+    if (!gather) cluster_wait();  // no CTA leaves while another may still read its shared memory
 }
 
 constexpr size_t kDynSmem = 8 * (size_t)kListCap + sizeof(FindScratch) + 4 * (size_t)kGatherCap;
