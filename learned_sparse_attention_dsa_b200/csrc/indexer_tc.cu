@@ -15,14 +15,16 @@
 //   warp 0      TMA producer: Q tile of the unit once, then key tiles through
 //               a K_STAGES-deep ring (128-byte swizzle, K-major).
 //   warp 1      allocates TMEM; one thread issues tcgen05.mma (bf16 in, fp32
-//               accumulate) into one of two TMEM accumulators.
+//               accumulate) into the TMEM accumulators in turn (four when
+//               4 * N_TILE columns fit, else two).
 //   warps 2..   epilogue, EPI = 8 or 16 warps, EPI / 4 per TMEM lane quarter (each takes every
 //               other query of the tile; with one query per tile, as in
-//               decode, every other tile): tcgen05.ld of the accumulator,
-//               ReLU, weight and head sum with packed fp32x2 FMAs, one fp32
-//               score per (query, key), causal mask.
-// The two accumulators let the epilogue of tile n overlap the MMAs of tile
-// n+1. A work unit is (batch entry, query group, chunk of at most C key
+//               decode, the groups take the accumulators in turn):
+//               tcgen05.ld of the accumulator, ReLU, weight and head sum
+//               with packed fp32x2 FMAs, one fp32 score per (query, key),
+//               causal mask.
+// The accumulators let the epilogue of tile n overlap the MMAs of the tiles
+// after it. A work unit is (batch entry, query group, chunk of at most C key
 // tiles); units are spread over the CTAs round-robin. Causal: a query group
 // only visits key tiles up to its last query position.
 //
@@ -110,8 +112,11 @@ struct Cfg {
     static constexpr int kStagesRaw = (int)((kSmemBudget - kQBufs * kQBytes) / kKBytes);
     // as many key stages as fit: with 16 KB e4m3 stages, 13 keep ~200 KB in flight
     static constexpr int kStages = kStagesRaw > 16 ? 16 : kStagesRaw;
-    static constexpr uint32_t kTmemCols = 2 * N_TILE;
-    static constexpr int kBars = 2 * kStages + 2 * kQBufs + 4;
+    // accumulator buffers in TMEM: four when they fit (the MMA runs further
+    // ahead of the epilogue), else two
+    static constexpr int kAcc = 4 * N_TILE <= 512 ? 4 : 2;
+    static constexpr uint32_t kTmemCols = kAcc * N_TILE;
+    static constexpr int kBars = 2 * kStages + 2 * kQBufs + 2 * kAcc;
     static constexpr size_t kSmem = 1024 + (size_t)kQBufs * kQBytes + (size_t)kStages * kKBytes + kBars * 8 + 16;
     static_assert(kStages >= 2, "shared memory too small for the pipeline");
     static_assert(kTmemCols == 128 || kTmemCols == 256 || kTmemCols == 512, "TMEM columns");
@@ -132,8 +137,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     uint64_t *q_full = k_empty + C::kStages;
     uint64_t *q_empty = q_full + C::kQBufs;
     uint64_t *acc_full = q_empty + C::kQBufs;
-    uint64_t *acc_empty = acc_full + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
+    uint64_t *acc_empty = acc_full + C::kAcc;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + C::kAcc);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -147,11 +152,12 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             mbar_init(&q_full[s], 1);
             mbar_init(&q_empty[s], 1);
         }
-        // one query per tile (decode): the two warps of a TMEM lane quarter
-        // take alternate tiles (accumulators), else alternate queries
-        // decode: each tile is taken by one group of four warps (one per lane quarter)
+        // one query per tile (decode): each tile is taken by one group of
+        // four warps (one per TMEM lane quarter), the groups taking the
+        // accumulator buffers in turn; else every epilogue warp works on
+        // every tile (its share of the queries)
         const int releasers = p.QPT == 1 ? 128 : Threads<EPI>::kEpilogue;
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < C::kAcc; ++s) {
             mbar_init(&acc_full[s], 1);
             mbar_init(&acc_empty[s], releasers);
         }
@@ -229,7 +235,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     mma_commit(&k_empty[ks]);   // key stage free once these MMAs finish
                     mma_commit(&acc_full[ab]);  // accumulator ready for the epilogue
                     if (++ks == C::kStages) { ks = 0; kph ^= 1u; }
-                    if (++ab == 2) { ab = 0; aph ^= 1u; }
+                    if (++ab == C::kAcc) { ab = 0; aph ^= 1u; }
                 }
                 if (!ok) break;
                 mma_commit(&q_empty[qb]);
@@ -253,8 +259,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             const size_t row0 = (size_t)un.b * p.Tq + un.i0;
             const float4 *w4 = reinterpret_cast<const float4 *>(p.w + row0 * p.H);
             for (int kt = un.kt0; kt < un.kt1; ++kt) {
-                if (by_tile && ab != half) {  // the other warp of the quarter takes this tile
-                    if (++ab == 2) { ab = 0; aph ^= 1u; }
+                if (by_tile && ab % (EPI / 4) != half) {  // another warp of the quarter takes this tile
+                    if (++ab == C::kAcc) { ab = 0; aph ^= 1u; }
                     continue;
                 }
                 if (!mbar_wait(&acc_full[ab], aph)) { ok = false; break; }
@@ -294,7 +300,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 }
                 tc_fence_before();
                 mbar_arrive(&acc_empty[ab]);
-                if (++ab == 2) { ab = 0; aph ^= 1u; }
+                if (++ab == C::kAcc) { ab = 0; aph ^= 1u; }
             }
         }
     }
