@@ -486,19 +486,20 @@ attn_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Args a) {
         const float inv = l > 0.0f ? 1.0f / l : 0.0f;
         float4 *stage = reinterpret_cast<float4 *>(smem + h * (kHalfDv * 4));
 #pragma unroll 1
-        for (int c = 0; c < kHalfDv; c += 32) {
-            uint32_t o[32];
+        for (int c = 0; c < kHalfDv; c += 64) {  // two loads per wait
+            uint32_t o[64];
             if (have_o) {
                 tmem_ld_32x32b_x32(tmem + lane_addr + kColO + (uint32_t)c, o);
+                tmem_ld_32x32b_x32(tmem + lane_addr + kColO + (uint32_t)(c + 32), o + 32);
                 tmem_ld_wait();
             } else {
 #pragma unroll
-                for (int j = 0; j < 32; ++j) o[j] = 0u;
+                for (int j = 0; j < 64; ++j) o[j] = 0u;
             }
             if (a.splits == 1) {
                 uint4 *dst = reinterpret_cast<uint4 *>(a.out + pair * DV + part * kHalfDv + c);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
+                for (int q = 0; q < 8; ++q) {
                     uint32_t w[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
@@ -508,7 +509,7 @@ attn_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Args a) {
                 }
             } else {
 #pragma unroll
-                for (int v = 0; v < 8; ++v)
+                for (int v = 0; v < 16; ++v)
                     stage[rot_q(h, c / 4 + v)] =
                         make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
                                     __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));

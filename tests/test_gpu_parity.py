@@ -148,7 +148,10 @@ def test_indexer_stage_all_rows(cuda, name):
                                            (32768, 3, 32765, 1000), (70000, 2, 69998, 2048),
                                            (140000, 1, 139999, 2048), (2100, 2100, 0, 2048),
                                            # many rows of 16K-49K scores: the shared-memory kernel
-                                           (20003, 200, 19803, 2048), (49152, 150, 49002, 1000)])
+                                           (20003, 200, 19803, 2048), (49152, 150, 49002, 1000),
+                                           # fewer rows than SMs: clusters of 8, 4 and 2 CTAs per row
+                                           (20000, 20, 19980, 2048), (6000, 40, 5960, 2048),
+                                           (9000, 80, 8920, 1000)])
 def test_topk_stage(cuda, kind, L, Tq, q_pos0, k):
     gen = torch.Generator().manual_seed(L + Tq + k)
     scores = random_score_rows(gen, Tq, L, kind)[None]            # [1, Tq, L]
@@ -223,7 +226,7 @@ def test_invalid_arguments_enqueue_nothing(cuda):
 @pytest.mark.parametrize("kind", ["int", "normal", "mixed"])
 @pytest.mark.parametrize("L,Tq,q_pos0,k", [(37, 37, 0, 5), (5000, 3, 4997, 2048), (3000, 2, 2998, 1),
                                            (140000, 1, 139999, 2048), (2100, 2100, 0, 2048),
-                                           (20003, 200, 19803, 2048)])
+                                           (20003, 200, 19803, 2048), (6000, 40, 5960, 2048)])
 def test_topk_stage_include_self(cuda, kind, L, Tq, q_pos0, k):
     gen = torch.Generator().manual_seed(L + Tq + k + 1)
     scores = random_score_rows(gen, Tq, L, kind)[None]
