@@ -264,6 +264,17 @@ topk_kernel(const float *__restrict__ scores, int Tq, int L, int q_pos0, int k, 
     // the row's own position t = n - 1 sits at the end of the last slice
     sl.self_s = (SELF && t >= lo && t < lo + sl.cnt) ? t - lo : -1;
 
+    // ---- pass 1: bits 31..21 of every key. The keys' loads (into registers)
+    // are issued first, so that their latency overlaps the zeroing below.
+    RegKeys<KPT> rk;
+    if constexpr (KPT > 0) {
+#pragma unroll
+        for (int i = 0; i < KPT; ++i) {
+            const int s = sl.w_lo + i * kWarp + lane;
+            const float v = s < sl.w_hi ? __ldg(sl.src + s) : 0.0f;
+            rk.k[i] = slice_key<SELF>(sl, s, v);
+        }
+    }
     // zero the three local histograms and fs.red, which receives the
     // cluster-wide sum of the first-digit histograms
     {
@@ -282,16 +293,6 @@ topk_kernel(const float *__restrict__ scores, int Tq, int L, int q_pos0, int k, 
     __syncthreads();
     cluster_arrive();  // (1) this CTA's sum is zeroed; waited on after pass 1
 
-    // ---- pass 1: bits 31..21 of every key (the keys land in registers)
-    RegKeys<KPT> rk;
-    if constexpr (KPT > 0) {
-#pragma unroll
-        for (int i = 0; i < KPT; ++i) {
-            const int s = sl.w_lo + i * kWarp + lane;
-            const float v = s < sl.w_hi ? __ldg(sl.src + s) : 0.0f;
-            rk.k[i] = slice_key<SELF>(sl, s, v);
-        }
-    }
     sweep<KPT, SELF>(sl, rk, [&](int, uint32_t key, bool ok) {
         if (ok) atomicAdd(&hist[0][key >> 21], 1);
     });
