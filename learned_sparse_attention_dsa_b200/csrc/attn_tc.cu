@@ -106,6 +106,7 @@ template <int DQK, int DV>
 __global__ void __launch_bounds__(kThreads)
 attn_mma_kernel(const Args a) {
     using C = Cfg<DQK, DV>;
+    wait_prior_grid();  // the selection comes from the kernel before (when launched to overlap it)
     extern __shared__ __align__(128) uint8_t smem[];
     int32_t *sel = reinterpret_cast<int32_t *>(smem + (C::kPipeBytes > C::kMergeBytes ? C::kPipeBytes
                                                                                         : C::kMergeBytes));
@@ -566,13 +567,14 @@ cudaError_t launch_mma(const AttnProblem &p, const DeviceInfo &info, cudaStream_
         cfg.blockDim = dim3(kThreads);
         cfg.dynamicSmemBytes = C::kSmem;
         cfg.stream = stream;
-        cudaLaunchAttribute attr[1];
+        cudaLaunchAttribute attr[2];
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = 1;
         attr[0].val.clusterDim.y = 1;
         attr[0].val.clusterDim.z = splits;
+        attr[1] = overlap_launch_attr();
         cfg.attrs = attr;
-        cfg.numAttrs = 1;
+        cfg.numAttrs = 2;
         err = cudaLaunchKernelEx(&cfg, kern, a);
         count_launch();
         return err;
