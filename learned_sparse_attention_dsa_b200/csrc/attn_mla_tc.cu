@@ -586,7 +586,8 @@ __global__ void attn_mla_combine_kernel(const float4 *__restrict__ part_o, const
 }
 
 // Splits per row: one CTA per SM over (row, split, part), at most kMaxTiles
-// tiles per split, at most kMaxSplits splits (one per combine lane).
+// tiles per split, at most kMaxSplits splits (one per combine lane), and no
+// more splits than the longest one needs.
 int mla_tc_splits(const AttnProblem &p, int sm_count) {
     const long long rows = (long long)p.B * p.Tq;
     const int tiles = (p.k + kTileN - 1) / kTileN;
@@ -596,6 +597,10 @@ int mla_tc_splits(const AttnProblem &p, int sm_count) {
     if (s > tiles) s = tiles;
     if (s > kMaxSplits) s = kMaxSplits;
     if (s < 1) s = 1;
+    // as few splits as give the same longest split (whole tiles each): the
+    // same time, fewer partials to write and combine
+    const long long per = (tiles + s - 1) / s;
+    s = (tiles + per - 1) / per;
     return (int)s;
 }
 
