@@ -51,8 +51,16 @@ struct Cfg {
     // (plus one merge weight per split and head)
     static constexpr int kMergeBytes = (kWarps + 1) * kHeads * (DV + 10) * 4 + 8 * kHeads * 4;
     static constexpr int kPipeBytes = kStages * kStageBytes;
-    static constexpr size_t kSmem =
-        (size_t)(kPipeBytes > kMergeBytes ? kPipeBytes : kMergeBytes) + kMaxSel * 4 + 64;
+    static constexpr size_t kRegion = (size_t)(kPipeBytes > kMergeBytes ? kPipeBytes : kMergeBytes);
+    static constexpr size_t kSmem = kRegion + kMaxSel * 4 + 64;
+    // with the cluster merge: the selection list of one split, then the
+    // receive area of this CTA's output slice from every split (P <= 8)
+    static constexpr int kQuads = kHeads * DV / 4;
+    static size_t cluster_smem(int splits, int per_split) {
+        const int per = (kQuads + splits - 1) / splits;
+        return kRegion + (size_t)per_split * 4 + (size_t)splits * per * 16 + (size_t)splits * kHeads * 8 + 64;
+    }
+    static constexpr size_t kSmemMax = kSmem + (size_t)(kQuads + 8) * 16 + 8 * kHeads * 8;
 };
 
 struct Args {
@@ -360,11 +368,13 @@ attn_mma_kernel(const Args a) {
         if (a.lse != nullptr && c0 == 0)
             a.lse[(size_t)row * a.Hq + h] = l_all > 0.0f ? (m_all + log2f(l_all)) / kLog2e : -INFINITY;
     } else if (a.cluster_merge) {
-        // the splits of this (row, head group) form one cluster: publish this
-        // CTA's (max, sum, O) in shared memory, then every CTA merges a slice
-        // of the 16 x DV outputs from all of them through distributed shared
-        // memory
-        float *cta_o = mrg_ml + kWarps * kHeads * 2;  // [16][DV]
+        // The splits of this (row, head group) form one cluster. CTA r owns
+        // quads [r * per, (r + 1) * per) of the 16 x DV outputs; every CTA
+        // stores its (max, sum) of the 16 heads and its O quads of each
+        // owner's slice into that owner's receive area (past the selection
+        // list, untouched by the owner before the barrier), so that after
+        // one cluster barrier each owner merges from its own shared memory.
+        float *cta_o = mrg_ml + kWarps * kHeads * 2;  // [16][DV], this CTA's merged O
         float *cta_ml = cta_o + kHeads * DV;          // [16][2]
         for (int c = c0; c < DV; c += 8) {
             float acc = 0.0f;
@@ -376,11 +386,26 @@ attn_mma_kernel(const Args a) {
             cta_ml[hh * 2 + 0] = m_all;
             cta_ml[hh * 2 + 1] = l_all;
         }
+        __syncthreads();
         cg::cluster_group cluster = cg::this_cluster();
-        cluster.sync();
         const int P = a.splits;
-        // (max, sum) of every split for the 16 heads: read once, then one
-        // weight per (split, head) with the 1/sum folded in
+        constexpr int kQuads = kHeads * DV / 4;
+        const int per = (kQuads + P - 1) / P;
+        float4 *recv_o = reinterpret_cast<float4 *>(sel + a.per_split);  // [P][per]
+        float2 *recv_ml = reinterpret_cast<float2 *>(recv_o + P * per);   // [P][16]
+        for (int q = threadIdx.x; q < kQuads; q += kThreads) {
+            const int r = q / per;
+            cluster.map_shared_rank(recv_o, r)[split * per + (q - r * per)] =
+                reinterpret_cast<const float4 *>(cta_o)[q];
+        }
+        if (threadIdx.x < P * kHeads) {
+            const int r = threadIdx.x / kHeads, he = threadIdx.x % kHeads;
+            cluster.map_shared_rank(recv_ml, r)[split * kHeads + he] =
+                make_float2(cta_ml[he * 2], cta_ml[he * 2 + 1]);
+        }
+        cluster.sync();  // every slice delivered; no CTA touches another's memory after this
+        // (max, sum) of every split for the 16 heads: one weight per
+        // (split, head) with the 1/sum folded in
         float *wts = cta_ml + kHeads * 2;  // [8][16]
         if (threadIdx.x < kHeads) {
             const int he = threadIdx.x;
@@ -390,7 +415,7 @@ attn_mma_kernel(const Args a) {
                 ms[r] = -INFINITY;
                 ls[r] = 0.0f;
                 if (r < P) {
-                    const float2 v = *reinterpret_cast<const float2 *>(cluster.map_shared_rank(cta_ml, r) + he * 2);
+                    const float2 v = recv_ml[r * kHeads + he];
                     ms[r] = v.x;
                     ls[r] = v.y;
                 }
@@ -409,9 +434,7 @@ attn_mma_kernel(const Args a) {
                 a.lse[(size_t)row * a.Hq + h0 + he] = l_x > 0.0f ? (m_x + log2f(l_x)) / kLog2e : -INFINITY;
         }
         __syncthreads();
-        // this CTA writes a 1/P slice of the 16 x DV outputs, four columns per step
-        constexpr int kQuads = kHeads * DV / 4;
-        const int per = (kQuads + P - 1) / P;
+        // this CTA's slice of the 16 x DV outputs, four columns per step
         const int e0 = split * per, e1 = min(kQuads, e0 + per);
         for (int e = e0 + threadIdx.x; e < e1; e += kThreads) {
             const int he = (4 * e) / DV, ce = 4 * e - he * DV;
@@ -420,7 +443,7 @@ attn_mma_kernel(const Args a) {
             for (int r = 0; r < 8; ++r) {
                 if (r < P) {
                     const float f = wts[r * kHeads + he];
-                    const float4 v = *reinterpret_cast<const float4 *>(cluster.map_shared_rank(cta_o, r) + he * DV + ce);
+                    const float4 v = recv_o[r * per + (e - e0)];
                     acc.x = fmaf(f, v.x, acc.x);
                     acc.y = fmaf(f, v.y, acc.y);
                     acc.z = fmaf(f, v.z, acc.z);
@@ -434,7 +457,6 @@ attn_mma_kernel(const Args a) {
             packed.y = *reinterpret_cast<uint32_t *>(&hi2);
             *reinterpret_cast<uint2 *>(a.out + ((size_t)row * a.Hq + h0 + he) * DV + ce) = packed;
         }
-        cluster.sync();  // no CTA leaves while another may still read its shared memory
     } else {
         const size_t pidx = ((size_t)row * a.Hq + h) * a.splits + split;
         float *dst = a.part_o + pidx * DV;
@@ -558,14 +580,14 @@ cudaError_t launch_mma(const AttnProblem &p, const DeviceInfo &info, cudaStream_
         a.part_ml = a.part_o + n_pairs * splits * DV;
     }
     auto kern = attn_mma_kernel<DQK, DV>;
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmemMax);
     if (err != cudaSuccess) return err;
     dim3 grid(rows, p.Hq / kHeads, splits);
     if (a.cluster_merge) {  // the splits of one (row, head group) form a cluster
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = grid;
         cfg.blockDim = dim3(kThreads);
-        cfg.dynamicSmemBytes = C::kSmem;
+        cfg.dynamicSmemBytes = C::cluster_smem(splits, per_split);
         cfg.stream = stream;
         cudaLaunchAttribute attr[2];
         attr[0].id = cudaLaunchAttributeClusterDimension;
