@@ -13,9 +13,12 @@
 // S = Q K^T with mma.sync m16n8k16 (bf16 in, fp32 accumulate; Q stays in
 // registers), an online softmax in fp32 (exp2 with the log2(e) prescale, as in
 // FlashAttention), and O += P V with P re-packed from the S accumulators as
-// the A operand. The four warps' (max, sum, O) are merged at the end; with a
-// split selected list the CTA writes fp32 partials and a combine kernel
-// merges the splits. Every selected row is loaded once for all 16 heads.
+// the A operand. The four warps' (max, sum, O) are merged at the end. With a
+// split selected list, up to eight splits form a thread-block cluster and
+// merge through distributed shared memory (each split stores its share of
+// every owner's output slice there, then one cluster barrier); more splits
+// write fp32 partials that a combine kernel merges. Every selected row is
+// loaded once for all 16 heads.
 #include <math.h>
 
 #include <cooperative_groups.h>
