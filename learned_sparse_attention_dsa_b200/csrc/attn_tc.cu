@@ -118,6 +118,9 @@ __global__ void __launch_bounds__(kThreads)
 attn_mma_kernel(const Args a) {
     using C = Cfg<DQK, DV>;
     wait_prior_grid();  // the selection comes from the kernel before (when launched to overlap it)
+    // cluster merge: this CTA has started (waited on before any other CTA
+    // stores into its shared memory)
+    if (a.cluster_merge) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
     extern __shared__ __align__(128) uint8_t smem[];
     int32_t *sel = reinterpret_cast<int32_t *>(smem + (C::kPipeBytes > C::kMergeBytes ? C::kPipeBytes
                                                                                         : C::kMergeBytes));
@@ -390,6 +393,8 @@ attn_mma_kernel(const Args a) {
             cta_ml[hh * 2 + 1] = l_all;
         }
         __syncthreads();
+        // every CTA of the cluster has started: its shared memory may be written
+        asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
         cg::cluster_group cluster = cg::this_cluster();
         const int P = a.splits;
         constexpr int kQuads = kHeads * DV / 4;
