@@ -159,7 +159,6 @@ __device__ __forceinline__ void issue_qk(uint32_t d, uint32_t a_tmem, uint64_t k
 
 __global__ void __launch_bounds__(kThreads, 1)
 attn_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Args a) {
-    wait_prior_grid();  // the selection comes from the kernel before (launched to overlap its tail)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *k_sm = smem;               // ring; slots 0-1 first stage the Q part
@@ -547,7 +546,6 @@ attn_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Args a) {
 __global__ void attn_mla_combine_kernel(const float4 *__restrict__ part_o, const float *__restrict__ part_ml,
                                         int n_pairs, int splits, __nv_bfloat16 *__restrict__ out,
                                         float *__restrict__ lse) {
-    wait_prior_grid();  // the partials come from the kernel before (launched to overlap its tail)
     // four warps per (row, head): warp quarter qt owns output float4s
     // [32 qt, 32 qt + 32), one per lane, and loads every split's value for it
     // independently (all in flight at once)
@@ -658,30 +656,23 @@ cudaError_t launch_attn_mla_tc(const AttnProblem &p, const DeviceInfo &info, cud
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = kSmem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[2];
+    cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;  // the two column parts of a (row, split)
     attr[0].val.clusterDim.x = 1;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 2;
-    attr[1] = overlap_launch_attr();
     cfg.attrs = attr;
-    cfg.numAttrs = 2;
+    cfg.numAttrs = 1;
     err = cudaLaunchKernelEx(&cfg, attn_mla_tc_kernel, tm_q, a);
     count_launch();
     if (err != cudaSuccess) return err;
     if (splits > 1) {
         const int warps_per_block = 8;  // four warps per (row, head) pair
         const int blocks = (int)((4 * n_pairs + warps_per_block - 1) / warps_per_block);
-        cudaLaunchConfig_t cc = {};
-        cc.gridDim = dim3((unsigned)blocks);
-        cc.blockDim = dim3(warps_per_block * 32);
-        cc.stream = stream;
-        cudaLaunchAttribute ca[1] = {overlap_launch_attr()};
-        cc.attrs = ca;
-        cc.numAttrs = 1;
-        err = cudaLaunchKernelEx(&cc, attn_mla_combine_kernel, reinterpret_cast<const float4 *>(a.part_o),
-                                 static_cast<const float *>(a.part_ml), (int)n_pairs, splits, a.out, a.lse);
+        attn_mla_combine_kernel<<<blocks, warps_per_block * 32, 0, stream>>>(
+            reinterpret_cast<const float4 *>(a.part_o), a.part_ml, (int)n_pairs, splits, a.out, a.lse);
         count_launch();
+        err = cudaGetLastError();
     }
     return err;
 }

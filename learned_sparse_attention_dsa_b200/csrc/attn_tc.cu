@@ -117,7 +117,6 @@ template <int DQK, int DV>
 __global__ void __launch_bounds__(kThreads)
 attn_mma_kernel(const Args a) {
     using C = Cfg<DQK, DV>;
-    wait_prior_grid();  // the selection comes from the kernel before (when launched to overlap it)
     // cluster merge: this CTA has started (waited on before any other CTA
     // stores into its shared memory)
     if (a.cluster_merge) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
@@ -597,14 +596,13 @@ cudaError_t launch_mma(const AttnProblem &p, const DeviceInfo &info, cudaStream_
         cfg.blockDim = dim3(kThreads);
         cfg.dynamicSmemBytes = C::cluster_smem(splits, per_split);
         cfg.stream = stream;
-        cudaLaunchAttribute attr[2];
+        cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = 1;
         attr[0].val.clusterDim.y = 1;
         attr[0].val.clusterDim.z = splits;
-        attr[1] = overlap_launch_attr();
         cfg.attrs = attr;
-        cfg.numAttrs = 2;
+        cfg.numAttrs = 1;
         err = cudaLaunchKernelEx(&cfg, kern, a);
         count_launch();
         return err;

@@ -79,22 +79,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
-// Programmatic dependent launch: a kernel launched with the programmatic
-// stream serialization attribute may be scheduled before the kernel ahead of
-// it in the stream has finished. Such a kernel calls this before it touches
-// global memory: it waits for that kernel's completion and the visibility of
-// its writes (a no-op for a kernel launched without the attribute).
-__device__ __forceinline__ void wait_prior_grid() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-
-// The launch attribute that lets a kernel's launch overlap the tail of the
-// kernel before it (the kernel must call wait_prior_grid first).
-inline cudaLaunchAttribute overlap_launch_attr() {
-    cudaLaunchAttribute a = {};
-    a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    a.val.programmaticStreamSerializationAllowed = 1;
-    return a;
-}
-
 __host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 __host__ __device__ __forceinline__ size_t align_up(size_t a, size_t b) { return (a + b - 1) / b * b; }
 

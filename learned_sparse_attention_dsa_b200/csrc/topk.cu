@@ -226,7 +226,6 @@ __device__ __forceinline__ void sweep(const Slice &sl, const RegKeys<KPT> &rk, F
 template <int KPT, bool SELF>
 __global__ void __launch_bounds__(kThreads, 2)  // two CTAs per SM: at most 64 registers
 topk_kernel(const float *__restrict__ scores, int Tq, int L, int q_pos0, int k, int32_t *__restrict__ idx) {
-    wait_prior_grid();  // the scores come from the kernel before (launched to overlap its tail)
     __shared__ __align__(16) int hist[3][kBins];
     extern __shared__ __align__(16) uint8_t dyn_smem[];
     uint32_t *list_key = reinterpret_cast<uint32_t *>(dyn_smem);                // [kListCap]
@@ -567,14 +566,13 @@ static cudaError_t launch_parts(const TopkProblem &p, int P, cudaStream_t stream
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = kDynSmem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[2];
+    cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = P;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
-    attr[1] = overlap_launch_attr();
     cfg.attrs = attr;
-    cfg.numAttrs = 2;
+    cfg.numAttrs = 1;
     if (P > 8) {  // a non-portable cluster size: make sure one can be scheduled
         int clusters = 0;
         err = cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg);
