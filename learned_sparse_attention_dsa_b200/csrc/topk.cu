@@ -329,7 +329,9 @@ topk_kernel(const float *__restrict__ scores, int Tq, int L, int q_pos0, int k, 
     const int wbase = warp_sum_int(lane < warp ? w_cnt[lane] : 0);
     const int n_list = warp_sum_int(lane < kWarps ? w_cnt[lane] : 0);
     const bool use_list = n_list <= kListCap;
-    const int cap = kGatherCap / P;  // gather-buffer region of each CTA (a multiple of four keys)
+    // gather-buffer region of each CTA (a multiple of four keys); never more
+    // than the list holds, so a gathered CTA always has its list
+    const int cap = min(kGatherCap / P, kListCap);
 
     // ---- this CTA's candidates into its list, in position order
     if (use_list) {
