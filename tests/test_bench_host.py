@@ -85,3 +85,21 @@ def test_units_and_metric():
     assert (units, unit) == (10.0, "decode steps/s")
     units, unit = bench._units(WORKLOADS["prefill8k"], 2)
     assert (units, unit) == (2 * 8192.0, "prefill tokens/s")
+
+
+def test_oracle_timing_helpers():
+    """The CPU-baseline legs: a bounded sample of rows, timed on one thread,
+    scaled to a whole step."""
+    import oracle
+    oracle.build()
+    wl = WORKLOADS["toy16"]
+    cpu = bench.make_inputs(wl)
+    rows = bench._sample_rows_for(wl, 0.2, 1, cpu)
+    assert 1 <= rows <= wl.B * wl.Tq
+    sec, r = bench.time_oracle(wl, cpu, rows, 1)
+    assert r == rows and sec >= 0.0
+    # 4 of toy16's 16 query rows in 2 s: a full step takes 8 s, 16 tokens / 8 s
+    assert bench._oracle_rate(wl, 2.0, 4) == pytest.approx(2.0)
+    dec = WORKLOADS["decode32k"]
+    # 8 of 32 decode rows in 1 s: a step takes 4 s
+    assert bench._oracle_rate(dec, 1.0, 8) == pytest.approx(0.25)
