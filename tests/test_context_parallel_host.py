@@ -1,5 +1,5 @@
 """The context-parallel decode step (learned_sparse_attention_dsa_b200.
-context_parallel) on two gloo ranks on CPU.
+context_parallel) on two and three gloo ranks on CPU.
 
 The per-shard steps run as CPU stand-ins built on the oracle (its indexer,
 top-k and attention rows) plus the definitions of the candidate gather, the
@@ -112,17 +112,18 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def test_context_parallel_decode_two_gloo_ranks():
+@pytest.mark.parametrize("world", [P, 3])
+def test_context_parallel_decode_gloo_ranks(world):
     ctx = mp.get_context("spawn")
     qu = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank_main, args=(r, P, port, qu)) for r in range(P)]
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, qu)) for r in range(world)]
     for p in procs:
         p.start()
     for p in procs:
         p.join(timeout=180)
         assert p.exitcode == 0
-    res = {r: (i, o) for r, i, o in (qu.get(timeout=5) for _ in range(P))}
+    res = {r: (i, o) for r, i, o in (qu.get(timeout=5) for _ in range(world))}
     # the single-context oracle
     q_idx, k_idx, w, qq, kc, vc = _inputs()
     rows = np.arange(B, dtype=np.int32)
@@ -130,12 +131,12 @@ def test_context_parallel_decode_two_gloo_ranks():
     scores = oracle.indexer_rows(q_idx[:, 0].numpy(), w[:, 0].numpy(), k_idx.numpy(), rows, t)
     ref_idx = oracle.topk_rows(scores, t, K)
     ref_out = oracle.attn_rows(qq[:, 0].numpy(), kc.numpy(), vc.numpy(), ref_idx, rows, 1.0 / D ** 0.5)
-    for r in range(P):
+    for r in range(world):
         idx, out = res[r]
         assert np.array_equal(idx[:, 0], ref_idx), f"rank {r}: selection differs"
         assert np.allclose(out[:, 0], ref_out, atol=1e-9, rtol=1e-9), f"rank {r}: output differs"
-    # both shards contributed (the test would not exercise the merge otherwise)
-    assert (ref_idx < L // P).any() and (ref_idx >= L // P).any()
+    # at least two shards contributed (the test would not exercise the merge otherwise)
+    assert len(np.unique(ref_idx[ref_idx >= 0] // (L // world))) >= 2
 
 
 def test_local_candidates_rejects_multi_row_queries():
