@@ -59,7 +59,10 @@ typedef enum {
     DSA_ERR_UNSUPPORTED = 2,  /* valid but not implemented (dtype, head width) */
     DSA_ERR_WORKSPACE = 3,    /* workspace pointer null or ws_bytes too small */
     DSA_ERR_CUDA = 4,         /* a CUDA runtime call or a kernel launch failed */
-    DSA_ERR_TIMEOUT = 5       /* a bounded device-side wait gave up (dsa_device_error) */
+    DSA_ERR_TIMEOUT = 5,      /* a bounded device-side wait gave up (dsa_device_error) */
+    DSA_ERR_BAD_INDEX = 6     /* an attention call met a selected position that is
+                                 neither -1 nor inside [0, L); it was skipped
+                                 (dsa_device_error) */
 } dsa_status;
 
 typedef enum {
@@ -89,10 +92,15 @@ const char *dsa_status_string(dsa_status status);
  * return without finishing its outputs, instead of hanging the GPU.
  *   stream  cudaStream_t (as void*) that ran the calls to check; it is
  *           synchronised first.
+ * The attention kernels also record a selected position that is neither -1
+ * nor inside the cache [0, L): they skip it like padding (no memory outside
+ * the cache is read) and the call's outputs are those of the remaining
+ * positions, but the selection it was given was malformed.
  * Returns DSA_OK if no kernel recorded an error since the last call,
- * DSA_ERR_TIMEOUT if one did (the outputs of that call are invalid), and
- * DSA_ERR_CUDA if synchronising or reading the words failed. Blocking; not
- * for use inside stream capture.
+ * DSA_ERR_TIMEOUT if a wait gave up (the outputs of that call are invalid;
+ * reported first when both happened), DSA_ERR_BAD_INDEX if an attention call
+ * skipped a malformed position, and DSA_ERR_CUDA if synchronising or reading
+ * the words failed. Blocking; not for use inside stream capture.
  */
 dsa_status dsa_device_error(dsa_stream_t stream);
 
@@ -174,7 +182,8 @@ typedef struct dsa_attn_shape {
  *
  * q   [B, Tq, Hq, Dqk] dtype dt;  out [B, Tq, Hq, Dv] dtype dt
  * idx [B, Tq, k] int32: positions in [0, L) or -1 (skipped); order is free;
- *     a position must not appear twice in one row.
+ *     a position must not appear twice in one row. Any other value is
+ *     skipped as well and reported by dsa_device_error (DSA_ERR_BAD_INDEX).
  * lse [B, Tq, Hq] fp32 or NULL: log sum_{s in S} exp(scale * q.k_s).
  * A row whose idx holds only -1 gets out = 0 and lse = -inf.
  * Logits, softmax and the weighted sum are accumulated in fp32.
@@ -185,6 +194,8 @@ dsa_status dsa_sparse_attn(const void *q, const void *k_cache, const void *v_cac
                            void *out, float *lse, void *ws, size_t ws_bytes,
                            dsa_stream_t stream);
 
+/* Workspace dsa_sparse_attn needs for this shape; 0 when the shape is
+ * invalid or unsupported (the call itself then reports why). */
 size_t dsa_sparse_attn_workspace_bytes(const dsa_attn_shape *sh, dsa_dtype dt);
 
 /*
@@ -200,7 +211,8 @@ size_t dsa_sparse_attn_workspace_bytes(const dsa_attn_shape *sh, dsa_dtype dt);
  * by every GPU that loads libdsa.so until the process exits). It calls no
  * allocator.
  *
- * - Returns DSA_ERR_WORKSPACE without launching anything when the problem
+ * - Checks its arguments as dsa_sparse_attn does (same statuses), then
+ *   returns DSA_ERR_WORKSPACE without launching anything when the problem
  *   needs more scratch than that (dsa_sparse_attn_workspace_bytes(sh, dt) >
  *   the maximum); use dsa_sparse_attn with a workspace then.
  * - The first call on each device looks up the array's device address

@@ -21,7 +21,7 @@ DSA_E4M3 = 2
 DSA_FLAG_INCLUDE_SELF = 1
 
 STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED",
-                3: "DSA_ERR_WORKSPACE", 4: "DSA_ERR_CUDA", 5: "DSA_ERR_TIMEOUT"}
+                3: "DSA_ERR_WORKSPACE", 4: "DSA_ERR_CUDA", 5: "DSA_ERR_TIMEOUT", 6: "DSA_ERR_BAD_INDEX"}
 
 # Symbols declared in include/dsa.h.
 EXPORTED = ("dsa_version", "dsa_kernel_launch_count", "dsa_status_string", "dsa_indexer_scores", "dsa_topk",
@@ -117,7 +117,9 @@ def kernel_launch_count() -> int:
 
 
 def device_error(stream=None) -> None:
-    """Synchronise `stream` and raise DSAError if a kernel gave up on a bounded wait."""
+    """Synchronise `stream` and raise DSAError if a kernel recorded an error: a
+    bounded wait that gave up (DSA_ERR_TIMEOUT) or a selected position outside
+    [0, L) other than -1 that an attention call skipped (DSA_ERR_BAD_INDEX)."""
     _check(load_library().dsa_device_error(_stream(stream)), "dsa_device_error")
 
 

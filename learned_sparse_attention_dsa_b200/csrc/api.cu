@@ -104,9 +104,10 @@ dsa_status check_topk(const float *scores, int B, int Tq, int L, int q_pos0, int
     return DSA_OK;
 }
 
-dsa_status check_attn(const void *q, const void *k_cache, const void *v_cache, const int32_t *idx,
-                      const dsa_attn_shape *sh, dsa_dtype dt, const void *out, const float *lse) {
-    if (!sh || !q || !k_cache || !v_cache || !idx || !out) return DSA_ERR_INVALID_ARG;
+// The attention shape alone (no pointers): sizes, strides, dtype, and the
+// shared-memory staging of the CUDA-core kernel that every shape falls back to.
+dsa_status check_attn_shape(const dsa_attn_shape *sh, dsa_dtype dt) {
+    if (!sh) return DSA_ERR_INVALID_ARG;
     if (sh->B < 1 || sh->Tq < 1 || sh->L < 1 || sh->k < 1) return DSA_ERR_INVALID_ARG;
     if (sh->Hq < 1 || sh->Hkv < 1 || sh->Hq % sh->Hkv != 0) return DSA_ERR_INVALID_ARG;
     if (sh->Dqk < 1 || sh->Dv < 1) return DSA_ERR_INVALID_ARG;
@@ -115,14 +116,22 @@ dsa_status check_attn(const void *q, const void *k_cache, const void *v_cache, c
         sh->k_stride_h < 0 || sh->v_stride_h < 0)
         return DSA_ERR_INVALID_ARG;
     if (!valid_dtype(dt)) return DSA_ERR_UNSUPPORTED;
-    const size_t eb = dtype_bytes(dt);
-    if (!aligned(q, eb) || !aligned(k_cache, eb) || !aligned(v_cache, eb) || !aligned(out, eb) ||
-        !aligned(idx, 4) || (lse && !aligned(lse, 4)))
-        return DSA_ERR_INVALID_ARG;
     if (sh->Dv > 512) return DSA_ERR_UNSUPPORTED;
     const int lim = smem_limit();
     if (lim == 0) return DSA_ERR_CUDA;
     if (attn_cuda_core_smem_bytes(sh->Dqk, sh->k) > (size_t)lim) return DSA_ERR_UNSUPPORTED;
+    return DSA_OK;
+}
+
+dsa_status check_attn(const void *q, const void *k_cache, const void *v_cache, const int32_t *idx,
+                      const dsa_attn_shape *sh, dsa_dtype dt, const void *out, const float *lse) {
+    if (!sh || !q || !k_cache || !v_cache || !idx || !out) return DSA_ERR_INVALID_ARG;
+    dsa_status st = check_attn_shape(sh, dt);
+    if (st != DSA_OK) return st;
+    const size_t eb = dtype_bytes(dt);
+    if (!aligned(q, eb) || !aligned(k_cache, eb) || !aligned(v_cache, eb) || !aligned(out, eb) ||
+        !aligned(idx, 4) || (lse && !aligned(lse, 4)))
+        return DSA_ERR_INVALID_ARG;
     return DSA_OK;
 }
 
@@ -195,6 +204,13 @@ dsa_status check_forward(const dsa_forward_args *a) {
 
 }  // namespace
 
+namespace dsa {
+dsa_status validate_attn_call(const void *q, const void *k_cache, const void *v_cache, const int32_t *idx,
+                              const dsa_attn_shape *sh, dsa_dtype dt, const void *out, const float *lse) {
+    return check_attn(q, k_cache, v_cache, idx, sh, dt, out, lse);
+}
+}  // namespace dsa
+
 extern "C" {
 
 int dsa_version(void) { return 100; }
@@ -204,9 +220,12 @@ uint64_t dsa_kernel_launch_count(void) { return g_launches.load(std::memory_orde
 dsa_status dsa_device_error(dsa_stream_t stream) {
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return DSA_ERR_CUDA;
     unsigned int words = dsa::indexer_take_device_error() | dsa::attn_mla_tc_take_device_error() |
-                         dsa::indexer_bwd_take_device_error();
+                         dsa::indexer_bwd_take_device_error() | dsa::attn_tc_take_device_error() |
+                         dsa::attn_mla_take_device_error() | dsa::attn_perhead_take_device_error() |
+                         dsa::attn_cc_take_device_error();
     if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
-    return words ? DSA_ERR_TIMEOUT : DSA_OK;
+    if (words & kErrTimeout) return DSA_ERR_TIMEOUT;
+    return (words & kErrBadIndex) ? DSA_ERR_BAD_INDEX : DSA_OK;
 }
 
 const char *dsa_status_string(dsa_status status) {
@@ -217,6 +236,7 @@ const char *dsa_status_string(dsa_status status) {
         case DSA_ERR_WORKSPACE: return "DSA_ERR_WORKSPACE: workspace missing or too small";
         case DSA_ERR_CUDA: return "DSA_ERR_CUDA: CUDA runtime or launch failure";
         case DSA_ERR_TIMEOUT: return "DSA_ERR_TIMEOUT: bounded device wait expired";
+        case DSA_ERR_BAD_INDEX: return "DSA_ERR_BAD_INDEX: selected position outside [0, L) skipped";
     }
     return "unknown dsa_status";
 }
@@ -254,7 +274,7 @@ dsa_status dsa_topk(const float *scores, int B, int Tq, int L, int q_pos0, int k
 }
 
 size_t dsa_sparse_attn_workspace_bytes(const dsa_attn_shape *sh, dsa_dtype dt) {
-    if (!sh) return 0;
+    if (check_attn_shape(sh, dt) != DSA_OK) return 0;
     AttnProblem p = make_attn_problem(nullptr, nullptr, nullptr, nullptr, sh, dt, nullptr, nullptr, nullptr, 0);
     return attn_workspace_bytes(p);
 }

@@ -21,6 +21,8 @@ cudaError_t launch_attn_tc(const AttnProblem &p, cudaStream_t stream, bool *take
 
 namespace {
 
+__device__ unsigned int g_attn_cc_error = 0;  // kErrBadIndex bits
+
 constexpr int kHeadsPerBlock = 4;
 constexpr int kMaxCols = 16;  // Dv <= 32 * 16 = 512
 
@@ -67,7 +69,8 @@ attn_cuda_core_kernel(AttnArgs a) {
     const T *q = static_cast<const T *>(a.q);
     for (int x = threadIdx.x; x < a.k; x += blockDim.x) {
         const int s = a.idx[(size_t)row * a.k + x];
-        idx_sm[x] = (s >= 0 && s < a.L) ? s : -1;  // positions outside [0, L) are padding
+        note_bad_index(&g_attn_cc_error, s, a.L);
+        idx_sm[x] = (s >= 0 && s < a.L) ? s : -1;  // positions outside [0, L) are skipped
     }
     for (int x = threadIdx.x; x < kHeadsPerBlock * a.Dqk; x += blockDim.x) {
         const int hh = blockIdx.y * kHeadsPerBlock + x / a.Dqk;
@@ -154,6 +157,13 @@ cudaError_t launch_cuda_core(const AttnProblem &p, cudaStream_t stream) {
 }
 
 }  // namespace
+
+unsigned int attn_cc_take_device_error() {
+    unsigned int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_attn_cc_error, sizeof(v)) != cudaSuccess) return 0;
+    cudaMemcpyToSymbol(g_attn_cc_error, &zero, sizeof(zero));
+    return v;
+}
 
 size_t attn_cuda_core_smem_bytes(int Dqk, int k) {
     return sizeof(float) * kHeadsPerBlock * Dqk + sizeof(int32_t) * k;

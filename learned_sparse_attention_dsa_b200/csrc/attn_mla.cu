@@ -32,6 +32,8 @@ cudaError_t launch_attn_combine(const float *part_o, const float *part_ml, int n
 
 namespace {
 
+__device__ unsigned int g_attn_mla_error = 0;  // kErrBadIndex bits
+
 constexpr int DQK = 576;
 constexpr int DV = 512;
 constexpr int kRows = 64;                 // selected rows per stage
@@ -121,6 +123,7 @@ attn_mla_kernel(const Args a) {
         for (int c0 = j0; c0 < j1; c0 += kThreads) {
             const int j = c0 + threadIdx.x;
             const int s = j < j1 ? a.idx[(size_t)row * a.k + j] : -1;
+            note_bad_index(&g_attn_mla_error, s, a.L);
             const bool valid = s >= 0 && s < a.L;
             const unsigned m = __ballot_sync(0xffffffffu, valid);
             if (lane == 0) warp_cnt[warp] = __popc(m);
@@ -329,6 +332,13 @@ int mla_splits(const AttnProblem &p, int sm_count) {
 }
 
 }  // namespace
+
+unsigned int attn_mla_take_device_error() {
+    unsigned int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_attn_mla_error, sizeof(v)) != cudaSuccess) return 0;
+    cudaMemcpyToSymbol(g_attn_mla_error, &zero, sizeof(zero));
+    return v;
+}
 
 bool attn_mla_supported(const AttnProblem &p) {
     if (p.dt != DSA_BF16 || p.Dqk != DQK || p.Dv != DV) return false;

@@ -110,7 +110,7 @@ __host__ __device__ constexpr int q_box0(int p) { return p == 0 ? 0 : 5; }
 __host__ __device__ constexpr int q_boxes(int p) { return p == 0 ? 5 : 4; }
 __host__ __device__ constexpr int g_box0(int p) { return 4 * p; }
 
-__device__ unsigned int g_attn_mla_tc_error = 0;  // 1 = a bounded wait gave up
+__device__ unsigned int g_attn_mla_tc_error = 0;  // kErrTimeout, kErrBadIndex bits
 
 struct Args {
     const __nv_bfloat16 *kv;  // latent rows: element strides sb (batch), ss (position)
@@ -199,6 +199,7 @@ attn_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Args a) {
         int s = -1;
         if (j < n_split) {
             s = a.idx[(size_t)row * a.k + j0 + j];
+            note_bad_index(&g_attn_mla_tc_error, s, a.L);
             if (s < 0 || s >= a.L) s = -1;
         }
         sel[j] = s;
@@ -530,7 +531,7 @@ attn_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Args a) {
         }
     }
 
-    if (!ok) atomicOr(&g_attn_mla_tc_error, 1u);
+    if (!ok) atomicOr(&g_attn_mla_tc_error, kErrTimeout);
     tc_fence_before();
     cg::this_cluster().sync();  // no part leaves while the other may still write to it
     if (warp == kMmaWarp) {

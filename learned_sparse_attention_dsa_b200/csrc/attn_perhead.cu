@@ -28,6 +28,8 @@
 namespace dsa {
 namespace {
 
+__device__ unsigned int g_attn_perhead_error = 0;  // kErrBadIndex bits
+
 constexpr int kRows = 16;  // selected positions per stage
 constexpr int kMaxHeads = 16;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -101,6 +103,7 @@ attn_perhead_kernel(const Args a) {
         for (int c0 = 0; c0 < a.k; c0 += nthreads) {
             const int j = c0 + threadIdx.x;
             const int s = j < a.k ? a.idx[(size_t)row * a.k + j] : -1;
+            note_bad_index(&g_attn_perhead_error, s, a.L);
             const bool valid = s >= 0 && s < a.L;
             const unsigned m = __ballot_sync(0xffffffffu, valid);
             if (lane == 0) warp_cnt[warp] = __popc(m);
@@ -266,6 +269,13 @@ attn_perhead_kernel(const Args a) {
 }
 
 }  // namespace
+
+unsigned int attn_perhead_take_device_error() {
+    unsigned int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_attn_perhead_error, sizeof(v)) != cudaSuccess) return 0;
+    cudaMemcpyToSymbol(g_attn_perhead_error, &zero, sizeof(zero));
+    return v;
+}
 
 cudaError_t launch_attn_perhead(const AttnProblem &p, cudaStream_t stream, bool *taken) {
     *taken = false;

@@ -35,6 +35,8 @@ cudaError_t launch_attn_cuda_core(const AttnProblem &p, cudaStream_t stream);
 
 namespace {
 
+__device__ unsigned int g_attn_tc_error = 0;  // kErrBadIndex bits
+
 constexpr int kRowsPerTile = 64;
 constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
@@ -168,6 +170,7 @@ attn_mma_kernel(const Args a) {
         for (int it = 0; it < kIters; ++it) {
             if (j0 + it * kThreads >= j1) break;  // uniform
             const int s = sv[it];
+            note_bad_index(&g_attn_tc_error, s, a.L);
             const bool valid = s >= 0 && s < a.L;
             const unsigned m = __ballot_sync(0xffffffffu, valid);
             if (lane == 0) warp_base[warp] = __popc(m);
@@ -621,6 +624,13 @@ cudaError_t launch_mma(const AttnProblem &p, const DeviceInfo &info, cudaStream_
 }
 
 }  // namespace
+
+unsigned int attn_tc_take_device_error() {
+    unsigned int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_attn_tc_error, sizeof(v)) != cudaSuccess) return 0;
+    cudaMemcpyToSymbol(g_attn_tc_error, &zero, sizeof(zero));
+    return v;
+}
 
 bool attn_mla_supported(const AttnProblem &p);
 size_t attn_mla_workspace_bytes(const AttnProblem &p, int sm_count);

@@ -79,6 +79,19 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
+// ---------------------------------------------------------------- error words
+//
+// Each kernel family keeps a device-side error word (a __device__ variable of
+// its translation unit) that dsa_device_error reads and clears. Bits:
+constexpr unsigned int kErrTimeout = 1u;   // a bounded wait gave up: the launch's outputs are invalid
+constexpr unsigned int kErrBadIndex = 2u;  // a selected position outside [0, L) other than -1 was skipped
+
+// Attention kernels: a selected position s that is neither -1 (padding) nor
+// inside the cache [0, L) is skipped like padding and reported here.
+__device__ __forceinline__ void note_bad_index(unsigned int *word, int s, int L) {
+    if (s < -1 || s >= L) atomicOr(word, kErrBadIndex);
+}
+
 __host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 __host__ __device__ __forceinline__ size_t align_up(size_t a, size_t b) { return (a + b - 1) / b * b; }
 

@@ -534,7 +534,7 @@ indexer_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         }
     }
 
-    if (!ok) atomicOr(&g_indexer_bwd_error, 1u);
+    if (!ok) atomicOr(&g_indexer_bwd_error, kErrTimeout);
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {

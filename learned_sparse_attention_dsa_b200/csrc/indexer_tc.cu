@@ -305,7 +305,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
     }
 
-    if (!ok) atomicOr(&g_indexer_error, 1u);
+    if (!ok) atomicOr(&g_indexer_error, kErrTimeout);
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {

@@ -81,6 +81,10 @@ struct AttnProblem {
 size_t attn_workspace_bytes(const AttnProblem &p);
 cudaError_t launch_attn(const AttnProblem &p, cudaStream_t stream);
 
+// The argument checks of dsa_sparse_attn (everything but the workspace).
+dsa_status validate_attn_call(const void *q, const void *k_cache, const void *v_cache, const int32_t *idx,
+                              const dsa_attn_shape *sh, dsa_dtype dt, const void *out, const float *lse);
+
 // ----------------------------------------------------------------- indexer loss
 struct KlProblem {
     const float *scores;    // [B, Tq, L]
@@ -122,10 +126,15 @@ cudaError_t launch_localize(const int32_t *idx, long long n, int key_pos0, int L
 cudaError_t launch_combine_parts(const void *parts, const float *parts_lse, int P, long long pairs, int Dv,
                                  dsa_dtype dt, void *out, float *lse, cudaStream_t stream);
 
-// Read and clear the error word of a kernel family with bounded waits
-// (non-zero: some launch gave up on a wait).
+// Read and clear the error word of a kernel family (kErrTimeout: some launch
+// gave up on a bounded wait; kErrBadIndex: an attention launch skipped a
+// selected position outside [0, L) other than -1).
 unsigned int indexer_take_device_error();
 unsigned int attn_mla_tc_take_device_error();
 unsigned int indexer_bwd_take_device_error();
+unsigned int attn_tc_take_device_error();
+unsigned int attn_mla_take_device_error();
+unsigned int attn_perhead_take_device_error();
+unsigned int attn_cc_take_device_error();
 
 }  // namespace dsa

@@ -61,7 +61,10 @@ size_t dsa_sparse_attn_noalloc_max_scratch_bytes(void) { return dsa::kScratchByt
 dsa_status dsa_sparse_attn_noalloc(const void *q, const void *k_cache, const void *v_cache, const int32_t *idx,
                                    const dsa_attn_shape *sh, dsa_dtype dt, void *out, float *lse,
                                    dsa_stream_t stream) {
-    // Same argument checks as dsa_sparse_attn (no workspace arguments).
+    // The argument checks of dsa_sparse_attn come first, so that a malformed
+    // or unsupported shape gets its own status, never DSA_ERR_WORKSPACE.
+    const dsa_status st = dsa::validate_attn_call(q, k_cache, v_cache, idx, sh, dt, out, lse);
+    if (st != DSA_OK) return st;
     const size_t need = dsa_sparse_attn_workspace_bytes(sh, dt);
     if (need > dsa::kScratchBytes) return DSA_ERR_WORKSPACE;  // needs more than the built-in scratch
     void *scratch = nullptr;

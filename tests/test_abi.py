@@ -35,8 +35,9 @@ def test_library_exports_every_declared_symbol(dsa_lib):
 
 def test_version_and_status_strings(dsa_lib):
     assert dsa_lib.dsa_version() >= 100
-    for code in range(6):
+    for code in range(7):
         assert dsa_lib.dsa_status_string(code)
+    assert b"DSA_ERR_BAD_INDEX" in dsa_lib.dsa_status_string(6)
     assert b"unknown" in dsa_lib.dsa_status_string(99)
 
 
@@ -72,6 +73,21 @@ def test_attention_shape_checks(dsa_lib):
     assert dsa_lib.dsa_sparse_attn(fake, fake, fake, fake, ctypes.byref(sh), 1, fake, None, None, 0, None) == 1
     sh = AttnShape(1, 1, 8, 4, 8, 4, 64, 64, 0.1, 512, 0, 64, 512, 64, 64)  # zero row stride
     assert dsa_lib.dsa_sparse_attn(fake, fake, fake, fake, ctypes.byref(sh), 1, fake, None, None, 0, None) == 1
+
+
+def test_workspace_size_of_an_invalid_attention_shape_is_zero(dsa_lib):
+    """Invalid shapes are rejected before any size arithmetic (a zero KV head
+    count would otherwise divide by zero on the host); the no-workspace entry
+    point returns the argument status, not DSA_ERR_WORKSPACE."""
+    from learned_sparse_attention_dsa_b200.binding import AttnShape
+    dsa_lib.dsa_sparse_attn_workspace_bytes.restype = ctypes.c_size_t
+    fake = ctypes.c_void_p(0x1000)  # never dereferenced: the checks fail first
+    for fields in ((16, 1, 128, 0), (-2, 1, 128, 1), (1, -1, 128, 1), (1, 1, 0, 1)):
+        B, Tq, Hq, Hkv = fields
+        sh = AttnShape(B, Tq, 64, 8, Hq, Hkv, 128, 128, 0.1, 8192, 128, 128, 8192, 128, 128)
+        assert dsa_lib.dsa_sparse_attn_workspace_bytes(ctypes.byref(sh), 1) == 0, fields
+        assert dsa_lib.dsa_sparse_attn_noalloc(fake, fake, fake, fake, ctypes.byref(sh), 1, fake, None,
+                                               None) == 1, fields
 
 
 def test_binding_fails_loudly_without_library(tmp_path):

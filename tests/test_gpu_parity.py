@@ -56,15 +56,18 @@ MEDIUM = {
                                 Hq=16, Hkv=1, Dqk=128, Dv=128, seed=24),
     "heads128_decode": Workload("heads128_decode", B=3, Tq=1, L=3000, q_pos0=2999, H_I=128, d_I=128, k=256,
                                 Hq=16, Hkv=1, Dqk=128, Dv=128, seed=25),
+    # 32 query heads over one latent row: the CUDA-core latent-row kernel
+    "latent_h32": Workload("latent_h32", B=2, Tq=1, L=3000, q_pos0=2999, H_I=64, d_I=128, k=256,
+                           Hq=32, Hkv=1, Dqk=576, Dv=512, kv_alias=True, seed=26),
 }
 
-FULL_ROWS = {
-    "toy16": None,  # every row
-    "decode32k": [0, 13, 31],
+FULL_ROWS = {  # None: every query row
+    "toy16": None,
+    "decode32k": None,
     "prefill8k": [0, 1, 2046, 2047, 2048, 5000, 8191],
     "prefill32k": [0, 2047, 2048, 20000, 32767],
-    "decode128k": [0, 5],
-    "decode32k_fp8": [0, 13, 31],
+    "decode128k": None,
+    "decode32k_fp8": None,
 }
 
 _cache = {}
@@ -151,7 +154,10 @@ def test_indexer_stage_all_rows(cuda, name):
                                            (20003, 200, 19803, 2048), (49152, 150, 49002, 1000),
                                            # fewer rows than SMs: clusters of 8, 4 and 2 CTAs per row
                                            (20000, 20, 19980, 2048), (6000, 40, 5960, 2048),
-                                           (9000, 80, 8920, 1000)])
+                                           (9000, 80, 8920, 1000),
+                                           # at least as many rows as SMs, rows longer than 49,152
+                                           # scores: the cluster kernel with one CTA per row
+                                           (60000, 160, 59840, 2048), (70000, 150, 69850, 1000)])
 def test_topk_stage(cuda, kind, L, Tq, q_pos0, k):
     gen = torch.Generator().manual_seed(L + Tq + k)
     scores = random_score_rows(gen, Tq, L, kind)[None]            # [1, Tq, L]
@@ -162,7 +168,7 @@ def test_topk_stage(cuda, kind, L, Tq, q_pos0, k):
 
 
 @pytest.mark.parametrize("name", ["prefill_mqa_700", "decode_latent_3000", "latent_chunk",
-                                  "latent_single", "prefill_perhead_520", "tiny_f32"])
+                                  "latent_single", "latent_h32", "prefill_perhead_520", "tiny_f32"])
 def test_sparse_attn_stage_shuffled_and_padded(cuda, name):
     """Attention on its own, with the oracle's index sets shuffled and padded."""
     wl = MEDIUM[name]
@@ -199,6 +205,41 @@ def test_sparse_attn_all_padding_row(cuda):
     assert torch.equal(out[:, 1], v0[:, g])
 
 
+@pytest.mark.parametrize("name", ["decode_5000", "decode_latent_3000", "latent_h32", "prefill_perhead_520",
+                                  "odd_heads", "tiny_f32"])
+def test_sparse_attn_reports_malformed_positions(cuda, name):
+    """Positions that are neither -1 nor inside [0, L) are skipped like -1
+    (no access outside the cache) and reported as DSA_ERR_BAD_INDEX by
+    dsa_device_error, which then clears the report. Each case reaches one
+    attention kernel: 16 heads per KV head, 128 and 32 heads over a latent
+    row, one KV head per query head, and the CUDA-core kernel."""
+    wl = MEDIUM[name]
+    _, dev = _inputs(wl)
+    gen = torch.Generator().manual_seed(7)
+    rows = wl.B * wl.Tq
+    k = min(wl.k, wl.L)
+    clean = torch.stack([torch.randperm(wl.L, generator=gen)[:k] for _ in range(rows)]).to(torch.int32)
+    bad = clean.clone()
+    bad[:, 1] = wl.L             # one past the cache
+    bad[:, k // 2] = -7          # negative, not the padding value
+    bad[:, k - 1] = wl.L + 4096  # far past the cache
+    clean[:, [1, k // 2, k - 1]] = -1
+    clean = clean.reshape(wl.B, wl.Tq, k).cuda()
+    bad = bad.reshape(wl.B, wl.Tq, k).cuda()
+    binding.device_error()  # nothing pending from earlier tests
+    out_clean, lse_clean = binding.sparse_attn(dev["q"], dev["k_cache"], dev["v_cache"], clean, wl.scale,
+                                               want_lse=True)
+    binding.device_error()
+    out_bad, lse_bad = binding.sparse_attn(dev["q"], dev["k_cache"], dev["v_cache"], bad, wl.scale,
+                                           want_lse=True)
+    with pytest.raises(binding.DSAError) as exc:
+        binding.device_error()
+    assert exc.value.status == 6  # DSA_ERR_BAD_INDEX
+    binding.device_error()        # cleared by the previous call
+    assert torch.equal(out_bad, out_clean)
+    assert torch.equal(lse_bad, lse_clean)
+
+
 def test_forward_equals_stage_calls(cuda):
     wl = MEDIUM["prefill_mqa_700"]
     _, dev = _inputs(wl)
@@ -226,7 +267,8 @@ def test_invalid_arguments_enqueue_nothing(cuda):
 @pytest.mark.parametrize("kind", ["int", "normal", "mixed"])
 @pytest.mark.parametrize("L,Tq,q_pos0,k", [(37, 37, 0, 5), (5000, 3, 4997, 2048), (3000, 2, 2998, 1),
                                            (140000, 1, 139999, 2048), (2100, 2100, 0, 2048),
-                                           (20003, 200, 19803, 2048), (6000, 40, 5960, 2048)])
+                                           (20003, 200, 19803, 2048), (6000, 40, 5960, 2048),
+                                           (60000, 160, 59840, 2048)])
 def test_topk_stage_include_self(cuda, kind, L, Tq, q_pos0, k):
     gen = torch.Generator().manual_seed(L + Tq + k + 1)
     scores = random_score_rows(gen, Tq, L, kind)[None]

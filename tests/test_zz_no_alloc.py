@@ -18,6 +18,7 @@ from parity_helpers import ATOL, RTOL
 
 pytestmark = pytest.mark.gpu
 
+DSA_ERR_INVALID_ARG = 1
 DSA_ERR_WORKSPACE = 3
 
 
@@ -71,16 +72,37 @@ def test_noalloc_matches_workspace_entry_point_twice(cuda, dsa_lib):
 
 def test_noalloc_rejects_problems_beyond_its_scratch(cuda, dsa_lib):
     _declare(dsa_lib)
-    # 16 sequences x 16 heads selecting 65,536 positions: the selection is
-    # split 32 ways, 16*16*32*(128+2)*4 bytes of partials > 4 MiB
-    B, L, k, Hq, D = 16, 65536, 65536, 16, 128
+    # One sequence decoding with 128 heads over a latent row, 2048 positions
+    # selected: the selection is split 32 ways, 128*32*(512+2)*4 bytes of
+    # partials (8.4 MB) > 4 MiB. dsa_sparse_attn runs this shape with a
+    # workspace; the no-workspace entry point must refuse it.
+    B, L, k, Hq, D, Dv = 1, 3000, 2048, 128, 576, 512
     q = torch.zeros((B, 1, Hq, D), dtype=torch.bfloat16, device="cuda")
     kc = torch.zeros((B, L, 1, D), dtype=torch.bfloat16, device="cuda")
-    vc = torch.zeros((B, L, 1, D), dtype=torch.bfloat16, device="cuda")
-    idx = torch.zeros((B, 1, k), dtype=torch.int32, device="cuda")
-    out = torch.empty((B, 1, Hq, D), dtype=torch.bfloat16, device="cuda")
+    vc = kc[..., :Dv]
+    gen = torch.Generator().manual_seed(3)
+    idx = torch.randperm(L, generator=gen)[:k].to(torch.int32).reshape(B, 1, k).cuda()
+    out = torch.empty((B, 1, Hq, Dv), dtype=torch.bfloat16, device="cuda")
     lse = torch.empty((B, 1, Hq), dtype=torch.float32, device="cuda")
     sh = binding.attn_shape(q, kc, vc, k, D ** -0.5)
     need = dsa_lib.dsa_sparse_attn_workspace_bytes(ctypes.byref(sh), binding._dt(q))
     assert need > dsa_lib.dsa_sparse_attn_noalloc_max_scratch_bytes()
+    binding.sparse_attn(q, kc, vc, idx, D ** -0.5, out=out)  # accepted with a workspace
+    torch.cuda.synchronize()
     assert _noalloc(dsa_lib, q, kc, vc, idx, sh, out, lse) == DSA_ERR_WORKSPACE
+
+
+def test_noalloc_checks_arguments_before_the_scratch_size(cuda, dsa_lib):
+    """A malformed shape gets the argument status, not DSA_ERR_WORKSPACE (and
+    no division by a zero head count on the host)."""
+    _declare(dsa_lib)
+    q = torch.zeros((1, 1, 16, 128), dtype=torch.bfloat16, device="cuda")
+    kc = torch.zeros((1, 64, 1, 128), dtype=torch.bfloat16, device="cuda")
+    idx = torch.zeros((1, 1, 8), dtype=torch.int32, device="cuda")
+    out = torch.empty((1, 1, 16, 128), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((1, 1, 16), dtype=torch.float32, device="cuda")
+    for field, value in (("Hkv", 0), ("B", -3), ("Tq", -1), ("k", 0)):
+        sh = binding.attn_shape(q, kc, kc, 8, 128 ** -0.5)
+        setattr(sh, field, value)
+        assert dsa_lib.dsa_sparse_attn_workspace_bytes(ctypes.byref(sh), binding._dt(q)) == 0
+        assert _noalloc(dsa_lib, q, kc, kc, idx, sh, out, lse) == DSA_ERR_INVALID_ARG, field
