@@ -38,11 +38,32 @@ from learned_sparse_attention_dsa_b200.inputs import WORKLOADS, make_inputs, to_
 METRIC = "prefill tokens/s and decode steps/s at k=2048; % HBM/tensor roofline per stage"
 
 # dram__bytes_read.sum + dram__bytes_write.sum per launch of a stage's kernel,
-# from one ncu capture of the current kernel (profiles/ holds each capture's
-# summary and command). An entry is removed when its kernel changes.
-DRAM_TRAFFIC_PER_LAUNCH = {
-    ("decode32k", "indexer"): 274.8e6,
-}
+# from an ncu capture (the profiles/ summary named here holds its command and
+# figures), with the SHA-256 prefix of the kernel sources it was taken on.
+# dram_traffic() reports an entry only while those sources are unchanged, so
+# a kernel edit turns its traffic into null until it is captured again.
+DRAM_TRAFFIC_PER_LAUNCH = {}
+
+
+def _sources_digest(files):
+    import hashlib
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "learned_sparse_attention_dsa_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def dram_traffic(workload, stage):
+    e = DRAM_TRAFFIC_PER_LAUNCH.get((workload, stage))
+    if e is None:
+        return None
+    try:
+        if _sources_digest(e["sources"]) != e["digest"]:
+            return None
+    except OSError:
+        return None
+    return e["bytes"]
 
 
 # ------------------------------------------------------------------ helpers
@@ -183,17 +204,35 @@ def _units(wl, steps: int) -> tuple[float, str]:
 
 # ------------------------------------------------------------------ oracle timing
 
-def time_oracle(wl, cpu, n_rows: int, nthreads: int = 0):
-    """Run the CPU oracle on the first n_rows query rows (flat order, evenly
-    spread over the batch) and return (seconds, rows)."""
+def sample_rows(wl, n_rows: int, tail: int = 0) -> np.ndarray:
+    """Flat query-row ids of an oracle sample: n_rows - tail rows spread
+    evenly over the batch, plus the last `tail` rows (the longest prefill
+    rows), without repeats."""
+    total = wl.B * wl.Tq
+    n_rows = min(n_rows, total)
+    tail = min(tail, n_rows)
+    spread = np.linspace(0, total - 1 - tail, num=n_rows - tail).round().astype(np.int64) if n_rows > tail \
+        else np.zeros(0, dtype=np.int64)
+    last = np.arange(total - tail, total, dtype=np.int64)
+    return np.unique(np.concatenate([spread, last]))
+
+
+def sample_pairs(wl, flat) -> int:
+    """Causal (query, key) pairs of the sampled rows: sum of t + 1."""
+    flat = np.asarray(flat, dtype=np.int64)
+    return int(((flat % wl.Tq) + wl.q_pos0 + 1).sum())
+
+
+def time_oracle(wl, cpu, n_rows: int, nthreads: int = 0, tail: int = 0):
+    """Run the CPU oracle (all three stages) on a sample of n_rows query rows
+    (sample_rows) and return (seconds, rows, causal pairs of those rows)."""
     import oracle
 
     def bits(t):
         t = t.contiguous()
         return t.view(torch.int16).numpy().view(np.uint16) if t.dtype == torch.bfloat16 else t.numpy()
 
-    total = wl.B * wl.Tq
-    flat = np.linspace(0, total - 1, num=min(n_rows, total)).round().astype(np.int64)
+    flat = sample_rows(wl, n_rows, tail)
     row_b = (flat // wl.Tq).astype(np.int32)
     row_i = (flat % wl.Tq).astype(np.int32)
     row_t = row_i + wl.q_pos0
@@ -215,13 +254,15 @@ def time_oracle(wl, cpu, n_rows: int, nthreads: int = 0):
     idx = oracle.topk_rows(scores, row_t, wl.k, nthreads)
     oracle.attn_rows(q, kbuf, vbuf, idx, row_b, wl.scale, k_strides=ks, v_strides=vs, Hkv=wl.Hkv,
                      Dv=wl.Dv, nthreads=nthreads)
-    return time.perf_counter() - t0, len(flat)
+    return time.perf_counter() - t0, len(flat), sample_pairs(wl, flat)
 
 
-def _oracle_rate(wl, seconds: float, rows: int) -> float:
-    """Metric value of the oracle: decode steps/s or prefill tokens/s."""
-    total = wl.B * wl.Tq
-    step_seconds = seconds * total / rows
+def _oracle_rate(wl, seconds: float, pairs: int) -> float:
+    """Metric value of the oracle (decode steps/s or prefill tokens/s) from
+    `seconds` spent on rows holding `pairs` causal pairs: the whole step is
+    extrapolated by the exact pair count (every decode row has the same
+    count; in prefill the indexer's work per row grows with t)."""
+    step_seconds = seconds * wl.causal_pairs() / pairs
     if wl.is_decode:
         return 1.0 / step_seconds
     return wl.B * wl.Tq / step_seconds
@@ -230,7 +271,7 @@ def _oracle_rate(wl, seconds: float, rows: int) -> float:
 def _sample_rows_for(wl, budget_s: float, nthreads: int, cpu) -> int:
     """Rows of the oracle that fit a wall-clock budget (probe with a few rows)."""
     probe = max(1, min(wl.B * wl.Tq, max(8, nthreads)))
-    sec, rows = time_oracle(wl, cpu, probe, nthreads)
+    sec, rows, _ = time_oracle(wl, cpu, probe, nthreads)
     per_row = sec / rows
     return int(max(1, min(wl.B * wl.Tq, budget_s / per_row)))
 
@@ -252,16 +293,17 @@ def run_reference(args, wl):
         time_oracle(wl, cpu, rows, nthreads)
     secs = []
     for _ in range(args.steps):
-        s, r = time_oracle(wl, cpu, rows, nthreads)
+        s, r, pairs = time_oracle(wl, cpu, rows, nthreads)
         secs.append(s)
     mean_s = sum(secs) / len(secs)
-    value = _oracle_rate(wl, mean_s, rows)
+    value = _oracle_rate(wl, mean_s, pairs)
     _, unit = _units(wl, 1)
-    sample = f"{rows} of {wl.B * wl.Tq} query rows per step (all three stages), scaled to a full step"
+    sample = (f"{rows} of {wl.B * wl.Tq} query rows per step (all three stages), extrapolated to a full "
+              f"step by the exact causal-pair count")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": 0,
         "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": 1000.0 * mean_s * (wl.B * wl.Tq) / rows,
+        "ms_per_step": 1000.0 * mean_s * wl.causal_pairs() / pairs,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": _config(wl, world),
         "cpu_baseline": {"value": value, "unit": unit, "cores": nthreads, "kind": "oracle",
@@ -283,20 +325,83 @@ def _config(wl, world):
 
 # ------------------------------------------------------------------ our arm
 
-def run_ours(args, wl):
-    from learned_sparse_attention_dsa_b200 import binding
+# The other configurations measured by the default run, each reported under
+# "workloads" in the same JSON line (the headline workload is decode32k).
+EXTRA_WORKLOADS = ("toy16", "prefill8k", "prefill32k", "decode128k")
+# Minimum length of the window of identical back-to-back steps over which
+# clocks are sampled (the steps queued right before the timed ones, then the
+# timed ones).
+CLOCK_WINDOW_S = 0.5
 
-    world, rank, local = _dist()
-    if world > 1:
-        import datetime
 
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    device = torch.device("cuda", local)
-    torch.cuda.set_device(device)
-    binding.load_library()
+def _stage_report(wl, stages, peaks):
+    work = stage_work(wl)
+    report = {}
+    for name, ms in stages.items():
+        nbytes, flops = work[name]
+        sec_s = ms / 1000.0
+        gbs = nbytes / sec_s / 1e9
+        entry = {"ms": ms, "GB/s": gbs, "hbm_frac": gbs / peaks["hbm_gbs"],
+                 "algorithmic_bytes": nbytes, "algorithmic_flops": flops}
+        if flops:
+            entry["TFLOP/s"] = flops / sec_s / 1e12
+            entry["tensor_frac"] = entry["TFLOP/s"] / _tensor_peak(wl, name, peaks)
+        report[name] = entry
+    return report
 
+
+def _roofline(wl, stage_report, peaks):
+    """The dominant stage against its bound: tensor for the prefill indexer,
+    HBM for every other stage."""
+    dominant = max(stage_report, key=lambda n: stage_report[n]["ms"])
+    d = stage_report[dominant]
+    traffic = dram_traffic(wl.name, dominant)
+    if dominant == "indexer" and not wl.is_decode:
+        tpeak = _tensor_peak(wl, dominant, peaks)
+        return {"bound": "tensor", "kernel": dominant, "achieved": d["TFLOP/s"], "peak": tpeak,
+                "unit": "TFLOP/s", "frac": d["TFLOP/s"] / tpeak, "traffic": traffic,
+                "peak_source": peaks["source"] + ("" if tpeak == peaks["bf16_tflops"] else
+                                                  " bf16 x 2 (nominal fp8 / bf16 dense ratio)")}
+    return {"bound": "hbm", "kernel": dominant, "achieved": d["GB/s"], "peak": peaks["hbm_gbs"],
+            "unit": "GB/s", "frac": d["GB/s"] / peaks["hbm_gbs"], "traffic": traffic,
+            "peak_source": peaks["source"]}
+
+
+def _timed_steps(run, steps, stream, device, world, local, step_s_estimate):
+    """Exactly `steps` calls of run() between two CUDA events on the launching
+    stream, barrier and synchronize on both sides, max over ranks. Identical
+    steps are queued right before the first event so that the clock sampler
+    sees at least CLOCK_WINDOW_S of this load; they are not timed.
+    Returns (seconds, clocks)."""
+    pre = int(min(100000, max(0, (CLOCK_WINDOW_S - steps * step_s_estimate) / max(step_s_estimate, 1e-7))))
+    sampler = ClockSampler(local)
+    sampler.start()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    _barrier(world)
+    torch.cuda.synchronize(device)
+    h0 = time.perf_counter()
+    for _ in range(pre):
+        run()
+    ev0.record(stream)
+    for _ in range(steps):
+        run()
+    ev1.record(stream)
+    torch.cuda.synchronize(device)
+    h1 = time.perf_counter()
+    _barrier(world)
+    sampler.stop()
+    sec = _max_over_ranks(ev0.elapsed_time(ev1) / 1000.0, world, device)
+    clocks = sampler.summary(h0, h1)
+    clocks["window"] = (f"{pre} identical steps queued before the {steps} timed ones, then the timed ones "
+                        f"({h1 - h0:.2f} s)")
+    return sec, clocks
+
+
+def measure_forward(wl, args, binding, device, world, rank, local, peaks):
+    """Device throughput of dsa_forward on one workload: CUDA-graph replays of
+    one forward per step, plus per-stage times and their roofline fractions.
+    Returns (report, context) where context holds what the e2e and CPU legs
+    reuse."""
     cpu = make_inputs(wl, seed=wl.seed + rank)
     dev = to_device(cpu, device)
     out = torch.empty((wl.B, wl.Tq, wl.Hq, wl.Dv), dtype=dev["q"].dtype, device=device)
@@ -320,116 +425,138 @@ def run_ours(args, wl):
     # as `eager` for comparison.
     graph, launches_per_step = _capture(step, binding, device)
     run = graph.replay if graph is not None else step
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
     for _ in range(args.warmup):
         run()
+    e1.record(stream)
     torch.cuda.synchronize(device)
+    est = e0.elapsed_time(e1) / 1000.0 / max(1, args.warmup)
 
-    sampler = ClockSampler(local)
-    sampler.start()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    _barrier(world)
-    torch.cuda.synchronize(device)
     launches0 = binding.kernel_launch_count()
-    h0 = time.perf_counter()
-    ev0.record(stream)
-    for _ in range(args.steps):
-        run()
-    ev1.record(stream)
-    torch.cuda.synchronize(device)
-    h1 = time.perf_counter()
+    sec_max, clocks = _timed_steps(run, args.steps, stream, device, world, local, est)
     launches = (launches_per_step * args.steps if graph is not None
                 else binding.kernel_launch_count() - launches0)
-    _barrier(world)
-    sampler.stop()
-    sec = ev0.elapsed_time(ev1) / 1000.0
-    sec_max = _max_over_ranks(sec, world, device)
     units, unit = _units(wl, args.steps)
     value = units * world / sec_max
-    clocks = sampler.summary(h0, h1)
 
     # eager: the same K steps as direct C-ABI calls from Python
     _barrier(world)
     torch.cuda.synchronize(device)
-    ev0.record(stream)
+    e0.record(stream)
     for _ in range(args.steps):
         step()
-    ev1.record(stream)
+    e1.record(stream)
     torch.cuda.synchronize(device)
-    eager_sec = _max_over_ranks(ev0.elapsed_time(ev1) / 1000.0, world, device)
-    eager = {"value": units * world / eager_sec, "unit": unit,
-             "ms_per_step": 1000.0 * eager_sec / args.steps,
+    eager_sec = _max_over_ranks(e0.elapsed_time(e1) / 1000.0, world, device)
+    eager = {"value": units * world / eager_sec, "unit": unit, "ms_per_step": 1000.0 * eager_sec / args.steps,
              "note": "one dsa_forward call per step from Python, no graph"}
 
-    # ---- per-stage timing (same stream, separate loops) for the roofline
+    # per-stage timing (same stream, separate loops) for the roofline
     stages = stage_timings(wl, dev, binding, stream, max(3, min(args.steps, 50)))
+    stage_report = _stage_report(wl, stages, peaks)
+    report = {"metric": METRIC, "value": value, "unit": unit, "ms_per_step": 1000.0 * sec_max / args.steps,
+              "steps": args.steps, "warmup": args.warmup, "config": _config(wl, world),
+              "roofline": _roofline(wl, stage_report, peaks), "stages": stage_report,
+              "gpu_launches": int(launches), "clocks": clocks, "eager": eager,
+              "timing": "CUDA-graph replay of one dsa_forward per step" if graph is not None
+              else "eager dsa_forward calls"}
+    if not wl.is_decode and stage_report["attn"]["algorithmic_bytes"] > 126e6:
+        report["stages"]["attn"]["note"] = (
+            "the gathered rows (algorithmic bytes) are mostly served by L2: the KV cache is smaller than "
+            "L2 and every row is selected by many queries; hbm_frac compares them with the HBM copy rate")
+    return report, {"cpu": cpu, "stream": stream}
+
+
+def cpu_baseline_for(wl, cpu, budget_s, repeat: bool):
+    """The oracle (all three stages) on a bounded sample of the workload's
+    query rows on every host core, sized to about budget_s seconds and
+    extrapolated to a whole step by the exact causal-pair count; for prefill
+    half of the sample is the longest (last) rows, the other half spread
+    evenly over the rest (at most 512 rows)."""
+    import oracle
+    oracle.build()
+    nthreads = oracle.max_threads()
+    _, unit = _units(wl, 1)
+    prefill = wl.Tq >= 1024
+    # the probe's rows are spread evenly (average cost); a sample that is half
+    # last rows costs about 1.5 times as much per row in prefill
+    rows = _sample_rows_for(wl, budget_s / (1.5 if prefill else 1.0), nthreads, cpu)
+    if prefill:
+        rows = max(16, min(512, rows))
+    tail = rows // 2 if prefill else 0
+    total_s, total_pairs, total_rows, reps = 0.0, 0, 0, 0
+    while reps == 0 or (repeat and total_s < 0.66 * budget_s and reps < 50):
+        secs, r, pairs = time_oracle(wl, cpu, rows, nthreads, tail=tail)
+        total_s += secs
+        total_pairs += pairs
+        total_rows += r
+        reps += 1
+    sample = (f"{r} of {wl.B * wl.Tq} query rows"
+              + (f" (the last {tail} and {r - tail} spread evenly)" if tail else "")
+              + f", all three stages, {reps} repetition(s), {total_s:.1f} s in total, "
+              + "extrapolated to a full step by the exact causal-pair count")
+    return {"value": _oracle_rate(wl, total_s, total_pairs), "unit": unit, "cores": nthreads, "kind": "oracle",
+            "sample": sample}
+
+
+def run_ours(args, wl):
+    from learned_sparse_attention_dsa_b200 import binding
+
+    world, rank, local = _dist()
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    binding.load_library()
     peaks = _peaks()
-    work = stage_work(wl)
-    stage_report = {}
-    for name, ms in stages.items():
-        nbytes, flops = work[name]
-        sec_s = ms / 1000.0
-        gbs = nbytes / sec_s / 1e9
-        tfs = flops / sec_s / 1e12 if flops else 0.0
-        entry = {"ms": ms, "GB/s": gbs, "hbm_frac": gbs / peaks["hbm_gbs"],
-                 "algorithmic_bytes": nbytes, "algorithmic_flops": flops}
-        if flops:
-            entry["TFLOP/s"] = tfs
-            entry["tensor_frac"] = tfs / _tensor_peak(wl, name, peaks)
-        stage_report[name] = entry
-    dominant = max(stages, key=lambda n: stages[n])
-    d = stage_report[dominant]
-    bound = "hbm"
-    if dominant == "indexer" and not wl.is_decode:
-        bound = "tensor"
-    traffic = DRAM_TRAFFIC_PER_LAUNCH.get((wl.name, dominant))
-    if bound == "tensor":
-        tpeak = _tensor_peak(wl, dominant, peaks)
-        roofline = {"bound": "tensor", "kernel": dominant, "achieved": d["TFLOP/s"],
-                    "peak": tpeak, "unit": "TFLOP/s", "frac": d["TFLOP/s"] / tpeak, "traffic": traffic,
-                    "peak_source": peaks["source"] + ("" if tpeak == peaks["bf16_tflops"] else
-                                                      " bf16 x 2 (nominal fp8 / bf16 dense ratio)")}
-    else:
-        roofline = {"bound": "hbm", "kernel": dominant, "achieved": d["GB/s"], "peak": peaks["hbm_gbs"],
-                    "unit": "GB/s", "frac": d["GB/s"] / peaks["hbm_gbs"], "traffic": traffic,
-                    "peak_source": peaks["source"]}
+
+    report, ctx = measure_forward(wl, args, binding, device, world, rank, local, peaks)
+    cpu = ctx["cpu"]
 
     # ---- end to end through the public API with host buffers
-    e2e = run_e2e(wl, cpu, binding, device, stream, max(1, min(args.steps, args.e2e_steps)), world)
+    e2e = run_e2e(wl, cpu, binding, device, ctx["stream"], max(1, min(args.steps, args.e2e_steps)), world)
 
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
     cpu_baseline = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        import oracle
-        oracle.build()
-        nthreads = oracle.max_threads()
-        rows = _sample_rows_for(wl, args.cpu_budget, nthreads, cpu)
-        # repeat the sample until about cpu_budget seconds of oracle time
-        total_s, total_rows, reps = 0.0, 0, 0
-        while reps == 0 or (total_s < 0.66 * args.cpu_budget and reps < 50):
-            secs, r = time_oracle(wl, cpu, rows, nthreads)
-            total_s += secs
-            total_rows += r
-            reps += 1
-        cpu_baseline = {"value": _oracle_rate(wl, total_s, total_rows), "unit": unit, "cores": nthreads,
-                        "kind": "oracle",
-                        "sample": f"{rows} of {wl.B * wl.Tq} query rows (all three stages), {reps} "
-                                  f"repetition(s), {total_s:.1f} s in total, scaled to a full step"}
+        cpu_baseline = cpu_baseline_for(wl, cpu, args.cpu_budget, repeat=True)
         # the same oracle on one core, on a smaller sample of the same rows
         rows1 = _sample_rows_for(wl, args.cpu_budget / 4, 1, cpu)
-        secs1, r1 = time_oracle(wl, cpu, rows1, 1)
-        cpu_baseline["single_core"] = {"value": _oracle_rate(wl, secs1, r1), "unit": unit, "cores": 1,
-                                       "sample": f"{r1} query rows, {secs1:.1f} s, scaled to a full step"}
+        secs1, r1, pairs1 = time_oracle(wl, cpu, rows1, 1)
+        cpu_baseline["single_core"] = {"value": _oracle_rate(wl, secs1, pairs1), "unit": report["unit"],
+                                       "cores": 1, "sample": f"{r1} query rows, {secs1:.1f} s, extrapolated "
+                                                             "to a full step"}
+    del cpu, ctx
+    torch.cuda.empty_cache()
+
+    # ---- the other configurations: device throughput, per-stage roofline
+    # fractions, clocks and an oracle baseline on a bounded row sample each
+    workloads = {}
+    extra = [] if args.workloads == "none" else (
+        [w for w in EXTRA_WORKLOADS if w != wl.name] if args.workloads == "all" else args.workloads.split(","))
+    for name in extra:
+        xwl = WORKLOADS[name]
+        xrep, xctx = measure_forward(xwl, args, binding, device, world, rank, local, peaks)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            xrep["cpu_baseline"] = cpu_baseline_for(xwl, xctx["cpu"], args.cpu_budget / 3, repeat=True)
+        workloads[name] = xrep
+        del xctx
+        torch.cuda.empty_cache()
 
     if rank == 0:
         line = {
-            "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": 1000.0 * sec_max / args.steps,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16"
-            if wl.dtype == "bf16" else "f32", "data": "synthetic", "config": _config(wl, world),
-            "roofline": roofline, "stages": stage_report, "cpu_baseline": cpu_baseline, "e2e": e2e,
-            "gpu_launches": int(launches), "clocks": clocks, "eager": eager,
-            "timing": "CUDA-graph replay of one dsa_forward per step" if graph is not None
-            else "eager dsa_forward calls",
+            "metric": METRIC, "value": report["value"], "unit": report["unit"], "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": report["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if wl.dtype == "bf16" else "f32", "data": "synthetic", "config": report["config"],
+            "roofline": report["roofline"], "stages": report["stages"], "cpu_baseline": cpu_baseline, "e2e": e2e,
+            "gpu_launches": report["gpu_launches"], "clocks": report["clocks"], "eager": report["eager"],
+            "timing": report["timing"], "workloads": workloads,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -927,6 +1054,9 @@ def main():
                     help="default: decode32k (forward), prefill8k (train)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--workloads", default="all",
+                    help="other configurations reported under \"workloads\": all (default), none, or a "
+                         "comma-separated list of names")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle wall time")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--pass", dest="pass_", default="forward", choices=["forward", "train", "cp"],

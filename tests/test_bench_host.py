@@ -96,10 +96,41 @@ def test_oracle_timing_helpers():
     cpu = bench.make_inputs(wl)
     rows = bench._sample_rows_for(wl, 0.2, 1, cpu)
     assert 1 <= rows <= wl.B * wl.Tq
-    sec, r = bench.time_oracle(wl, cpu, rows, 1)
+    sec, r, pairs = bench.time_oracle(wl, cpu, rows, 1)
     assert r == rows and sec >= 0.0
-    # 4 of toy16's 16 query rows in 2 s: a full step takes 8 s, 16 tokens / 8 s
-    assert bench._oracle_rate(wl, 2.0, 4) == pytest.approx(2.0)
+    assert pairs == bench.sample_pairs(wl, bench.sample_rows(wl, rows))
+    # rows holding a quarter of toy16's causal pairs in 2 s: a full step
+    # takes 8 s, 16 tokens / 8 s
+    assert bench._oracle_rate(wl, 2.0, wl.causal_pairs() // 4) == pytest.approx(2.0)
     dec = WORKLOADS["decode32k"]
-    # 8 of 32 decode rows in 1 s: a step takes 4 s
-    assert bench._oracle_rate(dec, 1.0, 8) == pytest.approx(0.25)
+    # 8 of 32 decode rows (32768 pairs each) in 1 s: a step takes 4 s
+    assert bench._oracle_rate(dec, 1.0, 8 * 32768) == pytest.approx(0.25)
+
+
+def test_oracle_row_sample_and_pair_count():
+    wl = WORKLOADS["prefill32k"]
+    flat = bench.sample_rows(wl, 512, tail=256)
+    assert len(flat) == 512 and len(set(flat.tolist())) == 512
+    assert flat[-256:].tolist() == list(range(32768 - 256, 32768))
+    assert flat[0] == 0
+    # sum of t + 1 over the rows, by brute force
+    assert bench.sample_pairs(wl, flat) == sum(int(t) + 1 for t in flat)
+    assert bench.sample_pairs(wl, range(wl.Tq)) == wl.causal_pairs()
+    dec = WORKLOADS["decode128k"]
+    assert bench.sample_pairs(dec, [0, 7]) == 2 * 131072
+
+
+def test_traffic_entries_expire_when_their_kernel_changes(monkeypatch):
+    files = ["indexer_tc.cu", "sm100.cuh"]
+    entry = {"bytes": 1.0e6, "sources": files, "digest": bench._sources_digest(files), "profile": "x"}
+    monkeypatch.setitem(bench.DRAM_TRAFFIC_PER_LAUNCH, ("w", "indexer"), entry)
+    assert bench.dram_traffic("w", "indexer") == 1.0e6
+    monkeypatch.setitem(bench.DRAM_TRAFFIC_PER_LAUNCH, ("w", "indexer"), dict(entry, digest="0" * 16))
+    assert bench.dram_traffic("w", "indexer") is None
+    assert bench.dram_traffic("w", "topk") is None
+
+
+def test_traffic_entries_name_their_profile():
+    """Every committed traffic figure names the profile summary it came from."""
+    for (wl, stage), e in bench.DRAM_TRAFFIC_PER_LAUNCH.items():
+        assert os.path.exists(os.path.join(bench.ROOT, e["profile"])), (wl, stage)
