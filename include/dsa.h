@@ -105,6 +105,21 @@ const char *dsa_status_string(dsa_status status);
 dsa_status dsa_device_error(dsa_stream_t stream);
 
 /*
+ * dsa_set_wait_limit_ns -- the time limit of every bounded device-side wait
+ * of the library's kernels on the current device (default 2,000,000,000 ns).
+ * A diagnostic with no counterpart on the pages, for testing the give-up
+ * path: with ns = 0 every bounded wait gives up at its first call, so each
+ * role of those kernels stops before it issues a copy or an MMA; the kernels
+ * release their resources, return without their outputs and record
+ * DSA_ERR_TIMEOUT (dsa_device_error). Copies and MMAs a CTA did issue are
+ * always waited for before it frees tensor memory or exits.
+ * Call it while none of the library's kernels runs on the device (it writes
+ * device variables like cudaMemcpyToSymbol). Returns DSA_ERR_CUDA if a write
+ * failed.
+ */
+dsa_status dsa_set_wait_limit_ns(uint64_t ns);
+
+/*
  * dsa_indexer_scores -- stage 1, lightning-indexer scores ("Learned Token Selection" §2.1).
  *
  *   scores[b,i,s] = sum_{j<H_I} w[b,i,j] * max(0, sum_{e<d_I} q_idx[b,i,j,e] * k_idx[b,s,e])

@@ -26,7 +26,7 @@ STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED",
 # Symbols declared in include/dsa.h.
 EXPORTED = ("dsa_version", "dsa_kernel_launch_count", "dsa_status_string", "dsa_indexer_scores", "dsa_topk",
             "dsa_topk_workspace_bytes", "dsa_sparse_attn", "dsa_sparse_attn_workspace_bytes",
-            "dsa_forward", "dsa_forward_workspace_bytes", "dsa_device_error", "dsa_topk_ex",
+            "dsa_forward", "dsa_forward_workspace_bytes", "dsa_device_error", "dsa_set_wait_limit_ns", "dsa_topk_ex",
             "dsa_indexer_kl", "dsa_indexer_backward", "dsa_indexer_backward_workspace_bytes",
             "dsa_cp_select_candidates", "dsa_cp_merge", "dsa_cp_localize", "dsa_cp_combine")
 
@@ -93,6 +93,7 @@ def load_library(path: str = LIB_PATH):
     lib.dsa_forward_workspace_bytes.argtypes = [ctypes.POINTER(ForwardArgs)]
     lib.dsa_forward_workspace_bytes.restype = sz
     lib.dsa_device_error.argtypes, lib.dsa_device_error.restype = [vp], ci
+    lib.dsa_set_wait_limit_ns.argtypes, lib.dsa_set_wait_limit_ns.restype = [ctypes.c_uint64], ci
     lib.dsa_indexer_kl.argtypes = [vp, vp, vp, ci, ci, ci, ci, ci, vp, vp, vp, vp]
     lib.dsa_indexer_kl.restype = ci
     lib.dsa_indexer_backward.argtypes = [vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, vp, vp, vp, vp, sz, vp]
@@ -121,6 +122,15 @@ def device_error(stream=None) -> None:
     bounded wait that gave up (DSA_ERR_TIMEOUT) or a selected position outside
     [0, L) other than -1 that an attention call skipped (DSA_ERR_BAD_INDEX)."""
     _check(load_library().dsa_device_error(_stream(stream)), "dsa_device_error")
+
+
+DEFAULT_WAIT_LIMIT_NS = 2_000_000_000
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    """dsa_set_wait_limit_ns: the limit of the kernels' bounded device-side
+    waits on the current device (0: every such wait gives up at once)."""
+    _check(load_library().dsa_set_wait_limit_ns(int(ns)), "dsa_set_wait_limit_ns")
 
 
 def _check(status: int, what: str):

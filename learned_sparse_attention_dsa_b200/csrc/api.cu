@@ -228,6 +228,13 @@ dsa_status dsa_device_error(dsa_stream_t stream) {
     return (words & kErrBadIndex) ? DSA_ERR_BAD_INDEX : DSA_OK;
 }
 
+dsa_status dsa_set_wait_limit_ns(uint64_t ns) {
+    if (dsa::indexer_set_wait_limit(ns) != cudaSuccess || dsa::indexer_bwd_set_wait_limit(ns) != cudaSuccess ||
+        dsa::attn_mla_tc_set_wait_limit(ns) != cudaSuccess)
+        return DSA_ERR_CUDA;
+    return DSA_OK;
+}
+
 const char *dsa_status_string(dsa_status status) {
     switch (status) {
         case DSA_OK: return "DSA_OK";

@@ -23,28 +23,31 @@
 // on B200: ~48 cycles, ~65 for N=128, ~129 for N=256), so a tile is 64 keys.
 // TMEM: Q part [0,160), S [160,224), O [256,512). Shared memory: a three-slot
 // ring of gathered boxes (3 x 40 KB), P (16 KB), the partial-S send and
-// receive buffers (2 x 32 KB). A partial S crosses to the other part as one
-// 32 KB bulk copy between the CTAs' shared memories.
+// receive buffers (2 x 32 KB).
 //
 // Per CTA (one per SM):
-//   warps 0-3  softmax, one head per thread: the Q part into TMEM (staged by
-//              TMA, then tcgen05.st); per tile tcgen05.ld of S_p (released at
-//              once, so the next QK^T overlaps), S_p to the other part, S =
-//              S_0 + S_1, online softmax in fp32 against a reference max that
-//              moves only when the row max grows by more than 2^8 (then O is
-//              rescaled in TMEM), P in bf16 to shared memory (128-byte
-//              swizzle); at the end O leaves TMEM for the output or the split
-//              partials (one bulk copy per head row).
-//   warps 4-6  gather the 5 boxes of 64 selected rows per tile with 16-byte
+//   warps 0-7  softmax, two warps per TMEM lane quarter: warp w takes heads
+//              32 (w % 4) .. + 31 (one per thread) and keys 32 (w / 4) .. + 31
+//              of every tile. Each warp swaps its 32 x 32 block of S_p with
+//              the same warp of the other part directly: a 4 KB bulk copy
+//              into the other part's receive buffer that completes on a
+//              barrier of that warp alone. The next tile's S_p is loaded and
+//              sent before this tile's softmax, so the swap of tile t + 1 runs
+//              under the softmax of tile t. The two warps of a lane quarter
+//              agree on the tile's row max through shared memory; the online
+//              softmax keeps a reference max that moves only when the row max
+//              grows by more than 2^8 (then O is rescaled in TMEM); P goes to
+//              shared memory in bf16 (128-byte swizzle). At the end O leaves
+//              TMEM for the output or for a bf16 partial normalised by its
+//              own sum.
+//   warps 8-10 gather the 5 boxes of 64 selected rows per tile with 16-byte
 //              cp.async (one warp instruction fills 4 rows x 128 bytes).
-//   warp 7     one thread moves S_p: bulk copy of the send buffer into the
-//              other part's receive buffer, then re-arms this part's receive
-//              barrier and frees the other part's sends.
-//   warp 8     TMEM allocation, the Q staging by TMA, and one thread issuing
+//   warp 11    TMEM allocation, the Q staging by TMA, and one thread issuing
 //              the MMAs with descriptors built once.
-// With several splits, attn_mla_combine_kernel merges the fp32 partials.
+// With several splits, attn_mla_combine_kernel merges the partials.
 // Every mbarrier wait is bounded; on a timeout the CTA records an error word,
-// drains its copies and MMAs, frees TMEM and returns.
+// waits for the copies and MMAs it issued and for the swaps sent to it, frees
+// TMEM and returns.
 #include <math.h>
 
 #include <cooperative_groups.h>
@@ -72,24 +75,28 @@ constexpr int kMaxTiles = 8;                       // tiles per split
 constexpr int kMaxSel = kMaxTiles * kTileN;        // selected entries per split
 constexpr int kMaxSplits = 32;
 constexpr int kSlots = 3;
+constexpr int kSoftWarps = 8;
+constexpr int kSoftmaxThreads = kSoftWarps * 32;   // 256
+constexpr int kGatherThreads = 96;
+constexpr int kMmaWarp = (kSoftmaxThreads + kGatherThreads) / 32;  // 11
+constexpr int kThreads = (kMmaWarp + 1) * 32;                      // 384
 constexpr uint32_t kQBox = kHeads * 128;           // 16,384
 constexpr uint32_t kKBox = kTileN * 128;           // 8,192
 constexpr uint32_t kKSlot = kGBoxes * kKBox;       // 40,960
 constexpr uint32_t kPBytes = kHeads * kTileN * 2;  // 16,384
 constexpr uint32_t kXBytes = kHeads * kTileN * 4;  // 32,768: one partial S tile
+constexpr uint32_t kXWarpBytes = kXBytes / kSoftWarps;  // 4,096: one warp's 32 heads x 32 keys
 constexpr uint32_t kOffP = kSlots * kKSlot;
 constexpr uint32_t kOffXs = kOffP + kPBytes;       // this part's S_p, sent to the other part
 constexpr uint32_t kOffXr = kOffXs + kXBytes;      // the other part's S_p, received
 constexpr uint32_t kOffSel = kOffXr + kXBytes;
-constexpr uint32_t kOffBar = kOffSel + kMaxSel * 4;
-constexpr uint32_t kStageBytes = kHeads * kHalfDv * 4;  // O staging for the partials
-constexpr int kNumBars = 18;
+constexpr uint32_t kOffMx = kOffSel + kMaxSel * 4;          // [tile parity][key half][head] row maxima
+constexpr uint32_t kOffL = kOffMx + 2 * 2 * kHeads * 4;     // [key half][head] row sums
+constexpr uint32_t kOffCnt = kOffL + 2 * kHeads * 4;        // [warp] S_p blocks the other part sent here
+constexpr uint32_t kOffBar = kOffCnt + kSoftWarps * 4;
+constexpr uint32_t kHalfRowBytes = kHalfDv * 2;             // one head's bf16 partial of a part
+constexpr int kNumBars = 17 + 2 * kSoftWarps;
 constexpr size_t kSmem = 1024 + kOffBar + kNumBars * 8 + 16;  // + slack to align the base to 1024
-constexpr int kSoftmaxThreads = 128;
-constexpr int kGatherThreads = 96;
-constexpr int kXchgWarp = (kSoftmaxThreads + kGatherThreads) / 32;  // 7
-constexpr int kMmaWarp = kXchgWarp + 1;                              // 8
-constexpr int kThreads = (kMmaWarp + 1) * 32;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColQ = 0;
 constexpr uint32_t kColS = 160;
@@ -100,7 +107,8 @@ constexpr uint32_t kIdescMnMajorB = 1u << 16;
 
 static_assert(kOffP % 1024 == 0 && kKSlot % 1024 == 0, "operand tiles must sit on 1024-byte boundaries");
 static_assert(5 * kQBox <= 2 * kKSlot, "the Q staging must fit over ring slots 0 and 1");
-static_assert(kStageBytes <= kOffXs, "the O staging must fit over the ring and P");
+static_assert(kHeads * kHalfRowBytes <= kOffXs, "the partial staging must fit over the ring and P");
+static_assert(kOffBar % 8 == 0, "mbarrier alignment");
 static_assert(kColS + kTileN <= kColO, "TMEM columns");
 static_assert(kSmem <= 232448, "shared memory budget");
 
@@ -120,19 +128,20 @@ struct Args {
     int64_t sb, ss;
     __nv_bfloat16 *out;       // [rows, 128, 512]
     float *lse;               // [rows, 128] or null
-    float *part_o, *part_ml;  // split partials (splits > 1)
+    uint4 *part_o;            // split partials (splits > 1), bf16, see attn_mla_tc_workspace_bytes
+    float *part_ml;           // [rows, 128, splits, 2]: (max in log2 units, sum)
 };
-
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
-// Where float4 q (0..63) of head h's half row sits in the O staging and in
-// the partials: rotated by h, so that a warp's 32 rows spread over the
-// shared-memory banks. The combine kernel undoes the rotation.
-__host__ __device__ __forceinline__ int rot_q(int h, int q) { return (q + h) & (kHalfDv / 4 - 1); }
+// Where 16-byte chunk q (0..31) of head h's bf16 half row of partials sits:
+// rotated by h, so that a warp's 32 rows spread over the shared-memory banks
+// of the staging and the combine kernel's loads stay coalesced. The combine
+// kernel undoes the rotation.
+__host__ __device__ __forceinline__ int rot_chunk(int h, int q) { return (q + h) & 31; }
 
 // Descriptor field arithmetic: the start address sits in the low bits in
 // units of 16 bytes, so moving an operand by b bytes adds b >> 4.
@@ -146,6 +155,12 @@ __device__ __forceinline__ void bulk_store(void *gdst, const void *ssrc, uint32_
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+
+__device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
 
 // QK^T of one tile: the part's Q columns (A, TMEM) against its boxes of the
 // gathered rows (B, K-major); QB boxes of 4 K=16 steps each.
@@ -163,23 +178,25 @@ attn_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Args a) {
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *k_sm = smem;               // ring; slots 0-1 first stage the Q part
     uint8_t *p_sm = smem + kOffP;
-    float4 *xs_sm = reinterpret_cast<float4 *>(smem + kOffXs);
-    float4 *xr_sm = reinterpret_cast<float4 *>(smem + kOffXr);
+    uint8_t *xs_sm = smem + kOffXs;
+    uint8_t *xr_sm = smem + kOffXr;
     int32_t *sel = reinterpret_cast<int32_t *>(smem + kOffSel);
+    float *mx_sm = reinterpret_cast<float *>(smem + kOffMx);
+    float *l_sm = reinterpret_cast<float *>(smem + kOffL);
+    uint32_t *cnt_sm = reinterpret_cast<uint32_t *>(smem + kOffCnt);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
     uint64_t *q_full = bars;            // TMA bytes of the staged Q part
-    uint64_t *q_copied = bars + 1;      // 128 softmax threads: Q part in TMEM, staging free
-    uint64_t *kv_full = bars + 2;       // [3] 128 gather threads (cp.async arrivals)
+    uint64_t *q_copied = bars + 1;      // 256 softmax threads: Q part in TMEM, staging free
+    uint64_t *kv_full = bars + 2;       // [3] 96 gather threads (cp.async arrivals)
     uint64_t *kv_empty = bars + 5;      // [3] MMA commit after PV
     uint64_t *s_full = bars + 8;        // MMA commit after QK^T
-    uint64_t *s_free = bars + 9;        // 128 softmax threads (S_p is in registers)
-    uint64_t *p_full = bars + 10;       // 128 softmax threads
+    uint64_t *s_free = bars + 9;        // 256 softmax threads (S_p is in registers)
+    uint64_t *p_full = bars + 10;       // 256 softmax threads
     uint64_t *pv_done = bars + 11;      // MMA commit after PV
     uint64_t *drained = bars + 12;      // MMA commit before teardown
-    uint64_t *x_full = bars + 13;       // bytes of the other part's S_p in xr_sm (armed per tile)
-    uint64_t *x_free = bars + 14;       // the other part has read what we sent
-    uint64_t *xs_full = bars + 15;      // 128 softmax threads: send buffer written
-    uint64_t *xr_done = bars + 16;      // 128 softmax threads: receive buffer read
+    uint64_t *mx_bar = bars + 13;       // [4] the two warps of a lane quarter posted their row maxima
+    uint64_t *x_full = bars + 17;       // [8] the other part's block of S_p for warp w landed
+    uint64_t *x_free = bars + 17 + kSoftWarps;  // [8] the other part's warp w read what we sent
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kNumBars);
 
     const int row = blockIdx.x;
@@ -216,29 +233,34 @@ attn_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Args a) {
         mbar_init(p_full, kSoftmaxThreads);
         mbar_init(pv_done, 1);
         mbar_init(drained, 1);
-        mbar_init(x_full, 1);
-        mbar_init(x_free, 1);
-        mbar_init(xs_full, kSoftmaxThreads);
-        mbar_init(xr_done, kSoftmaxThreads);
+        for (int i = 0; i < 4; ++i) mbar_init(&mx_bar[i], 64);
+        for (int w = 0; w < kSoftWarps; ++w) {
+            mbar_init(&x_full[w], 1);
+            mbar_init(&x_free[w], 1);
+        }
         fence_barrier_init();
-        mbar_arrive_expect_tx(x_full, kXBytes);  // armed for the first tile
+        // armed for the first tile: 4 KB from the other part's warp w
+        for (int w = 0; w < kSoftWarps; ++w) mbar_arrive_expect_tx(&x_full[w], kXWarpBytes);
     }
     if (warp == kMmaWarp) {
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
     tc_fence_before();
-    cg::this_cluster().sync();  // both parts' barriers exist before any remote arrival
+    cg::this_cluster().sync();  // both parts' barriers exist before any remote arrival or copy
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     bool ok = true;
-    float m_ref = -INFINITY, l = 0.0f;  // softmax threads: reference max (log2 units) and sum
+    float m_ref = -INFINITY, l = 0.0f;  // softmax threads: reference max (log2 units), partial sum
+    uint32_t sent = 0, recv = 0;        // softmax threads: S_p blocks sent to / received from the other part
 
     // Tile t lands in ring slot (t + 2) % 3 (its (t / 3)-th use): slots 0-1
     // first hold the Q staging, so tiles 1 and 2 wait for the copy to TMEM.
     if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0 && n_tiles > 0) {
+        // a wait limit of 0 gives up here, before the first copy is issued
+        if (lane == 0 && n_tiles > 0 && __ldg(&g_wait_limit_ns) == 0) ok = false;
+        if (lane == 0 && n_tiles > 0 && ok) {
             prefetch_tensor_map(&tm_q);
             mbar_arrive_expect_tx(q_full, (uint32_t)q_boxes(part) * kQBox);
 #pragma unroll 1
@@ -284,29 +306,13 @@ attn_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Args a) {
                 if (t > 0 && !issue_pv(t - 1)) ok = false;
             }
             if (ok) ok = issue_pv(n_tiles - 1);
-            // nothing of this CTA may still run on the tensor core at teardown
+            // nothing of this CTA may still run on the tensor core at teardown,
+            // and the Q load has landed
             mma_commit(drained);
-            if (!mbar_wait(drained, 0)) ok = false;
+            if (!mbar_drain(drained, 0)) ok = false;
+            if (!mbar_drain(q_full, 0)) ok = false;
         }
-    } else if (warp == kXchgWarp) {
-        // ------------------------------------------------------------ S_p exchange
-        if (lane == 0) {
-            const uint32_t peer = (uint32_t)(part ^ 1);
-            const uint32_t peer_xr = cluster_smem_addr(xr_sm, peer);
-            const uint32_t peer_x_full = cluster_smem_addr(x_full, peer);
-            const uint32_t peer_x_free = cluster_smem_addr(x_free, peer);
-            for (int t = 0; t < n_tiles; ++t) {
-                // the softmax threads have written S_p (after the other part
-                // had read the previous one)
-                if (!mbar_wait(xs_full, (uint32_t)t & 1u)) { ok = false; break; }
-                bulk_copy_to_cluster(peer_xr, xs_sm, kXBytes, peer_x_full);
-                // they have read the other part's S_p: re-arm, let it send again
-                if (!mbar_wait(xr_done, (uint32_t)t & 1u)) { ok = false; break; }
-                if (t + 1 < n_tiles) mbar_arrive_expect_tx(x_full, kXBytes);
-                mbar_arrive_remote(peer_x_free);
-            }
-        }
-    } else if (warp >= kSoftmaxThreads / 32) {
+    } else if (warp >= kSoftWarps) {
         // ------------------------------------------------------------ gather
         const int gt = threadIdx.x - kSoftmaxThreads;
         const __nv_bfloat16 *kvb = a.kv + (int64_t)b * a.sb + g_box0(part) * 64;
@@ -333,14 +339,26 @@ attn_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Args a) {
         cp_async_wait_all();
     } else {
         // ------------------------------------------------------------ softmax
-        const int h = warp * 32 + lane;                      // head = TMEM lane
-        const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
+        const int quarter = warp & 3;                        // TMEM lane quarter
+        const int kh = warp >> 2;                            // key half of every tile
+        const int h = quarter * 32 + lane;                   // head = TMEM lane
+        const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+        const uint32_t peer = (uint32_t)(part ^ 1);
+        // this warp's 4 KB block of S_p in the send and receive buffers:
+        // [key half][head][32 floats], the thread's row of 8 chunks rotated by h
+        const uint32_t blk = (uint32_t)(kh * kHeads + quarter * 32) * 128;
+        float4 *xs_row = reinterpret_cast<float4 *>(xs_sm + blk + lane * 128);
+        const float4 *xr_row = reinterpret_cast<const float4 *>(xr_sm + blk + lane * 128);
+        const uint32_t peer_xr_blk = cluster_smem_addr(xr_sm + blk, peer);
+        const uint32_t peer_x_full = cluster_smem_addr(&x_full[warp], peer);
+        const uint32_t peer_x_free = cluster_smem_addr(&x_free[warp], peer);
         if (n_tiles > 0) {
             // the part's Q columns of head h, staged by TMA (row h of each box,
-            // 128-byte swizzle), into its TMEM lane as raw bf16 pairs
+            // 128-byte swizzle), into its TMEM lane as raw bf16 pairs; the two
+            // warps of a lane quarter take alternate boxes
             if (!mbar_wait(q_full, 0)) ok = false;
             if (__all_sync(0xffffffffu, ok)) {
-                for (int c = 0; c < q_boxes(part); ++c) {  // warp-uniform trip count
+                for (int c = kh; c < q_boxes(part); c += 2) {  // warp-uniform trip count
                     const uint8_t *box = smem + c * kQBox + h * 128;
                     uint32_t w[32];
 #pragma unroll
@@ -356,70 +374,94 @@ attn_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Args a) {
             tc_fence_before();
             mbar_arrive(q_copied);
         }
-        for (int t = 0; ok && t < n_tiles; ++t) {
-            if (!mbar_wait(s_full, (uint32_t)t & 1u)) ok = false;
-            ok = __all_sync(0xffffffffu, ok);
-            if (!ok) break;
+        ok = __all_sync(0xffffffffu, ok);
+
+        // S_p of tile t (this warp's 32 keys) out of TMEM into registers
+        auto load_sp = [&](int t, uint32_t *v) -> bool {
+            if (!mbar_wait(s_full, (uint32_t)t & 1u)) return false;
             tc_fence_after();
-            uint32_t x[64];
-            tmem_ld_32x32b_x32(tmem + lane_addr + kColS, x);
-            tmem_ld_32x32b_x32(tmem + lane_addr + kColS + 32, x + 32);
+            tmem_ld_32x32b_x32(tmem + lane_addr + kColS + (uint32_t)(kh * 32), v);
             tmem_ld_wait();
             tc_fence_before();
             mbar_arrive(s_free);  // the next QK^T may overwrite S_p
-
-            // S_p to the other part: row h of the send buffer (16-byte chunks
-            // rotated by h), then one bulk copy into its receive buffer. The
-            // send buffer is free again once the other part has read the
-            // previous tile (every wait here is bounded).
-            if (t > 0 && !mbar_wait_cluster(x_free, (uint32_t)(t - 1) & 1u)) ok = false;
-            if (!__all_sync(0xffffffffu, ok)) break;
-            float4 *xsr = xs_sm + h * (kTileN / 4);
+            return true;
+        };
+        // send this warp's block of S_p to the same warp of the other part
+        auto send_sp = [&](const uint32_t *v) {
 #pragma unroll
-            for (int c = 0; c < kTileN / 4; ++c)
-                xsr[(c + h) & (kTileN / 4 - 1)] =
-                    make_float4(__uint_as_float(x[4 * c]), __uint_as_float(x[4 * c + 1]),
-                                __uint_as_float(x[4 * c + 2]), __uint_as_float(x[4 * c + 3]));
+            for (int c = 0; c < 8; ++c)
+                xs_row[(c + lane) & 7] = make_float4(__uint_as_float(v[4 * c]), __uint_as_float(v[4 * c + 1]),
+                                                     __uint_as_float(v[4 * c + 2]), __uint_as_float(v[4 * c + 3]));
             fence_proxy_async_smem();  // read by the bulk copy
-            mbar_arrive(xs_full);
-            if (!mbar_wait_cluster(x_full, (uint32_t)t & 1u)) ok = false;
+            __syncwarp();
+            if (lane == 0) bulk_copy_to_cluster(peer_xr_blk, xs_sm + blk, kXWarpBytes, peer_x_full);
+            ++sent;
+        };
+
+        uint32_t x[32], y[32];
+        if (ok && n_tiles > 0) {
+            if (!load_sp(0, x)) ok = false;
+            ok = __all_sync(0xffffffffu, ok);
+            if (ok) send_sp(x);
+        }
+        for (int t = 0; ok && t < n_tiles; ++t) {
+            // the other part's block of S_p for tile t: S = S_0 + S_1
+            if (!mbar_wait_cluster(&x_full[warp], (uint32_t)t & 1u)) ok = false;
             if (!__all_sync(0xffffffffu, ok)) break;
-            // S = S_0 + S_1 (the same sum on both parts)
-            const float4 *xr = xr_sm + h * (kTileN / 4);
 #pragma unroll
-            for (int c = 0; c < kTileN / 4; ++c) {
-                const float4 v = xr[(c + h) & (kTileN / 4 - 1)];
+            for (int c = 0; c < 8; ++c) {
+                const float4 v = xr_row[(c + lane) & 7];
                 x[4 * c] = __float_as_uint(__uint_as_float(x[4 * c]) + v.x);
                 x[4 * c + 1] = __float_as_uint(__uint_as_float(x[4 * c + 1]) + v.y);
                 x[4 * c + 2] = __float_as_uint(__uint_as_float(x[4 * c + 2]) + v.z);
                 x[4 * c + 3] = __float_as_uint(__uint_as_float(x[4 * c + 3]) + v.w);
             }
-            mbar_arrive(xr_done);
+            ++recv;
+            __syncwarp();  // every lane has read the block
+            if (lane == 0 && t + 1 < n_tiles) {
+                mbar_arrive_expect_tx(&x_full[warp], kXWarpBytes);  // armed for the next block
+                mbar_arrive_remote(peer_x_free);                    // the other part may send it
+            }
+            // the next tile's S_p goes out now, so that its swap runs under
+            // this tile's softmax; the send buffer is free again once the
+            // other part has read this tile's block
+            if (t + 1 < n_tiles) {
+                if (!load_sp(t + 1, y)) ok = false;
+                if (ok && !mbar_wait_cluster(&x_free[warp], (uint32_t)t & 1u)) ok = false;
+                if (!__all_sync(0xffffffffu, ok)) break;
+                send_sp(y);
+            }
 
-            const unsigned vm0 = __ballot_sync(0xffffffffu, sel[t * kTileN + lane] >= 0);
-            const unsigned vm1 = __ballot_sync(0xffffffffu, sel[t * kTileN + 32 + lane] >= 0);
+            // scale, mask entries that are padding, this half's max
+            const unsigned vm = __ballot_sync(0xffffffffu, sel[t * kTileN + kh * 32 + lane] >= 0);
             float mt = -INFINITY;
-            if ((vm0 & vm1) == 0xffffffffu) {  // every entry of the tile is a valid position
+            if (vm == 0xffffffffu) {
 #pragma unroll
-                for (int j = 0; j < 64; ++j) {
+                for (int j = 0; j < 32; ++j) {
                     const float z = __uint_as_float(x[j]) * a.scale_log2;
                     x[j] = __float_as_uint(z);
                     mt = fmaxf(mt, z);
                 }
             } else {
 #pragma unroll
-                for (int j = 0; j < 64; ++j) {
-                    const bool valid = ((j < 32 ? vm0 >> j : vm1 >> (j - 32)) & 1u) != 0;
-                    const float z = valid ? __uint_as_float(x[j]) * a.scale_log2 : -INFINITY;
+                for (int j = 0; j < 32; ++j) {
+                    const float z = ((vm >> j) & 1u) ? __uint_as_float(x[j]) * a.scale_log2 : -INFINITY;
                     x[j] = __float_as_uint(z);
                     mt = fmaxf(mt, z);
                 }
             }
-            // PV of the previous tile must be done before P is rewritten or O rescaled
-            if (t > 0 && !mbar_wait(pv_done, (uint32_t)(t - 1) & 1u)) ok = false;
+            // the row max over both key halves: each warp of the lane quarter
+            // posts its half's max (double-buffered by tile) and waits for the
+            // other's on a bounded barrier. PV of the previous tile must be
+            // done before P is rewritten or O rescaled.
+            mx_sm[((t & 1) * 2 + kh) * kHeads + h] = mt;
+            mbar_arrive(&mx_bar[quarter]);
+            if (!mbar_wait(&mx_bar[quarter], (uint32_t)t & 1u)) ok = false;
+            if (t > 0 && ok && !mbar_wait(pv_done, (uint32_t)(t - 1) & 1u)) ok = false;
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
+            mt = fmaxf(mt, mx_sm[((t & 1) * 2 + (kh ^ 1)) * kHeads + h]);
             float m_new = m_ref;
             bool grow = false;
             if (mt > -INFINITY) {
@@ -433,7 +475,7 @@ attn_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Args a) {
             if (__any_sync(0xffffffffu, grow)) {  // tcgen05.ld/st are warp-wide
                 const float f = grow ? exp2f(m_ref - m_new) : 1.0f;
 #pragma unroll 1
-                for (int c = 0; c < kHalfDv; c += 32) {
+                for (int c = kh * (kHalfDv / 2); c < (kh + 1) * (kHalfDv / 2); c += 32) {
                     uint32_t o[32];
                     tmem_ld_32x32b_x32(tmem + lane_addr + kColO + (uint32_t)c, o);
                     tmem_ld_wait();
@@ -448,10 +490,10 @@ attn_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Args a) {
             // p = 2^(z - m_ref); masked keys have z = -inf, so p = 0 (also when
             // no key of the row is valid yet: then every z is -inf)
             const float mr = m_ref == -INFINITY ? 0.0f : m_ref;
-            uint32_t pk[32];
+            uint32_t pk[16];
             float ps0 = 0.0f, ps1 = 0.0f;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
+            for (int j = 0; j < 16; ++j) {
                 const float p0 = ex2_approx(__uint_as_float(x[2 * j]) - mr);
                 const float p1 = ex2_approx(__uint_as_float(x[2 * j + 1]) - mr);
                 ps0 += p0;
@@ -459,99 +501,126 @@ attn_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Args a) {
                 pk[j] = pack_bf16x2(p0, p1);
             }
             l += ps0 + ps1;
-            // P row h: 128 bytes, 16-byte chunk c at chunk c ^ (h % 8)
+            // P row h: 128 bytes, 16-byte chunk c at chunk c ^ (h % 8); this
+            // warp's keys are chunks 4 kh .. 4 kh + 3
             uint8_t *prow = p_sm + h * 128;
 #pragma unroll
-            for (int c = 0; c < 8; ++c)
-                *reinterpret_cast<uint4 *>(prow + ((c ^ (h & 7)) << 4)) =
+            for (int c = 0; c < 4; ++c)
+                *reinterpret_cast<uint4 *>(prow + (((4 * kh + c) ^ (h & 7)) << 4)) =
                     make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
             fence_proxy_async_smem();  // P is read by the tensor core
             tc_fence_before();
             mbar_arrive(p_full);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) x[j] = y[j];
         }
         if (ok && n_tiles > 0 && !mbar_wait(pv_done, (uint32_t)(n_tiles - 1) & 1u)) ok = false;
         ok = __all_sync(0xffffffffu, ok);
+        l_sm[kh * kHeads + h] = l;
     }
 
-    // ---------------------------------------------------------------- outputs
-    // Every role is done here: MMAs drained, copies landed, O final in TMEM,
-    // so the ring and P may be reused as the O staging.
+    // ---------------------------------------------------------------- teardown
+    // Every S_p block sent to this CTA must have landed before it exits: each
+    // softmax warp tells the same warp of the other part how many blocks it
+    // sent, and after a cluster barrier a warp that received fewer waits for
+    // the one outstanding block (a warp sends block t + 1 only after the
+    // other part has read block t, so at most one can be in flight). The
+    // barrier is split around the output stores.
+    if (warp < kSoftWarps && lane == 0)
+        st_cluster_u32(cluster_smem_addr(&cnt_sm[warp], (uint32_t)(part ^ 1)), sent);
     tc_fence_before();
     const bool cta_ok = __syncthreads_and(ok ? 1 : 0) != 0;
     tc_fence_after();
+    cluster_arrive();
+
+    // ---------------------------------------------------------------- outputs
+    // Every role is done here: MMAs drained, copies landed, O final in TMEM,
+    // so the ring and P may be reused as the output staging.
     if (threadIdx.x < kSoftmaxThreads && cta_ok) {
-        const int h = threadIdx.x;
-        const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
+        const int quarter = warp & 3, kh = warp >> 2;
+        const int h = quarter * 32 + lane;
+        const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
         const size_t pair = (size_t)row * kHeads + h;
         const bool have_o = n_tiles > 0;
-        const float inv = l > 0.0f ? 1.0f / l : 0.0f;
-        float4 *stage = reinterpret_cast<float4 *>(smem + h * (kHalfDv * 4));
+        const float l_all = l_sm[h] + l_sm[kHeads + h];
+        const float inv = l_all > 0.0f ? 1.0f / l_all : 0.0f;
+        // this thread: value columns [128 kh, 128 kh + 128) of the part's 256
+        uint4 *stage = reinterpret_cast<uint4 *>(smem + h * kHalfRowBytes);
 #pragma unroll 1
-        for (int c = 0; c < kHalfDv; c += 64) {  // two loads per wait
+        for (int c = 0; c < kHalfDv / 2; c += 64) {  // two loads per wait
             uint32_t o[64];
+            const uint32_t col = (uint32_t)(kh * (kHalfDv / 2) + c);
             if (have_o) {
-                tmem_ld_32x32b_x32(tmem + lane_addr + kColO + (uint32_t)c, o);
-                tmem_ld_32x32b_x32(tmem + lane_addr + kColO + (uint32_t)(c + 32), o + 32);
+                tmem_ld_32x32b_x32(tmem + lane_addr + kColO + col, o);
+                tmem_ld_32x32b_x32(tmem + lane_addr + kColO + col + 32, o + 32);
                 tmem_ld_wait();
             } else {
 #pragma unroll
                 for (int j = 0; j < 64; ++j) o[j] = 0u;
             }
+            uint4 w[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                w[q] = make_uint4(pack_bf16x2(__uint_as_float(o[8 * q]) * inv, __uint_as_float(o[8 * q + 1]) * inv),
+                                  pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv, __uint_as_float(o[8 * q + 3]) * inv),
+                                  pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv, __uint_as_float(o[8 * q + 5]) * inv),
+                                  pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv, __uint_as_float(o[8 * q + 7]) * inv));
+            const int q0 = (int)col / 8;  // first 16-byte chunk of these 64 columns in the half row
             if (a.splits == 1) {
-                uint4 *dst = reinterpret_cast<uint4 *>(a.out + pair * DV + part * kHalfDv + c);
+                uint4 *dst = reinterpret_cast<uint4 *>(a.out + pair * DV + part * kHalfDv) + q0;
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    uint32_t w[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        w[e] = pack_bf16x2(__uint_as_float(o[8 * q + 2 * e]) * inv,
-                                           __uint_as_float(o[8 * q + 2 * e + 1]) * inv);
-                    dst[q] = make_uint4(w[0], w[1], w[2], w[3]);
-                }
+                for (int q = 0; q < 8; ++q) dst[q] = w[q];
             } else {
 #pragma unroll
-                for (int v = 0; v < 16; ++v)
-                    stage[rot_q(h, c / 4 + v)] =
-                        make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
-                                    __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
+                for (int q = 0; q < 8; ++q) stage[rot_chunk(h, q0 + q)] = w[q];
             }
         }
         if (a.splits == 1) {
-            if (part == 0 && a.lse != nullptr) a.lse[pair] = l > 0.0f ? (m_ref + log2f(l)) / kLog2e : -INFINITY;
+            if (part == 0 && kh == 0 && a.lse != nullptr)
+                a.lse[pair] = l_all > 0.0f ? (m_ref + log2f(l_all)) / kLog2e : -INFINITY;
         } else {
-            // one bulk copy of this head's (rotated) half row of partials
+            // the head's half row of partials, normalised by its own sum, once
+            // both warps of the lane quarter have staged their columns (every
+            // softmax thread gets here: cta_ok is the same for the whole CTA)
             fence_proxy_async_smem();
-            bulk_store(a.part_o + (pair * a.splits + split) * DV + part * kHalfDv, stage, kHalfDv * 4);
-            bulk_commit();
-            if (part == 0) {
-                a.part_ml[(pair * a.splits + split) * 2 + 0] = m_ref;
-                a.part_ml[(pair * a.splits + split) * 2 + 1] = l;
+            asm volatile("bar.sync %0, 64;" ::"r"(1 + quarter) : "memory");
+            if (kh == 0) {
+                bulk_store(a.part_o + (pair * a.splits + split) * (DV / 8) + part * (kHalfDv / 8), stage,
+                           kHalfRowBytes);
+                bulk_commit();
+                if (part == 0) {
+                    a.part_ml[(pair * a.splits + split) * 2 + 0] = m_ref;
+                    a.part_ml[(pair * a.splits + split) * 2 + 1] = l_all;
+                }
+                bulk_wait_read();  // the staging must outlive the copy's reads
             }
-            bulk_wait_read();  // the staging must outlive the copy's reads
         }
     }
 
+    cluster_wait();
+    if (warp < kSoftWarps && lane == 0 && cnt_sm[warp] > recv) {
+        if (!mbar_drain_cluster(&x_full[warp], recv & 1u)) ok = false;
+    }
     if (!ok) atomicOr(&g_attn_mla_tc_error, kErrTimeout);
     tc_fence_before();
-    cg::this_cluster().sync();  // no part leaves while the other may still write to it
+    cg::this_cluster().sync();  // no part leaves while the other may still read or write its memory
     if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
 }
 
-// Merge the split partials of one (row, head): lane j of each warp holds the
-// (max, sum) of split j; the pair's 128 output float4s are spread over four
-// warps, and every lane sums the splits' partials for its float4, undoing the
-// rotation of the half rows.
-__global__ void attn_mla_combine_kernel(const float4 *__restrict__ part_o, const float *__restrict__ part_ml,
+// Merge the split partials of one (row, head): two warps per pair, one per
+// part's half row. Lane j of each warp holds the (max, sum) of split j; every
+// lane owns 8 output columns (one 16-byte chunk of bf16) and loads every
+// split's chunk for them independently (all in flight at once), undoing the
+// rotation of the half rows. Each split's partial is normalised by its own
+// sum l_s, so it is weighted by l_s 2^(m_s - max).
+__global__ void attn_mla_combine_kernel(const uint4 *__restrict__ part_o, const float *__restrict__ part_ml,
                                         int n_pairs, int splits, __nv_bfloat16 *__restrict__ out,
                                         float *__restrict__ lse) {
-    // four warps per (row, head): warp quarter qt owns output float4s
-    // [32 qt, 32 qt + 32), one per lane, and loads every split's value for it
-    // independently (all in flight at once)
     const int gw = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    const int pair = gw >> 2, qt = gw & 3;
+    const int pair = gw >> 1, half = gw & 1;
     const int lane = threadIdx.x & 31;
     if (pair >= n_pairs) return;
     const int h = pair % kHeads;
@@ -559,28 +628,28 @@ __global__ void attn_mla_combine_kernel(const float4 *__restrict__ part_o, const
     const float m_s = lane < splits ? ml[2 * lane] : -INFINITY;
     const float l_s = lane < splits ? ml[2 * lane + 1] : 0.0f;
     const float m_all = warp_max(m_s);
-    const float f_s = (m_all == -INFINITY || lane >= splits) ? 0.0f : ex2_approx(m_s - m_all);
-    const float l_all = warp_sum(f_s * l_s);
+    const float f_s = (m_all == -INFINITY || lane >= splits) ? 0.0f : l_s * ex2_approx(m_s - m_all);
+    const float l_all = warp_sum(f_s);
     const float inv = l_all > 0.0f ? 1.0f / l_all : 0.0f;
-    const float4 *po = part_o + (size_t)pair * splits * (DV / 4);
-    const int c4 = qt * 32 + lane;  // output float4 index in [0, 128)
-    const int hf = c4 / (kHalfDv / 4), q = c4 % (kHalfDv / 4);
-    const int pos = hf * (kHalfDv / 4) + rot_q(h, q);
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    const uint4 *po = part_o + (size_t)pair * splits * (DV / 8) + half * (kHalfDv / 8) + rot_chunk(h, lane);
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
 #pragma unroll 8
     for (int sp = 0; sp < splits; ++sp) {
         const float f = __shfl_sync(0xffffffffu, f_s, sp);
-        const float4 v = po[(size_t)sp * (DV / 4) + pos];
-        acc.x = fmaf(f, v.x, acc.x);
-        acc.y = fmaf(f, v.y, acc.y);
-        acc.z = fmaf(f, v.z, acc.z);
-        acc.w = fmaf(f, v.w, acc.w);
+        float e8[8];
+        bf16x8_to_f32(po[(size_t)sp * (DV / 8)], e8);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = fmaf(f, e8[e], acc[e]);
     }
-    uint2 w;
-    w.x = pack_bf16x2(acc.x * inv, acc.y * inv);
-    w.y = pack_bf16x2(acc.z * inv, acc.w * inv);
-    *reinterpret_cast<uint2 *>(out + (size_t)pair * DV + 4 * c4) = w;
-    if (lse != nullptr && qt == 0 && lane == 0)
+    uint4 w;
+    w.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+    w.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+    w.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
+    w.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
+    reinterpret_cast<uint4 *>(out + (size_t)pair * DV + half * kHalfDv)[lane] = w;
+    if (lse != nullptr && half == 0 && lane == 0)
         lse[pair] = l_all > 0.0f ? (m_all + log2f(l_all)) / kLog2e : -INFINITY;
 }
 
@@ -605,6 +674,8 @@ int mla_tc_splits(const AttnProblem &p, int sm_count) {
 
 }  // namespace
 
+cudaError_t attn_mla_tc_set_wait_limit(unsigned long long ns) { return set_wait_limit_ns(ns); }
+
 unsigned int attn_mla_tc_take_device_error() {
     unsigned int v = 0, zero = 0;
     if (cudaMemcpyFromSymbol(&v, g_attn_mla_tc_error, sizeof(v)) != cudaSuccess) return 0;
@@ -624,10 +695,14 @@ bool attn_mla_tc_supported(const AttnProblem &p) {
     return info.cc_major == 10 && (size_t)info.max_smem_optin >= kSmem;
 }
 
+// Split partials: bf16 [rows, 128, splits, 512], each head's two half rows
+// (one per part) with their 16-byte chunks rotated by the head and normalised
+// by the split's own sum; then fp32 (max in log2 units, sum) [rows, 128,
+// splits, 2].
 size_t attn_mla_tc_workspace_bytes(const AttnProblem &p, int sm_count) {
     const int splits = mla_tc_splits(p, sm_count);
     if (splits <= 1) return 0;
-    return (size_t)p.B * p.Tq * kHeads * splits * ((size_t)DV + 2) * sizeof(float);
+    return (size_t)p.B * p.Tq * kHeads * splits * ((size_t)DV * 2 + 2 * sizeof(float));
 }
 
 cudaError_t launch_attn_mla_tc(const AttnProblem &p, const DeviceInfo &info, cudaStream_t stream) {
@@ -648,8 +723,9 @@ cudaError_t launch_attn_mla_tc(const AttnProblem &p, const DeviceInfo &info, cud
     a.out = static_cast<__nv_bfloat16 *>(p.out);
     a.lse = p.lse;
     const size_t n_pairs = (size_t)rows * kHeads;
-    a.part_o = splits > 1 ? static_cast<float *>(p.ws) : nullptr;
-    a.part_ml = splits > 1 ? a.part_o + n_pairs * splits * DV : nullptr;
+    a.part_o = splits > 1 ? static_cast<uint4 *>(p.ws) : nullptr;
+    a.part_ml = splits > 1 ? reinterpret_cast<float *>(static_cast<char *>(p.ws) + n_pairs * splits * DV * 2)
+                           : nullptr;
     cudaError_t err = cudaFuncSetAttribute(attn_mla_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
@@ -668,10 +744,10 @@ cudaError_t launch_attn_mla_tc(const AttnProblem &p, const DeviceInfo &info, cud
     count_launch();
     if (err != cudaSuccess) return err;
     if (splits > 1) {
-        const int warps_per_block = 8;  // four warps per (row, head) pair
-        const int blocks = (int)((4 * n_pairs + warps_per_block - 1) / warps_per_block);
-        attn_mla_combine_kernel<<<blocks, warps_per_block * 32, 0, stream>>>(
-            reinterpret_cast<const float4 *>(a.part_o), a.part_ml, (int)n_pairs, splits, a.out, a.lse);
+        const int warps_per_block = 8;  // two warps per (row, head) pair
+        const int blocks = (int)((2 * n_pairs + warps_per_block - 1) / warps_per_block);
+        attn_mla_combine_kernel<<<blocks, warps_per_block * 32, 0, stream>>>(a.part_o, a.part_ml, (int)n_pairs,
+                                                                            splits, a.out, a.lse);
         count_launch();
         err = cudaGetLastError();
     }

@@ -267,9 +267,9 @@ indexer_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             }
             // no copy may still be landing when the CTA exits
             for (int s = 0; s < kStages; ++s)
-                if (st_armed[s] >= 0 && !mbar_wait(&st_full[s], (uint32_t)st_armed[s])) ok = false;
+                if (st_armed[s] >= 0 && !mbar_drain(&st_full[s], (uint32_t)st_armed[s])) ok = false;
             for (int s = 0; s < kResBufs; ++s)
-                if (res_armed[s] >= 0 && !mbar_wait(&res_full[s], (uint32_t)res_armed[s])) ok = false;
+                if (res_armed[s] >= 0 && !mbar_drain(&res_full[s], (uint32_t)res_armed[s])) ok = false;
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -332,8 +332,10 @@ indexer_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                         idle = 0;
                     } else {
                         // bounded: give up after the wait limit without progress
+                        const unsigned long long limit = __ldg(&g_wait_limit_ns);
+                        if (limit == 0) { ok = false; break; }
                         if (idle == 0) t_idle = global_timer_ns();
-                        if ((++idle & 63u) == 0u && global_timer_ns() - t_idle > kWaitTimeoutNs) { ok = false; break; }
+                        if ((++idle & 63u) == 0u && global_timer_ns() - t_idle > limit) { ok = false; break; }
                         __nanosleep(20);
                     }
                 }
@@ -345,7 +347,7 @@ indexer_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             }
             // every MMA issued here has finished before TMEM is freed
             mma_commit(drain);
-            if (!mbar_wait(drain, 0)) ok = false;
+            if (!mbar_drain(drain, 0)) ok = false;
         }
     } else {
         // ---------------------------------------------------- epilogue
@@ -609,6 +611,8 @@ size_t part_bytes(const Params &p) {
 }
 
 }  // namespace
+
+cudaError_t indexer_bwd_set_wait_limit(unsigned long long ns) { return set_wait_limit_ns(ns); }
 
 unsigned int indexer_bwd_take_device_error() {
     unsigned int v = 0, zero = 0;

@@ -116,7 +116,7 @@ struct Cfg {
     // ahead of the epilogue), else two
     static constexpr int kAcc = 4 * N_TILE <= 512 ? 4 : 2;
     static constexpr uint32_t kTmemCols = kAcc * N_TILE;
-    static constexpr int kBars = 2 * kStages + 2 * kQBufs + 2 * kAcc;
+    static constexpr int kBars = 2 * kStages + 2 * kQBufs + 2 * kAcc + 1;
     static constexpr size_t kSmem = 1024 + (size_t)kQBufs * kQBytes + (size_t)kStages * kKBytes + kBars * 8 + 16;
     static_assert(kStages >= 2, "shared memory too small for the pipeline");
     static_assert(kTmemCols == 128 || kTmemCols == 256 || kTmemCols == 512, "TMEM columns");
@@ -138,7 +138,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     uint64_t *q_empty = q_full + C::kQBufs;
     uint64_t *acc_full = q_empty + C::kQBufs;
     uint64_t *acc_empty = acc_full + C::kAcc;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + C::kAcc);
+    uint64_t *drained = acc_empty + C::kAcc;  // MMA commit at teardown
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drained + 1);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -161,6 +162,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             mbar_init(&acc_full[s], 1);
             mbar_init(&acc_empty[s], releasers);
         }
+        mbar_init(drained, 1);
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -180,10 +182,15 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             prefetch_tensor_map(&tm_k);
             int ks = 0, qb = 0;
             uint32_t kph = 0, qph = 0;
+            // stages and query buffers armed at least once, and the parity of
+            // their last arming (drained before the CTA exits)
+            uint32_t k_armed = 0, k_par = 0, q_armed = 0, q_par = 0;
             for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
                 Unit un;
                 if (!decode_unit(u, p, un)) continue;
                 if (!mbar_wait(&q_empty[qb], qph ^ 1u)) { ok = false; break; }
+                q_armed |= 1u << qb;
+                q_par = (q_par & ~(1u << qb)) | (qph << qb);
                 mbar_arrive_expect_tx(&q_full[qb], C::kQBytes);
                 const int qrow = (un.b * p.Tq + un.i0) * p.H;
 #pragma unroll
@@ -192,6 +199,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 if (++qb == C::kQBufs) { qb = 0; qph ^= 1u; }
                 for (int kt = un.kt0; kt < un.kt1; ++kt) {
                     if (!mbar_wait(&k_empty[ks], kph ^ 1u)) { ok = false; break; }
+                    k_armed |= 1u << ks;
+                    k_par = (k_par & ~(1u << ks)) | (kph << ks);
                     mbar_arrive_expect_tx(&k_full[ks], C::kKBytes);
                     const int krow = un.b * p.L + kt * kBlockM;
 #pragma unroll
@@ -200,6 +209,12 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     if (++ks == C::kStages) { ks = 0; kph ^= 1u; }
                 }
             }
+            // every TMA load this CTA issued has landed before it exits (on
+            // the normal path these phases were consumed already)
+            for (int s = 0; s < C::kStages; ++s)
+                if (((k_armed >> s) & 1u) && !mbar_drain(&k_full[s], (k_par >> s) & 1u)) ok = false;
+            for (int s = 0; s < C::kQBufs; ++s)
+                if (((q_armed >> s) & 1u) && !mbar_drain(&q_full[s], (q_par >> s) & 1u)) ok = false;
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -241,6 +256,9 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 mma_commit(&q_empty[qb]);
                 if (++qb == C::kQBufs) { qb = 0; qph ^= 1u; }
             }
+            // no MMA of this CTA may still run when TMEM is freed
+            mma_commit(drained);
+            if (!mbar_drain(drained, 0)) ok = false;
         }
     } else {
         // ---------------------------------------------------- epilogue
@@ -396,6 +414,8 @@ cudaError_t dispatch_tc(const IndexerProblem &p, const DeviceInfo &info, cudaStr
 }
 
 }  // namespace
+
+cudaError_t indexer_set_wait_limit(unsigned long long ns) { return set_wait_limit_ns(ns); }
 
 unsigned int indexer_take_device_error() {
     unsigned int v = 0, zero = 0;

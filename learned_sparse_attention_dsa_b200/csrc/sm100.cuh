@@ -5,13 +5,29 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_runtime.h>
 #include <stdint.h>
 
 namespace dsa {
 namespace sm100 {
 
-// Bounded waits give up after this many nanoseconds of %globaltimer.
+// Bounded waits give up after this many nanoseconds of %globaltimer: the
+// default of the settable limit below, and the fixed limit of the drains at
+// teardown.
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s
+
+// Limit of the bounded waits of the kernels in the translation unit that
+// includes this header (internal linkage: one copy per unit, written by that
+// unit's set_wait_limit_ns). 0 makes every bounded wait give up at its first
+// call, even when its phase has completed, so that every role of a kernel
+// stops before it issues a copy or an MMA (the test setting of the give-up
+// path).
+static __device__ unsigned long long g_wait_limit_ns = kWaitTimeoutNs;
+
+// Host: set this translation unit's wait limit on the current device.
+static inline cudaError_t set_wait_limit_ns(unsigned long long ns) {
+    return cudaMemcpyToSymbol(g_wait_limit_ns, &ns, sizeof(ns));
+}
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -75,6 +91,20 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
 // Wait for the phase with the given parity to complete. Returns false when
 // the wait gives up (the caller records an error and winds down).
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+    const unsigned long long limit = __ldg(&g_wait_limit_ns);
+    if (limit == 0) return false;
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 15u) == 0u && global_timer_ns() - t0 > limit) return false;
+    }
+}
+
+// Teardown: wait for copies or MMAs this CTA issued to land before it frees
+// TMEM or exits, with the fixed 2 s limit (they complete on their own; the
+// limit only keeps a broken case from hanging).
+__device__ __forceinline__ bool mbar_drain(uint64_t *bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t i = 1;; ++i) {
@@ -97,6 +127,16 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t pa
     return done != 0;
 }
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity) {
+    const unsigned long long limit = __ldg(&g_wait_limit_ns);
+    if (limit == 0) return false;
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait_cluster(bar, parity)) return true;
+        if ((i & 15u) == 0u && global_timer_ns() - t0 > limit) return false;
+    }
+}
+__device__ __forceinline__ bool mbar_drain_cluster(uint64_t *bar, uint32_t parity) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t i = 1;; ++i) {

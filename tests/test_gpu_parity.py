@@ -240,6 +240,43 @@ def test_sparse_attn_reports_malformed_positions(cuda, name):
     assert torch.equal(lse_bad, lse_clean)
 
 
+def test_bounded_waits_give_up_and_report_timeout(cuda):
+    """With a wait limit of 0 every bounded wait of the tensor-core kernels
+    gives up at its first call, before its role has issued a copy or an MMA:
+    the indexer, the latent-row attention and the indexer backward return
+    without their outputs and dsa_device_error reports DSA_ERR_TIMEOUT. With
+    the default limit restored, the same calls pass parity again."""
+    wl = MEDIUM["decode_5000"]             # tensor-core indexer (one query per tile)
+    lat = MEDIUM["decode_latent_3000"]     # latent-row tensor-core attention
+    bwd = MEDIUM["heads128_prefill"]       # tensor-core indexer backward
+    _, dev = _inputs(wl)
+    binding.device_error()
+    try:
+        binding.set_wait_limit_ns(0)
+        binding.indexer_scores(dev["q_idx"], dev["k_idx"], dev["w"], wl.q_pos0)
+        with pytest.raises(binding.DSAError) as exc:
+            binding.device_error()
+        assert exc.value.status == 5  # DSA_ERR_TIMEOUT
+        _, ldev = _inputs(lat)
+        idx = torch.arange(lat.k, dtype=torch.int32, device="cuda").expand(lat.B, lat.Tq, lat.k).contiguous()
+        binding.sparse_attn(ldev["q"], ldev["k_cache"], ldev["v_cache"], idx, lat.scale)
+        with pytest.raises(binding.DSAError) as exc:
+            binding.device_error()
+        assert exc.value.status == 5
+        _, bdev = _inputs(bwd)
+        grad = torch.ones((bwd.B, bwd.Tq, bwd.L), dtype=torch.float32, device="cuda")
+        binding.indexer_backward(bdev["q_idx"], bdev["k_idx"], bdev["w"], grad, bwd.q_pos0,
+                                 dq=torch.empty((bwd.B, bwd.Tq, bwd.H_I, bwd.d_I), device="cuda"))
+        with pytest.raises(binding.DSAError) as exc:
+            binding.device_error()
+        assert exc.value.status == 5
+    finally:
+        binding.set_wait_limit_ns(binding.DEFAULT_WAIT_LIMIT_NS)
+    binding.device_error()  # cleared; nothing pending
+    _check_forward(wl, None)
+    _check_forward(lat, None)
+
+
 def test_forward_equals_stage_calls(cuda):
     wl = MEDIUM["prefill_mqa_700"]
     _, dev = _inputs(wl)

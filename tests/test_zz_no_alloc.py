@@ -72,16 +72,17 @@ def test_noalloc_matches_workspace_entry_point_twice(cuda, dsa_lib):
 
 def test_noalloc_rejects_problems_beyond_its_scratch(cuda, dsa_lib):
     _declare(dsa_lib)
-    # One sequence decoding with 128 heads over a latent row, 2048 positions
-    # selected: the selection is split 32 ways, 128*32*(512+2)*4 bytes of
-    # partials (8.4 MB) > 4 MiB. dsa_sparse_attn runs this shape with a
+    # Two sequences decoding with 128 heads over a latent row, 2048 positions
+    # selected: the selection is split 32 ways, 2*128*32*(512*2+8) bytes of
+    # partials (8.5 MB) > 4 MiB. dsa_sparse_attn runs this shape with a
     # workspace; the no-workspace entry point must refuse it.
-    B, L, k, Hq, D, Dv = 1, 3000, 2048, 128, 576, 512
+    B, L, k, Hq, D, Dv = 2, 3000, 2048, 128, 576, 512
     q = torch.zeros((B, 1, Hq, D), dtype=torch.bfloat16, device="cuda")
     kc = torch.zeros((B, L, 1, D), dtype=torch.bfloat16, device="cuda")
     vc = kc[..., :Dv]
     gen = torch.Generator().manual_seed(3)
-    idx = torch.randperm(L, generator=gen)[:k].to(torch.int32).reshape(B, 1, k).cuda()
+    idx = torch.stack([torch.randperm(L, generator=gen)[:k] for _ in range(B)]).to(torch.int32)
+    idx = idx.reshape(B, 1, k).cuda()
     out = torch.empty((B, 1, Hq, Dv), dtype=torch.bfloat16, device="cuda")
     lse = torch.empty((B, 1, Hq), dtype=torch.float32, device="cuda")
     sh = binding.attn_shape(q, kc, vc, k, D ** -0.5)
