@@ -108,11 +108,11 @@ dsa_status dsa_device_error(dsa_stream_t stream);
  * dsa_set_wait_limit_ns -- the time limit of every bounded device-side wait
  * of the library's kernels on the current device (default 2,000,000,000 ns).
  * A diagnostic with no counterpart on the pages, for testing the give-up
- * path: with ns = 0 every bounded wait gives up at its first call, so each
- * role of those kernels stops before it issues a copy or an MMA; the kernels
- * release their resources, return without their outputs and record
- * DSA_ERR_TIMEOUT (dsa_device_error). Copies and MMAs a CTA did issue are
- * always waited for before it frees tensor memory or exits.
+ * path: with ns = 0 those kernels start every role as having given up (they
+ * read the limit once at their start), so no role issues a copy or an MMA;
+ * the kernels release their resources, return without their outputs and
+ * record DSA_ERR_TIMEOUT (dsa_device_error). Copies and MMAs a CTA did issue
+ * are always waited for before it frees tensor memory or exits.
  * Call it while none of the library's kernels runs on the device (it writes
  * device variables like cudaMemcpyToSymbol). Returns DSA_ERR_CUDA if a write
  * failed.

@@ -22,8 +22,9 @@
 // An MMA of M=128, K=16 costs about the same for every N up to 64 (measured
 // on B200: ~48 cycles, ~65 for N=128, ~129 for N=256), so a tile is 64 keys.
 // TMEM: Q part [0,160), S [160,224), O [256,512). Shared memory: a three-slot
-// ring of gathered boxes (3 x 40 KB), P (16 KB), the partial-S send and
-// receive buffers (2 x 32 KB).
+// ring of gathered boxes (3 x 40 KB), P twice (2 x 16 KB), the partial-S send
+// and receive buffers (2 x 32 KB); the Q part is staged over P and those
+// buffers before the first tile, so the ring gathers from the start.
 //
 // Per CTA (one per SM):
 //   warps 0-7  softmax, two warps per TMEM lane quarter: warp w takes heads
@@ -37,12 +38,16 @@
 //              agree on the tile's row max through shared memory; the online
 //              softmax keeps a reference max that moves only when the row max
 //              grows by more than 2^8 (then O is rescaled in TMEM); P goes to
-//              shared memory in bf16 (128-byte swizzle). At the end O leaves
-//              TMEM for the output or for a bf16 partial normalised by its
-//              own sum.
-//   warps 8-10 gather the 5 boxes of 64 selected rows per tile with 16-byte
-//              cp.async (one warp instruction fills 4 rows x 128 bytes).
-//   warp 11    TMEM allocation, the Q staging by TMA, and one thread issuing
+//              shared memory in bf16 (128-byte swizzle), alternating
+//              between two buffers so that the softmax of tile t + 1 does not
+//              wait for PV of tile t (only a rescale of O does). At the end O
+//              leaves TMEM for the output or for a bf16 partial normalised by
+//              its own sum.
+//   warps 8-14 gather the 5 boxes of 64 selected rows per tile with 16-byte
+//              cp.async (one warp instruction fills 4 rows x 128 bytes); the
+//              rate at which cp.async is issued grows with the number of
+//              issuing warps (measured on B200: ~22 GB/s per SM with three).
+//   warp 15    TMEM allocation, the Q staging by TMA, and one thread issuing
 //              the MMAs with descriptors built once.
 // With several splits, attn_mla_combine_kernel merges the partials.
 // Every mbarrier wait is bounded; on a timeout the CTA records an error word,
@@ -77,17 +82,17 @@ constexpr int kMaxSplits = 32;
 constexpr int kSlots = 3;
 constexpr int kSoftWarps = 8;
 constexpr int kSoftmaxThreads = kSoftWarps * 32;   // 256
-constexpr int kGatherThreads = 96;
-constexpr int kMmaWarp = (kSoftmaxThreads + kGatherThreads) / 32;  // 11
-constexpr int kThreads = (kMmaWarp + 1) * 32;                      // 384
+constexpr int kGatherThreads = 224;
+constexpr int kMmaWarp = (kSoftmaxThreads + kGatherThreads) / 32;  // 15
+constexpr int kThreads = (kMmaWarp + 1) * 32;                      // 512
 constexpr uint32_t kQBox = kHeads * 128;           // 16,384
 constexpr uint32_t kKBox = kTileN * 128;           // 8,192
 constexpr uint32_t kKSlot = kGBoxes * kKBox;       // 40,960
 constexpr uint32_t kPBytes = kHeads * kTileN * 2;  // 16,384
 constexpr uint32_t kXBytes = kHeads * kTileN * 4;  // 32,768: one partial S tile
 constexpr uint32_t kXWarpBytes = kXBytes / kSoftWarps;  // 4,096: one warp's 32 heads x 32 keys
-constexpr uint32_t kOffP = kSlots * kKSlot;
-constexpr uint32_t kOffXs = kOffP + kPBytes;       // this part's S_p, sent to the other part
+constexpr uint32_t kOffP = kSlots * kKSlot;        // P, two buffers; the Q staging from here on
+constexpr uint32_t kOffXs = kOffP + 2 * kPBytes;   // this part's S_p, sent to the other part
 constexpr uint32_t kOffXr = kOffXs + kXBytes;      // the other part's S_p, received
 constexpr uint32_t kOffSel = kOffXr + kXBytes;
 constexpr uint32_t kOffMx = kOffSel + kMaxSel * 4;          // [tile parity][key half][head] row maxima
@@ -95,7 +100,7 @@ constexpr uint32_t kOffL = kOffMx + 2 * 2 * kHeads * 4;     // [key half][head] 
 constexpr uint32_t kOffCnt = kOffL + 2 * kHeads * 4;        // [warp] S_p blocks the other part sent here
 constexpr uint32_t kOffBar = kOffCnt + kSoftWarps * 4;
 constexpr uint32_t kHalfRowBytes = kHalfDv * 2;             // one head's bf16 partial of a part
-constexpr int kNumBars = 17 + 2 * kSoftWarps;
+constexpr int kNumBars = 19 + 2 * kSoftWarps;
 constexpr size_t kSmem = 1024 + kOffBar + kNumBars * 8 + 16;  // + slack to align the base to 1024
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColQ = 0;
@@ -106,7 +111,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kIdescMnMajorB = 1u << 16;
 
 static_assert(kOffP % 1024 == 0 && kKSlot % 1024 == 0, "operand tiles must sit on 1024-byte boundaries");
-static_assert(5 * kQBox <= 2 * kKSlot, "the Q staging must fit over ring slots 0 and 1");
+static_assert(5 * kQBox <= kOffSel - kOffP, "the Q staging must fit over P and the S_p buffers");
 static_assert(kHeads * kHalfRowBytes <= kOffXs, "the partial staging must fit over the ring and P");
 static_assert(kOffBar % 8 == 0, "mbarrier alignment");
 static_assert(kColS + kTileN <= kColO, "TMEM columns");
@@ -128,7 +133,7 @@ struct Args {
     int64_t sb, ss;
     __nv_bfloat16 *out;       // [rows, 128, 512]
     float *lse;               // [rows, 128] or null
-    uint4 *part_o;            // split partials (splits > 1), bf16, see attn_mla_tc_workspace_bytes
+    uint4 *part_o;            // split partials (splits > 1), bf16 [rows, splits, 2, 128, 256]
     float *part_ml;           // [rows, 128, splits, 2]: (max in log2 units, sum)
 };
 
@@ -187,16 +192,19 @@ attn_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Args a) {
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
     uint64_t *q_full = bars;            // TMA bytes of the staged Q part
     uint64_t *q_copied = bars + 1;      // 256 softmax threads: Q part in TMEM, staging free
-    uint64_t *kv_full = bars + 2;       // [3] 96 gather threads (cp.async arrivals)
+    uint64_t *kv_full = bars + 2;       // [3] gather threads (cp.async arrivals)
     uint64_t *kv_empty = bars + 5;      // [3] MMA commit after PV
     uint64_t *s_full = bars + 8;        // MMA commit after QK^T
     uint64_t *s_free = bars + 9;        // 256 softmax threads (S_p is in registers)
-    uint64_t *p_full = bars + 10;       // 256 softmax threads
-    uint64_t *pv_done = bars + 11;      // MMA commit after PV
-    uint64_t *drained = bars + 12;      // MMA commit before teardown
-    uint64_t *mx_bar = bars + 13;       // [4] the two warps of a lane quarter posted their row maxima
-    uint64_t *x_full = bars + 17;       // [8] the other part's block of S_p for warp w landed
-    uint64_t *x_free = bars + 17 + kSoftWarps;  // [8] the other part's warp w read what we sent
+    uint64_t *p_full = bars + 10;       // [2] 256 softmax threads: P buffer b written
+    uint64_t *pv_done = bars + 12;      // [2] MMA commit after PV from P buffer b
+    uint64_t *drained = bars + 14;      // MMA commit before teardown
+    uint64_t *mx_bar = bars + 15;       // [4] the two warps of a lane quarter posted their row maxima
+    uint64_t *x_full = bars + 19;       // [8] the other part's block of S_p for warp w landed
+    // [8] the other part's warp w may be sent its next block: phase 0 once
+    // its receive buffer no longer holds the Q staging, phase t + 1 once it
+    // has read block t
+    uint64_t *x_free = bars + 19 + kSoftWarps;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kNumBars);
 
     const int row = blockIdx.x;
@@ -230,8 +238,10 @@ attn_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Args a) {
         }
         mbar_init(s_full, 1);
         mbar_init(s_free, kSoftmaxThreads);
-        mbar_init(p_full, kSoftmaxThreads);
-        mbar_init(pv_done, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&p_full[i], kSoftmaxThreads);
+            mbar_init(&pv_done[i], 1);
+        }
         mbar_init(drained, 1);
         for (int i = 0; i < 4; ++i) mbar_init(&mx_bar[i], 64);
         for (int w = 0; w < kSoftWarps; ++w) {
@@ -250,62 +260,76 @@ attn_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Args a) {
     cg::this_cluster().sync();  // both parts' barriers exist before any remote arrival or copy
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    bool ok = true;
+    bool ok = waits_enabled();  // false: the wait limit is 0 (give-up test)
     float m_ref = -INFINITY, l = 0.0f;  // softmax threads: reference max (log2 units), partial sum
     uint32_t sent = 0, recv = 0;        // softmax threads: S_p blocks sent to / received from the other part
 
-    // Tile t lands in ring slot (t + 2) % 3 (its (t / 3)-th use): slots 0-1
-    // first hold the Q staging, so tiles 1 and 2 wait for the copy to TMEM.
+    // Tile t lands in ring slot t % 3 (its (t / 3)-th use) and its P in
+    // buffer t % 2.
     if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
-        // a wait limit of 0 gives up here, before the first copy is issued
-        if (lane == 0 && n_tiles > 0 && __ldg(&g_wait_limit_ns) == 0) ok = false;
         if (lane == 0 && n_tiles > 0 && ok) {
             prefetch_tensor_map(&tm_q);
             mbar_arrive_expect_tx(q_full, (uint32_t)q_boxes(part) * kQBox);
 #pragma unroll 1
             for (int c = 0; c < q_boxes(part); ++c)
-                tma_load_2d(smem + c * kQBox, &tm_q, q_full, (q_box0(part) + c) * 64, row * kHeads);
+                tma_load_2d(smem + kOffP + c * kQBox, &tm_q, q_full, (q_box0(part) + c) * 64, row * kHeads);
             ok = mbar_wait(q_copied, 0);
             tc_fence_after();
             const uint32_t idesc_qk = idesc_bf16_f32(kHeads, kTileN);
             const uint32_t idesc_pv = idesc_bf16_f32(kHeads, kHalfDv) | kIdescMnMajorB;
-            const uint64_t p_desc = smem_desc_k_sw128(smem_addr(p_sm));
+            const uint64_t p_desc0 = smem_desc_k_sw128(smem_addr(p_sm));
             // QK^T reads local boxes [q_box0 - g_box0, +q_boxes); PV local boxes 0-3
             const uint64_t k_desc0 =
                 smem_desc_k_sw128(smem_addr(k_sm) + (uint32_t)(q_box0(part) - g_box0(part)) * kKBox);
             const uint64_t v_desc0 = smem_desc_mn_sw128(smem_addr(k_sm), kKBox);
-            auto issue_pv = [&](int u) -> bool {
-                if (!mbar_wait(p_full, (uint32_t)(u & 1))) return false;
-                tc_fence_after();
-                const int slot = (u + 2) % kSlots;
-                const uint64_t vd = v_desc0 + desc_step((uint32_t)slot * kKSlot);
-#pragma unroll
-                for (int kk = 0; kk < kTileN / 16; ++kk)  // 16 keys = two 8-row groups = 2048 bytes
-                    mma_f16_ss(tmem + kColO, p_desc + desc_step(kk * 32), vd + desc_step(kk * 2048), idesc_pv,
-                               (u > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(&kv_empty[slot]);  // the slot may be refilled
-                mma_commit(pv_done);          // P may be rewritten, O is current
-                return true;
-            };
-            for (int t = 0; ok && t < n_tiles; ++t) {
-                const int slot = (t + 2) % kSlots;
-                if (!mbar_wait(&kv_full[slot], (uint32_t)(t / kSlots) & 1u) ||
-                    !mbar_wait(s_free, ((uint32_t)t & 1u) ^ 1u)) {
-                    ok = false;
-                    break;
+            // Two streams of MMAs, each issued as soon as its inputs are ready:
+            // QK^T of the next tile (its rows landed, the previous S_p read
+            // out of TMEM) and PV of the oldest tile whose P is written. QK^T
+            // of tile t + 1 is needed before the softmax of tile t finishes
+            // (its S_p block is sent first), so it must not wait behind PV.
+            int nq = 0, np = 0;
+            uint32_t idle = 0;
+            uint64_t t_idle = 0;
+            while (ok && np < n_tiles) {
+                bool progress = false;
+                if (nq < n_tiles && mbar_test_wait(&kv_full[nq % kSlots], (uint32_t)(nq / kSlots) & 1u) &&
+                    mbar_test_wait(s_free, ((uint32_t)nq & 1u) ^ 1u)) {
+                    fence_proxy_async_smem();  // the rows were written by cp.async
+                    tc_fence_after();
+                    const uint64_t kd = k_desc0 + desc_step((uint32_t)(nq % kSlots) * kKSlot);
+                    if (part == 0)
+                        issue_qk<5>(tmem + kColS, tmem + kColQ, kd, idesc_qk);
+                    else
+                        issue_qk<4>(tmem + kColS, tmem + kColQ, kd, idesc_qk);
+                    mma_commit(s_full);
+                    ++nq;
+                    progress = true;
                 }
-                fence_proxy_async_smem();  // the rows were written by cp.async
-                tc_fence_after();
-                const uint64_t kd = k_desc0 + desc_step((uint32_t)slot * kKSlot);
-                if (part == 0)
-                    issue_qk<5>(tmem + kColS, tmem + kColQ, kd, idesc_qk);
-                else
-                    issue_qk<4>(tmem + kColS, tmem + kColQ, kd, idesc_qk);
-                mma_commit(s_full);
-                if (t > 0 && !issue_pv(t - 1)) ok = false;
+                if (np < nq && mbar_test_wait(&p_full[np & 1], (uint32_t)(np >> 1) & 1u)) {
+                    tc_fence_after();
+                    const int slot = np % kSlots;
+                    const uint64_t vd = v_desc0 + desc_step((uint32_t)slot * kKSlot);
+                    const uint64_t pd = p_desc0 + desc_step((uint32_t)(np & 1) * kPBytes);
+#pragma unroll
+                    for (int kk = 0; kk < kTileN / 16; ++kk)  // 16 keys = two 8-row groups = 2048 bytes
+                        mma_f16_ss(tmem + kColO, pd + desc_step(kk * 32), vd + desc_step(kk * 2048), idesc_pv,
+                                   (np > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(&kv_empty[slot]);   // the slot may be refilled
+                    mma_commit(&pv_done[np & 1]);  // P buffer np % 2 may be rewritten; O holds every PV so far
+                    ++np;
+                    progress = true;
+                }
+                if (progress) {
+                    idle = 0;
+                } else {
+                    // bounded: give up after the wait limit without progress
+                    const unsigned long long limit = __ldg(&g_wait_limit_ns);
+                    if (idle == 0) t_idle = global_timer_ns();
+                    if ((++idle & 63u) == 0u && global_timer_ns() - t_idle > limit) ok = false;
+                    __nanosleep(32);
+                }
             }
-            if (ok) ok = issue_pv(n_tiles - 1);
             // nothing of this CTA may still run on the tensor core at teardown,
             // and the Q load has landed
             mma_commit(drained);
@@ -318,9 +342,8 @@ attn_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Args a) {
         const __nv_bfloat16 *kvb = a.kv + (int64_t)b * a.sb + g_box0(part) * 64;
         const uint32_t k_base = smem_addr(k_sm);
         for (int t = 0; t < n_tiles; ++t) {
-            const int slot = (t + 2) % kSlots;
-            if ((t == 1 || t == 2) && !mbar_wait(q_copied, 0)) ok = false;
-            if (ok && !mbar_wait(&kv_empty[slot], ((uint32_t)(t / kSlots) & 1u) ^ 1u)) ok = false;
+            const int slot = t % kSlots;
+            if (!mbar_wait(&kv_empty[slot], ((uint32_t)(t / kSlots) & 1u) ^ 1u)) ok = false;
             if (!ok) break;
             const uint32_t dst0 = k_base + (uint32_t)slot * kKSlot;
             // chunk c: local box c / 512, row (c / 8) % 64, 16-byte chunk c % 8
@@ -359,7 +382,7 @@ attn_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Args a) {
             if (!mbar_wait(q_full, 0)) ok = false;
             if (__all_sync(0xffffffffu, ok)) {
                 for (int c = kh; c < q_boxes(part); c += 2) {  // warp-uniform trip count
-                    const uint8_t *box = smem + c * kQBox + h * 128;
+                    const uint8_t *box = smem + kOffP + c * kQBox + h * 128;
                     uint32_t w[32];
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
@@ -370,15 +393,19 @@ attn_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Args a) {
                 }
                 tmem_st_wait();
             }
-            fence_proxy_async_smem();  // the staging is overwritten by the gathers next
+            fence_proxy_async_smem();  // the staging is overwritten by P and the S_p blocks next
             tc_fence_before();
             mbar_arrive(q_copied);
+            // every warp has copied its boxes: P and the send buffer may be
+            // written, and the other part may send into the receive buffer
+            if (ok && !mbar_wait(q_copied, 0)) ok = false;
+            if (lane == 0) mbar_arrive_remote(peer_x_free);
         }
         ok = __all_sync(0xffffffffu, ok);
 
         // S_p of tile t (this warp's 32 keys) out of TMEM into registers
         auto load_sp = [&](int t, uint32_t *v) -> bool {
-            if (!mbar_wait(s_full, (uint32_t)t & 1u)) return false;
+            if (!mbar_spin(s_full, (uint32_t)t & 1u)) return false;
             tc_fence_after();
             tmem_ld_32x32b_x32(tmem + lane_addr + kColS + (uint32_t)(kh * 32), v);
             tmem_ld_wait();
@@ -386,8 +413,11 @@ attn_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Args a) {
             mbar_arrive(s_free);  // the next QK^T may overwrite S_p
             return true;
         };
-        // send this warp's block of S_p to the same warp of the other part
-        auto send_sp = [&](const uint32_t *v) {
+        // this warp's block of S_p of tile t to the same warp of the other
+        // part, once that warp may be sent block t (x_free phase t); the block
+        // stays in the send buffer, where this warp reads it back
+        auto send_sp = [&](int t, const uint32_t *v) -> bool {
+            if (!mbar_spin_cluster(&x_free[warp], (uint32_t)t & 1u)) return false;
 #pragma unroll
             for (int c = 0; c < 8; ++c)
                 xs_row[(c + lane) & 7] = make_float4(__uint_as_float(v[4 * c]), __uint_as_float(v[4 * c + 1]),
@@ -396,40 +426,39 @@ attn_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Args a) {
             __syncwarp();
             if (lane == 0) bulk_copy_to_cluster(peer_xr_blk, xs_sm + blk, kXWarpBytes, peer_x_full);
             ++sent;
+            return true;
         };
 
-        uint32_t x[32], y[32];
+        uint32_t x[32];
         if (ok && n_tiles > 0) {
-            if (!load_sp(0, x)) ok = false;
+            if (!load_sp(0, x) || !send_sp(0, x)) ok = false;
             ok = __all_sync(0xffffffffu, ok);
-            if (ok) send_sp(x);
         }
         for (int t = 0; ok && t < n_tiles; ++t) {
             // the other part's block of S_p for tile t: S = S_0 + S_1
-            if (!mbar_wait_cluster(&x_full[warp], (uint32_t)t & 1u)) ok = false;
+            if (!mbar_spin_cluster(&x_full[warp], (uint32_t)t & 1u)) ok = false;
             if (!__all_sync(0xffffffffu, ok)) break;
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
+                const float4 u = xs_row[(c + lane) & 7];
                 const float4 v = xr_row[(c + lane) & 7];
-                x[4 * c] = __float_as_uint(__uint_as_float(x[4 * c]) + v.x);
-                x[4 * c + 1] = __float_as_uint(__uint_as_float(x[4 * c + 1]) + v.y);
-                x[4 * c + 2] = __float_as_uint(__uint_as_float(x[4 * c + 2]) + v.z);
-                x[4 * c + 3] = __float_as_uint(__uint_as_float(x[4 * c + 3]) + v.w);
+                x[4 * c] = __float_as_uint(u.x + v.x);
+                x[4 * c + 1] = __float_as_uint(u.y + v.y);
+                x[4 * c + 2] = __float_as_uint(u.z + v.z);
+                x[4 * c + 3] = __float_as_uint(u.w + v.w);
             }
             ++recv;
-            __syncwarp();  // every lane has read the block
+            __syncwarp();  // every lane has read both blocks
             if (lane == 0 && t + 1 < n_tiles) {
                 mbar_arrive_expect_tx(&x_full[warp], kXWarpBytes);  // armed for the next block
                 mbar_arrive_remote(peer_x_free);                    // the other part may send it
             }
             // the next tile's S_p goes out now, so that its swap runs under
-            // this tile's softmax; the send buffer is free again once the
-            // other part has read this tile's block
+            // this tile's softmax
             if (t + 1 < n_tiles) {
-                if (!load_sp(t + 1, y)) ok = false;
-                if (ok && !mbar_wait_cluster(&x_free[warp], (uint32_t)t & 1u)) ok = false;
+                uint32_t y[32];
+                if (!load_sp(t + 1, y) || !send_sp(t + 1, y)) ok = false;
                 if (!__all_sync(0xffffffffu, ok)) break;
-                send_sp(y);
             }
 
             // scale, mask entries that are padding, this half's max
@@ -452,12 +481,12 @@ attn_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Args a) {
             }
             // the row max over both key halves: each warp of the lane quarter
             // posts its half's max (double-buffered by tile) and waits for the
-            // other's on a bounded barrier. PV of the previous tile must be
-            // done before P is rewritten or O rescaled.
+            // other's on a bounded barrier
             mx_sm[((t & 1) * 2 + kh) * kHeads + h] = mt;
             mbar_arrive(&mx_bar[quarter]);
-            if (!mbar_wait(&mx_bar[quarter], (uint32_t)t & 1u)) ok = false;
-            if (t > 0 && ok && !mbar_wait(pv_done, (uint32_t)(t - 1) & 1u)) ok = false;
+            if (!mbar_spin(&mx_bar[quarter], (uint32_t)t & 1u)) ok = false;
+            // P buffer t % 2 was last read by PV of tile t - 2
+            if (t >= 2 && ok && !mbar_wait(&pv_done[t & 1], (uint32_t)((t - 2) >> 1) & 1u)) ok = false;
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
@@ -473,6 +502,10 @@ attn_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Args a) {
                 }
             }
             if (__any_sync(0xffffffffu, grow)) {  // tcgen05.ld/st are warp-wide
+                // O may be rescaled once every PV so far (through tile t - 1) is done
+                if (!mbar_wait(&pv_done[(t - 1) & 1], (uint32_t)((t - 1) >> 1) & 1u)) ok = false;
+                if (!__all_sync(0xffffffffu, ok)) break;
+                tc_fence_after();
                 const float f = grow ? exp2f(m_ref - m_new) : 1.0f;
 #pragma unroll 1
                 for (int c = kh * (kHalfDv / 2); c < (kh + 1) * (kHalfDv / 2); c += 32) {
@@ -501,20 +534,20 @@ attn_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Args a) {
                 pk[j] = pack_bf16x2(p0, p1);
             }
             l += ps0 + ps1;
-            // P row h: 128 bytes, 16-byte chunk c at chunk c ^ (h % 8); this
-            // warp's keys are chunks 4 kh .. 4 kh + 3
-            uint8_t *prow = p_sm + h * 128;
+            // P row h of buffer t % 2: 128 bytes, 16-byte chunk c at chunk
+            // c ^ (h % 8); this warp's keys are chunks 4 kh .. 4 kh + 3
+            uint8_t *prow = p_sm + (t & 1) * kPBytes + h * 128;
 #pragma unroll
             for (int c = 0; c < 4; ++c)
                 *reinterpret_cast<uint4 *>(prow + (((4 * kh + c) ^ (h & 7)) << 4)) =
                     make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
             fence_proxy_async_smem();  // P is read by the tensor core
             tc_fence_before();
-            mbar_arrive(p_full);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) x[j] = y[j];
+            mbar_arrive(&p_full[t & 1]);
         }
-        if (ok && n_tiles > 0 && !mbar_wait(pv_done, (uint32_t)(n_tiles - 1) & 1u)) ok = false;
+        if (ok && n_tiles > 0 &&
+            !mbar_wait(&pv_done[(n_tiles - 1) & 1], (uint32_t)((n_tiles - 1) >> 1) & 1u))
+            ok = false;
         ok = __all_sync(0xffffffffu, ok);
         l_sm[kh * kHeads + h] = l;
     }
@@ -579,19 +612,22 @@ attn_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Args a) {
             if (part == 0 && kh == 0 && a.lse != nullptr)
                 a.lse[pair] = l_all > 0.0f ? (m_ref + log2f(l_all)) / kLog2e : -INFINITY;
         } else {
-            // the head's half row of partials, normalised by its own sum, once
-            // both warps of the lane quarter have staged their columns (every
-            // softmax thread gets here: cta_ok is the same for the whole CTA)
+            if (part == 0 && kh == 0) {
+                a.part_ml[(pair * a.splits + split) * 2 + 0] = m_ref;
+                a.part_ml[(pair * a.splits + split) * 2 + 1] = l_all;
+            }
+            // this part's partials of all 128 heads, normalised by their own
+            // sums, are one contiguous 64 KB block: one bulk copy once every
+            // softmax thread has staged its columns (a bulk copy costs about
+            // the same per operation up to several KB, so one large copy
+            // instead of one per head; every softmax thread gets here, since
+            // cta_ok is the same for the whole CTA)
             fence_proxy_async_smem();
-            asm volatile("bar.sync %0, 64;" ::"r"(1 + quarter) : "memory");
-            if (kh == 0) {
-                bulk_store(a.part_o + (pair * a.splits + split) * (DV / 8) + part * (kHalfDv / 8), stage,
-                           kHalfRowBytes);
+            asm volatile("bar.sync 1, %0;" ::"n"(kSoftmaxThreads) : "memory");
+            if (threadIdx.x == 0) {
+                bulk_store(a.part_o + (((size_t)row * a.splits + split) * 2 + part) * (kHeads * kHalfRowBytes / 16),
+                           smem, kHeads * kHalfRowBytes);
                 bulk_commit();
-                if (part == 0) {
-                    a.part_ml[(pair * a.splits + split) * 2 + 0] = m_ref;
-                    a.part_ml[(pair * a.splits + split) * 2 + 1] = l_all;
-                }
                 bulk_wait_read();  // the staging must outlive the copy's reads
             }
         }
@@ -631,7 +667,10 @@ __global__ void attn_mla_combine_kernel(const uint4 *__restrict__ part_o, const 
     const float f_s = (m_all == -INFINITY || lane >= splits) ? 0.0f : l_s * ex2_approx(m_s - m_all);
     const float l_all = warp_sum(f_s);
     const float inv = l_all > 0.0f ? 1.0f / l_all : 0.0f;
-    const uint4 *po = part_o + (size_t)pair * splits * (DV / 8) + half * (kHalfDv / 8) + rot_chunk(h, lane);
+    const int row = pair / kHeads;
+    // chunk rot_chunk(h, lane) of head h's half row `half` in split sp:
+    // part_o[row][sp][half][h][32 chunks]
+    const uint4 *po = part_o + (((size_t)row * splits) * 2 + half) * (kHeads * 32) + h * 32 + rot_chunk(h, lane);
     float acc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
@@ -639,7 +678,7 @@ __global__ void attn_mla_combine_kernel(const uint4 *__restrict__ part_o, const 
     for (int sp = 0; sp < splits; ++sp) {
         const float f = __shfl_sync(0xffffffffu, f_s, sp);
         float e8[8];
-        bf16x8_to_f32(po[(size_t)sp * (DV / 8)], e8);
+        bf16x8_to_f32(po[(size_t)sp * 2 * (kHeads * 32)], e8);
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[e] = fmaf(f, e8[e], acc[e]);
     }
@@ -695,10 +734,9 @@ bool attn_mla_tc_supported(const AttnProblem &p) {
     return info.cc_major == 10 && (size_t)info.max_smem_optin >= kSmem;
 }
 
-// Split partials: bf16 [rows, 128, splits, 512], each head's two half rows
-// (one per part) with their 16-byte chunks rotated by the head and normalised
-// by the split's own sum; then fp32 (max in log2 units, sum) [rows, 128,
-// splits, 2].
+// Split partials: bf16 [rows, splits, 2 parts, 128 heads, 256], each head's
+// half row with its 16-byte chunks rotated by the head and normalised by the
+// split's own sum; then fp32 (max in log2 units, sum) [rows, 128, splits, 2].
 size_t attn_mla_tc_workspace_bytes(const AttnProblem &p, int sm_count) {
     const int splits = mla_tc_splits(p, sm_count);
     if (splits <= 1) return 0;

@@ -135,26 +135,11 @@ attn_mma_kernel(const Args a) {
     const int h0 = hgroup * kHeads;
     const int g = h0 / (a.Hq / a.Hkv);
 
-    // ---- Q fragments (A operand, 16 heads x DQK) straight from global memory
-    uint32_t qf[DQK / 16][4];
-    {
-        const int hr = lane >> 2, kc = (lane & 3) * 2;
-        const __nv_bfloat16 *q0 = a.q + ((size_t)row * a.Hq + h0 + hr) * DQK;
-        const __nv_bfloat16 *q8 = q0 + 8 * DQK;
-#pragma unroll
-        for (int kk = 0; kk < DQK / 16; ++kk) {
-            qf[kk][0] = *reinterpret_cast<const uint32_t *>(q0 + kk * 16 + kc);
-            qf[kk][1] = *reinterpret_cast<const uint32_t *>(q8 + kk * 16 + kc);
-            qf[kk][2] = *reinterpret_cast<const uint32_t *>(q0 + kk * 16 + 8 + kc);
-            qf[kk][3] = *reinterpret_cast<const uint32_t *>(q8 + kk * 16 + 8 + kc);
-        }
-    }
-
-    // ---- compact this split's valid selected positions (order kept)
+    // ---- this split's selected positions first: the gathers wait for them.
+    // When every entry is a position in [0, L) (decode) they are used as
+    // they are; otherwise the valid ones are compacted (order kept).
     const int j0 = split * a.per_split;
     const int j1 = min(a.k, j0 + a.per_split);
-    if (threadIdx.x == 0) s_count = 0;
-    __syncthreads();
     {
         __shared__ int warp_base[kWarps];
         // all of this split's entries are loaded up front: one memory latency
@@ -165,25 +150,41 @@ attn_mma_kernel(const Args a) {
             const int j = j0 + it * kThreads + threadIdx.x;
             sv[it] = j < j1 ? __ldg(a.idx + (size_t)row * a.k + j) : -1;
         }
-        int base = 0;
+        bool mine_valid = true;
 #pragma unroll
         for (int it = 0; it < kIters; ++it) {
-            if (j0 + it * kThreads >= j1) break;  // uniform
-            const int s = sv[it];
-            note_bad_index(&g_attn_tc_error, s, a.L);
-            const bool valid = s >= 0 && s < a.L;
-            const unsigned m = __ballot_sync(0xffffffffu, valid);
-            if (lane == 0) warp_base[warp] = __popc(m);
-            __syncthreads();
-            int off = base;
-            for (int w = 0; w < warp; ++w) off += warp_base[w];
-            if (valid) sel[off + __popc(m & ((1u << lane) - 1u))] = s;
-            int tot = 0;
-            for (int w = 0; w < kWarps; ++w) tot += warp_base[w];
-            base += tot;
-            __syncthreads();
+            if (j0 + it * kThreads + (int)threadIdx.x < j1) {
+                note_bad_index(&g_attn_tc_error, sv[it], a.L);
+                mine_valid = mine_valid && sv[it] >= 0 && sv[it] < a.L;
+            }
         }
-        if (threadIdx.x == 0) s_count = base;
+        if (__syncthreads_and(mine_valid ? 1 : 0)) {
+#pragma unroll
+            for (int it = 0; it < kIters; ++it) {
+                const int j = it * kThreads + threadIdx.x;
+                if (j0 + j < j1) sel[j] = sv[it];
+            }
+            if (threadIdx.x == 0) s_count = j1 - j0;
+        } else {
+            int base = 0;
+#pragma unroll
+            for (int it = 0; it < kIters; ++it) {
+                if (j0 + it * kThreads >= j1) break;  // uniform
+                const int s = sv[it];
+                const bool valid = s >= 0 && s < a.L;
+                const unsigned m = __ballot_sync(0xffffffffu, valid);
+                if (lane == 0) warp_base[warp] = __popc(m);
+                __syncthreads();
+                int off = base;
+                for (int w = 0; w < warp; ++w) off += warp_base[w];
+                if (valid) sel[off + __popc(m & ((1u << lane) - 1u))] = s;
+                int tot = 0;
+                for (int w = 0; w < kWarps; ++w) tot += warp_base[w];
+                base += tot;
+                __syncthreads();
+            }
+            if (threadIdx.x == 0) s_count = base;
+        }
     }
     __syncthreads();
     const int n_sel = s_count;
@@ -227,6 +228,22 @@ attn_mma_kernel(const Args a) {
     for (int st = 0; st < C::kStages - 1; ++st) {
         if (st < n_tiles) issue_tile(st, st);
         cp_async_commit();
+    }
+
+    // ---- Q fragments (A operand, 16 heads x DQK) straight from global
+    // memory, while the first tiles are in flight
+    uint32_t qf[DQK / 16][4];
+    {
+        const int hr = lane >> 2, kc = (lane & 3) * 2;
+        const __nv_bfloat16 *q0 = a.q + ((size_t)row * a.Hq + h0 + hr) * DQK;
+        const __nv_bfloat16 *q8 = q0 + 8 * DQK;
+#pragma unroll
+        for (int kk = 0; kk < DQK / 16; ++kk) {
+            qf[kk][0] = *reinterpret_cast<const uint32_t *>(q0 + kk * 16 + kc);
+            qf[kk][1] = *reinterpret_cast<const uint32_t *>(q8 + kk * 16 + kc);
+            qf[kk][2] = *reinterpret_cast<const uint32_t *>(q0 + kk * 16 + 8 + kc);
+            qf[kk][3] = *reinterpret_cast<const uint32_t *>(q8 + kk * 16 + 8 + kc);
+        }
     }
 
     for (int tile = 0; tile < n_tiles; ++tile) {

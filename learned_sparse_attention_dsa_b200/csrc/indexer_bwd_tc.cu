@@ -225,7 +225,7 @@ indexer_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    bool ok = true;
+    bool ok = waits_enabled();  // false: the wait limit is 0 (give-up test)
 
     if (warp == 0) {
         if (lane == 0) {

@@ -18,11 +18,15 @@ constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s
 
 // Limit of the bounded waits of the kernels in the translation unit that
 // includes this header (internal linkage: one copy per unit, written by that
-// unit's set_wait_limit_ns). 0 makes every bounded wait give up at its first
-// call, even when its phase has completed, so that every role of a kernel
-// stops before it issues a copy or an MMA (the test setting of the give-up
-// path).
+// unit's set_wait_limit_ns). It is read only once a wait has to poll, so the
+// waits that find their phase complete cost no extra load. 0 is the test
+// setting of the give-up path: the kernels start every role as having given
+// up (waits_enabled), so no role issues a copy or an MMA, and a wait that has
+// to poll gives up at once.
 static __device__ unsigned long long g_wait_limit_ns = kWaitTimeoutNs;
+
+// The initial state of a kernel role: false when the wait limit is 0.
+__device__ __forceinline__ bool waits_enabled() { return __ldg(&g_wait_limit_ns) != 0; }
 
 // Host: set this translation unit's wait limit on the current device.
 static inline cudaError_t set_wait_limit_ns(unsigned long long ns) {
@@ -91,9 +95,9 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
 // Wait for the phase with the given parity to complete. Returns false when
 // the wait gives up (the caller records an error and winds down).
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long limit = __ldg(&g_wait_limit_ns);
     if (limit == 0) return false;
-    if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
@@ -127,13 +131,47 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t pa
     return done != 0;
 }
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
     const unsigned long long limit = __ldg(&g_wait_limit_ns);
     if (limit == 0) return false;
-    if (mbar_try_wait_cluster(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait_cluster(bar, parity)) return true;
         if ((i & 15u) == 0u && global_timer_ns() - t0 > limit) return false;
+    }
+}
+// Polling variants for waits on a latency-critical path: the thread keeps
+// testing instead of suspending, so it resumes as soon as the phase completes
+// (bounded by the same limit).
+__device__ __forceinline__ bool mbar_test_wait_cluster(uint64_t *bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+__device__ __forceinline__ bool mbar_spin(uint64_t *bar, uint32_t parity) {
+    if (mbar_test_wait(bar, parity)) return true;
+    const unsigned long long limit = __ldg(&g_wait_limit_ns);
+    if (limit == 0) return false;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_test_wait(bar, parity)) return true;
+        if ((i & 63u) == 0u && global_timer_ns() - t0 > limit) return false;
+    }
+}
+__device__ __forceinline__ bool mbar_spin_cluster(uint64_t *bar, uint32_t parity) {
+    if (mbar_test_wait_cluster(bar, parity)) return true;
+    const unsigned long long limit = __ldg(&g_wait_limit_ns);
+    if (limit == 0) return false;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_test_wait_cluster(bar, parity)) return true;
+        if ((i & 63u) == 0u && global_timer_ns() - t0 > limit) return false;
     }
 }
 __device__ __forceinline__ bool mbar_drain_cluster(uint64_t *bar, uint32_t parity) {
