@@ -453,7 +453,12 @@ def measure_forward(wl, args, binding, device, world, rank, local, peaks):
              "note": "one dsa_forward call per step from Python, no graph"}
 
     # per-stage timing (same stream, separate loops) for the roofline
-    stages = stage_timings(wl, dev, binding, stream, max(3, min(args.steps, 50)))
+    # the L2-served prefill gathers (large selections over a KV cache that fits
+    # in L2) are also compared with the gather of the same rows alone
+    kv_row = wl.Hkv * (wl.Dqk + (0 if wl.kv_alias else wl.Dv)) * (4 if wl.dtype == "f32" else 2)
+    ceiling = {} if (not wl.is_decode and wl.selected_rows() * kv_row > 126e6
+                     and wl.Hkv * max(wl.Dqk, wl.Dv) * (4 if wl.dtype == "f32" else 2) <= 1024) else None
+    stages = stage_timings(wl, dev, binding, stream, max(3, min(args.steps, 50)), gather_ceiling=ceiling)
     stage_report = _stage_report(wl, stages, peaks)
     report = {"metric": METRIC, "value": value, "unit": unit, "ms_per_step": 1000.0 * sec_max / args.steps,
               "steps": args.steps, "warmup": args.warmup, "config": _config(wl, world),
@@ -461,10 +466,20 @@ def measure_forward(wl, args, binding, device, world, rank, local, peaks):
               "gpu_launches": int(launches), "clocks": clocks, "eager": eager,
               "timing": "CUDA-graph replay of one dsa_forward per step" if graph is not None
               else "eager dsa_forward calls"}
-    if not wl.is_decode and stage_report["attn"]["algorithmic_bytes"] > 126e6:
-        report["stages"]["attn"]["note"] = (
-            "the gathered rows (algorithmic bytes) are mostly served by L2: the KV cache is smaller than "
-            "L2 and every row is selected by many queries; hbm_frac compares them with the HBM copy rate")
+    if ceiling:
+        # prefill: the KV cache fits in L2 and every row is selected by many
+        # queries, so the gathers are served by L2; the attention is compared
+        # with the gather of the same rows alone
+        att = report["stages"]["attn"]
+        gbs = ceiling["gathered_bytes"] / (att["ms"] / 1e3) / 1e9
+        att["gather"] = {"gathered_bytes": ceiling["gathered_bytes"], "GB/s": gbs,
+                         "ceiling_GB/s": ceiling["GB/s"], "frac_of_ceiling": gbs / ceiling["GB/s"],
+                         "ceiling": "builder-measured: the same selected K and V rows gathered into shared memory "
+                                    "with no arithmetic (dsa_diag_gather, 16-byte cp.async), "
+                                    f"{ceiling['ms']:.3f} ms"}
+        att["note"] = ("the gathered rows are mostly served by L2 (the KV cache is smaller than L2 and each row "
+                       "is selected by many queries): hbm_frac compares them with the HBM copy rate, "
+                       "gather.frac_of_ceiling with the gather alone")
     return report, {"cpu": cpu, "stream": stream}
 
 
@@ -585,7 +600,7 @@ def _capture(fn, binding, device):
     return g, binding.kernel_launch_count() - n0
 
 
-def stage_timings(wl, dev, binding, stream, iters):
+def stage_timings(wl, dev, binding, stream, iters, gather_ceiling=None):
     """Average device time (ms) per launch of each stage: the stage call is
     captured in a CUDA graph and replayed `iters` times between CUDA events on
     the launching stream (the stage-API indexer also writes the -inf upper
@@ -622,6 +637,21 @@ def stage_timings(wl, dev, binding, stream, iters):
     res["topk"] = t_of(lambda: binding.topk(scores, wl.k, wl.q_pos0, idx=idx))
     res["attn"] = t_of(lambda: binding.sparse_attn(dev["q"], dev["k_cache"], dev["v_cache"], idx, wl.scale,
                                                    out=out, ws=ws))
+    if gather_ceiling is not None and wl.B == 1:
+        # the gather of the same selected K and V rows alone (dsa_diag_gather)
+        sink = torch.zeros(1, dtype=torch.int32, device=device)
+        kc, vc = dev["k_cache"], dev["v_cache"]
+        krow, vrow = wl.Hkv * wl.Dqk * kc.element_size(), wl.Hkv * wl.Dv * vc.element_size()
+        flat = idx.reshape(-1)
+
+        def gather_kv():
+            binding.diag_gather(kc, krow, wl.L, flat, sink, pitch_bytes=kc.stride(1) * kc.element_size())
+            if not wl.kv_alias:
+                binding.diag_gather(vc, vrow, wl.L, flat, sink, pitch_bytes=vc.stride(1) * vc.element_size())
+
+        ms = t_of(gather_kv)
+        gathered = wl.selected_rows() * (krow + (0 if wl.kv_alias else vrow))
+        gather_ceiling.update({"ms": ms, "GB/s": gathered / (ms / 1e3) / 1e9, "gathered_bytes": gathered})
     return res
 
 

@@ -378,6 +378,24 @@ dsa_status dsa_indexer_backward(const void *q_idx, const void *k_idx, const floa
 size_t dsa_indexer_backward_workspace_bytes(int B, int Tq, int L, int q_pos0, int H_I, int d_I,
                                             dsa_dtype dt);
 
+/*
+ * dsa_diag_gather -- a measurement aid with no counterpart on the pages: the
+ * gather of selected rows alone, without the attention's arithmetic. It
+ * moves rows idx[0..n) of src (row r at src + r * pitch_bytes, row_bytes
+ * bytes each) into shared memory with the 16-byte cp.async copies the
+ * attention kernels use, and discards them. Timed on the rows an attention
+ * call selects, it gives the rate at which those rows can be gathered at all,
+ * the ceiling of the attention's gather-bound time.
+ *   idx      int32; entries outside [0, n_src_rows) are skipped.
+ *   sink     one uint32 in device memory; written at most rarely (keeps the
+ *            copies live).
+ * Requires 16 <= row_bytes <= 1024, row_bytes and pitch_bytes multiples of 16,
+ * pitch_bytes >= row_bytes, src 16-byte aligned, n >= 1 (else
+ * DSA_ERR_INVALID_ARG).
+ */
+dsa_status dsa_diag_gather(const void *src, int64_t pitch_bytes, int row_bytes, int n_src_rows,
+                           const int32_t *idx, int64_t n, uint32_t *sink, dsa_stream_t stream);
+
 /* ------------------------------------------------------------------------
  * Context parallelism: the indexer keys and the KV cache split by position
  * over P ranks (rank r holds positions [key_pos0_r, key_pos0_r + L_r)), every

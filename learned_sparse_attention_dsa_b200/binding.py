@@ -27,6 +27,7 @@ STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED",
 EXPORTED = ("dsa_version", "dsa_kernel_launch_count", "dsa_status_string", "dsa_indexer_scores", "dsa_topk",
             "dsa_topk_workspace_bytes", "dsa_sparse_attn", "dsa_sparse_attn_workspace_bytes",
             "dsa_forward", "dsa_forward_workspace_bytes", "dsa_device_error", "dsa_set_wait_limit_ns", "dsa_topk_ex",
+            "dsa_diag_gather",
             "dsa_indexer_kl", "dsa_indexer_backward", "dsa_indexer_backward_workspace_bytes",
             "dsa_cp_select_candidates", "dsa_cp_merge", "dsa_cp_localize", "dsa_cp_combine")
 
@@ -93,6 +94,8 @@ def load_library(path: str = LIB_PATH):
     lib.dsa_forward_workspace_bytes.argtypes = [ctypes.POINTER(ForwardArgs)]
     lib.dsa_forward_workspace_bytes.restype = sz
     lib.dsa_device_error.argtypes, lib.dsa_device_error.restype = [vp], ci
+    lib.dsa_diag_gather.argtypes = [vp, ctypes.c_int64, ci, ci, vp, ctypes.c_int64, vp, vp]
+    lib.dsa_diag_gather.restype = ci
     lib.dsa_set_wait_limit_ns.argtypes, lib.dsa_set_wait_limit_ns.restype = [ctypes.c_uint64], ci
     lib.dsa_indexer_kl.argtypes = [vp, vp, vp, ci, ci, ci, ci, ci, vp, vp, vp, vp]
     lib.dsa_indexer_kl.restype = ci
@@ -125,6 +128,16 @@ def device_error(stream=None) -> None:
 
 
 DEFAULT_WAIT_LIMIT_NS = 2_000_000_000
+
+
+def diag_gather(src: torch.Tensor, row_bytes: int, n_src_rows: int, idx: torch.Tensor, sink: torch.Tensor,
+                pitch_bytes=None, stream=None) -> None:
+    """dsa_diag_gather: the gather of rows idx of src (row_bytes each, pitch_bytes
+    apart, default row_bytes) into shared memory alone, a measurement aid."""
+    _need_cuda(src, idx, sink)
+    pitch = row_bytes if pitch_bytes is None else pitch_bytes
+    _check(load_library().dsa_diag_gather(_p(src), pitch, row_bytes, n_src_rows, _p(idx), idx.numel(), _p(sink),
+                                          _stream(stream)), "dsa_diag_gather")
 
 
 def set_wait_limit_ns(ns: int) -> None:

@@ -381,6 +381,16 @@ dsa_status dsa_indexer_backward(const void *q_idx, const void *k_idx, const floa
     return from_cuda(launch_indexer_bwd(p, static_cast<cudaStream_t>(stream)));
 }
 
+dsa_status dsa_diag_gather(const void *src, int64_t pitch_bytes, int row_bytes, int n_src_rows, const int32_t *idx,
+                           int64_t n, uint32_t *sink, dsa_stream_t stream) {
+    if (!src || !idx || !sink || n < 1 || n_src_rows < 1) return DSA_ERR_INVALID_ARG;
+    if (row_bytes < 16 || row_bytes > 1024 || row_bytes % 16 != 0) return DSA_ERR_INVALID_ARG;
+    if (pitch_bytes < row_bytes || pitch_bytes % 16 != 0) return DSA_ERR_INVALID_ARG;
+    if (!aligned(src, 16) || !aligned(idx, 4) || !aligned(sink, 4)) return DSA_ERR_INVALID_ARG;
+    return from_cuda(launch_diag_gather(src, pitch_bytes, row_bytes, n_src_rows, idx, n, sink,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
 dsa_status dsa_cp_select_candidates(const float *scores, const int32_t *idx, int rows, int L, int k, int key_pos0,
                                     float *cand_scores, int32_t *cand_idx, dsa_stream_t stream) {
     if (!scores || !idx || !cand_scores || !cand_idx) return DSA_ERR_INVALID_ARG;

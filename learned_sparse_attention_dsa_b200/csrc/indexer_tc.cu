@@ -271,7 +271,62 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
         int ab = 0;
         uint32_t aph = 0;
-        for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
+        // the query's score of this thread's key from a tile's 64 head columns
+        // (x) and weights (wr), in the same order as the general loop below
+        auto head_sum64 = [](const uint32_t *x, const float4 *wr) -> float {
+            uint64_t part[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const float r0 = fmaxf(__uint_as_float(x[4 * j + 0]), 0.0f);
+                const float r1 = fmaxf(__uint_as_float(x[4 * j + 1]), 0.0f);
+                const float r2 = fmaxf(__uint_as_float(x[4 * j + 2]), 0.0f);
+                const float r3 = fmaxf(__uint_as_float(x[4 * j + 3]), 0.0f);
+                fma2(part[(2 * j) & 3], wr[j].x, wr[j].y, r0, r1);
+                fma2(part[(2 * j + 1) & 3], wr[j].z, wr[j].w, r2, r3);
+            }
+            return (lo_f32(part[0]) + hi_f32(part[0]) + (lo_f32(part[1]) + hi_f32(part[1]))) +
+                   (lo_f32(part[2]) + hi_f32(part[2]) + (lo_f32(part[3]) + hi_f32(part[3])));
+        };
+        // Decode with 64 indexer heads (one query per tile): the query's
+        // weights stay in registers for the whole work unit, and both halves
+        // of the accumulator are loaded before one wait.
+        const bool decode64 = EPI == 8 && N_TILE == 64 && p.H == 64;
+        for (int u = blockIdx.x; ok && decode64 && u < p.units; u += gridDim.x) {
+            Unit un;
+            if (!decode_unit(u, p, un)) continue;
+            const size_t row0 = (size_t)un.b * p.Tq + un.i0;
+            float4 wr[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) wr[j] = __ldg(reinterpret_cast<const float4 *>(p.w + row0 * 64) + j);
+            const int t = p.q_pos0 + un.i0;
+            float *dst_row = p.scores + row0 * (size_t)p.L;
+            for (int kt = un.kt0; kt < un.kt1; ++kt) {
+                if (ab % (EPI / 4) != half) {  // another warp of the quarter takes this tile
+                    if (++ab == C::kAcc) { ab = 0; aph ^= 1u; }
+                    continue;
+                }
+                if (!mbar_wait(&acc_full[ab], aph)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t tbase = tmem_base + lane_addr + (uint32_t)(ab * N_TILE);
+                uint32_t x[64];
+                tmem_ld_32x32b_x32(tbase, x);
+                tmem_ld_32x32b_x32(tbase + 32, x + 32);
+                tmem_ld_wait();
+                tc_fence_before();
+                mbar_arrive(&acc_empty[ab]);  // the accumulator is in registers
+                if (++ab == C::kAcc) { ab = 0; aph ^= 1u; }
+                const float acc = head_sum64(x, wr);
+                const int s = kt * kBlockM + key_in_tile;
+                if (s < p.L) {
+                    if (s <= t) {
+                        dst_row[s] = acc;
+                    } else if (p.fill) {
+                        dst_row[s] = -INFINITY;
+                    }
+                }
+            }
+        }
+        for (int u = blockIdx.x; ok && !decode64 && u < p.units; u += gridDim.x) {
             Unit un;
             if (!decode_unit(u, p, un)) continue;
             const size_t row0 = (size_t)un.b * p.Tq + un.i0;

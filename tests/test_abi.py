@@ -75,6 +75,19 @@ def test_attention_shape_checks(dsa_lib):
     assert dsa_lib.dsa_sparse_attn(fake, fake, fake, fake, ctypes.byref(sh), 1, fake, None, None, 0, None) == 1
 
 
+def test_diag_gather_argument_checks(dsa_lib):
+    fake = ctypes.c_void_p(0x1000)  # never dereferenced: the checks fail first
+    g = dsa_lib.dsa_diag_gather
+    g.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_int64,
+                  ctypes.c_void_p, ctypes.c_void_p]
+    assert g(None, 256, 256, 10, fake, 4, fake, None) == 1      # null source
+    assert g(fake, 256, 24, 10, fake, 4, fake, None) == 1       # row not a multiple of 16 bytes
+    assert g(fake, 2048, 2048, 10, fake, 4, fake, None) == 1    # row longer than 1024 bytes
+    assert g(fake, 128, 256, 10, fake, 4, fake, None) == 1      # pitch shorter than the row
+    assert g(fake, 256, 256, 10, fake, 0, fake, None) == 1      # no rows
+    assert g(ctypes.c_void_p(0x1008), 256, 256, 10, fake, 4, fake, None) == 1  # source not 16-byte aligned
+
+
 def test_workspace_size_of_an_invalid_attention_shape_is_zero(dsa_lib):
     """Invalid shapes are rejected before any size arithmetic (a zero KV head
     count would otherwise divide by zero on the host); the no-workspace entry

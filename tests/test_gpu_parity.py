@@ -277,6 +277,21 @@ def test_bounded_waits_give_up_and_report_timeout(cuda):
     _check_forward(lat, None)
 
 
+def test_diag_gather_runs_on_selected_rows(cuda):
+    """The measurement aid gathers selected rows (skipping invalid entries)
+    without error and without touching memory outside the source."""
+    wl = MEDIUM["prefill_mqa_700"]
+    _, dev = _inputs(wl)
+    kc = dev["k_cache"]
+    idx = torch.randint(-3, wl.L + 3, (5000,), dtype=torch.int32, device="cuda")  # some out of range
+    sink = torch.zeros(1, dtype=torch.int32, device="cuda")
+    n0 = binding.kernel_launch_count()
+    binding.diag_gather(kc, wl.Dqk * 2, wl.L, idx, sink, pitch_bytes=kc.stride(1) * 2)
+    binding.diag_gather(dev["v_cache"], wl.Dv * 2, wl.L, idx[:37], sink)
+    torch.cuda.synchronize()
+    assert binding.kernel_launch_count() - n0 == 2
+
+
 def test_forward_equals_stage_calls(cuda):
     wl = MEDIUM["prefill_mqa_700"]
     _, dev = _inputs(wl)
