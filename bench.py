@@ -42,7 +42,27 @@ METRIC = "prefill tokens/s and decode steps/s at k=2048; % HBM/tensor roofline p
 # figures), with the SHA-256 prefix of the kernel sources it was taken on.
 # dram_traffic() reports an entry only while those sources are unchanged, so
 # a kernel edit turns its traffic into null until it is captured again.
-DRAM_TRAFFIC_PER_LAUNCH = {}
+_IDX = ["indexer_tc.cu", "sm100.cuh", "common.cuh", "tma_map.cu"]
+_TOPK = ["topk.cu", "topk_block.cu", "common.cuh"]
+DRAM_TRAFFIC_PER_LAUNCH = {
+    ("decode32k", "indexer"): {"bytes": 271.64e6, "sources": _IDX, "digest": "d81e94d6c7647034",
+                               "profile": "profiles/dram_stages_decode32k.md"},
+    ("decode32k", "topk"): {"bytes": 4.27e6, "sources": _TOPK, "digest": "65454fadbee778ff",
+                            "profile": "profiles/dram_stages_decode32k.md"},
+    ("decode32k", "attn"): {"bytes": 34.02e6, "sources": ["attn_tc.cu", "common.cuh"],
+                            "digest": "fabd86ecdcf3fe4e", "profile": "profiles/dram_stages_decode32k.md"},
+    ("decode128k", "indexer"): {"bytes": 271.51e6, "sources": _IDX, "digest": "d81e94d6c7647034",
+                                "profile": "profiles/dram_stages_decode128k.md"},
+    ("decode128k", "topk"): {"bytes": 4.27e6, "sources": _TOPK, "digest": "65454fadbee778ff",
+                             "profile": "profiles/dram_stages_decode128k.md"},
+    # the stage's two kernels: the attention and the combine of its split partials
+    ("decode128k", "attn"): {"bytes": 28.65e6, "sources": ["attn_mla_tc.cu", "sm100.cuh", "common.cuh", "tma_map.cu"],
+                             "digest": "398fd6177746f459", "profile": "profiles/dram_stages_decode128k.md"},
+    ("prefill8k", "topk"): {"bytes": 170.64e6, "sources": _TOPK, "digest": "65454fadbee778ff",
+                            "profile": "profiles/dram_stages_prefill8k.md"},
+    ("prefill8k", "attn"): {"bytes": 94.3e6, "sources": ["attn_perhead.cu", "common.cuh"],
+                            "digest": "4201938db5e01efb", "profile": "profiles/dram_stages_prefill8k.md"},
+}
 
 
 def _sources_digest(files):
@@ -342,7 +362,8 @@ def _stage_report(wl, stages, peaks):
         sec_s = ms / 1000.0
         gbs = nbytes / sec_s / 1e9
         entry = {"ms": ms, "GB/s": gbs, "hbm_frac": gbs / peaks["hbm_gbs"],
-                 "algorithmic_bytes": nbytes, "algorithmic_flops": flops}
+                 "algorithmic_bytes": nbytes, "algorithmic_flops": flops,
+                 "dram_traffic": dram_traffic(wl.name, name)}
         if flops:
             entry["TFLOP/s"] = flops / sec_s / 1e12
             entry["tensor_frac"] = entry["TFLOP/s"] / _tensor_peak(wl, name, peaks)
@@ -475,8 +496,8 @@ def measure_forward(wl, args, binding, device, world, rank, local, peaks):
         att["gather"] = {"gathered_bytes": ceiling["gathered_bytes"], "GB/s": gbs,
                          "ceiling_GB/s": ceiling["GB/s"], "frac_of_ceiling": gbs / ceiling["GB/s"],
                          "ceiling": "builder-measured: the same selected K and V rows gathered into shared memory "
-                                    "with no arithmetic (dsa_diag_gather, 16-byte cp.async), "
-                                    f"{ceiling['ms']:.3f} ms"}
+                                    "with no arithmetic (dsa_diag_gather, 16-byte cp.async; fastest of 8-, 16- and "
+                                    f"32-row tiles: {ceiling['tile_rows']}), {ceiling['ms']:.3f} ms"}
         att["note"] = ("the gathered rows are mostly served by L2 (the KV cache is smaller than L2 and each row "
                        "is selected by many queries): hbm_frac compares them with the HBM copy rate, "
                        "gather.frac_of_ceiling with the gather alone")
@@ -644,14 +665,20 @@ def stage_timings(wl, dev, binding, stream, iters, gather_ceiling=None):
         krow, vrow = wl.Hkv * wl.Dqk * kc.element_size(), wl.Hkv * wl.Dv * vc.element_size()
         flat = idx.reshape(-1)
 
-        def gather_kv():
-            binding.diag_gather(kc, krow, wl.L, flat, sink, pitch_bytes=kc.stride(1) * kc.element_size())
+        def gather_kv(tile_rows):
+            binding.diag_gather(kc, krow, wl.L, flat, sink, pitch_bytes=kc.stride(1) * kc.element_size(),
+                                tile_rows=tile_rows)
             if not wl.kv_alias:
-                binding.diag_gather(vc, vrow, wl.L, flat, sink, pitch_bytes=vc.stride(1) * vc.element_size())
+                binding.diag_gather(vc, vrow, wl.L, flat, sink, pitch_bytes=vc.stride(1) * vc.element_size(),
+                                    tile_rows=tile_rows)
 
-        ms = t_of(gather_kv)
+        # the fastest of three tile sizes (more CTAs per SM with smaller tiles)
+        trial = {tr: t_of(lambda tr=tr: gather_kv(tr)) for tr in (8, 16, 32)}
+        best = min(trial, key=trial.get)
+        ms = trial[best]
         gathered = wl.selected_rows() * (krow + (0 if wl.kv_alias else vrow))
-        gather_ceiling.update({"ms": ms, "GB/s": gathered / (ms / 1e3) / 1e9, "gathered_bytes": gathered})
+        gather_ceiling.update({"ms": ms, "GB/s": gathered / (ms / 1e3) / 1e9, "gathered_bytes": gathered,
+                               "tile_rows": best, "ms_by_tile_rows": trial})
     return res
 
 

@@ -387,14 +387,16 @@ size_t dsa_indexer_backward_workspace_bytes(int B, int Tq, int L, int q_pos0, in
  * call selects, it gives the rate at which those rows can be gathered at all,
  * the ceiling of the attention's gather-bound time.
  *   idx      int32; entries outside [0, n_src_rows) are skipped.
+ *   tile_rows  8, 16 or 32: rows per shared-memory tile of a CTA (three
+ *            tiles in flight); smaller tiles fit more CTAs on an SM.
  *   sink     one uint32 in device memory; written at most rarely (keeps the
  *            copies live).
  * Requires 16 <= row_bytes <= 1024, row_bytes and pitch_bytes multiples of 16,
- * pitch_bytes >= row_bytes, src 16-byte aligned, n >= 1 (else
- * DSA_ERR_INVALID_ARG).
+ * pitch_bytes >= row_bytes, src 16-byte aligned, n >= 1, tile_rows in {8, 16,
+ * 32} (else DSA_ERR_INVALID_ARG).
  */
 dsa_status dsa_diag_gather(const void *src, int64_t pitch_bytes, int row_bytes, int n_src_rows,
-                           const int32_t *idx, int64_t n, uint32_t *sink, dsa_stream_t stream);
+                           const int32_t *idx, int64_t n, int tile_rows, uint32_t *sink, dsa_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * Context parallelism: the indexer keys and the KV cache split by position

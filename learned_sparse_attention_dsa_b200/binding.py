@@ -94,7 +94,7 @@ def load_library(path: str = LIB_PATH):
     lib.dsa_forward_workspace_bytes.argtypes = [ctypes.POINTER(ForwardArgs)]
     lib.dsa_forward_workspace_bytes.restype = sz
     lib.dsa_device_error.argtypes, lib.dsa_device_error.restype = [vp], ci
-    lib.dsa_diag_gather.argtypes = [vp, ctypes.c_int64, ci, ci, vp, ctypes.c_int64, vp, vp]
+    lib.dsa_diag_gather.argtypes = [vp, ctypes.c_int64, ci, ci, vp, ctypes.c_int64, ci, vp, vp]
     lib.dsa_diag_gather.restype = ci
     lib.dsa_set_wait_limit_ns.argtypes, lib.dsa_set_wait_limit_ns.restype = [ctypes.c_uint64], ci
     lib.dsa_indexer_kl.argtypes = [vp, vp, vp, ci, ci, ci, ci, ci, vp, vp, vp, vp]
@@ -131,13 +131,13 @@ DEFAULT_WAIT_LIMIT_NS = 2_000_000_000
 
 
 def diag_gather(src: torch.Tensor, row_bytes: int, n_src_rows: int, idx: torch.Tensor, sink: torch.Tensor,
-                pitch_bytes=None, stream=None) -> None:
+                pitch_bytes=None, tile_rows: int = 32, stream=None) -> None:
     """dsa_diag_gather: the gather of rows idx of src (row_bytes each, pitch_bytes
     apart, default row_bytes) into shared memory alone, a measurement aid."""
     _need_cuda(src, idx, sink)
     pitch = row_bytes if pitch_bytes is None else pitch_bytes
-    _check(load_library().dsa_diag_gather(_p(src), pitch, row_bytes, n_src_rows, _p(idx), idx.numel(), _p(sink),
-                                          _stream(stream)), "dsa_diag_gather")
+    _check(load_library().dsa_diag_gather(_p(src), pitch, row_bytes, n_src_rows, _p(idx), idx.numel(), tile_rows,
+                                          _p(sink), _stream(stream)), "dsa_diag_gather")
 
 
 def set_wait_limit_ns(ns: int) -> None:

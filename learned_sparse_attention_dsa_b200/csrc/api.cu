@@ -382,12 +382,13 @@ dsa_status dsa_indexer_backward(const void *q_idx, const void *k_idx, const floa
 }
 
 dsa_status dsa_diag_gather(const void *src, int64_t pitch_bytes, int row_bytes, int n_src_rows, const int32_t *idx,
-                           int64_t n, uint32_t *sink, dsa_stream_t stream) {
+                           int64_t n, int tile_rows, uint32_t *sink, dsa_stream_t stream) {
     if (!src || !idx || !sink || n < 1 || n_src_rows < 1) return DSA_ERR_INVALID_ARG;
+    if (tile_rows != 8 && tile_rows != 16 && tile_rows != 32) return DSA_ERR_INVALID_ARG;
     if (row_bytes < 16 || row_bytes > 1024 || row_bytes % 16 != 0) return DSA_ERR_INVALID_ARG;
     if (pitch_bytes < row_bytes || pitch_bytes % 16 != 0) return DSA_ERR_INVALID_ARG;
     if (!aligned(src, 16) || !aligned(idx, 4) || !aligned(sink, 4)) return DSA_ERR_INVALID_ARG;
-    return from_cuda(launch_diag_gather(src, pitch_bytes, row_bytes, n_src_rows, idx, n, sink,
+    return from_cuda(launch_diag_gather(src, pitch_bytes, row_bytes, n_src_rows, idx, n, tile_rows, sink,
                                         static_cast<cudaStream_t>(stream)));
 }
 

@@ -6,7 +6,8 @@
 // compared with.
 //
 // Each CTA (256 threads) walks a contiguous share of the index list in tiles
-// of 32 rows through a three-stage ring; thread i always moves the 16-byte
+// of 8, 16 or 32 rows (smaller tiles: more CTAs per SM) through a three-stage
+// ring; thread i always moves the 16-byte
 // chunk column i % C of rows i / C, i / C + 256 / C, ... (C = row_bytes / 16),
 // like the attention kernels' copies. Negative or out-of-range indices are
 // skipped (zero-filled, no memory traffic). One word of every landed tile is
@@ -18,7 +19,6 @@ namespace dsa {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kTileRows = 32;
 constexpr int kStages = 3;
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid) {
@@ -31,7 +31,7 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 
 __global__ void __launch_bounds__(kThreads)
 diag_gather_kernel(const uint8_t *__restrict__ src, int64_t pitch, int row_bytes, int n_src, const int32_t *__restrict__ idx,
-                   int64_t n, int64_t per_cta, unsigned int *sink) {
+                   int64_t n, int64_t per_cta, int tile_rows, unsigned int *sink) {
     extern __shared__ __align__(16) uint8_t smem[];
     const int64_t r0 = (int64_t)blockIdx.x * per_cta;
     const int64_t r1 = min(n, r0 + per_cta);
@@ -39,13 +39,13 @@ diag_gather_kernel(const uint8_t *__restrict__ src, int64_t pitch, int row_bytes
     const int chunks = row_bytes / 16;
     const int rows_per_pass = kThreads / chunks;
     const int ch = threadIdx.x % chunks, rr = threadIdx.x / chunks;
-    const int tile_bytes = kTileRows * row_bytes;
-    const int n_tiles = (int)((r1 - r0 + kTileRows - 1) / kTileRows);
+    const int tile_bytes = tile_rows * row_bytes;
+    const int n_tiles = (int)((r1 - r0 + tile_rows - 1) / tile_rows);
     const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
     auto issue = [&](int tile, int stage) {
         if (rr >= rows_per_pass) return;
-        for (int r = rr; r < kTileRows; r += rows_per_pass) {
-            const int64_t j = r0 + (int64_t)tile * kTileRows + r;
+        for (int r = rr; r < tile_rows; r += rows_per_pass) {
+            const int64_t j = r0 + (int64_t)tile * tile_rows + r;
             int s = j < r1 ? idx[j] : -1;
             const bool valid = s >= 0 && s < n_src;
             if (!valid) s = 0;
@@ -74,11 +74,11 @@ diag_gather_kernel(const uint8_t *__restrict__ src, int64_t pitch, int row_bytes
 }  // namespace
 
 cudaError_t launch_diag_gather(const void *src, int64_t pitch, int row_bytes, int n_src, const int32_t *idx, int64_t n,
-                               unsigned int *sink, cudaStream_t stream) {
+                               int tile_rows, unsigned int *sink, cudaStream_t stream) {
     DeviceInfo info;
     cudaError_t err = device_info(&info);
     if (err != cudaSuccess) return err;
-    const size_t smem = (size_t)kStages * kTileRows * row_bytes;
+    const size_t smem = (size_t)kStages * tile_rows * row_bytes;
     err = cudaFuncSetAttribute(diag_gather_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     int per_sm = 0;
@@ -86,11 +86,11 @@ cudaError_t launch_diag_gather(const void *src, int64_t pitch, int row_bytes, in
     if (err != cudaSuccess) return err;
     if (per_sm < 1) per_sm = 1;
     const int64_t ctas_max = (int64_t)info.sm_count * per_sm;
-    const int64_t tiles = (n + kTileRows - 1) / kTileRows;
+    const int64_t tiles = (n + tile_rows - 1) / tile_rows;
     const int64_t ctas = tiles < ctas_max ? tiles : ctas_max;
-    const int64_t per_cta = ((tiles + ctas - 1) / ctas) * kTileRows;
+    const int64_t per_cta = ((tiles + ctas - 1) / ctas) * tile_rows;
     diag_gather_kernel<<<(unsigned)ctas, kThreads, smem, stream>>>(static_cast<const uint8_t *>(src), pitch, row_bytes, n_src,
-                                                                   idx, n, per_cta, sink);
+                                                                   idx, n, per_cta, tile_rows, sink);
     count_launch();
     return cudaGetLastError();
 }

@@ -129,7 +129,7 @@ cudaError_t launch_combine_parts(const void *parts, const float *parts_lse, int 
 // Measurement aid: gather rows idx[0..n) of src (pitch bytes apart, row_bytes
 // each) into shared memory with 16-byte cp.async and discard them.
 cudaError_t launch_diag_gather(const void *src, int64_t pitch, int row_bytes, int n_src, const int32_t *idx, int64_t n,
-                               unsigned int *sink, cudaStream_t stream);
+                               int tile_rows, unsigned int *sink, cudaStream_t stream);
 
 // Read and clear the error word of a kernel family (kErrTimeout: some launch
 // gave up on a bounded wait; kErrBadIndex: an attention launch skipped a

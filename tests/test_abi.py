@@ -79,13 +79,14 @@ def test_diag_gather_argument_checks(dsa_lib):
     fake = ctypes.c_void_p(0x1000)  # never dereferenced: the checks fail first
     g = dsa_lib.dsa_diag_gather
     g.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_int64,
-                  ctypes.c_void_p, ctypes.c_void_p]
-    assert g(None, 256, 256, 10, fake, 4, fake, None) == 1      # null source
-    assert g(fake, 256, 24, 10, fake, 4, fake, None) == 1       # row not a multiple of 16 bytes
-    assert g(fake, 2048, 2048, 10, fake, 4, fake, None) == 1    # row longer than 1024 bytes
-    assert g(fake, 128, 256, 10, fake, 4, fake, None) == 1      # pitch shorter than the row
-    assert g(fake, 256, 256, 10, fake, 0, fake, None) == 1      # no rows
-    assert g(ctypes.c_void_p(0x1008), 256, 256, 10, fake, 4, fake, None) == 1  # source not 16-byte aligned
+                  ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
+    assert g(None, 256, 256, 10, fake, 4, 32, fake, None) == 1      # null source
+    assert g(fake, 256, 24, 10, fake, 4, 32, fake, None) == 1       # row not a multiple of 16 bytes
+    assert g(fake, 2048, 2048, 10, fake, 4, 32, fake, None) == 1    # row longer than 1024 bytes
+    assert g(fake, 128, 256, 10, fake, 4, 32, fake, None) == 1      # pitch shorter than the row
+    assert g(fake, 256, 256, 10, fake, 0, 32, fake, None) == 1      # no rows
+    assert g(fake, 256, 256, 10, fake, 4, 12, fake, None) == 1      # tile rows not 8, 16 or 32
+    assert g(ctypes.c_void_p(0x1008), 256, 256, 10, fake, 4, 32, fake, None) == 1  # source not 16-byte aligned
 
 
 def test_workspace_size_of_an_invalid_attention_shape_is_zero(dsa_lib):

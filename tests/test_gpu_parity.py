@@ -287,7 +287,7 @@ def test_diag_gather_runs_on_selected_rows(cuda):
     sink = torch.zeros(1, dtype=torch.int32, device="cuda")
     n0 = binding.kernel_launch_count()
     binding.diag_gather(kc, wl.Dqk * 2, wl.L, idx, sink, pitch_bytes=kc.stride(1) * 2)
-    binding.diag_gather(dev["v_cache"], wl.Dv * 2, wl.L, idx[:37], sink)
+    binding.diag_gather(dev["v_cache"], wl.Dv * 2, wl.L, idx[:37], sink, tile_rows=8)
     torch.cuda.synchronize()
     assert binding.kernel_launch_count() - n0 == 2
 
