@@ -108,9 +108,12 @@ struct Cfg {
     static constexpr uint32_t kQBytes = kQHalf * kHalves;
     static constexpr uint32_t kKHalf = kBlockM * 128;
     static constexpr uint32_t kKBytes = kKHalf * kHalves;
-    static constexpr int kQBufs = 2;
+    // query buffers: the producer can run at most kQBufs work units ahead of
+    // the MMA, so small query tiles (e4m3 decode, 8 KB, units of a few key
+    // tiles) get six, else the key ring would never fill
+    static constexpr int kQBufs = kQBytes <= 8192 ? 6 : 2;
     static constexpr int kStagesRaw = (int)((kSmemBudget - kQBufs * kQBytes) / kKBytes);
-    // as many key stages as fit: with 16 KB e4m3 stages, 13 keep ~200 KB in flight
+    // as many key stages as fit: with 16 KB e4m3 stages, 11 keep ~176 KB in flight
     static constexpr int kStages = kStagesRaw > 16 ? 16 : kStagesRaw;
     // accumulator buffers in TMEM: four when they fit (the MMA runs further
     // ahead of the epilogue), else two
@@ -233,14 +236,18 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     if (!mbar_wait(&k_full[ks], kph)) { ok = false; break; }
                     if (!mbar_wait(&acc_empty[ab], aph ^ 1u)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t k_base = smem_addr(k_sm + ks * C::kKBytes);
                     const uint32_t d_tmem = tmem_base + (uint32_t)(ab * N_TILE);
+                    // descriptors of the stage and query buffer once; each MMA
+                    // advances their start-address field (bytes / 16, 14 bits,
+                    // no carry below 256 KB of shared memory)
+                    const uint64_t a0 = smem_desc_k_sw128(smem_addr(k_sm + ks * C::kKBytes));
+                    const uint64_t b0 = smem_desc_k_sw128(q_base);
 #pragma unroll
                     for (int h = 0; h < C::kHalves; ++h) {
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk) {  // 4 MMAs of 32 bytes of K per 128-byte swizzle row
-                            const uint64_t a = smem_desc_k_sw128(k_base + h * C::kKHalf + kk * 32);
-                            const uint64_t b = smem_desc_k_sw128(q_base + h * C::kQHalf + kk * 32);
+                            const uint64_t a = a0 + (uint64_t)((h * C::kKHalf + kk * 32) >> 4);
+                            const uint64_t b = b0 + (uint64_t)((h * C::kQHalf + kk * 32) >> 4);
                             if constexpr (FP8)
                                 mma_f8_ss(d_tmem, a, b, idesc, (h | kk) != 0);
                             else
@@ -426,10 +433,14 @@ cudaError_t launch_tc(const IndexerProblem &pr, const DeviceInfo &info, cudaStre
         nkt_max = nkt > nkt_max ? nkt : nkt_max;
     }
     tiles *= pr.B;
-    // About 32 units per CTA when the query tile is small (decode: cheap
-    // reloads, fine balance), about 8 when it is 64 KB (prefill: each unit
-    // reloads its query tile).
-    const long long units_per_cta = pr.Tq == 1 ? 32 : 8;
+    // Units per CTA: about 8 when the query tile is 64 KB (prefill: each unit
+    // reloads its query tile). Decode: about 32 for bf16 keys (2-tile units;
+    // the query buffers then hold the producer to a few tiles ahead, and the
+    // deeper key ring that longer units allow measured slower), about 8 for
+    // e4m3 keys, whose 16 KB tiles arrive twice as often: with 2-tile units
+    // the MMA thread's per-unit work (unit decode, query wait and release)
+    // set the pace at ~0.5 us per tile.
+    const long long units_per_cta = pr.Tq == 1 ? (FP8 ? 8 : 32) : 8;
     long long chunk = (tiles + (long long)info.sm_count * units_per_cta - 1) / ((long long)info.sm_count * units_per_cta);
     p.C = (int)(chunk < 1 ? 1 : (chunk > 64 ? 64 : chunk));
     const long long units = (long long)ceil_div(nkt_max, p.C) * p.G;
