@@ -339,7 +339,7 @@ def _config(wl, world):
             "kv_heads": wl.Hkv, "d_qk": wl.Dqk, "d_v": wl.Dv, "kv_alias": wl.kv_alias,
             "parallelism": f"replicas{world}",
             "l2": "no flush: every step streams the indexer-key cache "
-                  f"({wl.B * wl.L * wl.d_I * (4 if wl.dtype == 'f32' else 2) / 1e6:.0f} MB), "
+                  f"({wl.B * wl.L * wl.d_I * (1 if wl.idx_dtype == 'e4m3' else 4 if wl.dtype == 'f32' else 2) / 1e6:.0f} MB), "
                   "larger than the 126 MB L2"}
 
 
@@ -347,7 +347,7 @@ def _config(wl, world):
 
 # The other configurations measured by the default run, each reported under
 # "workloads" in the same JSON line (the headline workload is decode32k).
-EXTRA_WORKLOADS = ("toy16", "prefill8k", "prefill32k", "decode128k")
+EXTRA_WORKLOADS = ("toy16", "prefill8k", "prefill32k", "decode128k", "decode32k_fp8")
 # Minimum length of the window of identical back-to-back steps over which
 # clocks are sampled (the steps queued right before the timed ones, then the
 # timed ones).

@@ -108,12 +108,11 @@ struct Cfg {
     static constexpr uint32_t kQBytes = kQHalf * kHalves;
     static constexpr uint32_t kKHalf = kBlockM * 128;
     static constexpr uint32_t kKBytes = kKHalf * kHalves;
-    // query buffers: the producer can run at most kQBufs work units ahead of
-    // the MMA, so small query tiles (e4m3 decode, 8 KB, units of a few key
-    // tiles) get six, else the key ring would never fill
-    static constexpr int kQBufs = kQBytes <= 8192 ? 6 : 2;
+    // query buffers: the producer runs at most kQBufs work units ahead of the
+    // MMA (bf16 decode keeps it to a few tiles ahead, which measured fastest)
+    static constexpr int kQBufs = 2;
     static constexpr int kStagesRaw = (int)((kSmemBudget - kQBufs * kQBytes) / kKBytes);
-    // as many key stages as fit: with 16 KB e4m3 stages, 11 keep ~176 KB in flight
+    // as many key stages as fit: with 16 KB e4m3 stages, 13 keep ~208 KB in flight
     static constexpr int kStages = kStagesRaw > 16 ? 16 : kStagesRaw;
     // accumulator buffers in TMEM: four when they fit (the MMA runs further
     // ahead of the epilogue), else two
