@@ -45,19 +45,25 @@ METRIC = "prefill tokens/s and decode steps/s at k=2048; % HBM/tensor roofline p
 _IDX = ["indexer_tc.cu", "sm100.cuh", "common.cuh", "tma_map.cu"]
 _TOPK = ["topk.cu", "topk_block.cu", "common.cuh"]
 DRAM_TRAFFIC_PER_LAUNCH = {
-    ("decode32k", "indexer"): {"bytes": 271.64e6, "sources": _IDX, "digest": "d81e94d6c7647034",
+    ("decode32k", "indexer"): {"bytes": 271.96e6, "sources": _IDX, "digest": "73a556a5f522a639",
                                "profile": "profiles/dram_stages_decode32k.md"},
     ("decode32k", "topk"): {"bytes": 4.27e6, "sources": _TOPK, "digest": "65454fadbee778ff",
                             "profile": "profiles/dram_stages_decode32k.md"},
     ("decode32k", "attn"): {"bytes": 34.02e6, "sources": ["attn_tc.cu", "common.cuh"],
                             "digest": "fabd86ecdcf3fe4e", "profile": "profiles/dram_stages_decode32k.md"},
-    ("decode128k", "indexer"): {"bytes": 271.51e6, "sources": _IDX, "digest": "d81e94d6c7647034",
+    ("decode128k", "indexer"): {"bytes": 271.42e6, "sources": _IDX, "digest": "73a556a5f522a639",
                                 "profile": "profiles/dram_stages_decode128k.md"},
     ("decode128k", "topk"): {"bytes": 4.27e6, "sources": _TOPK, "digest": "65454fadbee778ff",
                              "profile": "profiles/dram_stages_decode128k.md"},
     # the stage's two kernels: the attention and the combine of its split partials
     ("decode128k", "attn"): {"bytes": 28.65e6, "sources": ["attn_mla_tc.cu", "sm100.cuh", "common.cuh", "tma_map.cu"],
                              "digest": "398fd6177746f459", "profile": "profiles/dram_stages_decode128k.md"},
+    ("prefill8k", "indexer"): {"bytes": 219.44e6, "sources": _IDX, "digest": "73a556a5f522a639",
+                               "profile": "profiles/dram_stages_prefill8k.md"},
+    ("decode32k_fp8", "indexer"): {"bytes": 135.96e6, "sources": _IDX, "digest": "73a556a5f522a639",
+                                   "profile": "profiles/indexer_tc_e4m3_decode32k.md"},
+    ("decode32k_fp8", "topk"): {"bytes": 4.27e6, "sources": _TOPK, "digest": "65454fadbee778ff",
+                                "profile": "profiles/indexer_tc_e4m3_decode32k.md"},
     ("prefill8k", "topk"): {"bytes": 170.64e6, "sources": _TOPK, "digest": "65454fadbee778ff",
                             "profile": "profiles/dram_stages_prefill8k.md"},
     ("prefill8k", "attn"): {"bytes": 94.3e6, "sources": ["attn_perhead.cu", "common.cuh"],
@@ -243,14 +249,22 @@ def sample_pairs(wl, flat) -> int:
     return int(((flat % wl.Tq) + wl.q_pos0 + 1).sum())
 
 
+def bits(t):
+    """A CPU tensor as the oracle reads it: fp32 values, raw bf16 bits
+    (uint16) or e4m3 codes (uint8)."""
+    t = t.contiguous()
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).numpy().view(np.uint16)
+    if t.dtype == torch.float8_e4m3fn:
+        return t.view(torch.uint8).numpy()
+    return t.numpy()
+
+
 def time_oracle(wl, cpu, n_rows: int, nthreads: int = 0, tail: int = 0):
     """Run the CPU oracle (all three stages) on a sample of n_rows query rows
     (sample_rows) and return (seconds, rows, causal pairs of those rows)."""
     import oracle
 
-    def bits(t):
-        t = t.contiguous()
-        return t.view(torch.int16).numpy().view(np.uint16) if t.dtype == torch.bfloat16 else t.numpy()
 
     flat = sample_rows(wl, n_rows, tail)
     row_b = (flat // wl.Tq).astype(np.int32)
@@ -624,8 +638,9 @@ def _capture(fn, binding, device):
 def stage_timings(wl, dev, binding, stream, iters, gather_ceiling=None):
     """Average device time (ms) per launch of each stage: the stage call is
     captured in a CUDA graph and replayed `iters` times between CUDA events on
-    the launching stream (the stage-API indexer also writes the -inf upper
-    triangle, which the fused forward skips)."""
+    the launching stream. The indexer writes the causal entries only
+    (DSA_INDEXER_CAUSAL_ONLY), as the fused forward does; the top-k reads no
+    other entry."""
     device = dev["q"].device
     scores = torch.empty((wl.B, wl.Tq, wl.L), dtype=torch.float32, device=device)
     idx = torch.empty((wl.B, wl.Tq, wl.k), dtype=torch.int32, device=device)
@@ -654,7 +669,7 @@ def stage_timings(wl, dev, binding, stream, iters, gather_ceiling=None):
 
     res = {}
     res["indexer"] = t_of(lambda: binding.indexer_scores(dev["q_idx"], dev["k_idx"], dev["w"], wl.q_pos0,
-                                                         scores=scores))
+                                                         scores=scores, causal_only=True))
     res["topk"] = t_of(lambda: binding.topk(scores, wl.k, wl.q_pos0, idx=idx))
     res["attn"] = t_of(lambda: binding.sparse_attn(dev["q"], dev["k_cache"], dev["v_cache"], idx, wl.scale,
                                                    out=out, ws=ws))
@@ -738,11 +753,11 @@ def run_stage(args, wl):
     scores = torch.empty((wl.B, wl.Tq, wl.L), dtype=torch.float32, device=device)
     idx = torch.empty((wl.B, wl.Tq, wl.k), dtype=torch.int32, device=device)
     out = torch.empty((wl.B, wl.Tq, wl.Hq, wl.Dv), dtype=dev["q"].dtype, device=device)
-    binding.indexer_scores(dev["q_idx"], dev["k_idx"], dev["w"], wl.q_pos0, scores=scores)
+    binding.indexer_scores(dev["q_idx"], dev["k_idx"], dev["w"], wl.q_pos0, scores=scores, causal_only=True)
     binding.topk(scores, wl.k, wl.q_pos0, idx=idx)
     calls = {
         "indexer": lambda: binding.indexer_scores(dev["q_idx"], dev["k_idx"], dev["w"], wl.q_pos0,
-                                                  scores=scores),
+                                                  scores=scores, causal_only=True),
         "topk": lambda: binding.topk(scores, wl.k, wl.q_pos0, idx=idx),
         "attn": lambda: binding.sparse_attn(dev["q"], dev["k_cache"], dev["v_cache"], idx, wl.scale, out=out),
     }
@@ -829,9 +844,6 @@ def time_train_oracle(wl, cpu, target, n_rows: int, nthreads: int = 0):
     import oracle
     from oracle import kl as okl
 
-    def bits(t):
-        t = t.contiguous()
-        return t.view(torch.int16).numpy().view(np.uint16) if t.dtype == torch.bfloat16 else t.numpy()
 
     total = wl.B * wl.Tq
     flat = np.linspace(0, total - 1, num=min(n_rows, total)).round().astype(np.int64)

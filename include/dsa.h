@@ -141,6 +141,23 @@ dsa_status dsa_indexer_scores(const void *q_idx, const void *k_idx, const float 
                               int B, int Tq, int L, int q_pos0, int H_I, int d_I,
                               dsa_dtype dt, float *scores, dsa_stream_t stream);
 
+/* Indexer options (dsa_indexer_scores_ex flags). */
+typedef enum {
+    /* Write only the causal entries scores[b,i,s], s <= q_pos0 + i; the
+     * entries above the diagonal keep whatever the buffer held. What a
+     * consumer that reads only the causal part needs (dsa_topk reads
+     * scores[b,i,0..t]; the fused dsa_forward writes its scores this way),
+     * without the -inf writes of the upper triangle, about half the buffer
+     * in prefill. */
+    DSA_INDEXER_CAUSAL_ONLY = 1
+} dsa_indexer_flags;
+
+/* dsa_indexer_scores with options: flags is 0 or DSA_INDEXER_CAUSAL_ONLY; any
+ * other bit gives DSA_ERR_INVALID_ARG. Otherwise as dsa_indexer_scores. */
+dsa_status dsa_indexer_scores_ex(const void *q_idx, const void *k_idx, const float *w,
+                                 int B, int Tq, int L, int q_pos0, int H_I, int d_I,
+                                 dsa_dtype dt, unsigned flags, float *scores, dsa_stream_t stream);
+
 /*
  * dsa_topk -- stage 2, per-row top-k selection ("Learned Token Selection" §3.1).
  *

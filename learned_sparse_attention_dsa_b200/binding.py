@@ -19,12 +19,14 @@ DSA_F32 = 0
 DSA_BF16 = 1
 DSA_E4M3 = 2
 DSA_FLAG_INCLUDE_SELF = 1
+DSA_INDEXER_CAUSAL_ONLY = 1
 
 STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED",
                 3: "DSA_ERR_WORKSPACE", 4: "DSA_ERR_CUDA", 5: "DSA_ERR_TIMEOUT", 6: "DSA_ERR_BAD_INDEX"}
 
 # Symbols declared in include/dsa.h.
-EXPORTED = ("dsa_version", "dsa_kernel_launch_count", "dsa_status_string", "dsa_indexer_scores", "dsa_topk",
+EXPORTED = ("dsa_version", "dsa_kernel_launch_count", "dsa_status_string", "dsa_indexer_scores",
+            "dsa_indexer_scores_ex", "dsa_topk",
             "dsa_topk_workspace_bytes", "dsa_sparse_attn", "dsa_sparse_attn_workspace_bytes",
             "dsa_forward", "dsa_forward_workspace_bytes", "dsa_device_error", "dsa_set_wait_limit_ns", "dsa_topk_ex",
             "dsa_diag_gather",
@@ -79,6 +81,8 @@ def load_library(path: str = LIB_PATH):
     lib.dsa_status_string.argtypes, lib.dsa_status_string.restype = [ci], ctypes.c_char_p
     lib.dsa_indexer_scores.argtypes = [vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, vp, vp]
     lib.dsa_indexer_scores.restype = ci
+    lib.dsa_indexer_scores_ex.argtypes = [vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, ctypes.c_uint, vp, vp]
+    lib.dsa_indexer_scores_ex.restype = ci
     lib.dsa_topk.argtypes = [vp, ci, ci, ci, ci, ci, vp, vp, sz, vp]
     lib.dsa_topk.restype = ci
     lib.dsa_topk_ex.argtypes = [vp, ci, ci, ci, ci, ci, ctypes.c_uint, vp, vp, sz, vp]
@@ -193,17 +197,19 @@ def _workspace(nbytes: int, device, ws):
     return torch.empty(nbytes, dtype=torch.uint8, device=device)
 
 
-def indexer_scores(q_idx, k_idx, w, q_pos0: int = 0, scores=None, stream=None):
-    """dsa_indexer_scores: fp32 [B, Tq, L] scores, -inf above the diagonal."""
+def indexer_scores(q_idx, k_idx, w, q_pos0: int = 0, scores=None, stream=None, causal_only: bool = False):
+    """dsa_indexer_scores_ex: fp32 [B, Tq, L] scores, -inf above the diagonal
+    (with causal_only, the entries above the diagonal are not written)."""
     lib = load_library()
     _need_cuda(q_idx, k_idx, w, scores)
     B, Tq, H, d = q_idx.shape
     L = k_idx.shape[1]
     if scores is None:
         scores = torch.empty((B, Tq, L), dtype=torch.float32, device=q_idx.device)
-    st = lib.dsa_indexer_scores(_p(q_idx), _p(k_idx), _p(w), B, Tq, L, q_pos0, H, d, _dt(q_idx),
-                                _p(scores), _stream(stream))
-    _check(st, "dsa_indexer_scores")
+    flags = DSA_INDEXER_CAUSAL_ONLY if causal_only else 0
+    st = lib.dsa_indexer_scores_ex(_p(q_idx), _p(k_idx), _p(w), B, Tq, L, q_pos0, H, d, _dt(q_idx),
+                                   flags, _p(scores), _stream(stream))
+    _check(st, "dsa_indexer_scores_ex")
     return scores
 
 

@@ -248,14 +248,22 @@ const char *dsa_status_string(dsa_status status) {
     return "unknown dsa_status";
 }
 
+dsa_status dsa_indexer_scores_ex(const void *q_idx, const void *k_idx, const float *w, int B, int Tq, int L,
+                                 int q_pos0, int H_I, int d_I, dsa_dtype dt, unsigned flags, float *scores,
+                                 dsa_stream_t stream) {
+    dsa_status st = check_indexer(q_idx, k_idx, w, B, Tq, L, q_pos0, H_I, d_I, dt, scores);
+    if (st != DSA_OK) return st;
+    if (flags & ~(unsigned)DSA_INDEXER_CAUSAL_ONLY) return DSA_ERR_INVALID_ARG;
+    if ((st = check_indexer_fits(H_I, d_I)) != DSA_OK) return st;
+    const bool fill = (flags & DSA_INDEXER_CAUSAL_ONLY) == 0;
+    IndexerProblem p{q_idx, k_idx, w, B, Tq, L, q_pos0, H_I, d_I, dt, scores, fill};
+    return from_cuda(launch_indexer(p, static_cast<cudaStream_t>(stream)));
+}
+
 dsa_status dsa_indexer_scores(const void *q_idx, const void *k_idx, const float *w, int B, int Tq, int L,
                               int q_pos0, int H_I, int d_I, dsa_dtype dt, float *scores,
                               dsa_stream_t stream) {
-    dsa_status st = check_indexer(q_idx, k_idx, w, B, Tq, L, q_pos0, H_I, d_I, dt, scores);
-    if (st != DSA_OK) return st;
-    if ((st = check_indexer_fits(H_I, d_I)) != DSA_OK) return st;
-    IndexerProblem p{q_idx, k_idx, w, B, Tq, L, q_pos0, H_I, d_I, dt, scores, true};
-    return from_cuda(launch_indexer(p, static_cast<cudaStream_t>(stream)));
+    return dsa_indexer_scores_ex(q_idx, k_idx, w, B, Tq, L, q_pos0, H_I, d_I, dt, 0u, scores, stream);
 }
 
 size_t dsa_topk_workspace_bytes(int B, int Tq, int L, int q_pos0, int k) {

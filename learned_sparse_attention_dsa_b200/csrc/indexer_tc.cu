@@ -453,7 +453,9 @@ cudaError_t launch_tc(const IndexerProblem &pr, const DeviceInfo &info, cudaStre
     kern<<<grid, Threads<EPI>::kAll, C::kSmem, stream>>>(tm_q, tm_k, p);
     count_launch();
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    if (pr.fill_masked) {
+    // the first row (t = q_pos0) has the fewest tiles; when its tiles reach L,
+    // no row has keys beyond them (decode) and the fill would write nothing
+    if (pr.fill_masked && (long long)(pr.q_pos0 / kBlockM + 1) * kBlockM < pr.L) {
         fill_beyond_tiles_kernel<<<pr.B * pr.Tq, 256, 0, stream>>>(pr.scores, pr.Tq, pr.L, pr.q_pos0);
         count_launch();
         err = cudaGetLastError();

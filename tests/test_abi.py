@@ -62,6 +62,9 @@ def test_bad_sizes_rejected(dsa_lib):
     # misaligned bf16 pointer
     odd = ctypes.c_void_p(0x1001)
     assert dsa_lib.dsa_indexer_scores(odd, fake, fake, 1, 1, 4, 0, 2, 2, 1, fake, None) == 1
+    # an indexer flag other than DSA_INDEXER_CAUSAL_ONLY
+    assert dsa_lib.dsa_indexer_scores_ex(fake, fake, fake, 1, 1, 4, 0, 2, 2, 0, 2, fake, None) == 1
+    assert dsa_lib.dsa_indexer_scores_ex(None, fake, fake, 1, 1, 4, 0, 2, 2, 0, 1, fake, None) == 1
 
 
 def test_attention_shape_checks(dsa_lib):

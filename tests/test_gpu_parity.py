@@ -145,6 +145,31 @@ def test_indexer_stage_all_rows(cuda, name):
     assert np.array_equal(scores.reshape(-1, wl.L), ref)
 
 
+@pytest.mark.parametrize("name", ["prefill_mqa_700", "chunked_prefill", "decode_5000", "odd_heads", "tiny_f32"])
+@pytest.mark.parametrize("e4m3", [False, True])
+def test_indexer_causal_only_leaves_the_upper_triangle(cuda, name, e4m3):
+    """DSA_INDEXER_CAUSAL_ONLY: the causal entries equal the oracle bit for bit
+    (tensor-core and CUDA-core kernels, bf16 and e4m3) and every entry above
+    the diagonal keeps the sentinel that was in the buffer."""
+    wl = MEDIUM[name]
+    if e4m3:
+        if wl.dtype == "f32":
+            pytest.skip("the e4m3 indexer inputs replace bf16 ones")
+        wl = wl.replace(idx_dtype="e4m3", name=wl.name + "_e4m3")  # its own input cache entry
+    cpu, dev = _inputs(wl)
+    sentinel = 7.25
+    scores = torch.full((wl.B, wl.Tq, wl.L), sentinel, dtype=torch.float32, device="cuda")
+    binding.indexer_scores(dev["q_idx"], dev["k_idx"], dev["w"], wl.q_pos0, scores=scores, causal_only=True)
+    got = scores.cpu().numpy().reshape(-1, wl.L)
+    flat = np.arange(wl.B * wl.Tq)
+    row_b, row_i, row_t = rows_of(wl, flat)
+    ref = oracle.indexer_rows(bits(cpu["q_idx"][row_b, row_i]), cpu["w"][row_b, row_i].numpy(),
+                              bits(cpu["k_idx"]), row_b, row_t)
+    causal = np.arange(wl.L)[None, :] <= row_t[:, None]
+    assert np.array_equal(got[causal], ref[causal])
+    assert np.all(got[~causal] == sentinel)
+
+
 @pytest.mark.parametrize("kind", ["int", "equal", "normal", "neg", "mixed"])
 @pytest.mark.parametrize("L,Tq,q_pos0,k", [(37, 37, 0, 5), (5000, 3, 4997, 2048), (3000, 2, 2998, 1),
                                            (12000, 3, 11997, 2048), (32768, 2, 32766, 2048),
