@@ -43,14 +43,17 @@ constexpr int kThreads = kWarps * 32;
 constexpr int kHeads = 16;
 constexpr float kLog2e = 1.4426950408889634f;
 
-template <int DQK, int DV>
+// ROWS selected rows per pipeline stage: 64 (each warp 16 rows), or 32 (each
+// warp 8 rows) for wide rows without splits, where three 68 KB CTAs per SM
+// keep more copies in flight than two 88 KB ones.
+template <int DQK, int DV, int ROWS>
 struct Cfg {
     static constexpr int kKChunks = DQK / 8;  // 16-byte chunks per K row
     static constexpr int kVChunks = DV / 8;
-    static constexpr int kKBytes = kRowsPerTile * DQK * 2;
-    static constexpr int kVBytes = kRowsPerTile * DV * 2;
+    static constexpr int kKBytes = ROWS * DQK * 2;
+    static constexpr int kVBytes = ROWS * DV * 2;
     static constexpr int kStageBytes = kKBytes + kVBytes;
-    static constexpr int kStages = (DQK + DV) > 256 ? 2 : 3;
+    static constexpr int kStages = ROWS == 32 ? 3 : ((DQK + DV) > 256 ? 2 : 3);
     static constexpr int kMaxSel = 2048;  // selected entries one CTA handles
     // four warps' (O, m, l), then the CTA's merged (O, m, l) for the cluster merge
     // (plus one merge weight per split and head)
@@ -110,15 +113,25 @@ __device__ __forceinline__ void mma_bf16(float *c, const uint32_t *a, uint32_t b
         : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
+// m16n8k8: A 16 x 8 (two registers), B 8 x 8 (one register)
+__device__ __forceinline__ void mma_bf16_k8(float *c, const uint32_t *a, uint32_t b0) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5}, {%6}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(b0));
+}
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
-template <int DQK, int DV>
-__global__ void __launch_bounds__(kThreads)
+template <int DQK, int DV, int ROWS>
+__global__ void __launch_bounds__(kThreads, ROWS == 32 ? 3 : 1)
 attn_mma_kernel(const Args a) {
-    using C = Cfg<DQK, DV>;
+    using C = Cfg<DQK, DV, ROWS>;
+    constexpr int NT = ROWS / 32;  // 8-row n-tiles of S per warp
+    constexpr int WR = ROWS / 4;   // rows of a stage per warp
     // cluster merge: this CTA has started (waited on before any other CTA
     // stores into its shared memory)
     if (a.cluster_merge) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
@@ -188,7 +201,7 @@ attn_mma_kernel(const Args a) {
     }
     __syncthreads();
     const int n_sel = s_count;
-    const int n_tiles = (n_sel + kRowsPerTile - 1) / kRowsPerTile;
+    const int n_tiles = (n_sel + ROWS - 1) / ROWS;
 
     const __nv_bfloat16 *kbase = a.k_cache + b * a.k_sb + g * a.k_sh;
     const __nv_bfloat16 *vbase = a.v_cache + b * a.v_sb + g * a.v_sh;
@@ -204,8 +217,8 @@ attn_mma_kernel(const Args a) {
         if (r0 >= R) return;
         const __nv_bfloat16 *src0 = base + ch * 8;
 #pragma unroll 4
-        for (int r = r0; r < kRowsPerTile; r += R) {
-            const int jj = tile * kRowsPerTile + r;
+        for (int r = r0; r < ROWS; r += R) {
+            const int jj = tile * ROWS + r;
             const bool valid = jj < n_sel;
             const int s = valid ? sel[jj] : 0;
             cp_async16(dst0 + r * (CH * 16) + ((ch ^ (r & 7)) << 4), src0 + (int64_t)s * ss, valid);
@@ -259,9 +272,11 @@ attn_mma_kernel(const Args a) {
         const uint32_t kt = smem_base + stage * C::kStageBytes;
         const uint32_t vt = kt + C::kKBytes;
 
-        // S = Q K^T for this warp's 16 rows (two n-tiles of 8 rows)
-        float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-        {
+        // S = Q K^T for this warp's WR rows (NT n-tiles of 8 rows)
+        float s[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.0f;
+        if constexpr (NT == 2) {
             const int r = warp * 16 + (lane & 7) + ((lane >> 4) << 3);
             const uint32_t rbase = kt + r * (DQK * 2);
             const int rx = r & 7;
@@ -273,22 +288,37 @@ attn_mma_kernel(const Args a) {
                 mma_bf16(s[0], qf[kk], b0, b1);
                 mma_bf16(s[1], qf[kk], b2, b3);
             }
+        } else {
+            // 8 rows: one ldmatrix.x4 covers two 16-wide k-steps
+            const int r = warp * 8 + (lane & 7);
+            const uint32_t rbase = kt + r * (DQK * 2);
+            const int rx = r & 7;
+#pragma unroll
+            for (int kk = 0; kk < DQK / 16; kk += 2) {
+                const int ch = 2 * kk + (lane >> 3);
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4(rbase + ((ch ^ rx) << 4), b0, b1, b2, b3);
+                mma_bf16(s[0], qf[kk], b0, b1);
+                mma_bf16(s[0], qf[kk + 1], b2, b3);
+            }
         }
         // mask rows beyond the selected count, scale into log2 units
-        const int valid_rows = n_sel - tile * kRowsPerTile;
+        const int valid_rows = n_sel - tile * ROWS;
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
+        for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const int rr = warp * 16 + nt * 8 + (lane & 3) * 2 + (e & 1);
+                const int rr = warp * WR + nt * 8 + (lane & 3) * 2 + (e & 1);
                 s[nt][e] = rr < valid_rows ? s[nt][e] * a.scale_log2 : -INFINITY;
             }
         }
         // online softmax update for heads lane/4 (e = 0,1) and lane/4+8 (e = 2,3)
-        float p[2][4];
+        float p[NT][4];
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
-            float mx = fmaxf(fmaxf(s[0][2 * hh], s[0][2 * hh + 1]), fmaxf(s[1][2 * hh], s[1][2 * hh + 1]));
+            float mx = fmaxf(s[0][2 * hh], s[0][2 * hh + 1]);
+#pragma unroll
+            for (int nt = 1; nt < NT; ++nt) mx = fmaxf(mx, fmaxf(s[nt][2 * hh], s[nt][2 * hh + 1]));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
             const float m_new = fmaxf(m_r[hh], mx);
@@ -296,7 +326,7 @@ attn_mma_kernel(const Args a) {
             const float mr = m_new == -INFINITY ? 0.0f : m_new;  // masked entries: 2^-inf = 0
             float sum = 0.0f;
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
+            for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                     const float v = s[nt][2 * hh + e];
@@ -313,13 +343,13 @@ attn_mma_kernel(const Args a) {
                 o[n][2 * hh + 1] *= corr;
             }
         }
-        // O += P V: P (16 heads x 16 rows) as the A operand
-        uint32_t pa[4];
-        pa[0] = pack_bf16(p[0][0], p[0][1]);
-        pa[1] = pack_bf16(p[0][2], p[0][3]);
-        pa[2] = pack_bf16(p[1][0], p[1][1]);
-        pa[3] = pack_bf16(p[1][2], p[1][3]);
-        {
+        // O += P V: P (16 heads x WR rows) as the A operand
+        if constexpr (NT == 2) {
+            uint32_t pa[4];
+            pa[0] = pack_bf16(p[0][0], p[0][1]);
+            pa[1] = pack_bf16(p[0][2], p[0][3]);
+            pa[2] = pack_bf16(p[1][0], p[1][1]);
+            pa[3] = pack_bf16(p[1][2], p[1][3]);
             const int r = warp * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
             const uint32_t rbase = vt + r * (DV * 2);
             const int rx = r & 7;
@@ -330,6 +360,24 @@ attn_mma_kernel(const Args a) {
                 ldsm_x4_t(rbase + ((ch ^ rx) << 4), b0, b1, b2, b3);
                 mma_bf16(o[2 * nn], pa, b0, b1);
                 mma_bf16(o[2 * nn + 1], pa, b2, b3);
+            }
+        } else {
+            // 8 rows: k = 8 MMAs; one transposed ldmatrix.x4 gives four 8-column n-tiles
+            uint32_t pa[2];
+            pa[0] = pack_bf16(p[0][0], p[0][1]);
+            pa[1] = pack_bf16(p[0][2], p[0][3]);
+            const int r = warp * 8 + (lane & 7);
+            const uint32_t rbase = vt + r * (DV * 2);
+            const int rx = r & 7;
+#pragma unroll
+            for (int nn = 0; nn < DV / 32; ++nn) {
+                const int ch = 4 * nn + (lane >> 3);
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4_t(rbase + ((ch ^ rx) << 4), b0, b1, b2, b3);
+                mma_bf16_k8(o[4 * nn + 0], pa, b0);
+                mma_bf16_k8(o[4 * nn + 1], pa, b1);
+                mma_bf16_k8(o[4 * nn + 2], pa, b2);
+                mma_bf16_k8(o[4 * nn + 3], pa, b3);
             }
         }
         __syncthreads();  // this stage may be refilled next iteration
@@ -578,12 +626,9 @@ bool shape_supported(const AttnProblem &p, int *dqk_dv) {
     return true;
 }
 
-template <int DQK, int DV>
-cudaError_t launch_mma(const AttnProblem &p, const DeviceInfo &info, cudaStream_t stream) {
-    using C = Cfg<DQK, DV>;
-    const int splits = choose_splits(p, info.sm_count);
-    const int max_tiles = (p.k + kRowsPerTile - 1) / kRowsPerTile;
-    const int per_split = ((max_tiles + splits - 1) / splits) * kRowsPerTile;
+template <int DQK, int DV, int ROWS>
+cudaError_t launch_rows(const AttnProblem &p, int splits, int per_split, cudaStream_t stream) {
+    using C = Cfg<DQK, DV, ROWS>;
     if (per_split > C::kMaxSel) return cudaErrorInvalidValue;
     Args a;
     a.q = static_cast<const __nv_bfloat16 *>(p.q);
@@ -606,7 +651,7 @@ cudaError_t launch_mma(const AttnProblem &p, const DeviceInfo &info, cudaStream_
         a.part_o = static_cast<float *>(p.ws);
         a.part_ml = a.part_o + n_pairs * splits * DV;
     }
-    auto kern = attn_mma_kernel<DQK, DV>;
+    auto kern = attn_mma_kernel<DQK, DV, ROWS>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmemMax);
     if (err != cudaSuccess) return err;
     dim3 grid(rows, p.Hq / kHeads, splits);
@@ -638,6 +683,18 @@ cudaError_t launch_mma(const AttnProblem &p, const DeviceInfo &info, cudaStream_
         err = cudaGetLastError();
     }
     return err;
+}
+
+// Splits are whole 64-row tiles (a multiple of either stage height).
+template <int DQK, int DV>
+cudaError_t launch_mma(const AttnProblem &p, const DeviceInfo &info, cudaStream_t stream) {
+    const int splits = choose_splits(p, info.sm_count);
+    const int max_tiles = (p.k + kRowsPerTile - 1) / kRowsPerTile;
+    const int per_split = ((max_tiles + splits - 1) / splits) * kRowsPerTile;
+    if constexpr (DQK + DV > 256) {
+        if (splits == 1) return launch_rows<DQK, DV, 32>(p, splits, per_split, stream);
+    }
+    return launch_rows<DQK, DV, 64>(p, splits, per_split, stream);
 }
 
 }  // namespace
