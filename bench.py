@@ -50,7 +50,7 @@ DRAM_TRAFFIC_PER_LAUNCH = {
     ("decode32k", "topk"): {"bytes": 4.27e6, "sources": _TOPK, "digest": "65454fadbee778ff",
                             "profile": "profiles/dram_stages_decode32k.md"},
     ("decode32k", "attn"): {"bytes": 34.02e6, "sources": ["attn_tc.cu", "common.cuh"],
-                            "digest": "fabd86ecdcf3fe4e", "profile": "profiles/dram_stages_decode32k.md"},
+                            "digest": "dc4d1f57bbd48356", "profile": "profiles/dram_stages_decode32k.md"},
     ("decode128k", "indexer"): {"bytes": 271.42e6, "sources": _IDX, "digest": "73a556a5f522a639",
                                 "profile": "profiles/dram_stages_decode128k.md"},
     ("decode128k", "topk"): {"bytes": 4.27e6, "sources": _TOPK, "digest": "65454fadbee778ff",
@@ -66,8 +66,8 @@ DRAM_TRAFFIC_PER_LAUNCH = {
                                 "profile": "profiles/indexer_tc_e4m3_decode32k.md"},
     ("prefill8k", "topk"): {"bytes": 170.64e6, "sources": _TOPK, "digest": "65454fadbee778ff",
                             "profile": "profiles/dram_stages_prefill8k.md"},
-    ("prefill8k", "attn"): {"bytes": 94.3e6, "sources": ["attn_perhead.cu", "common.cuh"],
-                            "digest": "4201938db5e01efb", "profile": "profiles/dram_stages_prefill8k.md"},
+    ("prefill8k", "attn"): {"bytes": 92.63e6, "sources": ["attn_perhead.cu", "common.cuh"],
+                            "digest": "e351fb69a1804e15", "profile": "profiles/dram_stages_prefill8k.md"},
 }
 
 
@@ -115,7 +115,7 @@ def _tensor_peak(wl, stage, peaks):
     return peaks["bf16_tflops"]
 
 
-def stage_work(wl):
+def stage_work(wl, attn_rows=None):
     """Algorithmic bytes and flops per forward pass, per stage.
 
     indexer: reads K^I once, q^I and w once, writes one fp32 score per causal
@@ -123,7 +123,10 @@ def stage_work(wl):
     top-k:   reads one fp32 score per causal pair, writes k int32 per row.
     attn:    reads each selected KV row once per KV head (K and V; a V that is
              a view of the K row adds nothing), Q once, writes the output;
-             flops = 2 * Hq * (Dqk + Dv) per selected row.
+             flops = 2 * Hq * (Dqk + Dv) per selected row. attn_rows, when
+             given, replaces the selected rows in the bytes: the rows the
+             kernel has to fetch when query rows share the gathers of the
+             union of their selections (each union row once per group).
     """
     eb = 4 if wl.dtype == "f32" else 2
     ieb = 1 if wl.idx_dtype == "e4m3" else eb  # indexer input element bytes
@@ -135,7 +138,8 @@ def stage_work(wl):
     idx_flops = 2.0 * wl.H_I * wl.d_I * pairs
     topk_bytes = pairs * 4 + rows * wl.k * 4
     kv_row = wl.Hkv * (wl.Dqk if wl.kv_alias else wl.Dqk + wl.Dv) * eb
-    attn_bytes = sel * kv_row + rows * wl.Hq * (wl.Dqk + wl.Dv) * eb + rows * wl.k * 4
+    attn_bytes = (sel if attn_rows is None else attn_rows) * kv_row + rows * wl.Hq * (wl.Dqk + wl.Dv) * eb \
+        + rows * wl.k * 4
     attn_flops = 2.0 * wl.Hq * (wl.Dqk + wl.Dv) * sel
     return {"indexer": (idx_bytes, idx_flops), "topk": (topk_bytes, 0.0), "attn": (attn_bytes, attn_flops)}
 
@@ -368,8 +372,30 @@ EXTRA_WORKLOADS = ("toy16", "prefill8k", "prefill32k", "decode128k", "decode32k_
 CLOCK_WINDOW_S = 0.5
 
 
-def _stage_report(wl, stages, peaks):
-    work = stage_work(wl)
+def union_rows(idx, group: int, L: int) -> int:
+    """KV rows a grouped attention fetches: for every batch entry and every
+    group of `group` consecutive query rows, the number of distinct valid
+    positions in their selections (group 1: the valid entries)."""
+    B, Tq, k = idx.shape
+    if group <= 1:
+        return int(((idx >= 0) & (idx < L)).sum())
+    ng = (Tq + group - 1) // group
+    x = idx
+    if ng * group != Tq:
+        x = torch.cat([x, torch.full((B, ng * group - Tq, k), -1, dtype=idx.dtype, device=idx.device)], 1)
+    x = x.reshape(B * ng, group * k).long()
+    x = torch.where((x >= 0) & (x < L), x, torch.full_like(x, L))  # padding -> an extra column
+    total = 0
+    for c in range(0, x.shape[0], 64):
+        xs = x[c:c + 64]
+        m = torch.zeros((xs.shape[0], L + 1), dtype=torch.bool, device=x.device)
+        m.scatter_(1, xs, True)
+        total += int(m[:, :L].sum())
+    return total
+
+
+def _stage_report(wl, stages, peaks, attn_info=None):
+    work = stage_work(wl, attn_info["gathered_rows"] if attn_info and attn_info.get("row_group", 1) > 1 else None)
     report = {}
     for name, ms in stages.items():
         nbytes, flops = work[name]
@@ -382,6 +408,13 @@ def _stage_report(wl, stages, peaks):
             entry["TFLOP/s"] = flops / sec_s / 1e12
             entry["tensor_frac"] = entry["TFLOP/s"] / _tensor_peak(wl, name, peaks)
         report[name] = entry
+    if attn_info and attn_info.get("row_group", 1) > 1:
+        report["attn"]["row_group"] = attn_info["row_group"]
+        report["attn"]["gathered_rows"] = attn_info["gathered_rows"]
+        report["attn"]["selected_rows"] = wl.selected_rows()
+        report["attn"]["note_rows"] = (f"groups of {attn_info['row_group']} consecutive query rows share the gathers "
+                                       "of the union of their selections: algorithmic_bytes count each union row "
+                                       "once per group (selected_rows is the per-row count)")
     return report
 
 
@@ -493,8 +526,10 @@ def measure_forward(wl, args, binding, device, world, rank, local, peaks):
     kv_row = wl.Hkv * (wl.Dqk + (0 if wl.kv_alias else wl.Dv)) * (4 if wl.dtype == "f32" else 2)
     ceiling = {} if (not wl.is_decode and wl.selected_rows() * kv_row > 126e6
                      and wl.Hkv * max(wl.Dqk, wl.Dv) * (4 if wl.dtype == "f32" else 2) <= 1024) else None
-    stages = stage_timings(wl, dev, binding, stream, max(3, min(args.steps, 50)), gather_ceiling=ceiling)
-    stage_report = _stage_report(wl, stages, peaks)
+    attn_info = {}
+    stages = stage_timings(wl, dev, binding, stream, max(3, min(args.steps, 50)), gather_ceiling=ceiling,
+                           attn_info=attn_info)
+    stage_report = _stage_report(wl, stages, peaks, attn_info)
     report = {"metric": METRIC, "value": value, "unit": unit, "ms_per_step": 1000.0 * sec_max / args.steps,
               "steps": args.steps, "warmup": args.warmup, "config": _config(wl, world),
               "roofline": _roofline(wl, stage_report, peaks), "stages": stage_report,
@@ -506,8 +541,9 @@ def measure_forward(wl, args, binding, device, world, rank, local, peaks):
         # queries, so the gathers are served by L2; the attention is compared
         # with the gather of the same rows alone
         att = report["stages"]["attn"]
-        gbs = ceiling["gathered_bytes"] / (att["ms"] / 1e3) / 1e9
-        att["gather"] = {"gathered_bytes": ceiling["gathered_bytes"], "GB/s": gbs,
+        gathered = attn_info.get("gathered_rows", wl.selected_rows()) * kv_row
+        gbs = gathered / (att["ms"] / 1e3) / 1e9
+        att["gather"] = {"gathered_bytes": gathered, "GB/s": gbs,
                          "ceiling_GB/s": ceiling["GB/s"], "frac_of_ceiling": gbs / ceiling["GB/s"],
                          "ceiling": "builder-measured: the same selected K and V rows gathered into shared memory "
                                     "with no arithmetic (dsa_diag_gather, 16-byte cp.async; fastest of 8-, 16- and "
@@ -635,7 +671,7 @@ def _capture(fn, binding, device):
     return g, binding.kernel_launch_count() - n0
 
 
-def stage_timings(wl, dev, binding, stream, iters, gather_ceiling=None):
+def stage_timings(wl, dev, binding, stream, iters, gather_ceiling=None, attn_info=None):
     """Average device time (ms) per launch of each stage: the stage call is
     captured in a CUDA graph and replayed `iters` times between CUDA events on
     the launching stream. The indexer writes the causal entries only
@@ -673,6 +709,10 @@ def stage_timings(wl, dev, binding, stream, iters, gather_ceiling=None):
     res["topk"] = t_of(lambda: binding.topk(scores, wl.k, wl.q_pos0, idx=idx))
     res["attn"] = t_of(lambda: binding.sparse_attn(dev["q"], dev["k_cache"], dev["v_cache"], idx, wl.scale,
                                                    out=out, ws=ws))
+    if attn_info is not None:
+        group = binding.sparse_attn_row_group(dev["q"], dev["k_cache"], dev["v_cache"], wl.k)
+        attn_info["row_group"] = group
+        attn_info["gathered_rows"] = union_rows(idx, group, wl.L)
     if gather_ceiling is not None and wl.B == 1:
         # the gather of the same selected K and V rows alone (dsa_diag_gather)
         sink = torch.zeros(1, dtype=torch.int32, device=device)

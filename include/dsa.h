@@ -230,6 +230,15 @@ dsa_status dsa_sparse_attn(const void *q, const void *k_cache, const void *v_cac
  * invalid or unsupported (the call itself then reports why). */
 size_t dsa_sparse_attn_workspace_bytes(const dsa_attn_shape *sh, dsa_dtype dt);
 
+/* Query rows whose attention shares its copies: dsa_sparse_attn (and the
+ * fused forward) gather, for each group of this many consecutive query rows
+ * of one batch entry, the K and V rows of the union of the rows' selected
+ * sets once, and attend every row to its own set only. 1: every row gathers
+ * its own selected rows. The gathered bytes of a group are the union size
+ * times the row bytes of every KV head. Depends on the shape and the
+ * device's shared memory (the current device); 0 for an invalid shape. */
+int dsa_sparse_attn_row_group(const dsa_attn_shape *sh, dsa_dtype dt);
+
 /*
  * dsa_sparse_attn_noalloc -- dsa_sparse_attn for callers that cannot pass a
  * workspace. (The pages have no counterpart: this is a library convenience.)

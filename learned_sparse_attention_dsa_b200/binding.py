@@ -28,6 +28,7 @@ STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED",
 EXPORTED = ("dsa_version", "dsa_kernel_launch_count", "dsa_status_string", "dsa_indexer_scores",
             "dsa_indexer_scores_ex", "dsa_topk",
             "dsa_topk_workspace_bytes", "dsa_sparse_attn", "dsa_sparse_attn_workspace_bytes",
+            "dsa_sparse_attn_row_group",
             "dsa_forward", "dsa_forward_workspace_bytes", "dsa_device_error", "dsa_set_wait_limit_ns", "dsa_topk_ex",
             "dsa_diag_gather",
             "dsa_indexer_kl", "dsa_indexer_backward", "dsa_indexer_backward_workspace_bytes",
@@ -93,6 +94,8 @@ def load_library(path: str = LIB_PATH):
     lib.dsa_sparse_attn.restype = ci
     lib.dsa_sparse_attn_workspace_bytes.argtypes = [ctypes.POINTER(AttnShape), ci]
     lib.dsa_sparse_attn_workspace_bytes.restype = sz
+    lib.dsa_sparse_attn_row_group.argtypes = [ctypes.POINTER(AttnShape), ci]
+    lib.dsa_sparse_attn_row_group.restype = ci
     lib.dsa_forward.argtypes = [ctypes.POINTER(ForwardArgs), vp, sz, vp]
     lib.dsa_forward.restype = ci
     lib.dsa_forward_workspace_bytes.argtypes = [ctypes.POINTER(ForwardArgs)]
@@ -348,6 +351,14 @@ def attn_shape(q, k_cache, v_cache, k: int, scale=None) -> AttnShape:
     return AttnShape(B, Tq, k_cache.shape[1], k, Hq, k_cache.shape[2], Dqk, v_cache.shape[3],
                      float(scale if scale is not None else Dqk ** -0.5),
                      ksb, kss, ksh, vsb, vss, vsh)
+
+
+def sparse_attn_row_group(q, k_cache, v_cache, k: int) -> int:
+    """dsa_sparse_attn_row_group: consecutive query rows whose attention
+    shares the gathers of their selections (1: none share)."""
+    lib = load_library()
+    sh = attn_shape(q, k_cache, v_cache, k)
+    return int(lib.dsa_sparse_attn_row_group(ctypes.byref(sh), _dt(q)))
 
 
 def sparse_attn(q, k_cache, v_cache, idx, scale=None, out=None, lse=None, want_lse=False, ws=None,

@@ -288,6 +288,12 @@ dsa_status dsa_topk(const float *scores, int B, int Tq, int L, int q_pos0, int k
     return dsa_topk_ex(scores, B, Tq, L, q_pos0, k, 0u, idx, ws, ws_bytes, stream);
 }
 
+int dsa_sparse_attn_row_group(const dsa_attn_shape *sh, dsa_dtype dt) {
+    if (check_attn_shape(sh, dt) != DSA_OK) return 0;
+    AttnProblem p = make_attn_problem(nullptr, nullptr, nullptr, nullptr, sh, dt, nullptr, nullptr, nullptr, 0);
+    return attn_row_group(p);
+}
+
 size_t dsa_sparse_attn_workspace_bytes(const dsa_attn_shape *sh, dsa_dtype dt) {
     if (check_attn_shape(sh, dt) != DSA_OK) return 0;
     AttnProblem p = make_attn_problem(nullptr, nullptr, nullptr, nullptr, sh, dt, nullptr, nullptr, nullptr, 0);

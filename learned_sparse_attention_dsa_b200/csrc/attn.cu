@@ -190,6 +190,14 @@ cudaError_t launch_attn(const AttnProblem &p, cudaStream_t stream) {
 }
 
 size_t attn_tc_workspace_bytes(const AttnProblem &p);
+bool attn_tc_takes(const AttnProblem &p);
+int perhead_row_group(const AttnProblem &p);
+
+int attn_row_group(const AttnProblem &p) {
+    if (attn_tc_takes(p)) return 1;
+    const int g = perhead_row_group(p);
+    return g > 0 ? g : 1;
+}
 
 size_t attn_workspace_bytes(const AttnProblem &p) { return attn_tc_workspace_bytes(p); }
 

@@ -20,6 +20,8 @@
 // compute half of the logit of position r, the warp updates its running max
 // and sum (online softmax in fp32, exp2 with the log2(e) prescale), and the
 // lanes, each owning D/32 output columns, accumulate the weighted value rows.
+// With several query rows the group kernel below is used instead: rows share
+// the copies of the union of their selections.
 #include <math.h>
 
 #include "common.cuh"
@@ -268,6 +270,242 @@ attn_perhead_kernel(const Args a) {
         a.lse[(size_t)row * a.H + h] = l > 0.0f ? (m + log2f(l)) / kLog2e : -INFINITY;
 }
 
+
+// Query-row groups. QG consecutive query rows of one batch entry (QG in {2,
+// 4, 8, 16}) share one gather: their selected sets are marked in one bitmap
+// per row, the union is listed in ascending position order, and the K and V
+// rows of every union position are fetched once for the group. The head's
+// m16n8k16 logits then hold QG queries at once (A-operand row r is query
+// r * QG / 16; a single query would repeat in all 16 rows), each logit is
+// masked to -inf where its position is not in that query's own set, and each
+// lane keeps the online softmax of its two rows' queries (g and g + 8). The
+// result is the per-row attention over each row's own S_t; the union only
+// shares the copies. Positions are listed as 16-bit values (L <= 65,536).
+struct GroupArgs {
+    int B, ngroups;  // batch entries; row groups per batch entry
+    int W;           // 32-bit bitmap words per row: ceil(L / 32)
+};
+
+template <int D, int QG>
+__global__ void __launch_bounds__(D == 64 ? 512 : 256, 1)
+attn_perhead_group_kernel(const Args a, const GroupArgs ga) {
+    constexpr int STAGES = 2;
+    constexpr int R = 16 / QG;  // A-operand rows per query
+    extern __shared__ __align__(128) uint8_t smem[];
+    constexpr int kChunksPerHead = D / 8;
+    const int row_chunks = a.H * kChunksPerHead;
+    const int stage_bytes = 2 * kRows * row_chunks * 16;
+    const int W = ga.W;
+    uint32_t *bm = reinterpret_cast<uint32_t *>(smem + STAGES * stage_bytes);  // [QG][W]
+    uint16_t *ulist = reinterpret_cast<uint16_t *>(bm + QG * W);                // [union]
+    __shared__ int warp_tot[kMaxHeads];
+    __shared__ int s_count;
+
+    // heavy groups (the latest rows, the largest unions) first
+    const int b = blockIdx.x % ga.B;
+    const int gi = ga.ngroups - 1 - (int)(blockIdx.x / ga.B);
+    const int i0 = gi * QG;
+    const int qn = min(QG, a.Tq - i0);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nthreads = blockDim.x;
+    const size_t row0 = (size_t)b * a.Tq + i0;
+
+    // ---- one bitmap per row of the group, then the union in position order
+    for (int w = threadIdx.x; w < QG * W; w += nthreads) bm[w] = 0u;
+    __syncthreads();
+    for (int q = 0; q < qn; ++q) {
+        const int32_t *src = a.idx + (row0 + q) * a.k;
+        for (int j = threadIdx.x; j < a.k; j += nthreads) {
+            const int s = src[j];
+            note_bad_index(&g_attn_perhead_error, s, a.L);
+            if (s >= 0 && s < a.L) atomicOr(&bm[q * W + (s >> 5)], 1u << (s & 31));
+        }
+    }
+    __syncthreads();
+    {
+        // thread i owns words [i * per, (i + 1) * per): its union count, a
+        // block-wide exclusive scan of the counts, then its positions
+        const int per = (W + nthreads - 1) / nthreads;
+        const int w0 = min(W, threadIdx.x * per), w1 = min(W, w0 + per);
+        int cnt = 0;
+        for (int w = w0; w < w1; ++w) {
+            uint32_t u = 0u;
+            for (int q = 0; q < qn; ++q) u |= bm[q * W + w];
+            cnt += __popc(u);
+        }
+        const int incl = warp_inclusive_scan(cnt);
+        if (lane == 31) warp_tot[warp] = incl;
+        __syncthreads();
+        int base = incl - cnt;
+        for (int w = 0; w < warp; ++w) base += warp_tot[w];
+        for (int w = w0; w < w1; ++w) {
+            uint32_t u = 0u;
+            for (int q = 0; q < qn; ++q) u |= bm[q * W + w];
+            while (u) {
+                const int bit = __ffs(u) - 1;
+                ulist[base++] = (uint16_t)(w * 32 + bit);
+                u &= u - 1u;
+            }
+        }
+        if (threadIdx.x == nthreads - 1) s_count = base;
+    }
+    __syncthreads();
+    const int n_sel = s_count;
+    const int n_tiles = (n_sel + kRows - 1) / kRows;
+    const uint32_t smem_base = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+    const __nv_bfloat16 *kb = a.k_cache + b * a.k_sb;
+    const __nv_bfloat16 *vb = a.v_cache + b * a.v_sb;
+
+    // copies as in attn_perhead_kernel, positions from the union list
+    const int cstep = nthreads / row_chunks;
+    const int cx = threadIdx.x % row_chunks, cr0 = threadIdx.x / row_chunks;
+    const int64_t koff = (int64_t)(cx / kChunksPerHead) * a.k_sh + (cx % kChunksPerHead) * 8;
+    const int64_t voff = (int64_t)(cx / kChunksPerHead) * a.v_sh + (cx % kChunksPerHead) * 8;
+    const uint32_t vstage_off = kRows * row_chunks * 16;
+    auto issue = [&](int tile, int stage) {
+        const uint32_t kdst = smem_base + stage * stage_bytes;
+#pragma unroll 4
+        for (int r = cr0; r < kRows; r += cstep) {
+            const int jj = tile * kRows + r;
+            const bool valid = jj < n_sel;
+            const int s = valid ? (int)ulist[jj] : 0;
+            const uint32_t dst = kdst + (r * row_chunks + (cx ^ (r & 7))) * 16;
+            cp_async16(dst, kb + (int64_t)s * a.k_ss + koff, valid);
+            cp_async16(dst + vstage_off, vb + (int64_t)s * a.v_ss + voff, valid);
+        }
+    };
+
+    // ---- this warp's head h; lane (g, t) holds queries qx[0] = g / R (row g)
+    // and qx[1] = (g + 8) / R (row g + 8) of the group
+    const int h = warp;
+    const int t4 = lane & 3, g8 = lane >> 2;
+    const int qx[2] = {g8 / R, (g8 + 8) / R};
+    constexpr int kKSteps = D / 16;
+    constexpr int kNBlk = D / 8;
+    uint32_t qf[2][kKSteps][2];  // per query: k-low and k-high pairs of each 16-wide slice
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+        const bool live = qx[x] < qn;
+        const __nv_bfloat16 *qh = a.q + ((row0 + (live ? qx[x] : 0)) * a.H + h) * D;
+#pragma unroll
+        for (int ks = 0; ks < kKSteps; ++ks) {
+            qf[x][ks][0] = live ? *reinterpret_cast<const uint32_t *>(qh + ks * 16 + 2 * t4) : 0u;
+            qf[x][ks][1] = live ? *reinterpret_cast<const uint32_t *>(qh + ks * 16 + 8 + 2 * t4) : 0u;
+        }
+    }
+    const uint32_t *bmx[2] = {bm + qx[0] * W, bm + min(qx[1], QG - 1) * W};
+    float acc[kNBlk][4];
+#pragma unroll
+    for (int j = 0; j < kNBlk; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
+    float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.0f, 0.0f};
+    const int hx = h * kChunksPerHead;
+    const int row_bytes = row_chunks * 16;
+
+#pragma unroll
+    for (int st = 0; st < STAGES - 1; ++st) {
+        if (st < n_tiles) issue(st, st);
+        cp_async_commit();
+    }
+    for (int tile = 0; tile < n_tiles; ++tile) {
+        const int stage = tile % STAGES;
+        if (tile + STAGES - 1 < n_tiles) issue(tile + STAGES - 1, (tile + STAGES - 1) % STAGES);
+        cp_async_commit();
+        cp_async_wait<STAGES - 1>();
+        __syncthreads();
+
+        const uint32_t kt = smem_base + stage * stage_bytes;
+        const uint32_t vt = kt + kRows * row_bytes;
+        // logits: rows g (query qx[0]) and g + 8 (query qx[1]) of each 8-position block
+        float sc[2][2][2];  // [block][position pair][query]
+#pragma unroll
+        for (int nb = 0; nb < 2; ++nb) {
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int c = 0; c < kChunksPerHead; c += 4) {
+                const int p = nb * 8 + (lane & 7);
+                const int xx = hx + c + (lane >> 3);
+                uint32_t bf[4];
+                ldmatrix_x4(kt + p * row_bytes + ((xx ^ (p & 7)) << 4), bf);
+                mma_bf16_16816(d, qf[0][c / 2][0], qf[1][c / 2][0], qf[0][c / 2][1], qf[1][c / 2][1], bf[0], bf[1]);
+                mma_bf16_16816(d, qf[0][c / 2 + 1][0], qf[1][c / 2 + 1][0], qf[0][c / 2 + 1][1],
+                               qf[1][c / 2 + 1][1], bf[2], bf[3]);
+            }
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int jj = tile * kRows + nb * 8 + 2 * t4 + e;
+                const int s = jj < n_sel ? (int)ulist[jj] : -1;
+#pragma unroll
+                for (int x = 0; x < 2; ++x) {
+                    const bool in = s >= 0 && ((bmx[x][s >> 5] >> (s & 31)) & 1u);
+                    sc[nb][e][x] = in ? d[2 * x + e] * a.scale_log2 : -INFINITY;
+                }
+            }
+        }
+        // online softmax per query (the four lanes of a row share it)
+        float pr[2][2][2];
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+            float zmax = fmaxf(fmaxf(sc[0][0][x], sc[0][1][x]), fmaxf(sc[1][0][x], sc[1][1][x]));
+            zmax = fmaxf(zmax, __shfl_xor_sync(0xffffffffu, zmax, 1));
+            zmax = fmaxf(zmax, __shfl_xor_sync(0xffffffffu, zmax, 2));
+            const float m_new = fmaxf(m[x], zmax);
+            const float mr = m_new == -INFINITY ? 0.0f : m_new;
+            float psum = 0.0f;
+#pragma unroll
+            for (int nb = 0; nb < 2; ++nb)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    pr[nb][e][x] = ex2_approx(sc[nb][e][x] - mr);
+                    psum += pr[nb][e][x];
+                }
+            psum += __shfl_xor_sync(0xffffffffu, psum, 1);
+            psum += __shfl_xor_sync(0xffffffffu, psum, 2);
+            if (m_new != m[x]) {  // uniform over the row's four lanes
+                const float corr = ex2_approx(m[x] - mr);
+                l[x] *= corr;
+#pragma unroll
+                for (int j = 0; j < kNBlk; ++j) {
+                    acc[j][2 * x] *= corr;
+                    acc[j][2 * x + 1] *= corr;
+                }
+                m[x] = m_new;
+            }
+            l[x] += psum;
+        }
+        // weighted value rows: P rows g and g + 8 as the A operand
+        const uint32_t pa0 = pack_bf16x2(pr[0][0][0], pr[0][1][0]), pa1 = pack_bf16x2(pr[0][0][1], pr[0][1][1]);
+        const uint32_t pa2 = pack_bf16x2(pr[1][0][0], pr[1][1][0]), pa3 = pack_bf16x2(pr[1][0][1], pr[1][1][1]);
+#pragma unroll
+        for (int j = 0; j < kNBlk; j += 2) {
+            const int mi = lane >> 3;
+            const int p = (mi & 1) * 8 + (lane & 7);
+            const int xx = hx + j + (mi >> 1);
+            uint32_t bf[4];
+            ldmatrix_x4_trans(vt + p * row_bytes + ((xx ^ (p & 7)) << 4), bf);
+            mma_bf16_16816(acc[j], pa0, pa1, pa2, pa3, bf[0], bf[1]);
+            mma_bf16_16816(acc[j + 1], pa0, pa1, pa2, pa3, bf[2], bf[3]);
+        }
+        __syncthreads();  // the stage is refilled by a later iteration's issue
+    }
+    cp_async_wait<0>();
+
+    // the R rows of a query hold the same values: row g writes the column
+    // blocks j with j % R == g % R
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+        if (qx[x] >= qn) continue;
+        const float inv = l[x] > 0.0f ? 1.0f / l[x] : 0.0f;
+        __nv_bfloat16 *dst = a.out + ((row0 + qx[x]) * a.H + h) * D;
+#pragma unroll
+        for (int j = 0; j < kNBlk; ++j)
+            if ((j % R) == (g8 % R))
+                *reinterpret_cast<__nv_bfloat162 *>(dst + j * 8 + 2 * t4) =
+                    __floats2bfloat162_rn(acc[j][2 * x] * inv, acc[j][2 * x + 1] * inv);
+        if (a.lse != nullptr && t4 == 0 && g8 % R == 0)
+            a.lse[(row0 + qx[x]) * a.H + h] = l[x] > 0.0f ? (m[x] + log2f(l[x])) / kLog2e : -INFINITY;
+    }
+}
+
 }  // namespace
 
 unsigned int attn_perhead_take_device_error() {
@@ -277,24 +515,64 @@ unsigned int attn_perhead_take_device_error() {
     return v;
 }
 
-cudaError_t launch_attn_perhead(const AttnProblem &p, cudaStream_t stream, bool *taken) {
-    *taken = false;
-    if (p.dt != DSA_BF16 || p.Hq != p.Hkv || p.Hq > (p.Dqk == 64 ? kMaxHeads : 8)) return cudaSuccess;
-    if ((p.Hq & (p.Hq - 1)) != 0) return cudaSuccess;  // the row layout uses shifts
-    if (!((p.Dqk == 64 && p.Dv == 64) || (p.Dqk == 128 && p.Dv == 128))) return cudaSuccess;
+namespace {
+
+// Whether the per-head kernels take a shape, their shared-memory footprint,
+// and the query-row group: the largest QG whose bitmaps and union list fit
+// next to the stages within the single-row kernel's footprint or two CTAs
+// per SM (QG = 1: one row per CTA).
+struct PerheadPlan {
+    bool ok = false;
+    size_t smem = 0, smem_g = 0;
+    int qg = 1, W = 0;
+};
+
+PerheadPlan plan_perhead(const AttnProblem &p, const DeviceInfo &info) {
+    PerheadPlan pl;
+    if (p.dt != DSA_BF16 || p.Hq != p.Hkv || p.Hq > (p.Dqk == 64 ? kMaxHeads : 8)) return pl;
+    if ((p.Hq & (p.Hq - 1)) != 0) return pl;  // the row layout uses shifts
+    if (!((p.Dqk == 64 && p.Dv == 64) || (p.Dqk == 128 && p.Dv == 128))) return pl;
     if (((uintptr_t)p.k_cache | (uintptr_t)p.v_cache | (uintptr_t)p.q) % 16 != 0 || (uintptr_t)p.out % 4 != 0)
-        return cudaSuccess;
-    if (p.k_ss % 8 || p.k_sb % 8 || p.k_sh % 8 || p.v_ss % 8 || p.v_sb % 8 || p.v_sh % 8) return cudaSuccess;
-    DeviceInfo info;
-    cudaError_t err = device_info(&info);
-    if (err != cudaSuccess) return err;
+        return pl;
+    if (p.k_ss % 8 || p.k_sb % 8 || p.k_sh % 8 || p.v_ss % 8 || p.v_sb % 8 || p.v_sh % 8) return pl;
     const size_t stage_bytes = 2ull * kRows * p.Hq * p.Dqk * 2;
     const size_t sel_bytes = sizeof(int32_t) * (size_t)p.k;
     // two stages: more CTAs per SM issue copies (three stages only help when
     // the copies are few)
-    const int stages = 2;
-    const size_t smem = stages * stage_bytes + sel_bytes;
-    if (smem > (size_t)info.max_smem_optin) return cudaSuccess;
+    pl.smem = 2 * stage_bytes + sel_bytes;
+    if (pl.smem > (size_t)info.max_smem_optin) return pl;
+    pl.ok = true;
+    if (p.Tq >= 2 && p.L <= 65536) {
+        pl.W = (p.L + 31) / 32;
+        const size_t budget = pl.smem > 112 * 1024 ? pl.smem : 112 * 1024;
+        for (int qg = 16; qg >= 2; qg /= 2) {
+            const size_t ucap = (size_t)(p.L < qg * p.k ? p.L : qg * p.k);
+            const size_t smem_g = 2 * stage_bytes + (size_t)qg * pl.W * 4 + ((ucap * 2 + 15) & ~size_t(15));
+            if (smem_g > budget || smem_g > (size_t)info.max_smem_optin) continue;
+            pl.qg = qg;
+            pl.smem_g = smem_g;
+            break;
+        }
+    }
+    return pl;
+}
+
+}  // namespace
+
+int perhead_row_group(const AttnProblem &p) {
+    DeviceInfo info;
+    if (device_info(&info) != cudaSuccess) return 0;
+    const PerheadPlan pl = plan_perhead(p, info);
+    return pl.ok ? pl.qg : 0;
+}
+
+cudaError_t launch_attn_perhead(const AttnProblem &p, cudaStream_t stream, bool *taken) {
+    *taken = false;
+    DeviceInfo info;
+    cudaError_t err = device_info(&info);
+    if (err != cudaSuccess) return err;
+    const PerheadPlan pl = plan_perhead(p, info);
+    if (!pl.ok) return cudaSuccess;
     Args a;
     a.q = static_cast<const __nv_bfloat16 *>(p.q);
     a.k_cache = static_cast<const __nv_bfloat16 *>(p.k_cache);
@@ -309,10 +587,32 @@ cudaError_t launch_attn_perhead(const AttnProblem &p, cudaStream_t stream, bool 
     a.out = static_cast<__nv_bfloat16 *>(p.out);
     a.lse = p.lse;
     *taken = true;
+    if (pl.qg > 1) {  // groups of QG query rows share the gathers of their union
+        const int qg = pl.qg;
+        GroupArgs ga;
+        ga.B = p.B;
+        ga.ngroups = (p.Tq + qg - 1) / qg;
+        ga.W = pl.W;
+        void (*gk)(const Args, const GroupArgs) = nullptr;
+        if (p.Dqk == 64) {
+            gk = qg == 16 ? attn_perhead_group_kernel<64, 16> : qg == 8 ? attn_perhead_group_kernel<64, 8>
+               : qg == 4 ? attn_perhead_group_kernel<64, 4> : attn_perhead_group_kernel<64, 2>;
+        } else {
+            gk = qg == 16 ? attn_perhead_group_kernel<128, 16> : qg == 8 ? attn_perhead_group_kernel<128, 8>
+               : qg == 4 ? attn_perhead_group_kernel<128, 4> : attn_perhead_group_kernel<128, 2>;
+        }
+        err = cudaFuncSetAttribute(gk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem_g);
+        if (err != cudaSuccess) return err;
+        const long long grid = (long long)p.B * ga.ngroups;
+        if (grid > 0x7fffffffLL) return cudaErrorInvalidValue;
+        gk<<<(unsigned)grid, p.Hq * 32, pl.smem_g, stream>>>(a, ga);
+        count_launch();
+        return cudaGetLastError();
+    }
     auto kern = p.Dqk == 64 ? attn_perhead_kernel<64, 2> : attn_perhead_kernel<128, 2>;
-    err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem);
     if (err != cudaSuccess) return err;
-    kern<<<p.B * p.Tq, p.Hq * 32, smem, stream>>>(a);
+    kern<<<p.B * p.Tq, p.Hq * 32, pl.smem, stream>>>(a);
     count_launch();
     return cudaGetLastError();
 }

@@ -740,6 +740,12 @@ size_t attn_tc_workspace_bytes(const AttnProblem &p) {
     return n_pairs * splits * ((size_t)p.Dv + 2) * sizeof(float);
 }
 
+bool attn_tc_takes(const AttnProblem &p) {
+    if (attn_mla_tc_supported(p) || attn_mla_supported(p)) return true;
+    int which;
+    return shape_supported(p, &which);
+}
+
 cudaError_t launch_attn_tc(const AttnProblem &p, cudaStream_t stream, bool *taken) {
     *taken = false;
     DeviceInfo info;

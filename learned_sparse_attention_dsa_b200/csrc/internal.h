@@ -79,6 +79,9 @@ struct AttnProblem {
     size_t ws_bytes;
 };
 size_t attn_workspace_bytes(const AttnProblem &p);
+// Query rows of one batch entry whose attention shares the gathers of their
+// selections (1: every row gathers its own).
+int attn_row_group(const AttnProblem &p);
 cudaError_t launch_attn(const AttnProblem &p, cudaStream_t stream);
 
 // The argument checks of dsa_sparse_attn (everything but the workspace).

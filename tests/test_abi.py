@@ -76,6 +76,7 @@ def test_attention_shape_checks(dsa_lib):
     assert dsa_lib.dsa_sparse_attn(fake, fake, fake, fake, ctypes.byref(sh), 1, fake, None, None, 0, None) == 1
     sh = AttnShape(1, 1, 8, 4, 8, 4, 64, 64, 0.1, 512, 0, 64, 512, 64, 64)  # zero row stride
     assert dsa_lib.dsa_sparse_attn(fake, fake, fake, fake, ctypes.byref(sh), 1, fake, None, None, 0, None) == 1
+    assert dsa_lib.dsa_sparse_attn_row_group(ctypes.byref(sh), 1) == 0  # invalid shape
 
 
 def test_diag_gather_argument_checks(dsa_lib):

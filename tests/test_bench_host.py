@@ -134,3 +134,16 @@ def test_traffic_entries_name_their_profile():
     """Every committed traffic figure names the profile summary it came from."""
     for (wl, stage), e in bench.DRAM_TRAFFIC_PER_LAUNCH.items():
         assert os.path.exists(os.path.join(bench.ROOT, e["profile"])), (wl, stage)
+
+
+def test_union_rows_counts_each_group_once():
+    """The rows a grouped attention fetches: distinct valid positions per
+    group of consecutive query rows (padding and out-of-range entries not
+    counted), the plain valid count for groups of one."""
+    import torch
+    import bench
+    idx = torch.tensor([[[0, 1, 2, -1], [1, 2, 3, -1], [5, 6, -1, -1]],
+                        [[7, 7, -1, -1], [0, 9, -1, -1], [-1, -1, -1, -1]]], dtype=torch.int32)
+    assert bench.union_rows(idx, 1, 8) == 3 + 3 + 2 + 2 + 1 + 0  # 9 is out of range, 7 counted twice
+    assert bench.union_rows(idx, 2, 8) == 4 + 2 + 2 + 0          # {0..3}, {5, 6}, {0, 7}, {}
+    assert bench.union_rows(idx, 4, 8) == 6 + 2

@@ -59,6 +59,11 @@ MEDIUM = {
     # 32 query heads over one latent row: the CUDA-core latent-row kernel
     "latent_h32": Workload("latent_h32", B=2, Tq=1, L=3000, q_pos0=2999, H_I=64, d_I=128, k=256,
                            Hq=32, Hkv=1, Dqk=576, Dv=512, kv_alias=True, seed=26),
+    # one KV head per query head of width 128, a chunk of 45 rows (groups of
+    # query rows sharing their gathers, the last one partial) after 255
+    # positions, k not a multiple of the 16-position stage
+    "perhead_d128_chunk": Workload("perhead_d128_chunk", B=2, Tq=45, L=300, q_pos0=255, H_I=64, d_I=128, k=100,
+                                   Hq=4, Hkv=4, Dqk=128, Dv=128, seed=27),
 }
 
 FULL_ROWS = {  # None: every query row
@@ -192,8 +197,25 @@ def test_topk_stage(cuda, kind, L, Tq, q_pos0, k):
     assert np.array_equal(got, ref)
 
 
+def test_attention_row_groups(cuda):
+    """Per-head prefill shares gathers across 16 query rows (8 heads of 64,
+    L = 520) or fewer for wider rows; decode rows and the 16-head and
+    latent-row kernels gather per row."""
+    def group(name, Tq=None):
+        wl = MEDIUM[name] if Tq is None else MEDIUM[name].replace(Tq=Tq, q_pos0=MEDIUM[name].L - Tq,
+                                                                   name=f"{name}_tq{Tq}")
+        _, dev = _inputs(wl)
+        return binding.sparse_attn_row_group(dev["q"], dev["k_cache"], dev["v_cache"], wl.k)
+    assert group("prefill_perhead_520") == 16
+    assert group("perhead_d128_chunk") >= 2
+    assert group("prefill_perhead_520", Tq=1) == 1
+    assert group("prefill_mqa_700") == 1
+    assert group("decode_latent_3000") == 1
+
+
 @pytest.mark.parametrize("name", ["prefill_mqa_700", "decode_latent_3000", "latent_chunk",
-                                  "latent_single", "latent_h32", "prefill_perhead_520", "tiny_f32"])
+                                  "latent_single", "latent_h32", "prefill_perhead_520", "perhead_d128_chunk",
+                                  "tiny_f32"])
 def test_sparse_attn_stage_shuffled_and_padded(cuda, name):
     """Attention on its own, with the oracle's index sets shuffled and padded."""
     wl = MEDIUM[name]
