@@ -280,7 +280,8 @@ attn_perhead_kernel(const Args a) {
 // masked to -inf where its position is not in that query's own set, and each
 // lane keeps the online softmax of its two rows' queries (g and g + 8). The
 // result is the per-row attention over each row's own S_t; the union only
-// shares the copies. Positions are listed as 16-bit values (L <= 65,536).
+// shares the copies. A union entry packs the position (16 bits, L <= 65,536)
+// with the mask of the group's rows that selected it.
 struct GroupArgs {
     int B, ngroups;  // batch entries; row groups per batch entry
     int W;           // 32-bit bitmap words per row: ceil(L / 32)
@@ -297,7 +298,7 @@ attn_perhead_group_kernel(const Args a, const GroupArgs ga) {
     const int stage_bytes = 2 * kRows * row_chunks * 16;
     const int W = ga.W;
     uint32_t *bm = reinterpret_cast<uint32_t *>(smem + STAGES * stage_bytes);  // [QG][W]
-    uint16_t *ulist = reinterpret_cast<uint16_t *>(bm + QG * W);                // [union]
+    uint32_t *ulist = bm + QG * W;  // [union]: position | rows' mask << 16
     __shared__ int warp_tot[kMaxHeads];
     __shared__ int s_count;
 
@@ -339,11 +340,19 @@ attn_perhead_group_kernel(const Args a, const GroupArgs ga) {
         int base = incl - cnt;
         for (int w = 0; w < warp; ++w) base += warp_tot[w];
         for (int w = w0; w < w1; ++w) {
+            uint32_t wq[QG];
             uint32_t u = 0u;
-            for (int q = 0; q < qn; ++q) u |= bm[q * W + w];
+#pragma unroll
+            for (int q = 0; q < QG; ++q) {
+                wq[q] = q < qn ? bm[q * W + w] : 0u;
+                u |= wq[q];
+            }
             while (u) {
                 const int bit = __ffs(u) - 1;
-                ulist[base++] = (uint16_t)(w * 32 + bit);
+                uint32_t mask = 0u;
+#pragma unroll
+                for (int q = 0; q < QG; ++q) mask |= ((wq[q] >> bit) & 1u) << q;
+                ulist[base++] = (uint32_t)(w * 32 + bit) | (mask << 16);
                 u &= u - 1u;
             }
         }
@@ -368,7 +377,7 @@ attn_perhead_group_kernel(const Args a, const GroupArgs ga) {
         for (int r = cr0; r < kRows; r += cstep) {
             const int jj = tile * kRows + r;
             const bool valid = jj < n_sel;
-            const int s = valid ? (int)ulist[jj] : 0;
+            const int s = valid ? (int)(ulist[jj] & 0xFFFFu) : 0;
             const uint32_t dst = kdst + (r * row_chunks + (cx ^ (r & 7))) * 16;
             cp_async16(dst, kb + (int64_t)s * a.k_ss + koff, valid);
             cp_async16(dst + vstage_off, vb + (int64_t)s * a.v_ss + voff, valid);
@@ -393,7 +402,6 @@ attn_perhead_group_kernel(const Args a, const GroupArgs ga) {
             qf[x][ks][1] = live ? *reinterpret_cast<const uint32_t *>(qh + ks * 16 + 8 + 2 * t4) : 0u;
         }
     }
-    const uint32_t *bmx[2] = {bm + qx[0] * W, bm + min(qx[1], QG - 1) * W};
     float acc[kNBlk][4];
 #pragma unroll
     for (int j = 0; j < kNBlk; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
@@ -433,10 +441,10 @@ attn_perhead_group_kernel(const Args a, const GroupArgs ga) {
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
                 const int jj = tile * kRows + nb * 8 + 2 * t4 + e;
-                const int s = jj < n_sel ? (int)ulist[jj] : -1;
+                const uint32_t rows_in = jj < n_sel ? ulist[jj] >> 16 : 0u;  // rows that selected it
 #pragma unroll
                 for (int x = 0; x < 2; ++x) {
-                    const bool in = s >= 0 && ((bmx[x][s >> 5] >> (s & 31)) & 1u);
+                    const bool in = (rows_in >> qx[x]) & 1u;
                     sc[nb][e][x] = in ? d[2 * x + e] * a.scale_log2 : -INFINITY;
                 }
             }
@@ -547,7 +555,7 @@ PerheadPlan plan_perhead(const AttnProblem &p, const DeviceInfo &info) {
         const size_t budget = pl.smem > 112 * 1024 ? pl.smem : 112 * 1024;
         for (int qg = 16; qg >= 2; qg /= 2) {
             const size_t ucap = (size_t)(p.L < qg * p.k ? p.L : qg * p.k);
-            const size_t smem_g = 2 * stage_bytes + (size_t)qg * pl.W * 4 + ((ucap * 2 + 15) & ~size_t(15));
+            const size_t smem_g = 2 * stage_bytes + (size_t)qg * pl.W * 4 + ucap * 4;
             if (smem_g > budget || smem_g > (size_t)info.max_smem_optin) continue;
             pl.qg = qg;
             pl.smem_g = smem_g;
