@@ -66,8 +66,8 @@ DRAM_TRAFFIC_PER_LAUNCH = {
                                 "profile": "profiles/indexer_tc_e4m3_decode32k.md"},
     ("prefill8k", "topk"): {"bytes": 170.64e6, "sources": _TOPK, "digest": "65454fadbee778ff",
                             "profile": "profiles/dram_stages_prefill8k.md"},
-    ("prefill8k", "attn"): {"bytes": 92.63e6, "sources": ["attn_perhead.cu", "common.cuh"],
-                            "digest": "e351fb69a1804e15", "profile": "profiles/dram_stages_prefill8k.md"},
+    ("prefill8k", "attn"): {"bytes": 92.45e6, "sources": ["attn_perhead.cu", "common.cuh"],
+                            "digest": "f553d8ec079b5f95", "profile": "profiles/dram_stages_prefill8k.md"},
 }
 
 
