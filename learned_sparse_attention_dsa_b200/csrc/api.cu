@@ -222,7 +222,7 @@ dsa_status dsa_device_error(dsa_stream_t stream) {
     unsigned int words = dsa::indexer_take_device_error() | dsa::attn_mla_tc_take_device_error() |
                          dsa::indexer_bwd_take_device_error() | dsa::attn_tc_take_device_error() |
                          dsa::attn_mla_take_device_error() | dsa::attn_perhead_take_device_error() |
-                         dsa::attn_cc_take_device_error();
+                         dsa::attn_cc_take_device_error() | dsa::attn_mqa_tc_take_device_error();
     if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
     if (words & kErrTimeout) return DSA_ERR_TIMEOUT;
     return (words & kErrBadIndex) ? DSA_ERR_BAD_INDEX : DSA_OK;
@@ -230,7 +230,7 @@ dsa_status dsa_device_error(dsa_stream_t stream) {
 
 dsa_status dsa_set_wait_limit_ns(uint64_t ns) {
     if (dsa::indexer_set_wait_limit(ns) != cudaSuccess || dsa::indexer_bwd_set_wait_limit(ns) != cudaSuccess ||
-        dsa::attn_mla_tc_set_wait_limit(ns) != cudaSuccess)
+        dsa::attn_mla_tc_set_wait_limit(ns) != cudaSuccess || dsa::attn_mqa_tc_set_wait_limit(ns) != cudaSuccess)
         return DSA_ERR_CUDA;
     return DSA_OK;
 }

@@ -193,7 +193,11 @@ size_t attn_tc_workspace_bytes(const AttnProblem &p);
 bool attn_tc_takes(const AttnProblem &p);
 int perhead_row_group(const AttnProblem &p);
 
+bool attn_mqa_tc_supported(const AttnProblem &p);
+int attn_mqa_tc_row_group();
+
 int attn_row_group(const AttnProblem &p) {
+    if (attn_mqa_tc_supported(p)) return attn_mqa_tc_row_group();
     if (attn_tc_takes(p)) return 1;
     const int g = perhead_row_group(p);
     return g > 0 ? g : 1;

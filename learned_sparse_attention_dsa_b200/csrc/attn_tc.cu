@@ -712,6 +712,8 @@ cudaError_t launch_attn_mla(const AttnProblem &p, const DeviceInfo &info, cudaSt
 bool attn_mla_tc_supported(const AttnProblem &p);
 size_t attn_mla_tc_workspace_bytes(const AttnProblem &p, int sm_count);
 cudaError_t launch_attn_mla_tc(const AttnProblem &p, const DeviceInfo &info, cudaStream_t stream);
+bool attn_mqa_tc_supported(const AttnProblem &p);
+cudaError_t launch_attn_mqa_tc(const AttnProblem &p, cudaStream_t stream);
 
 cudaError_t launch_attn_combine(const float *part_o, const float *part_ml, int n_pairs, int splits, int DV,
                                 __nv_bfloat16 *out, float *lse, cudaStream_t stream) {
@@ -731,6 +733,7 @@ size_t attn_tc_workspace_bytes(const AttnProblem &p) {
     DeviceInfo info;
     if (device_info(&info) != cudaSuccess) return 0;
     if (attn_mla_tc_supported(p)) return attn_mla_tc_workspace_bytes(p, info.sm_count);
+    if (attn_mqa_tc_supported(p)) return 0;
     if (attn_mla_supported(p)) return attn_mla_workspace_bytes(p, info.sm_count);
     int which;
     if (!shape_supported(p, &which)) return 0;
@@ -741,7 +744,7 @@ size_t attn_tc_workspace_bytes(const AttnProblem &p) {
 }
 
 bool attn_tc_takes(const AttnProblem &p) {
-    if (attn_mla_tc_supported(p) || attn_mla_supported(p)) return true;
+    if (attn_mla_tc_supported(p) || attn_mla_supported(p) || attn_mqa_tc_supported(p)) return true;
     int which;
     return shape_supported(p, &which);
 }
@@ -760,6 +763,11 @@ cudaError_t launch_attn_tc(const AttnProblem &p, cudaStream_t stream, bool *take
         if (attn_tc_workspace_bytes(p) > p.ws_bytes) return cudaSuccess;
         *taken = true;
         return launch_attn_mla(p, info, stream);
+    }
+    // groups of 8 query rows of 16 heads sharing the gathers of their union
+    if (attn_mqa_tc_supported(p)) {
+        *taken = true;
+        return launch_attn_mqa_tc(p, stream);
     }
     int which;
     if (!shape_supported(p, &which)) return cudaSuccess;

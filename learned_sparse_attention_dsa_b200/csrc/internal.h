@@ -144,10 +144,12 @@ unsigned int attn_tc_take_device_error();
 unsigned int attn_mla_take_device_error();
 unsigned int attn_perhead_take_device_error();
 unsigned int attn_cc_take_device_error();
+unsigned int attn_mqa_tc_take_device_error();
 // Limit of the bounded waits of the kernel families that have them (0: every
 // bounded wait gives up before its role issues anything).
 cudaError_t indexer_set_wait_limit(unsigned long long ns);
 cudaError_t indexer_bwd_set_wait_limit(unsigned long long ns);
 cudaError_t attn_mla_tc_set_wait_limit(unsigned long long ns);
+cudaError_t attn_mqa_tc_set_wait_limit(unsigned long long ns);
 
 }  // namespace dsa

@@ -64,6 +64,11 @@ MEDIUM = {
     # positions, k not a multiple of the 16-position stage
     "perhead_d128_chunk": Workload("perhead_d128_chunk", B=2, Tq=45, L=300, q_pos0=255, H_I=64, d_I=128, k=100,
                                    Hq=4, Hkv=4, Dqk=128, Dv=128, seed=27),
+    # 16 heads over one KV head of width 128 in enough groups of 8 query rows
+    # for the tensor-core group kernel; k not a multiple of the 64-row tile,
+    # a partial last group in each batch entry
+    "mqa128_groups": Workload("mqa128_groups", B=3, Tq=397, L=600, q_pos0=203, H_I=64, d_I=128, k=300,
+                              Hq=16, Hkv=1, Dqk=128, Dv=128, seed=28),
 }
 
 FULL_ROWS = {  # None: every query row
@@ -199,8 +204,9 @@ def test_topk_stage(cuda, kind, L, Tq, q_pos0, k):
 
 def test_attention_row_groups(cuda):
     """Per-head prefill shares gathers across 16 query rows (8 heads of 64,
-    L = 520) or fewer for wider rows; decode rows and the 16-head and
-    latent-row kernels gather per row."""
+    L = 520) or fewer for wider rows, 16-head prefill across 8 rows when the
+    groups cover the GPU; decode rows and the latent-row kernels gather per
+    row."""
     def group(name, Tq=None):
         wl = MEDIUM[name] if Tq is None else MEDIUM[name].replace(Tq=Tq, q_pos0=MEDIUM[name].L - Tq,
                                                                    name=f"{name}_tq{Tq}")
@@ -209,13 +215,15 @@ def test_attention_row_groups(cuda):
     assert group("prefill_perhead_520") == 16
     assert group("perhead_d128_chunk") >= 2
     assert group("prefill_perhead_520", Tq=1) == 1
-    assert group("prefill_mqa_700") == 1
+    assert group("prefill_mqa_700") == 8
+    assert group("mqa128_groups") == 8
+    assert group("chunked_prefill") == 1  # too few groups of 8 rows to cover the GPU
     assert group("decode_latent_3000") == 1
 
 
 @pytest.mark.parametrize("name", ["prefill_mqa_700", "decode_latent_3000", "latent_chunk",
                                   "latent_single", "latent_h32", "prefill_perhead_520", "perhead_d128_chunk",
-                                  "tiny_f32"])
+                                  "mqa128_groups", "tiny_f32"])
 def test_sparse_attn_stage_shuffled_and_padded(cuda, name):
     """Attention on its own, with the oracle's index sets shuffled and padded."""
     wl = MEDIUM[name]
