@@ -26,9 +26,11 @@
 // P twice, the union list):
 //   warps 0-3   softmax, one thread per row (TMEM lane), the Q rows into TMEM
 //               first (staged by TMA over the ring)
-//   warps 4-11  gather the K and V boxes (64 columns, 128-byte swizzle) of 64
-//               union positions per tile with 16-byte cp.async
-//   warp 12     TMEM allocation, the Q staging by TMA, and one thread issuing
+//   warps 4-13  gather the K and V boxes (64 columns, 128-byte swizzle) of 64
+//               union positions per tile with 16-byte cp.async (the rate at
+//               which cp.async is issued grows with the number of issuing
+//               warps: ~2,450 cycles per 40 KB tile with eight)
+//   warp 14     TMEM allocation, the Q staging by TMA, and one thread issuing
 //               QK^T and PV as each becomes ready
 // Every mbarrier wait is bounded; on a timeout the CTA records an error word,
 // waits for the copies and MMAs it issued, frees TMEM and returns.
@@ -53,9 +55,9 @@ constexpr int DV = 128;
 constexpr int kTileN = 64;                   // union positions per tile
 constexpr int kSlots = 3;
 constexpr int kSoftThreads = kM;             // one per row
-constexpr int kGatherThreads = 256;
-constexpr int kMmaWarp = (kSoftThreads + kGatherThreads) / 32;  // 12
-constexpr int kThreads = (kMmaWarp + 1) * 32;                   // 416
+constexpr int kGatherThreads = 320;
+constexpr int kMmaWarp = (kSoftThreads + kGatherThreads) / 32;  // 14
+constexpr int kThreads = (kMmaWarp + 1) * 32;                   // 480
 constexpr uint32_t kBox = kTileN * 128;      // 8 KB: 64 rows of 64 bf16 columns
 constexpr uint32_t kQBox = kM * 128;         // 16 KB: 128 rows of 64 bf16 columns
 constexpr uint32_t kPBytes = kM * kTileN * 2;
@@ -365,19 +367,23 @@ attn_mqa_group_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MqaArgs
             const uint32_t mb0 = __ballot_sync(0xffffffffu, (e0 >> (16 + qb)) & 1u);
             const uint32_t mb1 = __ballot_sync(0xffffffffu, (e1 >> (16 + qb)) & 1u);
             const uint32_t mlo = lane < 16 ? ma0 : mb0, mhi = lane < 16 ? ma1 : mb1;
-            float mt = -INFINITY;
+            // positions either of the warp's queries selected (the same in
+            // every lane): the others need no exponent below
+            const uint32_t any_lo = ma0 | mb0, any_hi = ma1 | mb1;
+            float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
                 const float z = ((mlo >> j) & 1u) ? __uint_as_float(x[j]) * a.scale_log2 : -INFINITY;
                 x[j] = __float_as_uint(z);
-                mt = fmaxf(mt, z);
+                mq[j & 3] = fmaxf(mq[j & 3], z);
             }
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
                 const float z = ((mhi >> j) & 1u) ? __uint_as_float(x[32 + j]) * a.scale_log2 : -INFINITY;
                 x[32 + j] = __float_as_uint(z);
-                mt = fmaxf(mt, z);
+                mq[j & 3] = fmaxf(mq[j & 3], z);
             }
+            const float mt = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
             // P buffer t % 2 was last read by PV of tile t - 2
             if (t >= 2 && !mbar_wait(&pv_done[t & 1], (uint32_t)((t - 2) >> 1) & 1u)) ok = false;
             if (!__all_sync(0xffffffffu, ok)) break;
@@ -412,19 +418,23 @@ attn_mqa_group_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const MqaArgs
                 l *= f;
             }
             m_ref = m_new;
-            // p = 2^(z - m_ref); masked positions have z = -inf, so p = 0
+            // p = 2^(z - m_ref); masked positions have z = -inf, so p = 0, and
+            // positions neither query of the warp selected skip the exponent
             const float mr = m_ref == -INFINITY ? 0.0f : m_ref;
             uint32_t pk[32];
-            float ps0 = 0.0f, ps1 = 0.0f;
+            float ps[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
-                const float p0 = ex2_approx(__uint_as_float(x[2 * j]) - mr);
-                const float p1 = ex2_approx(__uint_as_float(x[2 * j + 1]) - mr);
-                ps0 += p0;
-                ps1 += p1;
+                const int e0 = 2 * j, e1 = 2 * j + 1;
+                const uint32_t any = e0 < 32 ? any_lo : any_hi;
+                float p0 = 0.0f, p1 = 0.0f;
+                if ((any >> (e0 & 31)) & 1u) p0 = ex2_approx(__uint_as_float(x[e0]) - mr);
+                if ((any >> (e1 & 31)) & 1u) p1 = ex2_approx(__uint_as_float(x[e1]) - mr);
+                ps[(2 * j) & 3] += p0;
+                ps[(2 * j + 1) & 3] += p1;
                 pk[j] = pack_bf16x2(p0, p1);
             }
-            l += ps0 + ps1;
+            l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
             // P row r of buffer t % 2: 128 bytes, 16-byte chunk c at c ^ (r % 8)
             uint8_t *prow = p_sm + (t & 1) * kPBytes + r * 128;
 #pragma unroll
