@@ -545,9 +545,12 @@ def measure_forward(wl, args, binding, device, world, rank, local, peaks):
         gbs = gathered / (att["ms"] / 1e3) / 1e9
         att["gather"] = {"gathered_bytes": gathered, "GB/s": gbs,
                          "ceiling_GB/s": ceiling["GB/s"], "frac_of_ceiling": gbs / ceiling["GB/s"],
-                         "ceiling": "builder-measured: the same selected K and V rows gathered into shared memory "
-                                    "with no arithmetic (dsa_diag_gather, 16-byte cp.async; fastest of 8-, 16- and "
-                                    f"32-row tiles: {ceiling['tile_rows']}), {ceiling['ms']:.3f} ms"}
+                         "ceiling": "builder-measured: the rate at which every query row's selected K and V rows "
+                                    "are gathered into shared memory with no arithmetic (dsa_diag_gather, 16-byte "
+                                    "cp.async; fastest of 8-, 16- and 32-row tiles: "
+                                    f"{ceiling['tile_rows']}; {ceiling['ms']:.3f} ms for "
+                                    f"{ceiling['gathered_bytes'] / 1e9:.1f} GB); gathered_bytes are the rows this "
+                                    "attention fetches (the union rows of each group when rows share gathers)"}
         att["note"] = ("the gathered rows are mostly served by L2 (the KV cache is smaller than L2 and each row "
                        "is selected by many queries): hbm_frac compares them with the HBM copy rate, "
                        "gather.frac_of_ceiling with the gather alone")
