@@ -147,3 +147,19 @@ def test_union_rows_counts_each_group_once():
     assert bench.union_rows(idx, 1, 8) == 3 + 3 + 2 + 2 + 1 + 0  # 9 is out of range, 7 counted twice
     assert bench.union_rows(idx, 2, 8) == 4 + 2 + 2 + 0          # {0..3}, {5, 6}, {0, 7}, {}
     assert bench.union_rows(idx, 4, 8) == 6 + 2
+
+
+def test_union_rows_matches_brute_force():
+    """union_rows against a plain set union on random selections with padding,
+    out-of-range entries and ragged last groups."""
+    import torch
+    import bench
+    gen = torch.Generator().manual_seed(7)
+    for B, Tq, k, L, group in ((2, 37, 9, 50, 8), (1, 16, 5, 20, 16), (3, 10, 4, 12, 4)):
+        idx = torch.randint(-2, L + 3, (B, Tq, k), generator=gen, dtype=torch.int32)
+        expect = 0
+        for b in range(B):
+            for g0 in range(0, Tq, group):
+                rows = idx[b, g0:g0 + group].reshape(-1).tolist()
+                expect += len({s for s in rows if 0 <= s < L})
+        assert bench.union_rows(idx, group, L) == expect
